@@ -1,0 +1,12 @@
+"""B200-native blockwise band Sinkhorn attention (C-ABI library libeot + thin binding).
+
+Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science
+2605.08123).  See include/eot.h for the C ABI.  Importing this package requires the built
+library (``python -m entropic_ot_attention_b200.build``); there is no fallback path.
+"""
+from . import _abi
+from .api import (SinkhornAttentionFn, make_problem, resolved_impl, sinkhorn_attention, sinkhorn_bwd,
+                  sinkhorn_fwd, workspace)
+
+__all__ = ["sinkhorn_attention", "sinkhorn_fwd", "sinkhorn_bwd", "SinkhornAttentionFn", "make_problem",
+           "workspace", "resolved_impl", "_abi"]

@@ -1,0 +1,127 @@
+"""ctypes binding of libeot's C ABI (include/eot.h): argument marshalling only.
+
+Every function here has the name of the C entry point it wraps and forwards plain
+pointers and sizes; all computation happens in the library's CUDA kernels.  Importing this
+module fails loudly when libeot.so is missing: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libeot.so")
+
+EOT_OK = 0
+EOT_ERR_INVALID_ARGUMENT = 1
+EOT_ERR_UNSUPPORTED = 2
+EOT_ERR_WORKSPACE_TOO_SMALL = 3
+EOT_ERR_CUDA = 4
+EOT_ERR_NONFINITE = 5
+EOT_ERR_TIMEOUT = 6
+
+EOT_FP32 = 0
+EOT_BF16 = 1
+EOT_IMPL_AUTO = 0
+EOT_IMPL_SIMT = 1
+EOT_IMPL_TCGEN05 = 2
+
+
+class eot_problem(ctypes.Structure):
+    """Mirror of ``eot_problem`` in include/eot.h (field order and types must match)."""
+
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("L", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("W", ctypes.c_int32), ("T", ctypes.c_int32), ("R", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("dustbin", ctypes.c_int32), ("dustbin_index", ctypes.c_int32),
+        ("dustbin_mass", ctypes.c_float), ("dustbin_self", ctypes.c_int32), ("impl", ctypes.c_int32),
+    ]
+
+
+class EotError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {eot_status_string(status)} (status {status})")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libeot.so not found at {LIB_PATH}; build it with "
+                      "`python entropic_ot_attention_b200/build.py` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.POINTER(eot_problem)
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+lib.eot_abi_version.restype = ctypes.c_int
+lib.eot_validate.argtypes = [_P]
+lib.eot_validate.restype = ctypes.c_int
+lib.eot_resolved_impl.argtypes = [_P]
+lib.eot_resolved_impl.restype = ctypes.c_int
+lib.eot_workspace_bytes.argtypes = [_P, ctypes.c_int]
+lib.eot_workspace_bytes.restype = _sz
+lib.eot_status_string.argtypes = [ctypes.c_int]
+lib.eot_status_string.restype = ctypes.c_char_p
+lib.eot_sinkhorn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.eot_sinkhorn_fwd.restype = ctypes.c_int
+lib.eot_sinkhorn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.eot_sinkhorn_bwd.restype = ctypes.c_int
+lib.eot_last_device_status.argtypes = [_vp, _vp]
+lib.eot_last_device_status.restype = ctypes.c_int
+lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+lib.eot_device_status_bits.restype = ctypes.c_int
+
+# Every symbol declared in include/eot.h (checked by the CPU tests).
+EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sinkhorn_bwd",
+            "eot_last_device_status", "eot_device_status_bits", "eot_status_string",
+            "eot_abi_version", "eot_resolved_impl")
+
+
+def eot_status_string(status: int) -> str:
+    return lib.eot_status_string(int(status)).decode()
+
+
+def eot_abi_version() -> int:
+    return lib.eot_abi_version()
+
+
+def eot_validate(p: eot_problem) -> int:
+    return lib.eot_validate(ctypes.byref(p))
+
+
+def eot_resolved_impl(p: eot_problem) -> int:
+    return lib.eot_resolved_impl(ctypes.byref(p))
+
+
+def eot_workspace_bytes(p: eot_problem, for_backward: bool) -> int:
+    return int(lib.eot_workspace_bytes(ctypes.byref(p), int(bool(for_backward))))
+
+
+def _check(status: int, what: str) -> None:
+    if status != EOT_OK:
+        raise EotError(status, what)
+
+
+def eot_sinkhorn_fwd(p: eot_problem, Q: int, K: int, V: int, mask: int | None, O: int, u_tail: int,
+                     v_tail: int, workspace: int, workspace_bytes: int, stream: int) -> None:
+    """Forward; all tensor arguments are raw device addresses (ints), mask may be None."""
+    _check(lib.eot_sinkhorn_fwd(ctypes.byref(p), Q, K, V, mask, O, u_tail, v_tail, workspace,
+                                workspace_bytes, stream), "eot_sinkhorn_fwd")
+
+
+def eot_sinkhorn_bwd(p: eot_problem, Q: int, K: int, V: int, mask: int | None, u_tail: int, v_tail: int,
+                     dO: int, dQ: int, dK: int, dV: int, workspace: int, workspace_bytes: int,
+                     stream: int) -> None:
+    """Backward; raw device addresses as in eot_sinkhorn_fwd."""
+    _check(lib.eot_sinkhorn_bwd(ctypes.byref(p), Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
+                                workspace_bytes, stream), "eot_sinkhorn_bwd")
+
+
+def eot_last_device_status(workspace: int, stream: int) -> int:
+    return lib.eot_last_device_status(workspace, stream)
+
+
+def eot_device_status_bits(workspace: int, stream: int) -> int:
+    bits = ctypes.c_uint32(0)
+    _check(lib.eot_device_status_bits(workspace, stream, ctypes.byref(bits)), "eot_device_status_bits")
+    return int(bits.value)

@@ -1,0 +1,384 @@
+// C-ABI entry points of libeot (declared in include/eot.h): validation, workspace layout,
+// and the order of the band sweeps that make up the forward and backward passes.
+//
+// Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science
+// 2605.08123).  §2.1: T stopped balanced steps, then R tail steps, then O = diag(1/a) P V.
+// §2.2: the exact tail adjoint is a chain of band sweeps over one reference plan P(R,R);
+// every other staircase factor is P(R,R) times per-row / per-column orbit factors.
+// §2.3: the dustbin token is one more active position linked to every real token.
+#include <math.h>
+#include <string.h>
+
+#include "kernels.cuh"
+
+using namespace eot;
+
+namespace {
+
+bool tensor_core_ok(const eot_problem& p) { return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128); }
+
+int resolve_impl(const eot_problem& p) {
+    if (p.impl == EOT_IMPL_SIMT) return EOT_IMPL_SIMT;
+    Geom g{};
+    g.d = p.d;
+    g.dtype = p.dtype;
+    const bool tc = tensor_core_ok(p) && tc_supported(g);
+    if (p.impl == EOT_IMPL_TCGEN05) return tc ? EOT_IMPL_TCGEN05 : -1;
+    return tc ? EOT_IMPL_TCGEN05 : EOT_IMPL_SIMT;
+}
+
+eot_status validate(const eot_problem* p) {
+    if (!p) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->B < 0 || p->H < 0 || p->L < 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->L % 128 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->d < 8 || p->d > 128 || p->d % 8 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->W < 0 || p->T < 0 || p->R < 0 || p->R > kMaxR) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->dtype != EOT_FP32 && p->dtype != EOT_BF16) return EOT_ERR_INVALID_ARGUMENT;
+    if (!(p->scale >= 0.f) || !isfinite(p->scale)) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->dustbin != 0 && p->dustbin != 1) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->dustbin_self != 0 && p->dustbin_self != 1) return EOT_ERR_INVALID_ARGUMENT;
+    if (p->dustbin) {
+        if (p->dustbin_index < 0 || p->dustbin_index >= p->L) return EOT_ERR_INVALID_ARGUMENT;
+        if (!(p->dustbin_mass >= 0.f && p->dustbin_mass < 1.f)) return EOT_ERR_INVALID_ARGUMENT;
+    }
+    if (p->impl < EOT_IMPL_AUTO || p->impl > EOT_IMPL_TCGEN05) return EOT_ERR_INVALID_ARGUMENT;
+    if (int64_t(p->B) * p->H > 65535) return EOT_ERR_UNSUPPORTED;
+    if (int64_t(p->B) * p->H * p->L * int64_t(p->d) >= (int64_t(1) << 40)) return EOT_ERR_UNSUPPORTED;
+    if (resolve_impl(*p) < 0) return EOT_ERR_UNSUPPORTED;
+    return EOT_OK;
+}
+
+bool empty(const eot_problem& p) { return int64_t(p.B) * p.H * p.L == 0; }
+
+Geom make_geom(const eot_problem& p) {
+    Geom g{};
+    g.B = p.B;
+    g.H = p.H;
+    g.BH = p.B * p.H;
+    g.L = p.L;
+    g.d = p.d;
+    g.h = p.W / 2;
+    g.D = p.dustbin ? p.dustbin_index : -1;
+    g.dself = p.dustbin_self;
+    g.scale = p.scale > 0.f ? p.scale : 1.0f / sqrtf(float(p.d));
+    g.dtype = p.dtype;
+    return g;
+}
+
+template <typename T> T* at(void* ws, size_t off) { return reinterpret_cast<T*>(static_cast<char*>(ws) + off); }
+
+#define EOT_TRY(expr)                                  \
+    do {                                               \
+        cudaError_t e_ = (expr);                       \
+        if (e_ != cudaSuccess) return EOT_ERR_CUDA;    \
+    } while (0)
+
+cudaError_t run_lse(int impl, const LsePass& lp, cudaStream_t st) {
+    return impl == EOT_IMPL_TCGEN05 ? launch_tc_lse(lp, st) : launch_simt_lse(lp, st);
+}
+
+cudaError_t run_bwd(int impl, const BwdPass& bp, cudaStream_t st) {
+    return impl == EOT_IMPL_TCGEN05 ? launch_tc_bwd(bp, st) : launch_simt_bwd(bp, st);
+}
+
+}  // namespace
+
+// Forward/backward bodies that take the workspace as an already-resolved device address.
+// (Also used by entry points that supply their own scratch.)
+namespace eot {
+
+eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
+                        void* O, float* u_tail, float* v_tail, void* ws, cudaStream_t st) {
+    const Geom g = make_geom(*p);
+    const int impl = resolve_impl(*p);
+    const WsLayout w = ws_layout(*p, false);
+    const size_t L = size_t(p->L), R = size_t(p->R);
+    const size_t pstride = (R + 1) * L;
+    uint32_t* status = at<uint32_t>(ws, w.status);
+    float* logm = at<float>(ws, w.logm);
+    float* sd_row = p->dustbin ? at<float>(ws, w.sd_row) : nullptr;
+    float* sd_col = p->dustbin ? at<float>(ws, w.sd_col) : nullptr;
+
+    EOT_TRY(launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st));
+    if (p->dustbin) EOT_TRY(launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st));
+    const size_t tail_bytes = size_t(g.BH) * pstride * sizeof(float);
+    EOT_TRY(cudaMemsetAsync(u_tail, 0, tail_bytes, st));
+    EOT_TRY(cudaMemsetAsync(v_tail, 0, tail_bytes, st));
+
+    LsePass row{};
+    row.g = g;
+    row.X = Q;
+    row.Y = K;
+    row.logm = logm;
+    row.pstride = pstride;
+    row.sd_term = sd_row;
+    row.sd_dense = sd_col;
+    row.status = status;
+    LsePass col = row;
+    col.X = K;
+    col.Y = Q;
+    col.sd_term = sd_col;
+    col.sd_dense = sd_row;
+
+    bool first = true;
+    auto step = [&](int k_in, int k_out) -> cudaError_t {
+        // row half-step: u(k_out) from v(k_in); column half-step: v(k_out) from u(k_out)
+        row.colpot = v_tail + size_t(k_in) * L;
+        row.stab = first ? nullptr : u_tail + size_t(k_in) * L;
+        row.out = u_tail + size_t(k_out) * L;
+        cudaError_t e = run_lse(impl, row, st);
+        if (e != cudaSuccess) return e;
+        first = false;
+        col.colpot = u_tail + size_t(k_out) * L;
+        col.stab = v_tail + size_t(k_in) * L;
+        col.out = v_tail + size_t(k_out) * L;
+        return run_lse(impl, col, st);
+    };
+    for (int t = 0; t < p->T; ++t) EOT_TRY(step(0, 0));                 // stopped base
+    for (int k = 1; k <= p->R; ++k) EOT_TRY(step(k - 1, k));            // differentiable tail
+
+    // Output O = diag(1/a) P(R,R) V (a vector sweep with coefficients P / a_r).
+    BwdVecArgs va{};
+    va.kind = kPassOut;
+    va.R = p->R;
+    va.H = g.H;
+    va.BH = g.BH;
+    va.L = g.L;
+    va.logm = logm;
+    va.u_tail = u_tail;
+    va.v_tail = v_tail;
+    va.pr = at<float>(ws, w.opr);
+    va.pc = at<float>(ws, w.opc);
+    va.f = va.hv = va.m = nullptr;            // unused by the output pass
+    EOT_TRY(launch_bwd_vectors(va, st));
+    BwdPass op{};
+    op.g = g;
+    op.X = Q;
+    op.Y = K;
+    op.Z = V;
+    op.logm = logm;
+    op.pr = va.pr;
+    op.pc = va.pc;
+    op.vout = O;
+    op.vscale = 1.f;
+    op.v_dp = 0;
+    op.nmod = 0;
+    op.sd_term = sd_row;
+    op.sd_dense = sd_col;
+    op.status = status;
+    EOT_TRY(run_bwd(impl, op, st));
+    return EOT_OK;
+}
+
+eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
+                         const float* u_tail, const float* v_tail, const void* dO, void* dQ, void* dK, void* dV,
+                         void* ws, cudaStream_t st) {
+    const Geom g = make_geom(*p);
+    const int impl = resolve_impl(*p);
+    const WsLayout w = ws_layout(*p, true);
+    const int R = p->R;
+    const size_t vecn = align256(size_t(g.BH) * g.L * sizeof(float)) / sizeof(float);
+    uint32_t* status = at<uint32_t>(ws, w.status);
+    float* logm = at<float>(ws, w.logm);
+    float *sd_row = nullptr, *sd_col = nullptr, *e1 = nullptr, *e2 = nullptr;
+    EOT_TRY(launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st));
+    if (p->dustbin) {
+        sd_row = at<float>(ws, w.sd_row);
+        sd_col = at<float>(ws, w.sd_col);
+        e1 = at<float>(ws, w.e1);
+        e2 = at<float>(ws, w.e2);
+        EOT_TRY(launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st));
+        EOT_TRY(launch_dustbin_dots(g, dO, V, 1.f, e1, e2, st));   // e1[r] = <dO_r, V_D>, e2[r] = <dO_D, V_r>
+    }
+    float* alpha = at<float>(ws, w.alpha);
+    float* beta = at<float>(ws, w.beta);
+
+    BwdVecArgs va{};
+    va.R = R;
+    va.H = g.H;
+    va.BH = g.BH;
+    va.L = g.L;
+    va.logm = logm;
+    va.u_tail = u_tail;
+    va.v_tail = v_tail;
+    va.alpha = alpha;
+    va.beta = beta;
+    va.pr = at<float>(ws, w.pr);
+    va.pc = at<float>(ws, w.pc);
+    va.f = at<float>(ws, w.f);
+    va.hv = at<float>(ws, w.hv);
+    va.m = at<float>(ws, w.m);
+    va.xr = R > 0 ? at<float>(ws, w.xr) : nullptr;
+    va.yc = R > 0 ? at<float>(ws, w.yc) : nullptr;
+
+    // Row orientation: S = Q K^T, dP = dO V^T.  Column orientation: S^T = K Q^T, dP^T = V dO^T.
+    BwdPass rowp{};
+    rowp.g = g;
+    rowp.X = Q;
+    rowp.Y = K;
+    rowp.A = dO;
+    rowp.Bm = V;
+    rowp.logm = logm;
+    rowp.pr = va.pr;
+    rowp.pc = va.pc;
+    rowp.sd_term = sd_row;
+    rowp.sd_dense = sd_col;
+    rowp.dp_term = e1;
+    rowp.dp_dense = e2;
+    rowp.status = status;
+    BwdPass colp = rowp;
+    colp.X = K;
+    colp.Y = Q;
+    colp.A = V;
+    colp.Bm = dO;
+    colp.sd_term = sd_col;
+    colp.sd_dense = sd_row;
+    colp.dp_term = e2;
+    colp.dp_dense = e1;
+
+    auto vec = [&](int kind, int k) -> cudaError_t {
+        va.kind = kind;
+        va.k = k;
+        return launch_bwd_vectors(va, st);
+    };
+    auto scalar_pass = [&](BwdPass bp, float* out, bool dp) -> cudaError_t {
+        bp.sout = out;
+        bp.f = va.f;
+        bp.hv = va.hv;
+        bp.m = va.m;
+        bp.s_dp = dp ? 1 : 0;
+        return run_bwd(impl, bp, st);
+    };
+
+    // C1: beta_R = colsum(P(R,R) * dP) and dV = P(R,R)^T (dO / a)   (one column sweep)
+    EOT_TRY(vec(kPassC1, 0));
+    {
+        BwdPass bp = colp;
+        if (R > 0) {
+            bp.sout = beta + size_t(R) * vecn;
+            bp.f = va.f;
+            bp.hv = va.hv;
+            bp.m = nullptr;
+            bp.s_dp = 1;
+        }
+        bp.vout = dV;
+        bp.Z = dO;
+        bp.vscale = 1.f;
+        bp.v_dp = 0;
+        bp.nmod = 0;
+        EOT_TRY(run_bwd(impl, bp, st));
+    }
+    if (R > 0) {
+        // R2: alpha_R = rowsum(P(R,R) * dP) - P(R,R) (beta_R / b)
+        EOT_TRY(vec(kPassR2, 0));
+        EOT_TRY(scalar_pass(rowp, alpha + size_t(R) * vecn, true));
+        for (int k = R - 1; k >= 1; --k) {
+            // beta_k = -P(k+1,k)^T (alpha_{k+1} / a), alpha_k = -P(k,k) (beta_k / b)
+            EOT_TRY(vec(kPassCk, k));
+            EOT_TRY(scalar_pass(colp, beta + size_t(k) * vecn, false));
+            EOT_TRY(vec(kPassRk, k));
+            EOT_TRY(scalar_pass(rowp, alpha + size_t(k) * vecn, false));
+        }
+    }
+    // dQ = scale dS K (row sweep), dK = scale dS^T Q (column sweep); dS = P(R,R) (dP - sum x y^T)
+    for (int orient = 0; orient < 2; ++orient) {
+        EOT_TRY(vec(orient == 0 ? kPassRF : kPassCF, 0));
+        BwdPass bp = orient == 0 ? rowp : colp;
+        bp.vout = orient == 0 ? dQ : dK;
+        bp.Z = orient == 0 ? K : Q;
+        bp.vscale = g.scale;
+        bp.v_dp = 1;
+        bp.nmod = 2 * R;
+        for (int k = 0; k < 2 * R; ++k) {
+            bp.xr[k] = va.xr + size_t(k) * vecn;
+            bp.yc[k] = va.yc + size_t(k) * vecn;
+        }
+        EOT_TRY(run_bwd(impl, bp, st));
+    }
+    return EOT_OK;
+}
+
+}  // namespace eot
+
+// ---------------------------------------------------------------------------------------
+// Exported C ABI
+// ---------------------------------------------------------------------------------------
+extern "C" {
+
+int eot_abi_version(void) { return EOT_ABI_VERSION; }
+
+eot_status eot_validate(const eot_problem* p) { return validate(p); }
+
+int eot_resolved_impl(const eot_problem* p) {
+    if (validate(p) != EOT_OK) return -1;
+    return resolve_impl(*p);
+}
+
+size_t eot_workspace_bytes(const eot_problem* p, int for_backward) {
+    if (validate(p) != EOT_OK || empty(*p)) return 0;
+    return ws_layout(*p, for_backward != 0).total;
+}
+
+const char* eot_status_string(eot_status s) {
+    switch (s) {
+        case EOT_OK: return "ok";
+        case EOT_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case EOT_ERR_UNSUPPORTED: return "unsupported problem for this build";
+        case EOT_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case EOT_ERR_CUDA: return "CUDA error";
+        case EOT_ERR_NONFINITE: return "non-finite potential produced on the device";
+        case EOT_ERR_TIMEOUT: return "a bounded device wait ran out";
+    }
+    return "unknown status";
+}
+
+eot_status eot_sinkhorn_fwd(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
+                            void* O, float* u_tail, float* v_tail, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (empty(*p)) return EOT_OK;
+    if (!Q || !K || !V || !O || !u_tail || !v_tail || !workspace) return EOT_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
+    return forward_impl(p, Q, K, V, mask, O, u_tail, v_tail, workspace, static_cast<cudaStream_t>(stream));
+}
+
+eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
+                            const float* u_tail, const float* v_tail, const void* dO, void* dQ, void* dK, void* dV,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (empty(*p)) return EOT_OK;
+    if (!Q || !K || !V || !u_tail || !v_tail || !dO || !dQ || !dK || !dV || !workspace)
+        return EOT_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < ws_layout(*p, true).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
+    return backward_impl(p, Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
+                         static_cast<cudaStream_t>(stream));
+}
+
+eot_status eot_device_status_bits(void* workspace, void* stream, uint32_t* bits) {
+    if (!workspace || !bits) return EOT_ERR_INVALID_ARGUMENT;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return EOT_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EOT_ERR_CUDA;
+    *bits = v;
+    return EOT_OK;
+}
+
+eot_status eot_last_device_status(void* workspace, void* stream) {
+    uint32_t bits = 0;
+    eot_status s = eot_device_status_bits(workspace, stream, &bits);
+    if (s != EOT_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st) != cudaSuccess) return EOT_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EOT_ERR_CUDA;
+    if (bits & kStatusTimeout) return EOT_ERR_TIMEOUT;
+    if (bits & kStatusNonFinite) return EOT_ERR_NONFINITE;
+    return EOT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Shared definitions of libeot: pass parameters, workspace layout, small device helpers.
+//
+// Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science
+// 2605.08123), §2.1-§2.3.  Every band sweep below evaluates, for each "row" r of one
+// (batch, head) unit and the columns c in its band |r - c| <= h (h = W / 2), the score
+// S_rc = scale <X_r, Y_c>.  A row half-step uses (X, Y) = (Q, K); a column half-step is the
+// same sweep with (X, Y) = (K, Q) because the band and the dustbin links are symmetric.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/eot.h"
+
+namespace eot {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxR = 8;
+constexpr int kMaxMods = 2 * kMaxR;
+
+// Device status bits (first word of every workspace).
+constexpr uint32_t kStatusNonFinite = 1u;
+constexpr uint32_t kStatusTimeout = 2u;
+
+// Problem geometry as the kernels see it.
+struct Geom {
+    int B, H, BH, L, d;
+    int h;          // band half-width W / 2
+    int D;          // dustbin position, or -1 (active iff logm[D] > -inf)
+    int dself;      // (D, D) in the support
+    float scale;    // score scale (natural units)
+    int dtype;      // eot_dtype
+};
+
+// One log-sum-exp half-step (§2.1):
+//   out_r = logm_r - LSE_{c in band(r), active, c != D} (S_rc + colpot_c) [+ dustbin entry]
+struct LsePass {
+    Geom g;
+    const void* X;          // [BH, L, d] row-side operand of S
+    const void* Y;          // [BH, L, d] column-side operand of S
+    const float* logm;      // [B, L] log marginals, -inf for inactive positions
+    const float* colpot;    // potential of the column side (natural log)
+    const float* stab;      // previous value of this row potential, or nullptr
+    float* out;             // new row potential (0 for inactive rows)
+    size_t pstride;         // unit stride of colpot / stab / out (elements): L or (R+1) L
+    const float* sd_term;   // [BH, L] S between row r and the dustbin column (dustbin only)
+    const float* sd_dense;  // [BH, L] S between the dustbin row and column c (dustbin only)
+    uint32_t* status;
+};
+
+// One backward sweep (§2.2).  With Pt_rc = exp(S_rc + pr_r + pc_c) on the support:
+//   scalar : sout_r = f_r * ( sum_c Pt_rc * dP_rc [if s_dp] + hv_r * sum_c Pt_rc * m_c )
+//   vector : vout_r = vscale * sum_c coef_rc Z_c,
+//            coef_rc = Pt_rc * ( (v_dp ? dP_rc : 1) - sum_k xr_k[r] * yc_k[c] )
+// where dP_rc = <A_r, Bm_c>.  Any of the vectors may be nullptr when unused.
+struct BwdPass {
+    Geom g;
+    const void* X;
+    const void* Y;
+    const void* A;          // row-side dP operand
+    const void* Bm;         // column-side dP operand
+    const void* Z;          // column-side operand of the vector output
+    const float* logm;
+    const float* pr;        // [BH, L]
+    const float* pc;        // [BH, L] (value at D used for the dustbin links)
+    float* sout;            // scalar output or nullptr
+    const float* f;
+    const float* hv;
+    const float* m;
+    int s_dp;
+    void* vout;             // vector output [BH, L, d] (dtype) or nullptr
+    float vscale;
+    int v_dp;
+    int nmod;
+    const float* xr[kMaxMods];
+    const float* yc[kMaxMods];
+    const float* sd_term;   // dustbin links of S (as in LsePass)
+    const float* sd_dense;
+    const float* dp_term;   // <A_r, Bm_D>
+    const float* dp_dense;  // <A_D, Bm_c>
+    uint32_t* status;
+};
+
+// Workspace layout.  Every region is 256-byte aligned; offsets in bytes.
+struct WsLayout {
+    size_t status, logm, sd_row, sd_col, e1, e2;
+    size_t opr, opc;        // forward output pass: row / column biases
+    size_t pr, pc, f, hv, m;
+    size_t xr, yc;          // kMaxMods vectors each, [BH, L]
+    size_t alpha, beta;     // (R + 1) vectors each, [BH, L]
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
+    WsLayout w{};
+    const size_t BH = size_t(p.B) * p.H, L = size_t(p.L);
+    const size_t vec = align256(BH * L * sizeof(float));
+    size_t o = 0;
+    w.status = o; o += 256;
+    w.logm = o; o += align256(size_t(p.B) * L * sizeof(float));
+    if (p.dustbin) {
+        w.sd_row = o; o += vec;
+        w.sd_col = o; o += vec;
+        if (bwd) { w.e1 = o; o += vec; w.e2 = o; o += vec; }
+    }
+    if (!bwd) {
+        w.opr = o; o += vec;
+        w.opc = o; o += vec;
+    }
+    if (bwd) {
+        w.pr = o; o += vec;
+        w.pc = o; o += vec;
+        w.f = o; o += vec;
+        w.hv = o; o += vec;
+        w.m = o; o += vec;
+        w.xr = o; o += vec * 2 * p.R;
+        w.yc = o; o += vec * 2 * p.R;
+        w.alpha = o; o += vec * (p.R + 1);
+        w.beta = o; o += vec * (p.R + 1);
+    }
+    w.total = o;
+    return w;
+}
+
+// ---------------------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// Merge two (max, sum) log-sum-exp partials in the log2 domain.
+__device__ __forceinline__ void lse2_merge(float& m, float& s, float m2, float s2) {
+    float M = fmaxf(m, m2);
+    if (M == neg_inf()) return;
+    float a = (m == neg_inf()) ? 0.f : s * exp2f(m - M);
+    float b = (m2 == neg_inf()) ? 0.f : s2 * exp2f(m2 - M);
+    m = M;
+    s = a + b;
+}
+
+__device__ __forceinline__ void lse2_add(float& m, float& s, float x) {
+    if (x == neg_inf()) return;
+    if (x > m) {
+        s = (m == neg_inf() ? 0.f : s * exp2f(m - x)) + 1.f;
+        m = x;
+    } else {
+        s += exp2f(x - m);
+    }
+}
+
+}  // namespace eot

@@ -1,0 +1,35 @@
+// Kernel launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace eot {
+
+// Kinds of per-position vector preparation (forward output and backward sweeps, §2.2).
+enum PassKind { kPassOut = 0, kPassC1, kPassR2, kPassCk, kPassRk, kPassRF, kPassCF };
+
+struct BwdVecArgs {
+    int kind, k, R, H, BH, L;
+    const float* logm;      // [B, L]
+    const float* u_tail;    // [BH, R+1, L]
+    const float* v_tail;    // [BH, R+1, L]
+    const float* alpha;     // [R+1][BH*L]
+    const float* beta;      // [R+1][BH*L]
+    float *pr, *pc, *f, *hv, *m;
+    float *xr, *yc;         // [2R][BH*L]
+};
+
+cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
+                                  uint32_t* status, cudaStream_t st);
+cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
+                                cudaStream_t st);
+cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st);
+cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
+cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
+
+// Tensor-core (tcgen05 + TMA) kernels; return cudaErrorNotSupported when not built.
+bool tc_supported(const Geom& g);
+cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st);
+cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
+
+}  // namespace eot

@@ -1,0 +1,569 @@
+// CUDA-core kernels of libeot: marginal/dustbin preparation, the fp32 (and reference bf16)
+// band sweeps, the dense dustbin row, and the backward vector preparation.
+//
+// Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science
+// 2605.08123): §2.1 balanced log-domain Sinkhorn on a fixed band support with the
+// temperature absorbed into S; §2.2 exact adjoint of the refinement tail through one
+// reference plan and per-row / per-column orbit factors; §2.3 dustbin token on an extended
+// state space.
+//
+// Tiling of the CUDA-core sweeps: a CTA owns 32 rows of one unit and walks the 32-column
+// tiles that intersect the band of those rows.  Each of its 8 warps owns 4 rows; lane l
+// owns column l of the current tile.  Row-side operands stay in shared memory for the
+// whole sweep, column-side operands are staged per tile.  Scores are exact fp32 dot
+// products (FFMA), which keeps fp32 inputs at fp32 accuracy.
+#include "kernels.cuh"
+
+namespace eot {
+
+constexpr int kSB = 32;    // rows per CTA == columns per tile
+constexpr int kSNT = 256;  // threads per CTA
+
+// ---------------------------------------------------------------------------------------
+// Preparation
+// ---------------------------------------------------------------------------------------
+
+// Uniform marginals over the active real tokens (§2.1), dustbin mass (§2.3).  One CTA per
+// batch row.  logm[b, i] = log a_i, -inf for inactive positions.
+__global__ void __launch_bounds__(256) prep_marginals_kernel(Geom g, const uint8_t* mask, int dustbin,
+                                                             float mass, float* logm, uint32_t* status) {
+    const int b = blockIdx.x;
+    const int L = g.L;
+    const int D = dustbin ? g.D : L;
+    __shared__ int red[256];
+    int cnt = 0;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+        int real = (mask ? (mask[size_t(b) * L + i] != 0) : 1) && (i < D);
+        cnt += real;
+    }
+    red[threadIdx.x] = cnt;
+    __syncthreads();
+    for (int s = 128; s > 0; s >>= 1) {
+        if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
+        __syncthreads();
+    }
+    const int n = red[0];
+    const bool use_db = dustbin && n > 0 && mass > 0.f;
+    const double real_mass = use_db ? (1.0 - double(mass)) : 1.0;
+    const float lr = n > 0 ? float(log(real_mass / double(n))) : neg_inf();
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+        int real = (mask ? (mask[size_t(b) * L + i] != 0) : 1) && (i < D);
+        float v = real ? lr : neg_inf();
+        if (dustbin && i == D) v = use_db ? float(log(double(mass))) : neg_inf();
+        logm[size_t(b) * L + i] = v;
+    }
+    if (b == 0 && threadIdx.x == 0 && status) *status = 0u;
+}
+
+// Dustbin link vectors: out_term[r] = s1 * <P_r, Q_D>, out_dense[r] = s1 * <P_D, Q_r> for
+// every position r of every unit (used for S and, in the backward, for dP).
+template <typename T>
+__global__ void __launch_bounds__(256) prep_dustbin_dots_kernel(Geom g, const T* P, const T* Qm, float s1,
+                                                                float* out_term, float* out_dense) {
+    const int bh = blockIdx.y;
+    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= g.L) return;
+    const size_t base = size_t(bh) * g.L;
+    const T* pr = P + (base + r) * g.d;
+    const T* pD = P + (base + g.D) * g.d;
+    const T* qr = Qm + (base + r) * g.d;
+    const T* qD = Qm + (base + g.D) * g.d;
+    float a = 0.f, b = 0.f;
+    for (int k = 0; k < g.d; ++k) {
+        a = fmaf(to_f(pr[k]), to_f(qD[k]), a);
+        b = fmaf(to_f(pD[k]), to_f(qr[k]), b);
+    }
+    out_term[base + r] = s1 * a;
+    out_dense[base + r] = s1 * b;
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward half-step on CUDA cores (online max; fp32 scores)
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
+    extern __shared__ float sm[];
+    const int d = p.g.d, ld = d + 1, L = p.g.L, h = p.g.h, D = p.g.D;
+    float* Xs = sm;
+    float* Ys = Xs + kSB * ld;
+    float* bs = Ys + kSB * ld;
+    const int bh = blockIdx.y, b = bh / p.g.H;
+    const int r0 = blockIdx.x * kSB;
+    const size_t base = size_t(bh) * L;
+    const size_t pb = size_t(bh) * p.pstride;
+    const T* X = static_cast<const T*>(p.X) + base * d;
+    const T* Y = static_cast<const T*>(p.Y) + base * d;
+    const float* logm = p.logm + size_t(b) * L;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float sl2 = p.g.scale * kLog2e;
+    const bool d_act = (D >= 0) && (logm[D] != neg_inf());
+
+    for (int e = threadIdx.x; e < kSB * d; e += kSNT) {
+        int r = e / d, k = e - r * d;
+        Xs[r * ld + k] = to_f(X[size_t(r0 + r) * d + k]);
+    }
+    float m[4], s[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) { m[q] = neg_inf(); s[q] = 0.f; }
+
+    const int clo = max(0, r0 - h), chi = min(L - 1, r0 + kSB - 1 + h);
+    for (int t = clo / kSB; t <= chi / kSB; ++t) {
+        const int c0 = t * kSB;
+        __syncthreads();
+        for (int e = threadIdx.x; e < kSB * d; e += kSNT) {
+            int r = e / d, k = e - r * d;
+            Ys[r * ld + k] = to_f(Y[size_t(c0 + r) * d + k]);
+        }
+        if (threadIdx.x < kSB) {
+            const int c = c0 + threadIdx.x;
+            const bool act = logm[c] != neg_inf() && c != D;
+            bs[threadIdx.x] = act ? p.colpot[pb + c] * kLog2e : neg_inf();
+        }
+        __syncthreads();
+        const int c = c0 + lane;
+        const float bc = bs[lane];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int rl = warp * 4 + q, r = r0 + rl;
+            float acc = 0.f;
+            for (int k = 0; k < d; ++k) acc = fmaf(Xs[rl * ld + k], Ys[lane * ld + k], acc);
+            float x = fmaf(acc, sl2, bc);
+            if (abs(r - c) > h) x = neg_inf();
+            lse2_add(m[q], s[q], x);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            float m2 = __shfl_xor_sync(0xffffffffu, m[q], off);
+            float s2 = __shfl_xor_sync(0xffffffffu, s[q], off);
+            lse2_merge(m[q], s[q], m2, s2);
+        }
+    }
+    if (lane < 4) {
+        const int q = lane;
+        const int r = r0 + warp * 4 + q;
+        float mq = m[0], sq = s[0];
+#pragma unroll
+        for (int j = 1; j < 4; ++j) if (q == j) { mq = m[j]; sq = s[j]; }
+        const float lm = logm[r];
+        if (r == D && d_act) return;  // written by the dense dustbin row
+        float outv = 0.f;
+        if (lm != neg_inf()) {
+            if (d_act) lse2_add(mq, sq, (p.sd_term[base + r] + p.colpot[pb + D]) * kLog2e);
+            outv = lm - (mq + log2f(sq)) * kLn2;
+            if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+        }
+        p.out[pb + r] = outv;
+    }
+}
+
+// Dense dustbin row of a half-step: out_D = logm_D - LSE_c (S_Dc + colpot_c) over every
+// active real c, plus (D, D) when it is in the support.  One CTA per unit.
+__global__ void __launch_bounds__(256) dustbin_lse_kernel(LsePass p) {
+    const int bh = blockIdx.x, b = bh / p.g.H, L = p.g.L, D = p.g.D;
+    const size_t base = size_t(bh) * L;
+    const size_t pb = size_t(bh) * p.pstride;
+    const float* logm = p.logm + size_t(b) * L;
+    if (D < 0 || logm[D] == neg_inf()) return;
+    float m = neg_inf(), s = 0.f;
+    for (int c = threadIdx.x; c < L; c += blockDim.x) {
+        if (c == D || logm[c] == neg_inf()) continue;
+        lse2_add(m, s, (p.sd_dense[base + c] + p.colpot[pb + c]) * kLog2e);
+    }
+    if (threadIdx.x == 0 && p.g.dself) lse2_add(m, s, (p.sd_term[base + D] + p.colpot[pb + D]) * kLog2e);
+    __shared__ float sm_m[256], sm_s[256];
+    sm_m[threadIdx.x] = m;
+    sm_s[threadIdx.x] = s;
+    __syncthreads();
+    for (int st = 128; st > 0; st >>= 1) {
+        if (threadIdx.x < st) {
+            float a = sm_m[threadIdx.x], bb = sm_s[threadIdx.x];
+            lse2_merge(a, bb, sm_m[threadIdx.x + st], sm_s[threadIdx.x + st]);
+            sm_m[threadIdx.x] = a;
+            sm_s[threadIdx.x] = bb;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        float outv = logm[D] - (sm_m[0] + log2f(sm_s[0])) * kLn2;
+        if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+        p.out[pb + D] = outv;
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward sweep on CUDA cores
+// ---------------------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSNT) simt_bwd_kernel(BwdPass p) {
+    extern __shared__ float sm[];
+    const int d = p.g.d, ld = d + 1, L = p.g.L, h = p.g.h, D = p.g.D;
+    const int nm = p.nmod;
+    const bool has_dp = (p.sout && p.s_dp) || (p.vout && p.v_dp);
+    float* Xs = sm;                       // [32][ld]
+    float* As = Xs + kSB * ld;            // [32][ld]
+    float* Ys = As + kSB * ld;            // [32][ld]
+    float* Bs = Ys + kSB * ld;            // [32][ld]
+    float* Zs = Bs + kSB * ld;            // [32][ld]
+    float* Cs = Zs + kSB * ld;            // [32][33] coefficients
+    float* colv = Cs + kSB * 33;          // [2 + nm][32]: pc, m, yc...
+    float* rowv = colv + (2 + kMaxMods) * kSB;  // [3 + nm][32]: pr, f, hv, xr...
+    const int bh = blockIdx.y, b = bh / p.g.H;
+    const int r0 = blockIdx.x * kSB;
+    const size_t base = size_t(bh) * L;
+    const float* logm = p.logm + size_t(b) * L;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float sc = p.g.scale;
+    const bool d_act = (D >= 0) && (logm[D] != neg_inf());
+    const T* X = static_cast<const T*>(p.X) + base * d;
+    const T* Y = static_cast<const T*>(p.Y) + base * d;
+    const T* A = has_dp ? static_cast<const T*>(p.A) + base * d : nullptr;
+    const T* Bm = has_dp ? static_cast<const T*>(p.Bm) + base * d : nullptr;
+    const T* Z = p.vout ? static_cast<const T*>(p.Z) + base * d : nullptr;
+
+    for (int e = threadIdx.x; e < kSB * d; e += kSNT) {
+        int r = e / d, k = e - r * d;
+        Xs[r * ld + k] = to_f(X[size_t(r0 + r) * d + k]);
+        if (has_dp) As[r * ld + k] = to_f(A[size_t(r0 + r) * d + k]);
+    }
+    if (threadIdx.x < kSB) {
+        const int r = r0 + threadIdx.x;
+        rowv[0 * kSB + threadIdx.x] = p.pr[base + r];
+        rowv[1 * kSB + threadIdx.x] = p.f ? p.f[base + r] : 1.f;
+        rowv[2 * kSB + threadIdx.x] = p.hv ? p.hv[base + r] : 0.f;
+        for (int k = 0; k < nm; ++k) rowv[(3 + k) * kSB + threadIdx.x] = p.xr[k][base + r];
+    }
+    float s1[4], s2[4], acc[4][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        s1[q] = s2[q] = 0.f;
+#pragma unroll
+        for (int z = 0; z < 4; ++z) acc[q][z] = 0.f;
+    }
+    const int clo = max(0, r0 - h), chi = min(L - 1, r0 + kSB - 1 + h);
+    for (int t = clo / kSB; t <= chi / kSB; ++t) {
+        const int c0 = t * kSB;
+        __syncthreads();
+        for (int e = threadIdx.x; e < kSB * d; e += kSNT) {
+            int r = e / d, k = e - r * d;
+            const size_t gi = size_t(c0 + r) * d + k;
+            Ys[r * ld + k] = to_f(Y[gi]);
+            if (has_dp) Bs[r * ld + k] = to_f(Bm[gi]);
+            if (Z) Zs[r * ld + k] = to_f(Z[gi]);
+        }
+        if (threadIdx.x < kSB) {
+            const int c = c0 + threadIdx.x;
+            const bool act = logm[c] != neg_inf() && c != D;
+            colv[threadIdx.x] = act ? p.pc[base + c] : neg_inf();
+            colv[kSB + threadIdx.x] = p.m ? p.m[base + c] : 0.f;
+            for (int k = 0; k < nm; ++k) colv[(2 + k) * kSB + threadIdx.x] = p.yc[k][base + c];
+        }
+        __syncthreads();
+        const int c = c0 + lane;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int rl = warp * 4 + q, r = r0 + rl;
+            float sacc = 0.f, dacc = 0.f;
+            for (int k = 0; k < d; ++k) sacc = fmaf(Xs[rl * ld + k], Ys[lane * ld + k], sacc);
+            if (has_dp)
+                for (int k = 0; k < d; ++k) dacc = fmaf(As[rl * ld + k], Bs[lane * ld + k], dacc);
+            float x = fmaf(sacc, sc, rowv[rl] + colv[lane]);
+            const bool in = (abs(r - c) <= h) && logm[r] != neg_inf() && r != D && x != neg_inf();
+            const float P = in ? expf(x) : 0.f;
+            if (p.sout) {
+                if (p.s_dp) s1[q] = fmaf(P, dacc, s1[q]);
+                s2[q] = fmaf(P, colv[kSB + lane], s2[q]);
+            }
+            if (p.vout) {
+                float mod = p.v_dp ? dacc : 1.f;
+                for (int k = 0; k < nm; ++k) mod -= rowv[(3 + k) * kSB + rl] * colv[(2 + k) * kSB + lane];
+                Cs[rl * 33 + lane] = P * mod;
+            }
+        }
+        if (p.vout) {
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int rl = warp * 4 + q;
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                    const int zc = lane + 32 * z;
+                    if (zc < d) {
+                        float a = acc[q][z];
+                        for (int cc = 0; cc < kSB; ++cc) a = fmaf(Cs[rl * 33 + cc], Zs[cc * ld + zc], a);
+                        acc[q][z] = a;
+                    }
+                }
+            }
+        }
+    }
+    // Finish the rows: lane reductions, dustbin link, writes.
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int rl = warp * 4 + q, r = r0 + rl;
+        if (p.sout) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                s1[q] += __shfl_xor_sync(0xffffffffu, s1[q], off);
+                s2[q] += __shfl_xor_sync(0xffffffffu, s2[q], off);
+            }
+        }
+        const bool ract = logm[r] != neg_inf();
+        if (r == D && d_act) continue;   // dense dustbin row kernel
+        float Pd = 0.f, dpd = 0.f, coefd = 0.f;
+        if (ract && d_act) {
+            Pd = expf(p.sd_term[base + r] + rowv[rl] + p.pc[base + D]);
+            if (has_dp) dpd = p.dp_term[base + r];
+            float mod = p.v_dp ? dpd : 1.f;
+            for (int k = 0; k < nm; ++k) mod -= rowv[(3 + k) * kSB + rl] * p.yc[k][base + D];
+            coefd = Pd * mod;
+        }
+        if (p.sout && lane == 0) {
+            float a = s1[q], bb = s2[q];
+            if (ract && d_act) {
+                if (p.s_dp) a = fmaf(Pd, dpd, a);
+                if (p.m) bb = fmaf(Pd, p.m[base + D], bb);
+            }
+            float outv = ract ? rowv[kSB + rl] * (a + rowv[2 * kSB + rl] * bb) : 0.f;
+            if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+            p.sout[base + r] = outv;
+        }
+        if (p.vout) {
+            T* vo = static_cast<T*>(p.vout) + (base + r) * d;
+            const T* zD = d_act ? static_cast<const T*>(p.Z) + (base + D) * d : nullptr;
+#pragma unroll
+            for (int z = 0; z < 4; ++z) {
+                const int zc = lane + 32 * z;
+                if (zc < d) {
+                    float a = acc[q][z];
+                    if (ract && d_act) a = fmaf(coefd, to_f(zD[zc]), a);
+                    vo[zc] = from_f<T>(ract ? p.vscale * a : 0.f);
+                }
+            }
+        }
+    }
+}
+
+// Dense dustbin row of a backward sweep (row r = D over every active real column, plus
+// (D, D)).  One CTA per unit.
+template <typename T>
+__global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
+    const int bh = blockIdx.x, b = bh / p.g.H, L = p.g.L, D = p.g.D, d = p.g.d;
+    const size_t base = size_t(bh) * L;
+    const float* logm = p.logm + size_t(b) * L;
+    if (D < 0 || logm[D] == neg_inf()) return;
+    const int nm = p.nmod;
+    const bool has_dp = (p.sout && p.s_dp) || (p.vout && p.v_dp);
+    const float prD = p.pr[base + D];
+    __shared__ float cs[256];
+    __shared__ float red1[256], red2[256];
+    __shared__ float vacc[256];
+    float a1 = 0.f, a2 = 0.f;
+    const T* Z = p.vout ? static_cast<const T*>(p.Z) + base * d : nullptr;
+    const int groups = d > 0 ? 256 / d : 1;      // threads per output element split over c
+    const int zc = threadIdx.x % d, grp = threadIdx.x / d;
+    float vpart = 0.f;
+    for (int c0 = 0; c0 < L + 1; c0 += 256) {
+        const int c = c0 + threadIdx.x;
+        float coef = 0.f;
+        // c == L stands for the (D, D) entry
+        const bool self = (c == L) && p.g.dself;
+        const bool band = (c < L) && c != D && logm[c] != neg_inf();
+        if (band || self) {
+            const int cc = self ? D : c;
+            const float s = self ? p.sd_term[base + D] : p.sd_dense[base + c];
+            const float P = expf(s + prD + p.pc[base + cc]);
+            const float dp = has_dp ? (self ? p.dp_term[base + D] : p.dp_dense[base + c]) : 0.f;
+            if (p.sout) {
+                if (p.s_dp) a1 = fmaf(P, dp, a1);
+                if (p.m) a2 = fmaf(P, p.m[base + cc], a2);
+            }
+            if (p.vout) {
+                float mod = p.v_dp ? dp : 1.f;
+                for (int k = 0; k < nm; ++k) mod -= p.xr[k][base + D] * p.yc[k][base + cc];
+                coef = P * mod;
+            }
+        }
+        if (p.vout) {
+            __syncthreads();
+            cs[threadIdx.x] = coef;
+            __syncthreads();
+            if (grp < groups) {
+                for (int j = grp; j < 256; j += groups) {
+                    const int cj = c0 + j;
+                    if (cj > L) break;
+                    const int row = (cj == L) ? D : cj;
+                    if (cs[j] != 0.f) vpart = fmaf(cs[j], to_f(Z[size_t(row) * d + zc]), vpart);
+                }
+            }
+        }
+    }
+    red1[threadIdx.x] = a1;
+    red2[threadIdx.x] = a2;
+    vacc[threadIdx.x] = (grp < groups) ? vpart : 0.f;
+    __syncthreads();
+    for (int st = 128; st > 0; st >>= 1) {
+        if (threadIdx.x < st) {
+            red1[threadIdx.x] += red1[threadIdx.x + st];
+            red2[threadIdx.x] += red2[threadIdx.x + st];
+        }
+        __syncthreads();
+    }
+    if (p.sout && threadIdx.x == 0) {
+        float outv = (p.f ? p.f[base + D] : 1.f) * (red1[0] + (p.hv ? p.hv[base + D] : 0.f) * red2[0]);
+        if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+        p.sout[base + D] = outv;
+    }
+    if (p.vout && threadIdx.x < d) {
+        float a = 0.f;
+        for (int g2 = 0; g2 < groups; ++g2) a += vacc[g2 * d + threadIdx.x];
+        static_cast<T*>(p.vout)[(base + D) * d + threadIdx.x] = from_f<T>(p.vscale * a);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward vector preparation (§2.2: orbit factors exp(u(k)-u(R)), exp(v(k)-v(R)))
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
+    const int bh = blockIdx.y, b = bh / a.H;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= a.L) return;
+    const size_t L = size_t(a.L);
+    const size_t idx = size_t(bh) * L + i;
+    const float lm = a.logm[size_t(b) * L + i];
+    const bool act = lm != neg_inf();
+    const int R = a.R;
+    auto U = [&](int k) { return a.u_tail[(size_t(bh) * (R + 1) + k) * L + i]; };
+    auto Vv = [&](int k) { return a.v_tail[(size_t(bh) * (R + 1) + k) * L + i]; };
+    auto AL = [&](int k) { return a.alpha[size_t(k) * a.BH * L + idx]; };
+    auto BE = [&](int k) { return a.beta[size_t(k) * a.BH * L + idx]; };
+    float pr = 0.f, pc = 0.f, f = 1.f, hv = 0.f, m = 0.f;
+    float xr[kMaxMods], yc[kMaxMods];
+    int nm = 0;
+    if (act) {
+        const float ea = expf(lm), ia = expf(-lm);
+        const float uR = U(R), vR = Vv(R);
+        switch (a.kind) {
+            case kPassOut: pr = uR - lm; pc = vR; break;
+            case kPassC1: pr = vR; pc = uR - lm; break;
+            case kPassR2: pr = uR - lm; pc = vR; hv = -ea; m = BE(R) * ia; break;
+            case kPassCk:
+                pr = vR; pc = uR; hv = 1.f;
+                f = -expf(Vv(a.k) - vR);
+                m = expf(U(a.k + 1) - uR) * AL(a.k + 1) * ia;
+                break;
+            case kPassRk:
+                pr = uR; pc = vR; hv = 1.f;
+                f = -expf(U(a.k) - uR);
+                m = expf(Vv(a.k) - vR) * BE(a.k) * ia;
+                break;
+            case kPassRF:
+                pr = uR - lm; pc = vR;
+                for (int k = 1; k <= R; ++k) {
+                    const float eu = expf(U(k) - uR);
+                    xr[nm] = ea * eu;                 yc[nm++] = expf(Vv(k) - vR) * BE(k) * ia;
+                    xr[nm] = eu * AL(k);              yc[nm++] = expf(Vv(k - 1) - vR);
+                }
+                break;
+            case kPassCF:
+                pr = vR; pc = uR - lm;
+                for (int k = 1; k <= R; ++k) {
+                    const float eu = expf(U(k) - uR);
+                    xr[nm] = expf(Vv(k) - vR) * BE(k) * ia;   yc[nm++] = ea * eu;
+                    xr[nm] = expf(Vv(k - 1) - vR);            yc[nm++] = eu * AL(k);
+                }
+                break;
+        }
+    } else {
+        if (a.kind == kPassRF || a.kind == kPassCF) {
+            for (int k = 0; k < 2 * R; ++k) { xr[k] = 0.f; yc[k] = 0.f; }
+            nm = 2 * R;
+        }
+    }
+    a.pr[idx] = pr;
+    a.pc[idx] = pc;
+    if (a.f) a.f[idx] = f;
+    if (a.hv) a.hv[idx] = hv;
+    if (a.m) a.m[idx] = m;
+    for (int k = 0; k < nm; ++k) {
+        a.xr[size_t(k) * a.BH * L + idx] = xr[k];
+        a.yc[size_t(k) * a.BH * L + idx] = yc[k];
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------------------
+cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
+                                  uint32_t* status, cudaStream_t st) {
+    prep_marginals_kernel<<<g.B, 256, 0, st>>>(g, mask, dustbin, mass, logm, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
+                                cudaStream_t st) {
+    dim3 grid((g.L + 255) / 256, g.BH);
+    if (g.dtype == EOT_BF16)
+        prep_dustbin_dots_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            g, static_cast<const __nv_bfloat16*>(P), static_cast<const __nv_bfloat16*>(Qm), s1, term, dense);
+    else
+        prep_dustbin_dots_kernel<float><<<grid, 256, 0, st>>>(g, static_cast<const float*>(P),
+                                                              static_cast<const float*>(Qm), s1, term, dense);
+    return cudaGetLastError();
+}
+
+static size_t simt_lse_smem(int d) { return size_t(2 * kSB * (d + 1) + kSB) * sizeof(float); }
+static size_t simt_bwd_smem(int d) {
+    return size_t(5 * kSB * (d + 1) + kSB * 33 + (2 + kMaxMods) * kSB + (3 + kMaxMods) * kSB) * sizeof(float);
+}
+
+cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st) {
+    dim3 grid(p.g.L / kSB, p.g.BH);
+    const size_t smem = simt_lse_smem(p.g.d);
+    cudaError_t e;
+    if (p.g.dtype == EOT_BF16) {
+        e = cudaFuncSetAttribute(simt_lse_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        simt_lse_kernel<__nv_bfloat16><<<grid, kSNT, smem, st>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(simt_lse_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        simt_lse_kernel<float><<<grid, kSNT, smem, st>>>(p);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.g.D < 0) return e;
+    dustbin_lse_kernel<<<p.g.BH, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st) {
+    dim3 grid(p.g.L / kSB, p.g.BH);
+    const size_t smem = simt_bwd_smem(p.g.d);
+    cudaError_t e;
+    if (p.g.dtype == EOT_BF16) {
+        e = cudaFuncSetAttribute(simt_bwd_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        simt_bwd_kernel<__nv_bfloat16><<<grid, kSNT, smem, st>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(simt_bwd_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        simt_bwd_kernel<float><<<grid, kSNT, smem, st>>>(p);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || p.g.D < 0) return e;
+    if (p.g.dtype == EOT_BF16)
+        dustbin_bwd_kernel<__nv_bfloat16><<<p.g.BH, 256, 0, st>>>(p);
+    else
+        dustbin_bwd_kernel<float><<<p.g.BH, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st) {
+    dim3 grid((a.L + 255) / 256, a.BH);
+    bwd_vectors_kernel<<<grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace eot

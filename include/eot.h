@@ -1,0 +1,143 @@
+/*
+ * eot.h -- C ABI of libeot, blockwise band-support balanced log-domain Sinkhorn attention
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science,
+ * paper 2605.08123).  Per (batch, head) unit, with S_ij = scale <q_i, k_j> (the entropic
+ * temperature absorbed into S, §2.1) on the fixed band support
+ *     Omega = { (i, j) : i, j active, |i - j| <= W / 2 }          (§2.1; W / 2 rounds down)
+ * and uniform marginals a = b over the active tokens, the forward pass runs
+ *     T stopped balanced Sinkhorn steps from v = 0                (§2.1, stopped base)
+ *         u_i = log a_i - LSE_{j : (i,j) in Omega} (S_ij + v_j)
+ *         v_j = log b_j - LSE_{i : (i,j) in Omega} (S_ij + u_i)
+ *     R more steps from (u0, v0), the differentiable tail          (§2.1, refinement tail)
+ *     O = diag(1/a) P V,  P = exp(S + u(R) + v(R)) on Omega
+ * and the backward pass is the exact adjoint of that tail w.r.t. Q, K, V with the base held
+ * fixed (§2.2), computed from one reference plan P(R,R) per tile plus per-row and per-column
+ * factors exp(u(k) - u(R)), exp(v(k) - v(R)) (the scaling-orbit identity of §2.2).
+ * With the dustbin flag (§2.3) a dustbin token at ``dustbin_index`` is linked to every
+ * active real token in both directions (and to itself when ``dustbin_self``); it carries
+ * marginal ``dustbin_mass`` and the real tokens share 1 - dustbin_mass.  Positions after the
+ * dustbin are inactive fillers.
+ *
+ * Conventions common to every call
+ *   - All tensors are caller-owned device buffers, contiguous, [B, H, L, d] row-major for
+ *     Q, K, V, O, dO, dQ, dK, dV (element type given by ``dtype``), [B, H, R+1, L] float32
+ *     for the tail potentials, [B, L] uint8 for the mask.
+ *   - The library never allocates device memory (all scratch lives in the caller's
+ *     workspace) and keeps no global device state.
+ *   - Calls are asynchronous and stream-ordered on ``stream`` (a cudaStream_t; NULL is the
+ *     legacy default stream).  No host synchronisation happens inside fwd/bwd.
+ *   - Argument errors are detected on the host before anything is enqueued; nothing is then
+ *     launched and the status says why.  Launch failures return EOT_ERR_CUDA.
+ *   - Conditions found on the device (a non-finite potential, a wait that ran out) set bits
+ *     in a status word inside the workspace; read them with eot_last_device_status.  The
+ *     kernels never trap.
+ *   - B * H * L == 0 is an empty problem: the call validates and returns EOT_OK at once.
+ *   - Rows of inactive tokens are written as 0 in O, dQ, dK, dV; their u and v are 0.
+ */
+#ifndef EOT_H_
+#define EOT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EOT_ABI_VERSION 1
+
+typedef enum {
+    EOT_OK = 0,
+    EOT_ERR_INVALID_ARGUMENT = 1,   /* bad size, pointer or flag; nothing was launched */
+    EOT_ERR_UNSUPPORTED = 2,        /* valid problem this build cannot run (e.g. impl/dtype) */
+    EOT_ERR_WORKSPACE_TOO_SMALL = 3,
+    EOT_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    EOT_ERR_NONFINITE = 5,          /* device status: a non-finite potential was produced */
+    EOT_ERR_TIMEOUT = 6             /* device status: a bounded wait inside a kernel ran out */
+} eot_status;
+
+typedef enum { EOT_FP32 = 0, EOT_BF16 = 1 } eot_dtype;
+
+/* Kernel family.  AUTO picks the tensor-core (tcgen05/TMA) kernels for bf16 with d in
+ * {64, 128} and the CUDA-core kernels otherwise (fp32 is always computed on CUDA cores,
+ * in fp32, so that its scores keep full fp32 precision). */
+typedef enum { EOT_IMPL_AUTO = 0, EOT_IMPL_SIMT = 1, EOT_IMPL_TCGEN05 = 2 } eot_impl;
+
+typedef struct {
+    int32_t B, H;          /* batch, heads */
+    int32_t L;             /* sequence length incl. dustbin and fillers; multiple of 128 */
+    int32_t d;             /* head dim: multiple of 8, <= 128 (tensor-core path: 64 or 128) */
+    int32_t W;             /* band width: support |i - j| <= W / 2 (integer division), W >= 0 */
+    int32_t T;             /* stopped base steps, T >= 0 */
+    int32_t R;             /* differentiable tail steps, 0 <= R <= 8 */
+    int32_t dtype;         /* eot_dtype of Q, K, V, O, dO, dQ, dK, dV; potentials are fp32 */
+    float scale;           /* score scale; 0 means 1 / sqrt(d) */
+    int32_t dustbin;       /* 0 or 1 */
+    int32_t dustbin_index; /* position of the dustbin token (0 <= index < L) when dustbin = 1 */
+    float dustbin_mass;    /* dustbin marginal in [0, 1); 0 makes the dustbin inactive */
+    int32_t dustbin_self;  /* 1: (D, D) is in the support; 0: it is not */
+    int32_t impl;          /* eot_impl */
+} eot_problem;
+
+/* Bytes of device workspace that eot_sinkhorn_fwd (for_backward = 0) or eot_sinkhorn_bwd
+ * (for_backward = 1) needs for problem *p.  Returns 0 when *p is invalid (see
+ * eot_validate) and for empty problems.  Workspace must be 256-byte aligned. */
+size_t eot_workspace_bytes(const eot_problem* p, int for_backward);
+
+/* Host-side validation only: EOT_OK, EOT_ERR_INVALID_ARGUMENT or EOT_ERR_UNSUPPORTED. */
+eot_status eot_validate(const eot_problem* p);
+
+/*
+ * Forward (§2.1).  Device pointers:
+ *   Q, K, V   [B, H, L, d] dtype, read only.
+ *   mask      [B, L] uint8, 1 = active real token; NULL = every position active.  With a
+ *             dustbin, the dustbin position and everything after it are ignored in the mask
+ *             (the dustbin is active iff mass > 0 and at least one real token is active;
+ *             positions after it are inactive fillers).
+ *   O         [B, H, L, d] dtype, written.  O_i = (1/a_i) sum_j P_ij V_j.
+ *   u_tail    [B, H, R+1, L] float32, written: u_tail[0] = u after the T base steps (0 when
+ *             T = 0), u_tail[k] = u(k) of tail step k.
+ *   v_tail    [B, H, R+1, L] float32, written: v_tail[0] = stopped base v0, v_tail[k] = v(k).
+ *   workspace eot_workspace_bytes(p, 0) bytes, device, contents clobbered.
+ */
+eot_status eot_sinkhorn_fwd(const eot_problem* p, const void* Q, const void* K, const void* V,
+                            const uint8_t* mask, void* O, float* u_tail, float* v_tail,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward: exact adjoint of the R-step tail w.r.t. Q, K, V, the base (u0, v0) held fixed
+ * (stop-gradient, §2.1-§2.2), for the loss gradient dO.  Inputs as in the forward plus
+ * u_tail/v_tail from it and dO [B, H, L, d].  dQ, dK, dV [B, H, L, d] are overwritten (not
+ * accumulated).  The gradient w.r.t. the dustbin token is written at ``dustbin_index`` per
+ * (batch, head); a caller sharing one learned token across the batch sums over B.
+ */
+eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, const void* V,
+                            const uint8_t* mask, const float* u_tail, const float* v_tail,
+                            const void* dO, void* dQ, void* dK, void* dV, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Synchronises ``stream``, reads the device status word that the last fwd/bwd call on this
+ * workspace left, clears it, and returns EOT_OK, EOT_ERR_NONFINITE or EOT_ERR_TIMEOUT
+ * (EOT_ERR_CUDA if the copy fails). */
+eot_status eot_last_device_status(void* workspace, void* stream);
+
+/* Raw device status bits of the last call (bit 0 non-finite, bit 1 timeout); syncs. */
+eot_status eot_device_status_bits(void* workspace, void* stream, uint32_t* bits);
+
+/* Static string for a status code. */
+const char* eot_status_string(eot_status s);
+
+/* EOT_ABI_VERSION of the loaded library. */
+int eot_abi_version(void);
+
+/* Kernel family that ``p`` would run with (EOT_IMPL_SIMT or EOT_IMPL_TCGEN05), or -1 if
+ * the problem is invalid or unsupported. */
+int eot_resolved_impl(const eot_problem* p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EOT_H_ */

@@ -233,6 +233,25 @@ static void unit_forward(unit_t *U, int T, double *O, double *u_tail, double *v_
     free(u); free(v);
 }
 
+/* Visit every support entry (i, j, S_ij) of column j: band rows plus the dustbin row. */
+#define FOR_COL_ENTRIES(U, j, i, sij, ...)                                           \
+    do {                                                                             \
+        const int w_ = wid(U), h_ = (U)->h;                                          \
+        if ((j) == (U)->D) {                                                         \
+            for (int i = 0; i < (U)->L; ++i)                                         \
+                if ((U)->real[i]) { double sij = (U)->sDr[i]; __VA_ARGS__ }          \
+            if ((U)->dself) { int i = (U)->D; double sij = (U)->sDD; __VA_ARGS__ }   \
+        } else if ((U)->real[j]) {                                                   \
+            for (int i = (j) - h_; i <= (j) + h_; ++i) {                             \
+                if (i < 0 || i >= (U)->L) continue;                                  \
+                double sij = (U)->S[(size_t)i * w_ + ((j) - i + h_)];                \
+                if (sij == -INFINITY) continue;                                      \
+                __VA_ARGS__                                                          \
+            }                                                                        \
+            if ((U)->D >= 0) { int i = (U)->D; double sij = (U)->sDc[j]; __VA_ARGS__ } \
+        }                                                                            \
+    } while (0)
+
 /*
  * Tail adjoint for one unit (§2.2), same chain as the dense oracle:
  *   dP_ij = <dO_i, V_j> / a_i, G = P(R,R) * dP
@@ -240,7 +259,8 @@ static void unit_forward(unit_t *U, int T, double *O, double *u_tail, double *v_
  *   beta_k = -P(k+1,k)^T (alpha_{k+1} / a), alpha_k = -P(k,k)(beta_k / b)
  *   dS = G - sum_k [P(k,k) (beta_k/b)_j + P(k,k-1) (alpha_k/a)_i]
  *   dQ = scale dS K, dK = scale dS^T Q, dV = P(R,R)^T (dO / a)
- * Column sums are accumulated row by row (serially over rows, in row order).
+ * Row-owned sums loop over the row's support, column-owned sums over the column's
+ * support, so every loop is parallel over its owner.
  */
 static void unit_backward(unit_t *U, const double *u_tail, const double *v_tail, const double *dO,
                           double *dQ, double *dK, double *dV)
@@ -253,41 +273,43 @@ static void unit_backward(unit_t *U, const double *u_tail, const double *v_tail,
     for (int i = 0; i < L; ++i) inv_a[i] = is_active(U, i) ? exp(-U->log_a[i]) : 0.0;
     double *alpha = (double *)calloc((size_t)(R + 1) * L, sizeof(double));
     double *beta = (double *)calloc((size_t)(R + 1) * L, sizeof(double));
-    double *rho = (double *)calloc((size_t)L, sizeof(double));
     memset(dQ, 0, sizeof(double) * (size_t)L * d);
     memset(dK, 0, sizeof(double) * (size_t)L * d);
     memset(dV, 0, sizeof(double) * (size_t)L * d);
 
-    /* rho = rowsum G, beta_R = colsum G */
-    for (int i = 0; i < L; ++i) {
-        if (!is_active(U, i)) continue;
-        const double *doi = dO + (size_t)i * d;
-        FOR_ROW_ENTRIES(U, i, j, sij, {
-            double p = exp(sij + UT(R, i) + VT(R, j));
-            double g = p * dot(doi, U->v + (size_t)j * d, d) * inv_a[i];
-            rho[i] += g;
-            if (R > 0) beta[(size_t)R * L + j] += g;
-        });
-    }
     if (R > 0) {
         double *Rb = beta + (size_t)R * L, *Ra = alpha + (size_t)R * L;
-#pragma omp parallel for schedule(static)
-        for (int i = 0; i < L; ++i) {
+#pragma omp parallel for schedule(dynamic, 64)
+        for (int j = 0; j < L; ++j) {            /* beta_R = colsum G */
+            if (!is_active(U, j)) continue;
+            double acc = 0.0;
+            FOR_COL_ENTRIES(U, j, i, sij, {
+                acc += exp(sij + UT(R, i) + VT(R, j)) * dot(dO + (size_t)i * d, U->v + (size_t)j * d, d) * inv_a[i];
+            });
+            Rb[j] = acc;
+        }
+#pragma omp parallel for schedule(dynamic, 64)
+        for (int i = 0; i < L; ++i) {            /* alpha_R = rowsum G - P(R,R)(beta_R/b) */
             if (!is_active(U, i)) continue;
             double acc = 0.0;
-            FOR_ROW_ENTRIES(U, i, j, sij, { acc += exp(sij + UT(R, i) + VT(R, j)) * Rb[j] * inv_a[j]; });
-            Ra[i] = rho[i] - acc;
+            const double *doi = dO + (size_t)i * d;
+            FOR_ROW_ENTRIES(U, i, j, sij, {
+                double p = exp(sij + UT(R, i) + VT(R, j));
+                acc += p * (dot(doi, U->v + (size_t)j * d, d) * inv_a[i] - Rb[j] * inv_a[j]);
+            });
+            Ra[i] = acc;
         }
         for (int kk = R - 1; kk >= 1; --kk) {
             double *bk = beta + (size_t)kk * L, *ak = alpha + (size_t)kk * L;
             const double *a1 = alpha + (size_t)(kk + 1) * L;
-            for (int i = 0; i < L; ++i) {        /* beta_k = -P(k+1,k)^T (alpha_{k+1}/a) */
-                if (!is_active(U, i)) continue;
-                FOR_ROW_ENTRIES(U, i, j, sij, {
-                    bk[j] -= exp(sij + UT(kk + 1, i) + VT(kk, j)) * a1[i] * inv_a[i];
-                });
+#pragma omp parallel for schedule(dynamic, 64)
+            for (int j = 0; j < L; ++j) {        /* beta_k = -P(k+1,k)^T (alpha_{k+1}/a) */
+                if (!is_active(U, j)) continue;
+                double acc = 0.0;
+                FOR_COL_ENTRIES(U, j, i, sij, { acc += exp(sij + UT(kk + 1, i) + VT(kk, j)) * a1[i] * inv_a[i]; });
+                bk[j] = -acc;
             }
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for schedule(dynamic, 64)
             for (int i = 0; i < L; ++i) {        /* alpha_k = -P(k,k)(beta_k/b) */
                 if (!is_active(U, i)) continue;
                 double acc = 0.0;
@@ -296,32 +318,42 @@ static void unit_backward(unit_t *U, const double *u_tail, const double *v_tail,
             }
         }
     }
-    /* dS entries, then dQ (row owner), dK and dV (accumulated in row order). */
+    /* dS_ij; dQ by rows, dK and dV by columns. */
+#define DS_ENTRY(i_, j_, sij_, p_, ds_)                                                        \
+    double p_ = exp((sij_) + UT(R, i_) + VT(R, j_));                                           \
+    double ds_ = p_ * dot(dO + (size_t)(i_) * d, U->v + (size_t)(j_) * d, d) * inv_a[i_];      \
+    for (int kk = 1; kk <= R; ++kk) {                                                          \
+        ds_ -= exp((sij_) + UT(kk, i_) + VT(kk, j_)) * beta[(size_t)kk * L + (j_)] * inv_a[j_]; \
+        ds_ -= exp((sij_) + UT(kk, i_) + VT(kk - 1, j_)) * alpha[(size_t)kk * L + (i_)] * inv_a[i_]; \
+    }
+#pragma omp parallel for schedule(dynamic, 64)
     for (int i = 0; i < L; ++i) {
         if (!is_active(U, i)) continue;
-        const double *doi = dO + (size_t)i * d;
-        const double *qi = U->q + (size_t)i * d;
         double *dqi = dQ + (size_t)i * d;
         FOR_ROW_ENTRIES(U, i, j, sij, {
-            double p = exp(sij + UT(R, i) + VT(R, j));
-            double g = p * dot(doi, U->v + (size_t)j * d, d) * inv_a[i];
-            double ds = g;
-            for (int kk = 1; kk <= R; ++kk) {
-                ds -= exp(sij + UT(kk, i) + VT(kk, j)) * beta[(size_t)kk * L + j] * inv_a[j];
-                ds -= exp(sij + UT(kk, i) + VT(kk - 1, j)) * alpha[(size_t)kk * L + i] * inv_a[i];
-            }
+            DS_ENTRY(i, j, sij, p, ds)
+            (void)p;
             const double *kj = U->k + (size_t)j * d;
-            double *dkj = dK + (size_t)j * d, *dvj = dV + (size_t)j * d;
+            for (int t = 0; t < d; ++t) dqi[t] += sc * ds * kj[t];
+        });
+    }
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int j = 0; j < L; ++j) {
+        if (!is_active(U, j)) continue;
+        double *dkj = dK + (size_t)j * d, *dvj = dV + (size_t)j * d;
+        FOR_COL_ENTRIES(U, j, i, sij, {
+            DS_ENTRY(i, j, sij, p, ds)
+            const double *qi = U->q + (size_t)i * d, *doi = dO + (size_t)i * d;
             for (int t = 0; t < d; ++t) {
-                dqi[t] += sc * ds * kj[t];
                 dkj[t] += sc * ds * qi[t];
                 dvj[t] += p * doi[t] * inv_a[i];
             }
         });
     }
+#undef DS_ENTRY
 #undef UT
 #undef VT
-    free(inv_a); free(alpha); free(beta); free(rho);
+    free(inv_a); free(alpha); free(beta);
 }
 
 /*
