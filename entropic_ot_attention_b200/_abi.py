@@ -71,10 +71,39 @@ lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
 lib.eot_device_status_bits.restype = ctypes.c_int
 
+lib.eot_kernel_launches.restype = ctypes.c_longlong
+lib.eot_profile_begin.restype = None
+lib.eot_profile_end.argtypes = [_vp]
+lib.eot_profile_end.restype = ctypes.c_int
+lib.eot_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+lib.eot_profile_read.restype = ctypes.c_int
+
 # Every symbol declared in include/eot.h (checked by the CPU tests).
 EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sinkhorn_bwd",
             "eot_last_device_status", "eot_device_status_bits", "eot_status_string",
-            "eot_abi_version", "eot_resolved_impl")
+            "eot_abi_version", "eot_resolved_impl", "eot_kernel_launches", "eot_profile_begin",
+            "eot_profile_end", "eot_profile_read")
+
+PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3}
+
+
+def eot_kernel_launches() -> int:
+    return int(lib.eot_kernel_launches())
+
+
+def eot_profile_begin() -> None:
+    lib.eot_profile_begin()
+
+
+def eot_profile_end(stream: int) -> None:
+    _check(lib.eot_profile_end(stream), "eot_profile_end")
+
+
+def eot_profile_read(kind: int):
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_longlong(0)
+    _check(lib.eot_profile_read(int(kind), ctypes.byref(ms), ctypes.byref(n)), "eot_profile_read")
+    return float(ms.value), int(n.value)
 
 
 def eot_status_string(status: int) -> str:

@@ -9,11 +9,53 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+#include <vector>
+
 #include "kernels.cuh"
 
 using namespace eot;
 
 namespace {
+
+// ---------------------------------------------------------------------------------------
+// Launch accounting and optional per-kind CUDA-event timing (benchmark support)
+// ---------------------------------------------------------------------------------------
+enum ProfKind { kProfLse = 0, kProfOut = 1, kProfBwd = 2, kProfAux = 3, kProfKinds = 4 };
+
+struct Profiler {
+    bool on = false;
+    std::vector<cudaEvent_t> ev[kProfKinds];   // start/stop pairs, reused across sessions
+    size_t used[kProfKinds] = {};
+    double ms[kProfKinds] = {};
+    long long count[kProfKinds] = {};
+};
+Profiler g_prof;
+std::atomic<long long> g_launches{0};
+
+// Runs f (which enqueues `nkernels` kernels on st) and, while profiling, brackets it with
+// a pair of CUDA events on the same stream.
+template <typename F>
+cudaError_t tracked(int kind, int nkernels, cudaStream_t st, F&& f) {
+    g_launches += nkernels;
+    if (!g_prof.on) return f();
+    auto& ev = g_prof.ev[kind];
+    const size_t i = g_prof.used[kind];
+    if (ev.size() < i + 2) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return cudaErrorMemoryAllocation;
+        ev.push_back(a);
+        ev.push_back(b);
+    }
+    cudaError_t e = cudaEventRecord(ev[i], st);
+    if (e != cudaSuccess) return e;
+    e = f();
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(ev[i + 1], st);
+    g_prof.used[kind] = i + 2;
+    g_prof.count[kind] += 1;
+    return e;
+}
 
 bool tensor_core_ok(const eot_problem& p) { return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128); }
 
@@ -44,6 +86,7 @@ eot_status validate(const eot_problem* p) {
     if (p->impl < EOT_IMPL_AUTO || p->impl > EOT_IMPL_TCGEN05) return EOT_ERR_INVALID_ARGUMENT;
     if (int64_t(p->B) * p->H > 65535) return EOT_ERR_UNSUPPORTED;
     if (int64_t(p->B) * p->H * p->L * int64_t(p->d) >= (int64_t(1) << 40)) return EOT_ERR_UNSUPPORTED;
+    if (int64_t(p->B) * p->H * p->L >= (int64_t(1) << 31)) return EOT_ERR_UNSUPPORTED;   // TMA row coordinate
     if (resolve_impl(*p) < 0) return EOT_ERR_UNSUPPORTED;
     return EOT_OK;
 }
@@ -74,12 +117,21 @@ template <typename T> T* at(void* ws, size_t off) { return reinterpret_cast<T*>(
     } while (0)
 
 cudaError_t run_lse(int impl, const LsePass& lp, cudaStream_t st) {
-    return impl == EOT_IMPL_TCGEN05 ? launch_tc_lse(lp, st) : launch_simt_lse(lp, st);
+    const int nk = lp.g.D >= 0 ? 2 : 1;
+    return tracked(kProfLse, nk, st, [&] {
+        return impl == EOT_IMPL_TCGEN05 ? launch_tc_lse(lp, st) : launch_simt_lse(lp, st);
+    });
 }
 
-cudaError_t run_bwd(int impl, const BwdPass& bp, cudaStream_t st) {
-    return impl == EOT_IMPL_TCGEN05 ? launch_tc_bwd(bp, st) : launch_simt_bwd(bp, st);
+cudaError_t run_bwd(int impl, const BwdPass& bp, cudaStream_t st, int kind = kProfBwd) {
+    const int nk = bp.g.D >= 0 ? 2 : 1;
+    return tracked(kind, nk, st, [&] {
+        return impl == EOT_IMPL_TCGEN05 ? launch_tc_bwd(bp, st) : launch_simt_bwd(bp, st);
+    });
 }
+
+template <typename F>
+cudaError_t aux(cudaStream_t st, F&& f) { return tracked(kProfAux, 1, st, f); }
 
 }  // namespace
 
@@ -99,8 +151,8 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     float* sd_row = p->dustbin ? at<float>(ws, w.sd_row) : nullptr;
     float* sd_col = p->dustbin ? at<float>(ws, w.sd_col) : nullptr;
 
-    EOT_TRY(launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st));
-    if (p->dustbin) EOT_TRY(launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st));
+    EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
+    if (p->dustbin) EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st); }));
     const size_t tail_bytes = size_t(g.BH) * pstride * sizeof(float);
     EOT_TRY(cudaMemsetAsync(u_tail, 0, tail_bytes, st));
     EOT_TRY(cudaMemsetAsync(v_tail, 0, tail_bytes, st));
@@ -114,7 +166,14 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     row.sd_term = sd_row;
     row.sd_dense = sd_col;
     row.status = status;
+    float* ub2 = at<float>(ws, w.ub2);
+    float* vb2 = at<float>(ws, w.vb2);
+    EOT_TRY(aux(st, [&] { return launch_init_bias2(g, logm, vb2, st); }));
+    row.colbias2 = vb2;
+    row.out_bias2 = ub2;
     LsePass col = row;
+    col.colbias2 = ub2;
+    col.out_bias2 = vb2;
     col.X = K;
     col.Y = Q;
     col.sd_term = sd_col;
@@ -147,10 +206,12 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     va.logm = logm;
     va.u_tail = u_tail;
     va.v_tail = v_tail;
+    va.D = g.D;
     va.pr = at<float>(ws, w.opr);
     va.pc = at<float>(ws, w.opc);
+    va.pcm2 = at<float>(ws, w.opcm);
     va.f = va.hv = va.m = nullptr;            // unused by the output pass
-    EOT_TRY(launch_bwd_vectors(va, st));
+    EOT_TRY(aux(st, [&] { return launch_bwd_vectors(va, st); }));
     BwdPass op{};
     op.g = g;
     op.X = Q;
@@ -159,6 +220,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     op.logm = logm;
     op.pr = va.pr;
     op.pc = va.pc;
+    op.pcm2 = va.pcm2;
     op.vout = O;
     op.vscale = 1.f;
     op.v_dp = 0;
@@ -166,7 +228,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     op.sd_term = sd_row;
     op.sd_dense = sd_col;
     op.status = status;
-    EOT_TRY(run_bwd(impl, op, st));
+    EOT_TRY(run_bwd(impl, op, st, kProfOut));
     return EOT_OK;
 }
 
@@ -181,14 +243,15 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     uint32_t* status = at<uint32_t>(ws, w.status);
     float* logm = at<float>(ws, w.logm);
     float *sd_row = nullptr, *sd_col = nullptr, *e1 = nullptr, *e2 = nullptr;
-    EOT_TRY(launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st));
+    EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
     if (p->dustbin) {
         sd_row = at<float>(ws, w.sd_row);
         sd_col = at<float>(ws, w.sd_col);
         e1 = at<float>(ws, w.e1);
         e2 = at<float>(ws, w.e2);
-        EOT_TRY(launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st));
-        EOT_TRY(launch_dustbin_dots(g, dO, V, 1.f, e1, e2, st));   // e1[r] = <dO_r, V_D>, e2[r] = <dO_D, V_r>
+        EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st); }));
+        // e1[r] = <dO_r, V_D>, e2[r] = <dO_D, V_r>
+        EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, dO, V, 1.f, e1, e2, st); }));
     }
     float* alpha = at<float>(ws, w.alpha);
     float* beta = at<float>(ws, w.beta);
@@ -203,8 +266,10 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     va.v_tail = v_tail;
     va.alpha = alpha;
     va.beta = beta;
+    va.D = g.D;
     va.pr = at<float>(ws, w.pr);
     va.pc = at<float>(ws, w.pc);
+    va.pcm2 = at<float>(ws, w.pcm);
     va.f = at<float>(ws, w.f);
     va.hv = at<float>(ws, w.hv);
     va.m = at<float>(ws, w.m);
@@ -221,6 +286,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.logm = logm;
     rowp.pr = va.pr;
     rowp.pc = va.pc;
+    rowp.pcm2 = va.pcm2;
     rowp.sd_term = sd_row;
     rowp.sd_dense = sd_col;
     rowp.dp_term = e1;
@@ -239,7 +305,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     auto vec = [&](int kind, int k) -> cudaError_t {
         va.kind = kind;
         va.k = k;
-        return launch_bwd_vectors(va, st);
+        return aux(st, [&] { return launch_bwd_vectors(va, st); });
     };
     auto scalar_pass = [&](BwdPass bp, float* out, bool dp) -> cudaError_t {
         bp.sout = out;
@@ -356,6 +422,39 @@ eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, 
     if (workspace_bytes < ws_layout(*p, true).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
     return backward_impl(p, Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
                          static_cast<cudaStream_t>(stream));
+}
+
+long long eot_kernel_launches(void) { return g_launches.load(); }
+
+void eot_profile_begin(void) {
+    g_prof.on = true;
+    for (int k = 0; k < kProfKinds; ++k) {
+        g_prof.used[k] = 0;
+        g_prof.ms[k] = 0.0;
+        g_prof.count[k] = 0;
+    }
+}
+
+eot_status eot_profile_end(void* stream) {
+    g_prof.on = false;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return EOT_ERR_CUDA;
+    for (int k = 0; k < kProfKinds; ++k) {
+        double t = 0.0;
+        for (size_t i = 0; i + 1 < g_prof.used[k]; i += 2) {
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, g_prof.ev[k][i], g_prof.ev[k][i + 1]) != cudaSuccess) return EOT_ERR_CUDA;
+            t += ms;
+        }
+        g_prof.ms[k] = t;
+    }
+    return EOT_OK;
+}
+
+eot_status eot_profile_read(int kind, double* total_ms, long long* launches) {
+    if (kind < 0 || kind >= kProfKinds || !total_ms || !launches) return EOT_ERR_INVALID_ARGUMENT;
+    *total_ms = g_prof.ms[kind];
+    *launches = g_prof.count[kind];
+    return EOT_OK;
 }
 
 eot_status eot_device_status_bits(void* workspace, void* stream, uint32_t* bits) {

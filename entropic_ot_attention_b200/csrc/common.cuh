@@ -45,6 +45,8 @@ struct LsePass {
     const float* stab;      // previous value of this row potential, or nullptr
     float* out;             // new row potential (0 for inactive rows)
     size_t pstride;         // unit stride of colpot / stab / out (elements): L or (R+1) L
+    const float* colbias2;  // [BH, L] log2(e) * colpot, -inf for inactive columns and the dustbin
+    float* out_bias2;       // [BH, L] same masking of the new potential (for the next half-step)
     const float* sd_term;   // [BH, L] S between row r and the dustbin column (dustbin only)
     const float* sd_dense;  // [BH, L] S between the dustbin row and column c (dustbin only)
     uint32_t* status;
@@ -65,6 +67,7 @@ struct BwdPass {
     const float* logm;
     const float* pr;        // [BH, L]
     const float* pc;        // [BH, L] (value at D used for the dustbin links)
+    const float* pcm2;      // [BH, L] log2(e) * pc, -inf for inactive columns and the dustbin
     float* sout;            // scalar output or nullptr
     const float* f;
     const float* hv;
@@ -86,7 +89,9 @@ struct BwdPass {
 // Workspace layout.  Every region is 256-byte aligned; offsets in bytes.
 struct WsLayout {
     size_t status, logm, sd_row, sd_col, e1, e2;
-    size_t opr, opc;        // forward output pass: row / column biases
+    size_t opr, opc, opcm;  // forward output pass: row / column biases
+    size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
+    size_t pcm;             // backward: masked log2 column bias
     size_t pr, pc, f, hv, m;
     size_t xr, yc;          // kMaxMods vectors each, [BH, L]
     size_t alpha, beta;     // (R + 1) vectors each, [BH, L]
@@ -110,6 +115,9 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     if (!bwd) {
         w.opr = o; o += vec;
         w.opc = o; o += vec;
+        w.opcm = o; o += vec;
+        w.ub2 = o; o += vec;
+        w.vb2 = o; o += vec;
     }
     if (bwd) {
         w.pr = o; o += vec;
@@ -117,6 +125,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.f = o; o += vec;
         w.hv = o; o += vec;
         w.m = o; o += vec;
+        w.pcm = o; o += vec;
         w.xr = o; o += vec * 2 * p.R;
         w.yc = o; o += vec * 2 * p.R;
         w.alpha = o; o += vec * (p.R + 1);

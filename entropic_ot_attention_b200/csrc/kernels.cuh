@@ -9,13 +9,13 @@ namespace eot {
 enum PassKind { kPassOut = 0, kPassC1, kPassR2, kPassCk, kPassRk, kPassRF, kPassCF };
 
 struct BwdVecArgs {
-    int kind, k, R, H, BH, L;
+    int kind, k, R, H, BH, L, D;
     const float* logm;      // [B, L]
     const float* u_tail;    // [BH, R+1, L]
     const float* v_tail;    // [BH, R+1, L]
     const float* alpha;     // [R+1][BH*L]
     const float* beta;      // [R+1][BH*L]
-    float *pr, *pc, *f, *hv, *m;
+    float *pr, *pc, *pcm2, *f, *hv, *m;
     float *xr, *yc;         // [2R][BH*L]
 };
 
@@ -26,6 +26,9 @@ cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, fl
 cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st);
 cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
 cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
+cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st);
+cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st);
+cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 
 // Tensor-core (tcgen05 + TMA) kernels; return cudaErrorNotSupported when not built.
 bool tc_supported(const Geom& g);

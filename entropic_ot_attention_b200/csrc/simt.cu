@@ -149,13 +149,15 @@ __global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
         for (int j = 1; j < 4; ++j) if (q == j) { mq = m[j]; sq = s[j]; }
         const float lm = logm[r];
         if (r == D && d_act) return;  // written by the dense dustbin row
-        float outv = 0.f;
+        float outv = 0.f, ob = neg_inf();
         if (lm != neg_inf()) {
             if (d_act) lse2_add(mq, sq, (p.sd_term[base + r] + p.colpot[pb + D]) * kLog2e);
             outv = lm - (mq + log2f(sq)) * kLn2;
             if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+            ob = outv * kLog2e;
         }
         p.out[pb + r] = outv;
+        p.out_bias2[base + r] = ob;
     }
 }
 
@@ -190,6 +192,7 @@ __global__ void __launch_bounds__(256) dustbin_lse_kernel(LsePass p) {
         float outv = logm[D] - (sm_m[0] + log2f(sm_s[0])) * kLn2;
         if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
         p.out[pb + D] = outv;
+        p.out_bias2[base + D] = neg_inf();   // the dustbin never enters a band sum
     }
 }
 
@@ -484,6 +487,7 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
     }
     a.pr[idx] = pr;
     a.pc[idx] = pc;
+    if (a.pcm2) a.pcm2[idx] = (act && i != a.D) ? pc * kLog2e : neg_inf();
     if (a.f) a.f[idx] = f;
     if (a.hv) a.hv[idx] = hv;
     if (a.m) a.m[idx] = m;
@@ -534,6 +538,10 @@ cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st) {
     }
     e = cudaGetLastError();
     if (e != cudaSuccess || p.g.D < 0) return e;
+    return launch_dustbin_lse(p, st);
+}
+
+cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st) {
     dustbin_lse_kernel<<<p.g.BH, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
@@ -553,10 +561,29 @@ cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st) {
     }
     e = cudaGetLastError();
     if (e != cudaSuccess || p.g.D < 0) return e;
+    return launch_dustbin_bwd(p, st);
+}
+
+cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st) {
     if (p.g.dtype == EOT_BF16)
         dustbin_bwd_kernel<__nv_bfloat16><<<p.g.BH, 256, 0, st>>>(p);
     else
         dustbin_bwd_kernel<float><<<p.g.BH, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// Masked log2 bias of the zero potential: 0 for active non-dustbin positions, -inf else.
+__global__ void __launch_bounds__(256) init_bias2_kernel(Geom g, const float* logm, float* bias2) {
+    const int bh = blockIdx.y, b = bh / g.H;
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= g.L) return;
+    const bool act = logm[size_t(b) * g.L + i] != neg_inf() && i != g.D;
+    bias2[size_t(bh) * g.L + i] = act ? 0.f : neg_inf();
+}
+
+cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st) {
+    dim3 grid((g.L + 255) / 256, g.BH);
+    init_bias2_kernel<<<grid, 256, 0, st>>>(g, logm, bias2);
     return cudaGetLastError();
 }
 

@@ -1,10 +1,885 @@
-// Tensor-core (tcgen05 + TMA) band sweeps for sm_100a.
+// Tensor-core band sweeps for sm_100a: TMA tile loads into 128-byte-swizzled shared memory,
+// tcgen05.mma (bf16 in, fp32 accumulate in TMEM) issued by one thread, warp-specialised
+// roles, and register epilogues that read the score tiles back with tcgen05.ld.
+//
+// Method: "Blockwise Differentiable Sinkhorn Attention", technical summary (gist.science
+// 2605.08123).  §2.1: each forward half-step is a band log-sum-exp
+//     u_r = log a_r - LSE_{c in band(r)} (S_rc + v_c),   S = scale X Y^T,
+// computed here with the previous potential as the shift (after a completed half-step every
+// plan entry exp(S + u_old + v) is at most 1, so no running maximum is needed; the very
+// first half-step of a call has no previous potential and keeps a running maximum).
+// §2.2: the backward sweeps re-form the one reference plan P(R,R) per tile from S and the
+// stored potentials, and apply the per-row / per-column orbit factors in registers.
+//
+// Roles in a CTA of 192 threads:
+//   warp 0      TMA producer (one elected lane): row tile once, column tiles into a ring
+//   warp 1      TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..5  epilogue: thread t of warp w owns TMEM lane / row 32 (w % 4) + t
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace eot {
 
-bool tc_supported(const Geom&) { return false; }
-cudaError_t launch_tc_lse(const LsePass&, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_tc_bwd(const BwdPass&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kThreads = 192;
+constexpr float kNegInf = -__builtin_huge_valf();
+
+// ---------------------------------------------------------------------------------------
+// Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
+// ---------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn || !base || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+    cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------------------
+// Device: band tile list shared by all roles of a CTA
+// ---------------------------------------------------------------------------------------
+// Columns of tile width BN intersecting the band of rows [r0, r0 + BM) that hold at least
+// one active band column (the dustbin position is excluded: its links are handled apart).
+// Returns the number of tiles; tile column indices go to tiles[].  Also reports whether
+// any row of the row tile is active.  Must be called by all threads.
+template <int BM, int BN>
+__device__ int build_tile_list(const float* logm, int L, int r0, int h, int D, int* tiles, int* flags,
+                               int* ntiles_smem, bool* any_row) {
+    const int tid = threadIdx.x;
+    const int clo = max(0, r0 - h), chi = min(L - 1, r0 + BM - 1 + h);
+    const int t_lo = clo / BN, t_hi = chi / BN;
+    for (int t = tid; t <= t_hi - t_lo; t += blockDim.x) flags[t] = 0;
+    __syncthreads();
+    for (int c = clo + tid; c <= chi; c += blockDim.x)
+        if (logm[c] != kNegInf && c != D) flags[c / BN - t_lo] = 1;
+    int rowact = 0;
+    for (int r = tid; r < BM; r += blockDim.x) rowact |= (logm[r0 + r] != kNegInf);
+    const int any = __syncthreads_or(rowact);
+    if (tid == 0) {
+        int n = 0;
+        for (int t = 0; t <= t_hi - t_lo; ++t)
+            if (flags[t]) tiles[n++] = t_lo + t;
+        *ntiles_smem = n;
+    }
+    __syncthreads();
+    *any_row = any != 0;
+    return *ntiles_smem;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ---------------------------------------------------------------------------------------
+// Forward half-step (band log-sum-exp), 128 x 128 tiles
+// ---------------------------------------------------------------------------------------
+struct TcLseArgs {
+    int H, L, h, D;
+    float sl2;              // scale * log2(e)
+    const float* logm;
+    const float* colbias2;  // [BH, L] masked log2 column bias
+    const float* colpot;    // natural column potential (pstride), read at D
+    const float* stab;      // natural previous row potential (pstride) or nullptr
+    float* out;             // natural (pstride)
+    float* out_bias2;       // [BH, L]
+    size_t pstride;
+    const float* sd_term;
+    uint32_t* status;
+};
+
+template <int DH>
+struct LseCfg {
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int KATOMS = DH / 64;
+    static constexpr int NS = DH == 128 ? 2 : 4;   // column-tile stages
+    static constexpr int NB = 4;                   // bias ring slots
+    static constexpr uint32_t XB = BM * DH * 2;    // row tile bytes
+    static constexpr uint32_t YB = BN * DH * 2;    // column tile bytes
+    static constexpr uint32_t ATOM = 128 * 128;    // one 64-element-wide atom column of 128 rows
+    static constexpr uint32_t OFF_Y = XB;
+    static constexpr uint32_t OFF_BIAS = OFF_Y + NS * YB;
+    static constexpr uint32_t OFF_BAR = OFF_BIAS + NB * BN * 4;
+    // barriers: full[NS] empty[NS] xfull tfull[2] tempty[2] bfull[NB] bempty[NB]
+    static constexpr uint32_t NBARS = 2 * NS + 1 + 4 + 2 * NB;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
+    static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
+    static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
+};
+
+template <int DH, bool ONLINE>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_lse_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                  const TcLseArgs a, int max_tiles) {
+    using C = LseCfg<DH>;
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = align1024(smraw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.y, b = bh / a.H, L = a.L, h = a.h, D = a.D;
+    const int r0 = blockIdx.x * C::BM;
+    const size_t base = size_t(bh) * L;
+    const size_t pb = size_t(bh) * a.pstride;
+    const float* logm = a.logm + size_t(b) * L;
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    const uint32_t bar0 = ptx::smem_u32(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (C::NS + s); };
+    const uint32_t xfull = bar0 + 8u * (2 * C::NS);
+    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 1 + i); };
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
+    auto bfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
+    auto bempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + C::NB + i); };
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
+    int* flags = tiles + max_tiles;
+    const float* bias_s = reinterpret_cast<const float*>(sm + C::OFF_BIAS);
+
+    if (tid == 0) *abort_flag = 0;
+    bool any_row;
+    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
+                                                 reinterpret_cast<int*>(misc + 2), &any_row);
+    if (!any_row) {
+        for (int r = tid; r < C::BM; r += kThreads) {
+            a.out[pb + r0 + r] = 0.f;
+            a.out_bias2[base + r0 + r] = kNegInf;
+        }
+        return;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            ptx::mbar_init(full(s), 1);
+            ptx::mbar_init(empty(s), 1);
+        }
+        ptx::mbar_init(xfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(tfull(i), 1);
+            ptx::mbar_init(tempty(i), 4);
+        }
+        for (int i = 0; i < C::NB; ++i) {
+            ptx::mbar_init(bfull(i), 1);
+            ptx::mbar_init(bempty(i), 4);
+        }
+        ptx::mbar_fence_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(misc), 256);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tbase = misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            ptx::prefetch_tmap(&tmX);
+            ptx::prefetch_tmap(&tmY);
+            const uint32_t xs = ptx::smem_u32(sm);
+            ptx::mbar_expect_tx(xfull, C::XB);
+            for (int ka = 0; ka < C::KATOMS; ++ka)
+                ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(base) + r0, xfull);
+            int issued = 0, bissued = 0;
+            for (int it = 0; it < n; ++it) {
+                const int s = it % C::NS, bs = it % C::NB;
+                const int c0 = tiles[it] * C::BN;
+                if (!ptx::mbar_wait(empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, a.status)) break;
+                ptx::mbar_expect_tx(full(s), C::YB);
+                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+                for (int ka = 0; ka < C::KATOMS; ++ka)
+                    ptx::tma_load_2d(ys + ka * C::ATOM, &tmY, ka * 64, int(base) + c0, full(s));
+                issued = it + 1;
+                if (!ptx::mbar_wait(bempty(bs), ((it / C::NB) & 1) ^ 1, abort_flag, a.status)) break;
+                ptx::mbar_expect_tx(bfull(bs), C::BN * 4);
+                ptx::bulk_load(ptx::smem_u32(sm + C::OFF_BIAS + bs * C::BN * 4), a.colbias2 + base + c0, C::BN * 4,
+                               bfull(bs));
+                bissued = it + 1;
+            }
+            if (*abort_flag) {
+                // Let every copy already issued land before the CTA retires.
+                volatile int dummy = 0;
+                for (int it = max(0, issued - C::NS); it < issued; ++it)
+                    ptx::mbar_wait(full(it % C::NS), (it / C::NS) & 1, &dummy, a.status);
+                for (int it = max(0, bissued - C::NB); it < bissued; ++it)
+                    ptx::mbar_wait(bfull(it % C::NB), (it / C::NB) & 1, &dummy, a.status);
+                ptx::mbar_wait(xfull, 0, &dummy, a.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t xs = ptx::smem_u32(sm);
+            int last = -1;
+            if (ptx::mbar_wait(xfull, 0, abort_flag, a.status)) {
+                for (int it = 0; it < n; ++it) {
+                    const int s = it % C::NS, bb = it & 1;
+                    if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) break;
+                    if (!ptx::mbar_wait(tempty(bb), ((it >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                    ptx::tc_fence_after();
+                    const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+                    const uint32_t dt = tbase + uint32_t(bb * C::BN);
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+                        ptx::mma_bf16(dt, ptx::smem_desc(xs + koff, 16, 1024), ptx::smem_desc(ys + koff, 16, 1024),
+                                      C::IDESC, kk > 0 ? 1u : 0u);
+                    }
+                    ptx::mma_commit(empty(s));
+                    ptx::mma_commit(tfull(bb));
+                    last = it;
+                }
+            }
+            if (*abort_flag && last >= 0) {
+                volatile int dummy = 0;
+                ptx::mbar_wait(tfull(last & 1), (last >> 1) & 1, &dummy, a.status);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;
+        const int row = q * 32 + lane, r = r0 + row;
+        const float lm = logm[r];
+        const bool is_dustbin_row = (r == D) && lm != kNegInf;
+        const float st = ONLINE ? 0.f : a.stab[pb + r];
+        const float st2 = st * kLog2e;
+        float m_run = kNegInf, sum = 0.f;
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        bool ok = true;
+        for (int it = 0; it < n && ok; ++it) {
+            const int bb = it & 1, bs = it % C::NB;
+            const int c0 = tiles[it] * C::BN;
+            const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
+            // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
+            bool w1 = ptx::mbar_wait(bfull(bs), (it / C::NB) & 1, abort_flag, a.status);
+            bool w2 = w1 && ptx::mbar_wait(tfull(bb), (it >> 1) & 1, abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN);
+#pragma unroll 1
+            for (int ch = 0; ch < C::BN / 32; ++ch) {
+                float v[32];
+                ptx::tmem_ld32(tbase + lane_base + uint32_t(bb * C::BN + ch * 32), v);
+                ptx::tmem_wait_ld(v);
+                if (ch == C::BN / 32 - 1) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(tempty(bb));
+                }
+                float x[32];
+#pragma unroll
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 bv = bias4[ch * 8 + j4];
+                    x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
+                    x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
+                    x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
+                    x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
+                }
+                if (!interior) {
+                    const int dlt0 = c0 + ch * 32 - r;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int dl = dlt0 + j;
+                        if (dl < -h || dl > h) x[j] = kNegInf;
+                    }
+                }
+                if (ONLINE) {
+                    float cm = kNegInf;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) cm = fmaxf(cm, x[j]);
+                    if (cm > m_run) {
+                        sum *= ptx::ex2(m_run - cm);
+                        m_run = cm;
+                    }
+                    if (m_run != kNegInf) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) sum += ptx::ex2(x[j] - m_run);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sum += ptx::ex2(x[j] + st2);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bempty(bs));
+        }
+        if (ok && !*abort_flag && !is_dustbin_row) {
+            float outv = 0.f, ob = kNegInf;
+            if (lm != kNegInf) {
+                const bool d_act = D >= 0 && logm[D] != kNegInf;
+                if (ONLINE) {
+                    if (d_act) lse2_add(m_run, sum, (a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e);
+                    outv = lm - (m_run + log2f(sum)) * kLn2;
+                } else {
+                    if (d_act) sum += ptx::ex2((a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e + st2);
+                    outv = lm - log2f(sum) * kLn2 + st;
+                }
+                if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+                ob = outv * kLog2e;
+            }
+            a.out[pb + r] = outv;
+            a.out_bias2[base + r] = ob;
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tbase, 256);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Backward / output sweep, 128-row x 64-column tiles
+// ---------------------------------------------------------------------------------------
+struct TcVecArgs {
+    int H, L, h, D, d;
+    float sc2;              // scale * log2(e)
+    const float* logm;
+    const float* pr;        // natural row bias [BH, L]
+    const float* pcm2;      // masked log2 column bias [BH, L]
+    const float* pc;        // natural column bias (read at D)
+    float* sout;
+    const float* f;
+    const float* hv;
+    const float* m;
+    int s_dp;
+    void* vout;
+    float vscale;
+    int v_dp;
+    int nmod;
+    const float* xr[kMaxMods];
+    const float* yc[kMaxMods];
+    const __nv_bfloat16* Zg;  // column-side vector operand (global), read at D
+    int z_from_w2;            // vector operand tile = second column tile (else the S tile)
+    int has_w2;               // a second column-side tensor is loaded
+    int has_dp;
+    const float* sd_term;
+    const float* dp_term;
+    uint32_t* status;
+};
+
+template <int DH>
+struct VecCfg {
+    static constexpr int BM = 128, BN = 64;
+    static constexpr int KATOMS = DH / 64;
+    static constexpr int NS = 3;
+    static constexpr uint32_t XB = BM * DH * 2;          // row tile bytes
+    static constexpr uint32_t YB = BN * DH * 2;          // column tile bytes
+    static constexpr uint32_t XATOM = BM * 128;          // 16 KB
+    static constexpr uint32_t YATOM = BN * 128;          // 8 KB
+    static constexpr uint32_t CB = BM * BN * 2;          // coefficient tile bytes (16 KB)
+    static constexpr int MAXV = 2 + kMaxMods;            // column vectors per stage
+    static constexpr uint32_t VB = MAXV * BN * 4;        // column vector bytes per stage
+    static constexpr uint32_t OFF_A = XB;
+    static constexpr uint32_t OFF_Y = 2 * XB;
+    static constexpr uint32_t OFF_W = OFF_Y + NS * YB;
+    static constexpr uint32_t OFF_C = OFF_W + NS * YB;
+    static constexpr uint32_t OFF_V = OFF_C + 2 * CB;
+    static constexpr uint32_t OFF_BAR = OFF_V + NS * VB;
+    // full[NS] empty[NS] xfull tfull[2] tempty[2] cfull[2] cempty[2] accfull
+    static constexpr uint32_t NBARS = 2 * NS + 1 + 8 + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
+    static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
+    static constexpr uint32_t IDESC_S = ptx::idesc_bf16(128, 64, false, false);
+    static constexpr uint32_t IDESC_O = ptx::idesc_bf16(128, DH, false, true);
+    static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_vec_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
+                  const TcVecArgs a, int max_tiles) {
+    using C = VecCfg<DH>;
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = align1024(smraw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.y, b = bh / a.H, L = a.L, h = a.h, D = a.D;
+    const int r0 = blockIdx.x * C::BM;
+    const size_t base = size_t(bh) * L;
+    const float* logm = a.logm + size_t(b) * L;
+    const bool vec = a.vout != nullptr, scal = a.sout != nullptr;
+    const int nv = 1 + (a.m ? 1 : 0) + a.nmod;   // column vectors per stage: pcm2, m, yc...
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+    const uint32_t bar0 = ptx::smem_u32(bars);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (C::NS + s); };
+    const uint32_t xfull = bar0 + 8u * (2 * C::NS);
+    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 1 + i); };
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
+    auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
+    auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 7 + i); };
+    const uint32_t accfull = bar0 + 8u * (2 * C::NS + 9);
+    uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
+    int* flags = tiles + max_tiles;
+
+    if (tid == 0) *abort_flag = 0;
+    bool any_row;
+    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
+                                                 reinterpret_cast<int*>(misc + 2), &any_row);
+    if (!any_row) {
+        for (int r = tid; r < C::BM; r += kThreads) {
+            if (scal) a.sout[base + r0 + r] = 0.f;
+        }
+        if (vec) {
+            __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
+            for (int e = tid; e < C::BM * DH / 8; e += kThreads)
+                reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            ptx::mbar_init(full(s), 1);
+            ptx::mbar_init(empty(s), 5);   // MMA commit + 4 epilogue warps
+        }
+        ptx::mbar_init(xfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(tfull(i), 1);
+            ptx::mbar_init(tempty(i), 4);
+            ptx::mbar_init(cfull(i), 4);
+            ptx::mbar_init(cempty(i), 1);
+        }
+        ptx::mbar_init(accfull, 1);
+        ptx::mbar_fence_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_u32(misc), 512);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tbase = misc[0];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            ptx::prefetch_tmap(&tmX);
+            ptx::prefetch_tmap(&tmY);
+            if (a.has_dp) ptx::prefetch_tmap(&tmA);
+            if (a.has_w2) ptx::prefetch_tmap(&tmW);
+            const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
+            ptx::mbar_expect_tx(xfull, C::XB * (a.has_dp ? 2 : 1));
+            for (int ka = 0; ka < C::KATOMS; ++ka) {
+                ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
+                if (a.has_dp) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
+            }
+            const float* vsrc[C::MAXV];
+            int k = 0;
+            vsrc[k++] = a.pcm2;
+            if (a.m) vsrc[k++] = a.m;
+            for (int i = 0; i < a.nmod; ++i) vsrc[k++] = a.yc[i];
+            const uint32_t stage_bytes = C::YB * (a.has_w2 ? 2 : 1) + uint32_t(nv) * C::BN * 4;
+            int issued = 0;
+            for (int it = 0; it < n; ++it) {
+                const int s = it % C::NS;
+                const int c0 = tiles[it] * C::BN;
+                if (!ptx::mbar_wait(empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, a.status)) break;
+                ptx::mbar_expect_tx(full(s), stage_bytes);
+                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+                const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
+                for (int ka = 0; ka < C::KATOMS; ++ka) {
+                    ptx::tma_load_2d(ys + ka * C::YATOM, &tmY, ka * 64, int(base) + c0, full(s));
+                    if (a.has_w2) ptx::tma_load_2d(ws + ka * C::YATOM, &tmW, ka * 64, int(base) + c0, full(s));
+                }
+                const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
+                for (int i = 0; i < nv; ++i)
+                    ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full(s));
+                issued = it + 1;
+            }
+            if (*abort_flag) {
+                volatile int dummy = 0;
+                for (int it = max(0, issued - C::NS); it < issued; ++it)
+                    ptx::mbar_wait(full(it % C::NS), (it / C::NS) & 1, &dummy, a.status);
+                ptx::mbar_wait(xfull, 0, &dummy, a.status);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
+            int vec_done = 0;        // vector products issued
+            bool ok = ptx::mbar_wait(xfull, 0, abort_flag, a.status);
+            auto do_vec = [&](int j) -> bool {
+                const int cb = j & 1;
+                if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) return false;
+                ptx::tc_fence_after();
+                const int s = j % C::NS;
+                const uint32_t zs = ptx::smem_u32(sm + (a.z_from_w2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
+                const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + kk * 32, 16, 1024),
+                                  ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::mma_commit(cempty(cb));
+                ptx::mma_commit(empty(s));
+                vec_done = j + 1;
+                return true;
+            };
+            int issued = 0;
+            for (int it = 0; it < n && ok; ++it) {
+                const int s = it % C::NS, bb = it & 1;
+                if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
+                if (!ptx::mbar_wait(tempty(bb), ((it >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+                const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk) {
+                    const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
+                    const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
+                    ptx::mma_bf16(tbase + C::TM_S + bb * C::BN, ptx::smem_desc(xs + xo, 16, 1024),
+                                  ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                if (a.has_dp) {
+#pragma unroll
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
+                        const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
+                        ptx::mma_bf16(tbase + C::TM_DP + bb * C::BN, ptx::smem_desc(as + xo, 16, 1024),
+                                      ptx::smem_desc(ws + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                }
+                ptx::mma_commit(tfull(bb));
+                if (!vec) ptx::mma_commit(empty(s));
+                issued = it + 1;
+                if (vec && it >= 1 && !do_vec(it - 1)) { ok = false; break; }
+            }
+            if (ok && vec && n > 0 && do_vec(n - 1)) ptx::mma_commit(accfull);
+            if (*abort_flag) {
+                volatile int dummy = 0;
+                if (issued > 0) ptx::mbar_wait(tfull((issued - 1) & 1), ((issued - 1) >> 1) & 1, &dummy, a.status);
+                if (vec_done > 0)
+                    ptx::mbar_wait(cempty((vec_done - 1) & 1), ((vec_done - 1) >> 1) & 1, &dummy, a.status);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3;
+        const int row = q * 32 + lane, r = r0 + row;
+        const float lm = logm[r];
+        const bool ract = lm != kNegInf;
+        const bool is_dustbin_row = (r == D) && ract;
+        const float pr2 = ract ? a.pr[base + r] * kLog2e : kNegInf;
+        float xr[kMaxMods];
+#pragma unroll
+        for (int k = 0; k < kMaxMods; ++k) xr[k] = (k < a.nmod && ract) ? a.xr[k][base + r] : 0.f;
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        float s1 = 0.f, s2 = 0.f;
+        bool ok = true;
+        const int voff_m = 1, voff_y = 1 + (a.m ? 1 : 0);
+        const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
+        for (int it = 0; it < n; ++it) {
+            const int s = it % C::NS, bb = it & 1, cb = it & 1;
+            const int c0 = tiles[it] * C::BN;
+            const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
+            // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
+            bool w1 = ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status);
+            bool w2 = w1 && ptx::mbar_wait(tfull(bb), (it >> 1) & 1, abort_flag, a.status);
+            bool w3 = w2 && (!vec || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
+            if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const float* cv = reinterpret_cast<const float*>(sm + C::OFF_V + s * C::VB);
+            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + crow;
+#pragma unroll 1
+            for (int ch = 0; ch < C::BN / 32; ++ch) {
+                float v[32], w[32];
+                ptx::tmem_ld32(tbase + lane_base + C::TM_S + uint32_t(bb * C::BN + ch * 32), v);
+                if (a.has_dp) {
+                    ptx::tmem_ld32(tbase + lane_base + C::TM_DP + uint32_t(bb * C::BN + ch * 32), w);
+                    ptx::tmem_wait_ld(v, w);
+                } else {
+                    ptx::tmem_wait_ld(v);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) w[j] = 0.f;
+                }
+                if (ch == C::BN / 32 - 1) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(tempty(bb));
+                }
+                const int cc0 = ch * 32;
+                float P[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) P[j] = fmaf(v[j], a.sc2, pr2 + cv[cc0 + j]);
+                if (!interior) {
+                    const int dlt0 = c0 + cc0 - r;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int dl = dlt0 + j;
+                        if (dl < -h || dl > h) P[j] = kNegInf;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) P[j] = ptx::ex2(P[j]);
+                if (scal) {
+                    if (a.s_dp) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) s1 = fmaf(P[j], w[j], s1);
+                    }
+                    if (a.m) {
+                        const float* mv = cv + voff_m * C::BN + cc0;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) s2 = fmaf(P[j], mv[j], s2);
+                    }
+                }
+                if (vec) {
+                    float cf[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) cf[j] = a.v_dp ? w[j] : 1.f;
+#pragma unroll
+                    for (int k = 0; k < kMaxMods; ++k) {
+                        if (k < a.nmod) {
+                            const float* yv = cv + (voff_y + k) * C::BN + cc0;
+                            const float xk = xr[k];
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) cf[j] = fmaf(-xk, yv[j], cf[j]);
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t unit = uint32_t(ch * 4 + t);
+                        const uint32_t addr = cbase + ((unit ^ uint32_t(row & 7)) << 4);
+                        ptx::st_shared_v4(addr, ptx::pack_bf16(P[8 * t + 0] * cf[8 * t + 0], P[8 * t + 1] * cf[8 * t + 1]),
+                                          ptx::pack_bf16(P[8 * t + 2] * cf[8 * t + 2], P[8 * t + 3] * cf[8 * t + 3]),
+                                          ptx::pack_bf16(P[8 * t + 4] * cf[8 * t + 4], P[8 * t + 5] * cf[8 * t + 5]),
+                                          ptx::pack_bf16(P[8 * t + 6] * cf[8 * t + 6], P[8 * t + 7] * cf[8 * t + 7]));
+                    }
+                }
+            }
+            if (vec) ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(empty(s));
+                if (vec) ptx::mbar_arrive(cfull(cb));
+            }
+        }
+        // Dustbin link of this row (the dustbin column), then the writes.
+        const bool d_act = D >= 0 && logm[D] != kNegInf;
+        float Pd = 0.f, dpd = 0.f, coefd = 0.f;
+        if (ract && d_act && !is_dustbin_row) {
+            Pd = ptx::ex2((a.sd_term[base + r] + a.pr[base + r] + a.pc[base + D]) * kLog2e);
+            if (a.has_dp) dpd = a.dp_term[base + r];
+            float mod = a.v_dp ? dpd : 1.f;
+#pragma unroll
+            for (int k = 0; k < kMaxMods; ++k)
+                if (k < a.nmod) mod -= xr[k] * a.yc[k][base + D];
+            coefd = Pd * mod;
+        }
+        if (ok && scal && !is_dustbin_row) {
+            if (d_act && ract) {
+                if (a.s_dp) s1 = fmaf(Pd, dpd, s1);
+                if (a.m) s2 = fmaf(Pd, a.m[base + D], s2);
+            }
+            float outv = 0.f;
+            if (ract) {
+                outv = (a.f ? a.f[base + r] : 1.f) * (s1 + (a.hv ? a.hv[base + r] : 0.f) * s2);
+                if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+            }
+            a.sout[base + r] = outv;
+        }
+        // The accumulator read is a warp-collective: every lane of the warp takes part; only
+        // the stores are predicated (the dustbin row is written by the dense dustbin kernel).
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && vec) {
+            const bool have_acc = n > 0;
+            bool wacc = !have_acc || ptx::mbar_wait(accfull, 0, abort_flag, a.status);
+            ok = __all_sync(0xffffffffu, wacc);
+            ptx::tc_fence_after();
+            if (ok) {
+                __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r) * DH;
+                const __nv_bfloat16* zD = d_act ? a.Zg + (base + D) * DH : nullptr;
+                const bool store = !is_dustbin_row;
+#pragma unroll 1
+                for (int ch = 0; ch < DH / 32; ++ch) {
+                    float v[32];
+                    if (have_acc) {
+                        ptx::tmem_ld32(tbase + lane_base + C::TM_ACC + uint32_t(ch * 32), v);
+                        ptx::tmem_wait_ld(v);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        float lo = v[2 * j], hi = v[2 * j + 1];
+                        if (ract && d_act && store) {
+                            lo = fmaf(coefd, __bfloat162float(zD[ch * 32 + 2 * j]), lo);
+                            hi = fmaf(coefd, __bfloat162float(zD[ch * 32 + 2 * j + 1]), hi);
+                        }
+                        pk[j] = ract ? ptx::pack_bf16(a.vscale * lo, a.vscale * hi) : 0u;
+                    }
+                    if (store) {
+                        uint4* dst = reinterpret_cast<uint4*>(vo + ch * 32);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                    }
+                }
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tbase, 512);
+    }
+}
+
+int max_tiles_for(int L, int h, int BM, int BN) {
+    const long span = long(BM) + 2L * h;
+    const long t = span / BN + 2;
+    return int(std::min<long>(t, L / BN));
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+}
+
+}  // namespace
+
+bool tc_supported(const Geom& g) { return g.dtype == EOT_BF16 && (g.d == 64 || g.d == 128) && encode_fn() != nullptr; }
+
+cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
+    const Geom& g = p.g;
+    CUtensorMap tmX, tmY;
+    const uint64_t rows = uint64_t(g.BH) * g.L;
+    if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
+    TcLseArgs a{};
+    a.H = g.H;
+    a.L = g.L;
+    a.h = g.h;
+    a.D = g.D;
+    a.sl2 = g.scale * kLog2e;
+    a.logm = p.logm;
+    a.colbias2 = p.colbias2;
+    a.colpot = p.colpot;
+    a.stab = p.stab;
+    a.out = p.out;
+    a.out_bias2 = p.out_bias2;
+    a.pstride = p.pstride;
+    a.sd_term = p.sd_term;
+    a.status = p.status;
+    const int mt = max_tiles_for(g.L, g.h, 128, 128);
+    dim3 grid(g.L / 128, g.BH);
+    cudaError_t e;
+    if (g.d == 128) {
+        const size_t smem = LseCfg<128>::smem_bytes(mt);
+        if (p.stab) {
+            if ((e = set_smem(tc_lse_kernel<128, false>, smem)) != cudaSuccess) return e;
+            tc_lse_kernel<128, false><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+        } else {
+            if ((e = set_smem(tc_lse_kernel<128, true>, smem)) != cudaSuccess) return e;
+            tc_lse_kernel<128, true><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+        }
+    } else {
+        const size_t smem = LseCfg<64>::smem_bytes(mt);
+        if (p.stab) {
+            if ((e = set_smem(tc_lse_kernel<64, false>, smem)) != cudaSuccess) return e;
+            tc_lse_kernel<64, false><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+        } else {
+            if ((e = set_smem(tc_lse_kernel<64, true>, smem)) != cudaSuccess) return e;
+            tc_lse_kernel<64, true><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+        }
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || g.D < 0) return e;
+    return launch_dustbin_lse(p, st);
+}
+
+cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
+    const Geom& g = p.g;
+    const bool has_dp = (p.sout && p.s_dp) || (p.vout && p.v_dp);
+    // Column-side tensors: Y always; the second one is the dP operand or, if different from
+    // Y, the vector operand Z.
+    const void* w2 = has_dp ? p.Bm : (p.vout && p.Z != p.Y ? p.Z : nullptr);
+    const uint64_t rows = uint64_t(g.BH) * g.L;
+    CUtensorMap tmX, tmA, tmY, tmW;
+    if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
+    if (!make_map(&tmA, has_dp ? p.A : p.X, rows, g.d, 128)) return cudaErrorInvalidValue;
+    if (!make_map(&tmW, w2 ? w2 : p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
+    if (p.vout && p.Z != p.Y && p.Z != w2) return cudaErrorInvalidValue;   // not a pass this library runs
+    TcVecArgs a{};
+    a.H = g.H;
+    a.L = g.L;
+    a.h = g.h;
+    a.D = g.D;
+    a.d = g.d;
+    a.sc2 = g.scale * kLog2e;
+    a.logm = p.logm;
+    a.pr = p.pr;
+    a.pcm2 = p.pcm2;
+    a.pc = p.pc;
+    a.sout = p.sout;
+    a.f = p.f;
+    a.hv = p.hv;
+    a.m = p.sout ? p.m : nullptr;
+    a.s_dp = p.s_dp;
+    a.vout = p.vout;
+    a.vscale = p.vscale;
+    a.v_dp = p.v_dp;
+    a.nmod = p.vout ? p.nmod : 0;
+    for (int k = 0; k < a.nmod; ++k) {
+        a.xr[k] = p.xr[k];
+        a.yc[k] = p.yc[k];
+    }
+    a.Zg = static_cast<const __nv_bfloat16*>(p.Z);
+    a.z_from_w2 = (p.vout && w2 && p.Z == w2) ? 1 : 0;
+    a.has_w2 = w2 ? 1 : 0;
+    a.has_dp = has_dp ? 1 : 0;
+    a.sd_term = p.sd_term;
+    a.dp_term = p.dp_term;
+    a.status = p.status;
+    const int mt = max_tiles_for(g.L, g.h, 128, 64);
+    dim3 grid(g.L / 128, g.BH);
+    cudaError_t e;
+    if (g.d == 128) {
+        const size_t smem = VecCfg<128>::smem_bytes(mt);
+        if ((e = set_smem(tc_vec_kernel<128>, smem)) != cudaSuccess) return e;
+        tc_vec_kernel<128><<<grid, kThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
+    } else {
+        // at least 120 KB so that one CTA owns the SM (the kernel allocates all 512 TMEM columns)
+        const size_t smem = std::max<size_t>(VecCfg<64>::smem_bytes(mt), 120 * 1024);
+        if ((e = set_smem(tc_vec_kernel<64>, smem)) != cudaSuccess) return e;
+        tc_vec_kernel<64><<<grid, kThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || g.D < 0) return e;
+    return launch_dustbin_bwd(p, st);
+}
 
 }  // namespace eot

@@ -132,6 +132,19 @@ const char* eot_status_string(eot_status s);
 /* EOT_ABI_VERSION of the loaded library. */
 int eot_abi_version(void);
 
+/* Benchmark support (process-wide, not thread-safe).
+ * eot_kernel_launches: number of kernels this library has enqueued since it was loaded.
+ * eot_profile_begin / eot_profile_end: between the two calls, every sweep that fwd/bwd
+ * enqueue is bracketed by a pair of CUDA events recorded on the call's stream;
+ * eot_profile_end synchronises ``stream`` and totals the elapsed times per kind.
+ * eot_profile_read(kind, ...): kind 0 = forward half-step sweeps, 1 = forward output sweep,
+ * 2 = backward sweeps, 3 = auxiliary kernels (marginals, vectors, dustbin links); returns
+ * the summed milliseconds and the number of bracketed launches of that kind. */
+long long eot_kernel_launches(void);
+void eot_profile_begin(void);
+eot_status eot_profile_end(void* stream);
+eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
+
 /* Kernel family that ``p`` would run with (EOT_IMPL_SIMT or EOT_IMPL_TCGEN05), or -1 if
  * the problem is invalid or unsupported. */
 int eot_resolved_impl(const eot_problem* p);
