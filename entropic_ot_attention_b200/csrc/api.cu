@@ -291,7 +291,9 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.sd_dense = sd_col;
     rowp.dp_term = e1;
     rowp.dp_dense = e2;
+    rowp.zero_vec = at<float>(ws, w.zero);
     rowp.status = status;
+    EOT_TRY(cudaMemsetAsync(at<float>(ws, w.zero), 0, vecn * sizeof(float), st));
     BwdPass colp = rowp;
     colp.X = K;
     colp.Y = Q;

@@ -83,6 +83,7 @@ struct BwdPass {
     const float* sd_dense;
     const float* dp_term;   // <A_r, Bm_D>
     const float* dp_dense;  // <A_D, Bm_c>
+    const float* zero_vec;  // [BH, L] zeros (padding of the modifier list), or nullptr
     uint32_t* status;
 };
 
@@ -92,6 +93,7 @@ struct WsLayout {
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t pcm;             // backward: masked log2 column bias
+    size_t zero;            // backward: a vector of zeros
     size_t pr, pc, f, hv, m;
     size_t xr, yc;          // kMaxMods vectors each, [BH, L]
     size_t alpha, beta;     // (R + 1) vectors each, [BH, L]
@@ -126,6 +128,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.hv = o; o += vec;
         w.m = o; o += vec;
         w.pcm = o; o += vec;
+        w.zero = o; o += vec;
         w.xr = o; o += vec * 2 * p.R;
         w.yc = o; o += vec * 2 * p.R;
         w.alpha = o; o += vec * (p.R + 1);

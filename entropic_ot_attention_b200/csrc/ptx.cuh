@@ -183,6 +183,55 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// ---- packed fp32x2 arithmetic (sm_100) ---------------------------------------------------
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipe (no MUFU): Cody-Waite reduction x = j + f with
+// j = round(x) (the 1.5 * 2^23 rounding constant), |f| <= 1/2, then 2^f by the degree-5
+// Chebyshev-interpolation polynomial of csrc/gen_exp2_poly.py (max relative error 2.4e-7,
+// the accuracy of ex2.approx), and 2^j applied by adding j to the exponent field.
+// Inputs are clamped to [-125, 127): below -125 the result is 2^-125 instead of 0, which is
+// only used where such entries are negligible against the sum they join.
+__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+    const uint64_t R2 = f2(kRound, kRound);
+    const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = fadd2(x, R2);
+    const uint64_t f = fsub2(x, fsub2(t, R2));
+    uint64_t p = ffma2(f2(1.339086331e-03f, 1.339086331e-03f), f, f2(9.676031768e-03f, 9.676031768e-03f));
+    p = ffma2(p, f, f2(5.550356954e-02f, 5.550356954e-02f));
+    p = ffma2(p, f, f2(2.402210683e-01f, 2.402210683e-01f));
+    p = ffma2(p, f, f2(6.931471825e-01f, 6.931471825e-01f));
+    p = ffma2(p, f, f2(1.000000119e+00f, 1.000000119e+00f));
+    float t0, t1, p0, p1;
+    f2split(t, t0, t1);
+    f2split(p, p0, p1);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

@@ -28,6 +28,9 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr float kNegInf = -__builtin_huge_valf();
+// Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
+// interior forward tiles (6 of 16 pairs: 37.5 %, where the two pipes balance).
+constexpr int kFmaPairs = 6;
 
 // ---------------------------------------------------------------------------------------
 // Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
@@ -130,7 +133,7 @@ struct LseCfg {
 };
 
 template <int DH, bool ONLINE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                   const TcLseArgs a, int max_tiles) {
     using C = LseCfg<DH>;
@@ -266,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool is_dustbin_row = (r == D) && lm != kNegInf;
         const float st = ONLINE ? 0.f : a.stab[pb + r];
         const float st2 = st * kLog2e;
-        float m_run = kNegInf, sum = 0.f;
+        float m_run = kNegInf;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums (no serial FADD chain)
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         bool ok = true;
         for (int it = 0; it < n && ok; ++it) {
@@ -279,53 +283,102 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
             ptx::tc_fence_after();
             const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN);
-#pragma unroll 1
-            for (int ch = 0; ch < C::BN / 32; ++ch) {
-                float v[32];
-                ptx::tmem_ld32(tbase + lane_base + uint32_t(bb * C::BN + ch * 32), v);
-                ptx::tmem_wait_ld(v);
-                if (ch == C::BN / 32 - 1) {
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(tempty(bb));
-                }
-                float x[32];
+            const uint32_t tcol = tbase + lane_base + uint32_t(bb * C::BN);
+            auto process = [&](const float (&v)[32], int ch) {
+                if (ONLINE || !interior) {
+                    // scalar path: running maximum (first half-step) or band-edge masking
+                    float x[32];
 #pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const float4 bv = bias4[ch * 8 + j4];
-                    x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
-                    x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
-                    x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
-                    x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
-                }
-                if (!interior) {
-                    const int dlt0 = c0 + ch * 32 - r;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int dl = dlt0 + j;
-                        if (dl < -h || dl > h) x[j] = kNegInf;
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 bv = bias4[ch * 8 + j4];
+                        x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
+                        x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
+                        x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
+                        x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
                     }
-                }
-                if (ONLINE) {
-                    float cm = kNegInf;
+                    if (!interior) {
+                        const int dlt0 = c0 + ch * 32 - r;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) cm = fmaxf(cm, x[j]);
-                    if (cm > m_run) {
-                        sum *= ptx::ex2(m_run - cm);
-                        m_run = cm;
+                        for (int j = 0; j < 32; ++j) {
+                            const int dl = dlt0 + j;
+                            if (dl < -h || dl > h) x[j] = kNegInf;
+                        }
                     }
-                    if (m_run != kNegInf) {
+                    if (ONLINE) {
+                        float cm = kNegInf;
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) sum += ptx::ex2(x[j] - m_run);
+                        for (int j = 0; j < 32; ++j) cm = fmaxf(cm, x[j]);
+                        if (cm > m_run) {
+                            const float sc = ptx::ex2(m_run - cm);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) acc[k] *= sc;
+                            m_run = cm;
+                        }
+                        if (m_run != kNegInf) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] - m_run);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] + st2);
                     }
                 } else {
+                    // interior tile, shifted by the previous potential: packed fp32x2 math;
+                    // the first kFmaPairs pairs of exponentials go to the FMA pipe, the rest
+                    // to the MUFU pipe, so that the two pipes share the exp2 work.
+                    const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
+                    uint64_t acc2[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) sum += ptx::ex2(x[j] + st2);
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 bv = bias4[ch * 8 + j4];
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            const int k = 2 * j4 + hh;
+                            uint64_t xx = ptx::ffma2(ptx::f2(v[2 * k], v[2 * k + 1]), SL2,
+                                                     hh ? ptx::f2(bv.z, bv.w) : ptx::f2(bv.x, bv.y));
+                            xx = ptx::fadd2(xx, ST2);
+                            float x0, x1, e0, e1;
+                            ptx::f2split(xx, x0, x1);
+                            if (k < kFmaPairs) {
+                                ptx::exp2_fma_x2(x0, x1, e0, e1);
+                            } else {
+                                e0 = ptx::ex2(x0);
+                                e1 = ptx::ex2(x1);
+                            }
+                            acc2[k & 1] = ptx::fadd2(acc2[k & 1], ptx::f2(e0, e1));
+                        }
+                    }
+                    float s0, s1, s2, s3;
+                    ptx::f2split(acc2[0], s0, s1);
+                    ptx::f2split(acc2[1], s2, s3);
+                    acc[0] += s0;
+                    acc[1] += s1;
+                    acc[2] += s2;
+                    acc[3] += s3;
                 }
-            }
+            };
+            // TMEM loads run one chunk ahead of the arithmetic.
+            float va[32], vb[32];
+            ptx::tmem_ld32(tcol + 0, va);
+            ptx::tmem_wait_ld(va);
+            ptx::tmem_ld32(tcol + 32, vb);
+            process(va, 0);
+            ptx::tmem_wait_ld(vb);
+            ptx::tmem_ld32(tcol + 64, va);
+            process(vb, 1);
+            ptx::tmem_wait_ld(va);
+            ptx::tmem_ld32(tcol + 96, vb);
+            process(va, 2);
+            ptx::tmem_wait_ld(vb);
+            // accumulator buffer fully read: hand it back to the MMA warp
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(tempty(bb));
+            process(vb, 3);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bempty(bs));
         }
+        float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
         if (ok && !*abort_flag && !is_dustbin_row) {
             float outv = 0.f, ob = kNegInf;
             if (lm != kNegInf) {
@@ -353,10 +406,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// Backward / output sweep, 128-row x 64-column tiles
+// Output / backward sweep, 128-row x 64-column tiles
 // ---------------------------------------------------------------------------------------
+// Pass kinds (compile-time, so that each variant carries only its own arithmetic):
+//   Out    O  = sum_c (P/a)_rc V_c                                   (forward output)
+//   C1     beta_R = sum_c Pt_rc dP_rc  and  dV = sum_c Pt_rc dO_c     (column sweep)
+//   R2     alpha_R = sum_c Pt dP + hv_r sum_c Pt m_c                  (row sweep)
+//   Stair  f_r * hv_r * sum_c P_rc m_c                                (staircase sweeps)
+//   Grad   dQ / dK = scale sum_c Pt_rc (dP_rc - sum_k xr_k yc_k) Y_c  (final sweeps)
+enum SweepMode { kModeOut = 0, kModeC1 = 1, kModeR2 = 2, kModeStair = 3, kModeGrad = 4 };
+
+template <int MODE>
+struct ModeT {
+    static constexpr bool SCAL = MODE == kModeC1 || MODE == kModeR2 || MODE == kModeStair;
+    static constexpr bool SDP = MODE == kModeC1 || MODE == kModeR2;
+    static constexpr bool SM = MODE == kModeR2 || MODE == kModeStair;
+    static constexpr bool VEC = MODE == kModeOut || MODE == kModeC1 || MODE == kModeGrad;
+    static constexpr bool VDP = MODE == kModeGrad;
+    static constexpr bool HASDP = SDP || VDP;
+    static constexpr bool W2 = HASDP || MODE == kModeOut;        // second column-side tensor
+    static constexpr bool ZW2 = MODE == kModeOut || MODE == kModeC1;  // vector operand = W2 tile
+};
+
 struct TcVecArgs {
-    int H, L, h, D, d;
+    int H, L, h, D;
     float sc2;              // scale * log2(e)
     const float* logm;
     const float* pr;        // natural row bias [BH, L]
@@ -366,24 +439,20 @@ struct TcVecArgs {
     const float* f;
     const float* hv;
     const float* m;
-    int s_dp;
     void* vout;
     float vscale;
-    int v_dp;
-    int nmod;
     const float* xr[kMaxMods];
     const float* yc[kMaxMods];
     const __nv_bfloat16* Zg;  // column-side vector operand (global), read at D
-    int z_from_w2;            // vector operand tile = second column tile (else the S tile)
-    int has_w2;               // a second column-side tensor is loaded
-    int has_dp;
     const float* sd_term;
     const float* dp_term;
     uint32_t* status;
 };
 
-template <int DH>
-struct VecCfg {
+constexpr int kSweepThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
+
+template <int DH, int NV>
+struct SweepCfg {
     static constexpr int BM = 128, BN = 64;
     static constexpr int KATOMS = DH / 64;
     static constexpr int NS = 3;
@@ -392,14 +461,14 @@ struct VecCfg {
     static constexpr uint32_t XATOM = BM * 128;          // 16 KB
     static constexpr uint32_t YATOM = BN * 128;          // 8 KB
     static constexpr uint32_t CB = BM * BN * 2;          // coefficient tile bytes (16 KB)
-    static constexpr int MAXV = 2 + kMaxMods;            // column vectors per stage
-    static constexpr uint32_t VB = MAXV * BN * 4;        // column vector bytes per stage
+    static constexpr uint32_t VB = NV * BN * 4;          // column vector bytes per stage
     static constexpr uint32_t OFF_A = XB;
     static constexpr uint32_t OFF_Y = 2 * XB;
     static constexpr uint32_t OFF_W = OFF_Y + NS * YB;
     static constexpr uint32_t OFF_C = OFF_W + NS * YB;
     static constexpr uint32_t OFF_V = OFF_C + 2 * CB;
-    static constexpr uint32_t OFF_BAR = OFF_V + NS * VB;
+    static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2][2][128] scalar partials
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
     // full[NS] empty[NS] xfull tfull[2] tempty[2] cfull[2] cempty[2] accfull
     static constexpr uint32_t NBARS = 2 * NS + 1 + 8 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -410,12 +479,15 @@ struct VecCfg {
     static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256;
 };
 
-template <int DH>
-__global__ void __launch_bounds__(kThreads, 1)
-    tc_vec_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
-                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
-                  const TcVecArgs a, int max_tiles) {
-    using C = VecCfg<DH>;
+template <int DH, int MODE, int NMOD>
+__global__ void __launch_bounds__(kSweepThreads, 1)
+    tc_sweep_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
+                    const TcVecArgs a, int max_tiles) {
+    using M = ModeT<MODE>;
+    constexpr int NV = 1 + (M::SM ? 1 : 0) + NMOD;   // column vectors per stage: pcm2, m, yc...
+    using C = SweepCfg<DH, NV>;
+    constexpr int VOFF_M = 1, VOFF_Y = 1 + (M::SM ? 1 : 0);
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -423,8 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r0 = blockIdx.x * C::BM;
     const size_t base = size_t(bh) * L;
     const float* logm = a.logm + size_t(b) * L;
-    const bool vec = a.vout != nullptr, scal = a.sout != nullptr;
-    const int nv = 1 + (a.m ? 1 : 0) + a.nmod;   // column vectors per stage: pcm2, m, yc...
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     const uint32_t bar0 = ptx::smem_u32(bars);
@@ -446,12 +516,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
                                                  reinterpret_cast<int*>(misc + 2), &any_row);
     if (!any_row) {
-        for (int r = tid; r < C::BM; r += kThreads) {
-            if (scal) a.sout[base + r0 + r] = 0.f;
-        }
-        if (vec) {
+        if (M::SCAL)
+            for (int r = tid; r < C::BM; r += kSweepThreads) a.sout[base + r0 + r] = 0.f;
+        if (M::VEC) {
             __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
-            for (int e = tid; e < C::BM * DH / 8; e += kThreads)
+            for (int e = tid; e < C::BM * DH / 8; e += kSweepThreads)
                 reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
         }
         return;
@@ -459,13 +528,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::NS; ++s) {
             ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 5);   // MMA commit + 4 epilogue warps
+            ptx::mbar_init(empty(s), 9);   // MMA commit + 8 epilogue warps
         }
         ptx::mbar_init(xfull, 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(tfull(i), 1);
-            ptx::mbar_init(tempty(i), 4);
-            ptx::mbar_init(cfull(i), 4);
+            ptx::mbar_init(tempty(i), 8);
+            ptx::mbar_init(cfull(i), 8);
             ptx::mbar_init(cempty(i), 1);
         }
         ptx::mbar_init(accfull, 1);
@@ -485,20 +554,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---------------- TMA producer ----------------
             ptx::prefetch_tmap(&tmX);
             ptx::prefetch_tmap(&tmY);
-            if (a.has_dp) ptx::prefetch_tmap(&tmA);
-            if (a.has_w2) ptx::prefetch_tmap(&tmW);
+            if (M::HASDP) ptx::prefetch_tmap(&tmA);
+            if (M::W2) ptx::prefetch_tmap(&tmW);
             const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
-            ptx::mbar_expect_tx(xfull, C::XB * (a.has_dp ? 2 : 1));
+            ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1));
             for (int ka = 0; ka < C::KATOMS; ++ka) {
                 ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
-                if (a.has_dp) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
+                if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
             }
-            const float* vsrc[C::MAXV];
-            int k = 0;
-            vsrc[k++] = a.pcm2;
-            if (a.m) vsrc[k++] = a.m;
-            for (int i = 0; i < a.nmod; ++i) vsrc[k++] = a.yc[i];
-            const uint32_t stage_bytes = C::YB * (a.has_w2 ? 2 : 1) + uint32_t(nv) * C::BN * 4;
+            const float* vsrc[NV];
+            {
+                int k = 0;
+                vsrc[k++] = a.pcm2;
+                if (M::SM) vsrc[k++] = a.m;
+                for (int i = 0; i < NMOD; ++i) vsrc[k++] = a.yc[i];
+            }
+            constexpr uint32_t stage_bytes = C::YB * (M::W2 ? 2 : 1) + uint32_t(NV) * C::BN * 4;
             int issued = 0;
             for (int it = 0; it < n; ++it) {
                 const int s = it % C::NS;
@@ -509,11 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
                 for (int ka = 0; ka < C::KATOMS; ++ka) {
                     ptx::tma_load_2d(ys + ka * C::YATOM, &tmY, ka * 64, int(base) + c0, full(s));
-                    if (a.has_w2) ptx::tma_load_2d(ws + ka * C::YATOM, &tmW, ka * 64, int(base) + c0, full(s));
+                    if (M::W2) ptx::tma_load_2d(ws + ka * C::YATOM, &tmW, ka * 64, int(base) + c0, full(s));
                 }
                 const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
-                for (int i = 0; i < nv; ++i)
-                    ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full(s));
+#pragma unroll
+                for (int i = 0; i < NV; ++i) ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full(s));
                 issued = it + 1;
             }
             if (*abort_flag) {
@@ -527,21 +598,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
             const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
-            int vec_done = 0;        // vector products issued
+            int vec_done = 0;
             bool ok = ptx::mbar_wait(xfull, 0, abort_flag, a.status);
             auto do_vec = [&](int j) -> bool {
                 const int cb = j & 1;
                 if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) return false;
                 ptx::tc_fence_after();
                 const int s = j % C::NS;
-                const uint32_t zs = ptx::smem_u32(sm + (a.z_from_w2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
+                const uint32_t zs = ptx::smem_u32(sm + (M::ZW2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
                 const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk) {
+                for (int kk = 0; kk < C::BN / 16; ++kk)
                     ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + kk * 32, 16, 1024),
                                   ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
                                   (j > 0 || kk > 0) ? 1u : 0u);
-                }
                 ptx::mma_commit(cempty(cb));
                 ptx::mma_commit(empty(s));
                 vec_done = j + 1;
@@ -562,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mma_bf16(tbase + C::TM_S + bb * C::BN, ptx::smem_desc(xs + xo, 16, 1024),
                                   ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
-                if (a.has_dp) {
+                if (M::HASDP) {
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk) {
                         const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
@@ -572,11 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 ptx::mma_commit(tfull(bb));
-                if (!vec) ptx::mma_commit(empty(s));
+                if (!M::VEC) ptx::mma_commit(empty(s));
                 issued = it + 1;
-                if (vec && it >= 1 && !do_vec(it - 1)) { ok = false; break; }
+                if (M::VEC && it >= 1 && !do_vec(it - 1)) { ok = false; break; }
             }
-            if (ok && vec && n > 0 && do_vec(n - 1)) ptx::mma_commit(accfull);
+            if (M::VEC && ok && n > 0 && do_vec(n - 1)) ptx::mma_commit(accfull);
             if (*abort_flag) {
                 volatile int dummy = 0;
                 if (issued > 0) ptx::mbar_wait(tfull((issued - 1) & 1), ((issued - 1) >> 1) & 1, &dummy, a.status);
@@ -585,21 +655,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue ----------------
-        const int q = warp & 3;
+        // ---------------- epilogue: 8 warps, two per TMEM lane quadrant ----------------
+        const int q = warp & 3;                  // lane quadrant
+        const int half = (warp - 2) >> 2;        // which 32 columns of each 64-column tile
         const int row = q * 32 + lane, r = r0 + row;
         const float lm = logm[r];
         const bool ract = lm != kNegInf;
         const bool is_dustbin_row = (r == D) && ract;
         const float pr2 = ract ? a.pr[base + r] * kLog2e : kNegInf;
-        float xr[kMaxMods];
+        const uint64_t PR2 = ptx::f2(pr2, pr2), SC2 = ptx::f2(a.sc2, a.sc2);
+        float xr[NMOD > 0 ? NMOD : 1];
 #pragma unroll
-        for (int k = 0; k < kMaxMods; ++k) xr[k] = (k < a.nmod && ract) ? a.xr[k][base + r] : 0.f;
+        for (int k = 0; k < NMOD; ++k) xr[k] = ract ? -a.xr[k][base + r] : 0.f;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        float s1 = 0.f, s2 = 0.f;
+        uint64_t s1a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
+        uint64_t s2a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
         bool ok = true;
-        const int voff_m = 1, voff_y = 1 + (a.m ? 1 : 0);
         const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
+        const int cc0 = half * 32;
         for (int it = 0; it < n; ++it) {
             const int s = it % C::NS, bb = it & 1, cb = it & 1;
             const int c0 = tiles[it] * C::BN;
@@ -607,100 +680,110 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
             bool w1 = ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status);
             bool w2 = w1 && ptx::mbar_wait(tfull(bb), (it >> 1) & 1, abort_flag, a.status);
-            bool w3 = w2 && (!vec || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
+            bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
             if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
             ptx::tc_fence_after();
             const float* cv = reinterpret_cast<const float*>(sm + C::OFF_V + s * C::VB);
-            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + crow;
-#pragma unroll 1
-            for (int ch = 0; ch < C::BN / 32; ++ch) {
-                float v[32], w[32];
-                ptx::tmem_ld32(tbase + lane_base + C::TM_S + uint32_t(bb * C::BN + ch * 32), v);
-                if (a.has_dp) {
-                    ptx::tmem_ld32(tbase + lane_base + C::TM_DP + uint32_t(bb * C::BN + ch * 32), w);
-                    ptx::tmem_wait_ld(v, w);
-                } else {
-                    ptx::tmem_wait_ld(v);
+            float v[32], w[32];
+            ptx::tmem_ld32(tbase + lane_base + C::TM_S + uint32_t(bb * C::BN + cc0), v);
+            if (M::HASDP) {
+                ptx::tmem_ld32(tbase + lane_base + C::TM_DP + uint32_t(bb * C::BN + cc0), w);
+                ptx::tmem_wait_ld(v, w);
+            } else {
+                ptx::tmem_wait_ld(v);
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(tempty(bb));
+            // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
+            const float4* pc4 = reinterpret_cast<const float4*>(cv + cc0);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) w[j] = 0.f;
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const float4 b4 = pc4[j4];
+                uint64_t x0 = ptx::ffma2(ptx::f2(v[4 * j4 + 0], v[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
+                uint64_t x1 = ptx::ffma2(ptx::f2(v[4 * j4 + 2], v[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
+                ptx::f2split(x0, v[4 * j4 + 0], v[4 * j4 + 1]);
+                ptx::f2split(x1, v[4 * j4 + 2], v[4 * j4 + 3]);
+            }
+            if (!interior) {
+                const int dlt0 = c0 + cc0 - r;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int dl = dlt0 + j;
+                    if (dl < -h || dl > h) v[j] = kNegInf;
                 }
-                if (ch == C::BN / 32 - 1) {
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(tempty(bb));
-                }
-                const int cc0 = ch * 32;
-                float P[32];
+            }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) P[j] = fmaf(v[j], a.sc2, pr2 + cv[cc0 + j]);
-                if (!interior) {
-                    const int dlt0 = c0 + cc0 - r;
+            for (int j = 0; j < 32; ++j) v[j] = ptx::ex2(v[j]);
+            if (M::SCAL) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int dl = dlt0 + j;
-                        if (dl < -h || dl > h) P[j] = kNegInf;
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) P[j] = ptx::ex2(P[j]);
-                if (scal) {
-                    if (a.s_dp) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) s1 = fmaf(P[j], w[j], s1);
-                    }
-                    if (a.m) {
-                        const float* mv = cv + voff_m * C::BN + cc0;
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) s2 = fmaf(P[j], mv[j], s2);
-                    }
-                }
-                if (vec) {
-                    float cf[32];
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) cf[j] = a.v_dp ? w[j] : 1.f;
-#pragma unroll
-                    for (int k = 0; k < kMaxMods; ++k) {
-                        if (k < a.nmod) {
-                            const float* yv = cv + (voff_y + k) * C::BN + cc0;
-                            const float xk = xr[k];
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) cf[j] = fmaf(-xk, yv[j], cf[j]);
-                        }
-                    }
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint32_t unit = uint32_t(ch * 4 + t);
-                        const uint32_t addr = cbase + ((unit ^ uint32_t(row & 7)) << 4);
-                        ptx::st_shared_v4(addr, ptx::pack_bf16(P[8 * t + 0] * cf[8 * t + 0], P[8 * t + 1] * cf[8 * t + 1]),
-                                          ptx::pack_bf16(P[8 * t + 2] * cf[8 * t + 2], P[8 * t + 3] * cf[8 * t + 3]),
-                                          ptx::pack_bf16(P[8 * t + 4] * cf[8 * t + 4], P[8 * t + 5] * cf[8 * t + 5]),
-                                          ptx::pack_bf16(P[8 * t + 6] * cf[8 * t + 6], P[8 * t + 7] * cf[8 * t + 7]));
+                for (int k = 0; k < 16; ++k) {
+                    const uint64_t P2 = ptx::f2(v[2 * k], v[2 * k + 1]);
+                    if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(w[2 * k], w[2 * k + 1]), s1a[k & 1]);
+                    if (M::SM) {
+                        const float2 mv = reinterpret_cast<const float2*>(cv + VOFF_M * C::BN + cc0)[k];
+                        s2a[k & 1] = ptx::ffma2(P2, ptx::f2(mv.x, mv.y), s2a[k & 1]);
                     }
                 }
             }
-            if (vec) ptx::fence_proxy_async_smem();
+            if (M::VEC) {
+                // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    uint64_t cf = M::VDP ? ptx::f2(w[2 * k], w[2 * k + 1]) : ptx::f2(1.f, 1.f);
+#pragma unroll
+                    for (int mm = 0; mm < NMOD; ++mm) {
+                        const float2 yv = reinterpret_cast<const float2*>(cv + (VOFF_Y + mm) * C::BN + cc0)[k];
+                        cf = ptx::ffma2(ptx::f2(xr[mm], xr[mm]), ptx::f2(yv.x, yv.y), cf);
+                    }
+                    float c0f, c1f;
+                    ptx::f2split(cf, c0f, c1f);
+                    pk[k] = ptx::pack_bf16(v[2 * k] * c0f, v[2 * k + 1] * c1f);
+                }
+                const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + crow;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const uint32_t unit = uint32_t(half * 4 + t);
+                    ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1], pk[4 * t + 2],
+                                      pk[4 * t + 3]);
+                }
+                ptx::fence_proxy_async_smem();
+            }
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(empty(s));
-                if (vec) ptx::mbar_arrive(cfull(cb));
+                if (M::VEC) ptx::mbar_arrive(cfull(cb));
             }
         }
+        // Scalar partials of the two column halves meet in shared memory.
+        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
+        if (M::SCAL) {
+            float a0, a1, b0, b1;
+            ptx::f2split(ptx::fadd2(s1a[0], s1a[1]), a0, a1);
+            ptx::f2split(ptx::fadd2(s2a[0], s2a[1]), b0, b1);
+            red[(0 * 2 + half) * 128 + row] = a0 + a1;
+            red[(1 * 2 + half) * 128 + row] = b0 + b1;
+        }
+        ptx::named_bar_sync(1, 256);
+        ok = __all_sync(0xffffffffu, ok);
         // Dustbin link of this row (the dustbin column), then the writes.
         const bool d_act = D >= 0 && logm[D] != kNegInf;
         float Pd = 0.f, dpd = 0.f, coefd = 0.f;
         if (ract && d_act && !is_dustbin_row) {
             Pd = ptx::ex2((a.sd_term[base + r] + a.pr[base + r] + a.pc[base + D]) * kLog2e);
-            if (a.has_dp) dpd = a.dp_term[base + r];
-            float mod = a.v_dp ? dpd : 1.f;
+            if (M::HASDP) dpd = a.dp_term[base + r];
+            float mod = M::VDP ? dpd : 1.f;
 #pragma unroll
-            for (int k = 0; k < kMaxMods; ++k)
-                if (k < a.nmod) mod -= xr[k] * a.yc[k][base + D];
+            for (int k = 0; k < NMOD; ++k) mod += xr[k] * a.yc[k][base + D];
             coefd = Pd * mod;
         }
-        if (ok && scal && !is_dustbin_row) {
+        if (M::SCAL && ok && half == 0 && !is_dustbin_row) {
+            float s1 = red[0 * 128 + row] + red[1 * 128 + row];
+            float s2 = red[2 * 128 + row] + red[3 * 128 + row];
             if (d_act && ract) {
-                if (a.s_dp) s1 = fmaf(Pd, dpd, s1);
-                if (a.m) s2 = fmaf(Pd, a.m[base + D], s2);
+                if (M::SDP) s1 = fmaf(Pd, dpd, s1);
+                if (M::SM) s2 = fmaf(Pd, a.m[base + D], s2);
             }
             float outv = 0.f;
             if (ract) {
@@ -709,10 +792,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             a.sout[base + r] = outv;
         }
-        // The accumulator read is a warp-collective: every lane of the warp takes part; only
-        // the stores are predicated (the dustbin row is written by the dense dustbin kernel).
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok && vec) {
+        // The accumulator read is a warp-collective: every lane takes part; only the stores
+        // are predicated (the dustbin row is written by the dense dustbin kernel).
+        if (M::VEC && ok) {
             const bool have_acc = n > 0;
             bool wacc = !have_acc || ptx::mbar_wait(accfull, 0, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, wacc);
@@ -721,11 +803,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r) * DH;
                 const __nv_bfloat16* zD = d_act ? a.Zg + (base + D) * DH : nullptr;
                 const bool store = !is_dustbin_row;
-#pragma unroll 1
-                for (int ch = 0; ch < DH / 32; ++ch) {
+#pragma unroll
+                for (int chh = 0; chh < DH / 64; ++chh) {
+                    const int col = half * (DH / 2) + chh * 32;
                     float v[32];
                     if (have_acc) {
-                        ptx::tmem_ld32(tbase + lane_base + C::TM_ACC + uint32_t(ch * 32), v);
+                        ptx::tmem_ld32(tbase + lane_base + C::TM_ACC + uint32_t(col), v);
                         ptx::tmem_wait_ld(v);
                     } else {
 #pragma unroll
@@ -736,13 +819,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int j = 0; j < 16; ++j) {
                         float lo = v[2 * j], hi = v[2 * j + 1];
                         if (ract && d_act && store) {
-                            lo = fmaf(coefd, __bfloat162float(zD[ch * 32 + 2 * j]), lo);
-                            hi = fmaf(coefd, __bfloat162float(zD[ch * 32 + 2 * j + 1]), hi);
+                            lo = fmaf(coefd, __bfloat162float(zD[col + 2 * j]), lo);
+                            hi = fmaf(coefd, __bfloat162float(zD[col + 2 * j + 1]), hi);
                         }
                         pk[j] = ract ? ptx::pack_bf16(a.vscale * lo, a.vscale * hi) : 0u;
                     }
                     if (store) {
-                        uint4* dst = reinterpret_cast<uint4*>(vo + ch * 32);
+                        uint4* dst = reinterpret_cast<uint4*>(vo + col);
 #pragma unroll
                         for (int t = 0; t < 4; ++t)
                             dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
@@ -821,24 +904,63 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     return launch_dustbin_lse(p, st);
 }
 
+template <int DH, int MODE, int NMOD>
+cudaError_t launch_sweep(const CUtensorMap& tmX, const CUtensorMap& tmA, const CUtensorMap& tmY, const CUtensorMap& tmW,
+                         const TcVecArgs& a, int mt, dim3 grid, cudaStream_t st) {
+    constexpr int NV = 1 + (ModeT<MODE>::SM ? 1 : 0) + NMOD;
+    const size_t smem = SweepCfg<DH, NV>::smem_bytes(mt);
+    cudaError_t e = set_smem(tc_sweep_kernel<DH, MODE, NMOD>, smem);
+    if (e != cudaSuccess) return e;
+    tc_sweep_kernel<DH, MODE, NMOD><<<grid, kSweepThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
+    return cudaGetLastError();
+}
+
+template <int DH>
+cudaError_t launch_sweep_dh(int mode, int nmod, const CUtensorMap& tmX, const CUtensorMap& tmA, const CUtensorMap& tmY,
+                            const CUtensorMap& tmW, const TcVecArgs& a, int mt, dim3 grid, cudaStream_t st) {
+    switch (mode) {
+        case kModeOut: return launch_sweep<DH, kModeOut, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+        case kModeC1: return launch_sweep<DH, kModeC1, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+        case kModeR2: return launch_sweep<DH, kModeR2, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+        case kModeStair: return launch_sweep<DH, kModeStair, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+        case kModeGrad:
+            switch (nmod) {
+                case 0: return launch_sweep<DH, kModeGrad, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+                case 2: return launch_sweep<DH, kModeGrad, 2>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+                case 4: return launch_sweep<DH, kModeGrad, 4>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+                case 8: return launch_sweep<DH, kModeGrad, 8>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+                case 16: return launch_sweep<DH, kModeGrad, 16>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+            }
+    }
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     const Geom& g = p.g;
-    const bool has_dp = (p.sout && p.s_dp) || (p.vout && p.v_dp);
-    // Column-side tensors: Y always; the second one is the dP operand or, if different from
-    // Y, the vector operand Z.
-    const void* w2 = has_dp ? p.Bm : (p.vout && p.Z != p.Y ? p.Z : nullptr);
+    // Which pass this is (the orchestration in api.cu only builds these five kinds).
+    int mode;
+    if (p.vout && !p.sout && !p.v_dp && p.nmod == 0 && p.Z != p.Y) mode = kModeOut;
+    else if (p.vout && p.sout && p.s_dp && !p.v_dp && p.nmod == 0 && p.Z == p.Bm) mode = kModeC1;
+    else if (!p.vout && p.sout && p.s_dp && p.m) mode = kModeR2;
+    else if (!p.vout && p.sout && !p.s_dp && p.m) mode = kModeStair;
+    else if (p.vout && !p.sout && p.v_dp && p.Z == p.Y) mode = kModeGrad;
+    else return cudaErrorInvalidValue;
+    // Modifier count rounded up to an instantiated one; the padding terms have xr = 0.
+    int nmod = p.nmod;
+    const int nmod_k = nmod == 0 ? 0 : nmod <= 2 ? 2 : nmod <= 4 ? 4 : nmod <= 8 ? 8 : 16;
+    if (nmod_k > nmod && !p.zero_vec) return cudaErrorInvalidValue;
+    const bool has_dp = mode == kModeC1 || mode == kModeR2 || mode == kModeGrad;
+    const void* w2 = has_dp ? p.Bm : (mode == kModeOut ? p.Z : nullptr);
     const uint64_t rows = uint64_t(g.BH) * g.L;
     CUtensorMap tmX, tmA, tmY, tmW;
     if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
     if (!make_map(&tmA, has_dp ? p.A : p.X, rows, g.d, 128)) return cudaErrorInvalidValue;
     if (!make_map(&tmW, w2 ? w2 : p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
-    if (p.vout && p.Z != p.Y && p.Z != w2) return cudaErrorInvalidValue;   // not a pass this library runs
     TcVecArgs a{};
     a.H = g.H;
     a.L = g.L;
     a.h = g.h;
     a.D = g.D;
-    a.d = g.d;
     a.sc2 = g.scale * kLog2e;
     a.logm = p.logm;
     a.pr = p.pr;
@@ -847,37 +969,21 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.sout = p.sout;
     a.f = p.f;
     a.hv = p.hv;
-    a.m = p.sout ? p.m : nullptr;
-    a.s_dp = p.s_dp;
+    a.m = p.m;
     a.vout = p.vout;
     a.vscale = p.vscale;
-    a.v_dp = p.v_dp;
-    a.nmod = p.vout ? p.nmod : 0;
-    for (int k = 0; k < a.nmod; ++k) {
-        a.xr[k] = p.xr[k];
-        a.yc[k] = p.yc[k];
+    for (int k = 0; k < nmod_k; ++k) {
+        a.xr[k] = k < nmod ? p.xr[k] : p.zero_vec;
+        a.yc[k] = k < nmod ? p.yc[k] : p.zero_vec;
     }
     a.Zg = static_cast<const __nv_bfloat16*>(p.Z);
-    a.z_from_w2 = (p.vout && w2 && p.Z == w2) ? 1 : 0;
-    a.has_w2 = w2 ? 1 : 0;
-    a.has_dp = has_dp ? 1 : 0;
     a.sd_term = p.sd_term;
     a.dp_term = p.dp_term;
     a.status = p.status;
     const int mt = max_tiles_for(g.L, g.h, 128, 64);
     dim3 grid(g.L / 128, g.BH);
-    cudaError_t e;
-    if (g.d == 128) {
-        const size_t smem = VecCfg<128>::smem_bytes(mt);
-        if ((e = set_smem(tc_vec_kernel<128>, smem)) != cudaSuccess) return e;
-        tc_vec_kernel<128><<<grid, kThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
-    } else {
-        // at least 120 KB so that one CTA owns the SM (the kernel allocates all 512 TMEM columns)
-        const size_t smem = std::max<size_t>(VecCfg<64>::smem_bytes(mt), 120 * 1024);
-        if ((e = set_smem(tc_vec_kernel<64>, smem)) != cudaSuccess) return e;
-        tc_vec_kernel<64><<<grid, kThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
-    }
-    e = cudaGetLastError();
+    cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st)
+                               : launch_sweep_dh<64>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st);
     if (e != cudaSuccess || g.D < 0) return e;
     return launch_dustbin_bwd(p, st);
 }
