@@ -71,6 +71,9 @@ lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
 lib.eot_device_status_bits.restype = ctypes.c_int
 
+lib.eot_sinkhorn_fwd_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+lib.eot_sinkhorn_fwd_static.restype = ctypes.c_int
+EOT_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 lib.eot_kernel_launches.restype = ctypes.c_longlong
 lib.eot_profile_begin.restype = None
 lib.eot_profile_end.argtypes = [_vp]
@@ -82,7 +85,7 @@ lib.eot_profile_read.restype = ctypes.c_int
 EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sinkhorn_bwd",
             "eot_last_device_status", "eot_device_status_bits", "eot_status_string",
             "eot_abi_version", "eot_resolved_impl", "eot_kernel_launches", "eot_profile_begin",
-            "eot_profile_end", "eot_profile_read")
+            "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static")
 
 PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3}
 
@@ -144,6 +147,12 @@ def eot_sinkhorn_bwd(p: eot_problem, Q: int, K: int, V: int, mask: int | None, u
     """Backward; raw device addresses as in eot_sinkhorn_fwd."""
     _check(lib.eot_sinkhorn_bwd(ctypes.byref(p), Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
                                 workspace_bytes, stream), "eot_sinkhorn_bwd")
+
+
+def eot_sinkhorn_fwd_static(p: eot_problem, Q: int, K: int, V: int, mask: int | None, O: int, u_tail: int,
+                            v_tail: int, stream: int) -> int:
+    """Forward with the library's static scratch (no workspace); returns the raw status."""
+    return lib.eot_sinkhorn_fwd_static(ctypes.byref(p), Q, K, V, mask, O, u_tail, v_tail, stream)
 
 
 def eot_last_device_status(workspace: int, stream: int) -> int:

@@ -139,6 +139,8 @@ cudaError_t aux(cudaStream_t st, F&& f) { return tracked(kProfAux, 1, st, f); }
 // (Also used by entry points that supply their own scratch.)
 namespace eot {
 
+eot_status validate_problem(const eot_problem* p) { return validate(p); }
+
 eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
                         void* O, float* u_tail, float* v_tail, void* ws, cudaStream_t st) {
     const Geom g = make_geom(*p);

@@ -145,6 +145,28 @@ void eot_profile_begin(void);
 eot_status eot_profile_end(void* stream);
 eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
 
+/* Forward pass that allocates nothing and takes no workspace.  The paper has no counterpart:
+ * this is a deployment variant of eot_sinkhorn_fwd for callers that cannot allocate device
+ * memory where they run it (a plug-in inside a host that owns all device memory and gives it
+ * no allocator; a serving loop that forbids cudaMalloc/cudaFree after start-up because those
+ * calls can synchronise the device).  Arguments and results are those of eot_sinkhorn_fwd;
+ * the scratch is a fixed array of EOT_STATIC_SCRATCH_BYTES in this library's device memory,
+ * held on every GPU that loads the library until the process exits.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ *   - Problems whose forward scratch, eot_workspace_bytes(p, 0), exceeds
+ *     EOT_STATIC_SCRATCH_BYTES are rejected with EOT_ERR_WORKSPACE_TOO_SMALL before anything
+ *     is launched.
+ *   - Every call on a device shares the one array and leaves its contents behind (the first
+ *     kernel of each call clears what must start at zero).  Calls that overlap on the GPU
+ *     (other streams, other host threads) race on it and corrupt each other: serialise them.
+ *   - The device status word of these calls lives in the shared array and is not readable
+ *     through eot_last_device_status. */
+#define EOT_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+eot_status eot_sinkhorn_fwd_static(const eot_problem* p, const void* Q, const void* K, const void* V,
+                                   const uint8_t* mask, void* O, float* u_tail, float* v_tail,
+                                   void* stream);
+
 /* Kernel family that ``p`` would run with (EOT_IMPL_SIMT or EOT_IMPL_TCGEN05), or -1 if
  * the problem is invalid or unsupported. */
 int eot_resolved_impl(const eot_problem* p);
