@@ -123,7 +123,8 @@ struct LseCfg {
     static constexpr uint32_t ATOM = 128 * 128;    // one 64-element-wide atom column of 128 rows
     static constexpr uint32_t OFF_Y = XB;
     static constexpr uint32_t OFF_BIAS = OFF_Y + NS * YB;
-    static constexpr uint32_t OFF_BAR = OFF_BIAS + NB * BN * 4;
+    static constexpr uint32_t OFF_RED = OFF_BIAS + NB * BN * 4;   // [2 halves][m, s][128 rows]
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
     // barriers: full[NS] empty[NS] xfull tfull[2] tempty[2] bfull[NB] bempty[NB]
     static constexpr uint32_t NBARS = 2 * NS + 1 + 4 + 2 * NB;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -132,8 +133,10 @@ struct LseCfg {
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
+constexpr int kLseThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
+
 template <int DH, bool ONLINE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kLseThreads, 2)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                   const TcLseArgs a, int max_tiles) {
     using C = LseCfg<DH>;
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
                                                  reinterpret_cast<int*>(misc + 2), &any_row);
     if (!any_row) {
-        for (int r = tid; r < C::BM; r += kThreads) {
+        for (int r = tid; r < C::BM; r += kLseThreads) {
             a.out[pb + r0 + r] = 0.f;
             a.out_bias2[base + r0 + r] = kNegInf;
         }
@@ -180,11 +183,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         ptx::mbar_init(xfull, 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(tfull(i), 1);
-            ptx::mbar_init(tempty(i), 4);
+            ptx::mbar_init(tempty(i), 8);
         }
         for (int i = 0; i < C::NB; ++i) {
             ptx::mbar_init(bfull(i), 1);
-            ptx::mbar_init(bempty(i), 4);
+            ptx::mbar_init(bempty(i), 8);
         }
         ptx::mbar_fence_init();
     }
@@ -262,8 +265,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     } else {
-        // ---------------- epilogue ----------------
-        const int q = warp & 3;
+        // ---------------- epilogue: 8 warps, two per TMEM lane quadrant ----------------
+        const int q = warp & 3;                  // lane quadrant
+        const int half = (warp - 2) >> 2;        // columns [64 half, 64 half + 64) of each tile
         const int row = q * 32 + lane, r = r0 + row;
         const float lm = logm[r];
         const bool is_dustbin_row = (r == D) && lm != kNegInf;
@@ -357,28 +361,32 @@ __global__ void __launch_bounds__(kThreads, 2)
                     acc[3] += s3;
                 }
             };
-            // TMEM loads run one chunk ahead of the arithmetic.
+            // TMEM load of the second chunk runs while the first is processed.
             float va[32], vb[32];
-            ptx::tmem_ld32(tcol + 0, va);
+            const int ch0 = 2 * half;
+            ptx::tmem_ld32(tcol + uint32_t(32 * ch0), va);
             ptx::tmem_wait_ld(va);
-            ptx::tmem_ld32(tcol + 32, vb);
-            process(va, 0);
+            ptx::tmem_ld32(tcol + uint32_t(32 * ch0 + 32), vb);
+            process(va, ch0);
             ptx::tmem_wait_ld(vb);
-            ptx::tmem_ld32(tcol + 64, va);
-            process(vb, 1);
-            ptx::tmem_wait_ld(va);
-            ptx::tmem_ld32(tcol + 96, vb);
-            process(va, 2);
-            ptx::tmem_wait_ld(vb);
-            // accumulator buffer fully read: hand it back to the MMA warp
+            // this warp's half of the accumulator buffer is read: hand it back to the MMA warp
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty(bb));
-            process(vb, 3);
+            process(vb, ch0 + 1);
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bempty(bs));
         }
         float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        // The two column halves of each row meet in shared memory.
+        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
+        red[(half * 2 + 0) * 128 + row] = m_run;
+        red[(half * 2 + 1) * 128 + row] = sum;
+        ptx::named_bar_sync(1, 256);
+        ok = __all_sync(0xffffffffu, ok);
+        if (half != 0) ok = false;   // the first half writes the row
+        else if (ONLINE) lse2_merge(m_run, sum, red[2 * 128 + row], red[3 * 128 + row]);
+        else sum += red[3 * 128 + row];
         if (ok && !*abort_flag && !is_dustbin_row) {
             float outv = 0.f, ob = kNegInf;
             if (lm != kNegInf) {
@@ -884,19 +892,19 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
         const size_t smem = LseCfg<128>::smem_bytes(mt);
         if (p.stab) {
             if ((e = set_smem(tc_lse_kernel<128, false>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<128, false><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+            tc_lse_kernel<128, false><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
         } else {
             if ((e = set_smem(tc_lse_kernel<128, true>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<128, true><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+            tc_lse_kernel<128, true><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
         }
     } else {
         const size_t smem = LseCfg<64>::smem_bytes(mt);
         if (p.stab) {
             if ((e = set_smem(tc_lse_kernel<64, false>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<64, false><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+            tc_lse_kernel<64, false><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
         } else {
             if ((e = set_smem(tc_lse_kernel<64, true>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<64, true><<<grid, kThreads, smem, st>>>(tmX, tmY, a, mt);
+            tc_lse_kernel<64, true><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
         }
     }
     e = cudaGetLastError();
