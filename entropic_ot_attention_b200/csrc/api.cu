@@ -171,6 +171,9 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     float* ub2 = at<float>(ws, w.ub2);
     float* vb2 = at<float>(ws, w.vb2);
     EOT_TRY(aux(st, [&] { return launch_init_bias2(g, logm, vb2, st); }));
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
+    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
+    row.tile_bits = tbits;
     row.colbias2 = vb2;
     row.out_bias2 = ub2;
     LsePass col = row;

@@ -47,6 +47,7 @@ struct LsePass {
     size_t pstride;         // unit stride of colpot / stab / out (elements): L or (R+1) L
     const float* colbias2;  // [BH, L] log2(e) * colpot, -inf for inactive columns and the dustbin
     float* out_bias2;       // [BH, L] same masking of the new potential (for the next half-step)
+    const uint32_t* tile_bits;  // [B][tile_words(L)]: 128-position tiles holding an active non-dustbin token
     const float* sd_term;   // [BH, L] S between row r and the dustbin column (dustbin only)
     const float* sd_dense;  // [BH, L] S between the dustbin row and column c (dustbin only)
     uint32_t* status;
@@ -92,6 +93,7 @@ struct WsLayout {
     size_t status, logm, sd_row, sd_col, e1, e2;
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
+    size_t tbits;           // forward: active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
     size_t zero;            // backward: a vector of zeros
     size_t pr, pc, f, hv, m;
@@ -101,6 +103,7 @@ struct WsLayout {
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+__host__ __device__ inline int tile_words(int L) { return (L / 128 + 31) / 32; }
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     WsLayout w{};
@@ -120,6 +123,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.opcm = o; o += vec;
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
+        w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     }
     if (bwd) {
         w.pr = o; o += vec;

@@ -581,6 +581,33 @@ __global__ void __launch_bounds__(256) init_bias2_kernel(Geom g, const float* lo
     bias2[size_t(bh) * g.L + i] = act ? 0.f : neg_inf();
 }
 
+// Bit t of word w of batch row b: positions [128 t, 128 t + 128) hold an active token other
+// than the dustbin (tiles without one contribute nothing to a band sum and are skipped).
+// One 1024-thread block per word; warp k examines tile 32 w + k.
+__global__ void __launch_bounds__(1024) tile_bits_kernel(Geom g, const float* logm, uint32_t* bits) {
+    const int words = tile_words(g.L);
+    const int b = blockIdx.x / words, w = blockIdx.x - b * words;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ uint32_t acc;
+    if (threadIdx.x == 0) acc = 0u;
+    __syncthreads();
+    const int t = w * 32 + warp;
+    bool any = false;
+    if (t * 128 < g.L) {
+        const float* lm = logm + size_t(b) * g.L + size_t(t) * 128;
+        for (int i = lane; i < 128; i += 32) any |= lm[i] != neg_inf() && (t * 128 + i) != g.D;
+    }
+    const unsigned vote = __ballot_sync(0xffffffffu, any);
+    if (lane == 0 && vote) atomicOr(&acc, 1u << warp);
+    __syncthreads();
+    if (threadIdx.x == 0) bits[blockIdx.x] = acc;
+}
+
+cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st) {
+    tile_bits_kernel<<<g.B * tile_words(g.L), 1024, 0, st>>>(g, logm, bits);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st) {
     dim3 grid((g.L + 255) / 256, g.BH);
     init_bias2_kernel<<<grid, 256, 0, st>>>(g, logm, bias2);

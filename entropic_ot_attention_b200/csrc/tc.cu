@@ -29,8 +29,8 @@ namespace {
 constexpr int kThreads = 192;
 constexpr float kNegInf = -__builtin_huge_valf();
 // Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
-// interior forward tiles (6 of 16 pairs: 37.5 %, where the two pipes balance).
-constexpr int kFmaPairs = 6;
+// interior forward tiles (3 of 16 pairs; measured best on the long workload).
+constexpr int kFmaPairs = 3;
 
 // ---------------------------------------------------------------------------------------
 // Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
@@ -96,12 +96,21 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Forward half-step (band log-sum-exp), 128 x 128 tiles
+// Forward half-step (band log-sum-exp): persistent kernel, 128 x 128 tiles
 // ---------------------------------------------------------------------------------------
+// One CTA per SM walks a contiguous range of (unit, row-tile) work items.  Barriers and TMEM
+// are set up once; the TMA warp runs ahead across item boundaries (two row-tile buffers,
+// NS column-tile stages, a bias ring), the MMA warp keeps up to four score tiles in flight
+// in TMEM (4 x 128 columns), and 16 epilogue warps (four per TMEM lane quadrant, one per
+// 32-column chunk of a tile) turn each tile into row partial sums.  All three roles walk
+// the same item / tile sequence, so ring indices and mbarrier phases follow from one
+// running tile counter.
 struct TcLseArgs {
-    int H, L, h, D;
+    int H, L, h, D, n_items, items_per_cta;
     float sl2;              // scale * log2(e)
     const float* logm;
+    const uint32_t* tile_bits;  // [B][words]: bit t = positions [128 t, 128 t + 128) hold an active non-dustbin token
+    int words;
     const float* colbias2;  // [BH, L] masked log2 column bias
     const float* colpot;    // natural column potential (pstride), read at D
     const float* stab;      // natural previous row potential (pstride) or nullptr
@@ -116,83 +125,90 @@ template <int DH>
 struct LseCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
-    static constexpr int NS = DH == 128 ? 2 : 4;   // column-tile stages
-    static constexpr int NB = 4;                   // bias ring slots
+    static constexpr int NS = DH == 128 ? 4 : 8;   // column-tile stages
+    static constexpr int NQ = 2;                   // row-tile buffers
+    static constexpr int NT = 4;                   // TMEM accumulator buffers (4 x 128 columns)
+    static constexpr int NB = 8;                   // bias ring slots
     static constexpr uint32_t XB = BM * DH * 2;    // row tile bytes
     static constexpr uint32_t YB = BN * DH * 2;    // column tile bytes
     static constexpr uint32_t ATOM = 128 * 128;    // one 64-element-wide atom column of 128 rows
-    static constexpr uint32_t OFF_Y = XB;
+    static constexpr uint32_t OFF_Y = NQ * XB;
     static constexpr uint32_t OFF_BIAS = OFF_Y + NS * YB;
-    static constexpr uint32_t OFF_RED = OFF_BIAS + NB * BN * 4;   // [2 halves][m, s][128 rows]
-    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
-    // barriers: full[NS] empty[NS] xfull tfull[2] tempty[2] bfull[NB] bempty[NB]
-    static constexpr uint32_t NBARS = 2 * NS + 1 + 4 + 2 * NB;
+    static constexpr uint32_t OFF_RED = OFF_BIAS + NB * BN * 4;   // [2 parity][4 chunks][m, s][128 rows]
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 2 * 128 * 4;
+    // full[NS] empty[NS] qfull[NQ] qempty[NQ] tfull[NT] tempty[NT] bfull[NB] bempty[NB]
+    static constexpr uint32_t NBARS = 2 * NS + 2 * NQ + 2 * NT + 2 * NB;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
-    static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
-    static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
+    static constexpr size_t SMEM = 1024 + OFF_MISC + 64;
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
-constexpr int kLseThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kLseThreads = 576;   // TMA warp, MMA warp, 16 epilogue warps
+
+// Decoded work item: the 128-row tile I of unit bh and its band of column tiles.
+struct LseItem {
+    int bh, b, r0, t_lo, t_hi;
+    bool rows_active;
+    size_t base;
+};
+
+__device__ __forceinline__ bool tile_bit(const uint32_t* bits, int t) { return (bits[t >> 5] >> (t & 31)) & 1u; }
 
 template <int DH, bool ONLINE>
-__global__ void __launch_bounds__(kLseThreads, 2)
+__global__ void __launch_bounds__(kLseThreads, 1)
     tc_lse_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-                  const TcLseArgs a, int max_tiles) {
+                  const TcLseArgs a) {
     using C = LseCfg<DH>;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.y, b = bh / a.H, L = a.L, h = a.h, D = a.D;
-    const int r0 = blockIdx.x * C::BM;
-    const size_t base = size_t(bh) * L;
-    const size_t pb = size_t(bh) * a.pstride;
-    const float* logm = a.logm + size_t(b) * L;
+    const int L = a.L, h = a.h, D = a.D;
+    const int tiles_per_unit = L / C::BM;
+    const int item0 = blockIdx.x * a.items_per_cta;
+    const int item1 = min(a.n_items, item0 + a.items_per_cta);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     const uint32_t bar0 = ptx::smem_u32(bars);
-    auto full = [&](int s) { return bar0 + 8u * s; };
-    auto empty = [&](int s) { return bar0 + 8u * (C::NS + s); };
-    const uint32_t xfull = bar0 + 8u * (2 * C::NS);
-    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 1 + i); };
-    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
-    auto bfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
-    auto bempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + C::NB + i); };
+    auto full = [&](int i) { return bar0 + 8u * i; };
+    auto empty = [&](int i) { return bar0 + 8u * (C::NS + i); };
+    auto qfull = [&](int i) { return bar0 + 8u * (2 * C::NS + i); };
+    auto qempty = [&](int i) { return bar0 + 8u * (2 * C::NS + C::NQ + i); };
+    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + i); };
+    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + C::NT + i); };
+    auto bfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + 2 * C::NT + i); };
+    auto bempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + 2 * C::NT + C::NB + i); };
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-    int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
-    int* flags = tiles + max_tiles;
     const float* bias_s = reinterpret_cast<const float*>(sm + C::OFF_BIAS);
 
-    if (tid == 0) *abort_flag = 0;
-    bool any_row;
-    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
-                                                 reinterpret_cast<int*>(misc + 2), &any_row);
-    if (!any_row) {
-        for (int r = tid; r < C::BM; r += kLseThreads) {
-            a.out[pb + r0 + r] = 0.f;
-            a.out_bias2[base + r0 + r] = kNegInf;
-        }
-        return;
-    }
+    auto decode = [&](int item) {
+        LseItem it;
+        it.bh = item / tiles_per_unit;
+        it.b = it.bh / a.H;
+        it.r0 = (item - it.bh * tiles_per_unit) * C::BM;
+        it.base = size_t(it.bh) * L;
+        it.t_lo = max(0, it.r0 - h) / C::BN;
+        it.t_hi = min(L - 1, it.r0 + C::BM - 1 + h) / C::BN;
+        it.rows_active = tile_bit(a.tile_bits + size_t(it.b) * a.words, it.r0 / C::BM);
+        return it;
+    };
+    auto count_tiles = [&](const LseItem& it) {
+        const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+        int n = 0;
+        for (int t = it.t_lo; t <= it.t_hi; ++t) n += tile_bit(bits, t);
+        return n;
+    };
+
     if (tid == 0) {
-        for (int s = 0; s < C::NS; ++s) {
-            ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 1);
-        }
-        ptx::mbar_init(xfull, 1);
-        for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(tfull(i), 1);
-            ptx::mbar_init(tempty(i), 8);
-        }
-        for (int i = 0; i < C::NB; ++i) {
-            ptx::mbar_init(bfull(i), 1);
-            ptx::mbar_init(bempty(i), 8);
-        }
+        *abort_flag = 0;
+        for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 1); }
+        for (int i = 0; i < C::NQ; ++i) { ptx::mbar_init(qfull(i), 1); ptx::mbar_init(qempty(i), 1); }
+        for (int i = 0; i < C::NT; ++i) { ptx::mbar_init(tfull(i), 1); ptx::mbar_init(tempty(i), 16); }
+        for (int i = 0; i < C::NB; ++i) { ptx::mbar_init(bfull(i), 1); ptx::mbar_init(bempty(i), 16); }
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(ptx::smem_u32(misc), 256);
+        ptx::tmem_alloc(ptx::smem_u32(misc), 512);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -205,49 +221,63 @@ __global__ void __launch_bounds__(kLseThreads, 2)
             // ---------------- TMA producer ----------------
             ptx::prefetch_tmap(&tmX);
             ptx::prefetch_tmap(&tmY);
-            const uint32_t xs = ptx::smem_u32(sm);
-            ptx::mbar_expect_tx(xfull, C::XB);
-            for (int ka = 0; ka < C::KATOMS; ++ka)
-                ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(base) + r0, xfull);
-            int issued = 0, bissued = 0;
-            for (int it = 0; it < n; ++it) {
-                const int s = it % C::NS, bs = it % C::NB;
-                const int c0 = tiles[it] * C::BN;
-                if (!ptx::mbar_wait(empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(full(s), C::YB);
-                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+            int g = 0, qi = 0;
+            bool ok = true;
+            for (int item = item0; item < item1 && ok; ++item) {
+                const LseItem it = decode(item);
+                if (!it.rows_active || count_tiles(it) == 0) continue;
+                const int qb = qi % C::NQ;
+                if (!ptx::mbar_wait(qempty(qb), ((qi / C::NQ) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                ptx::mbar_expect_tx(qfull(qb), C::XB);
+                const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
                 for (int ka = 0; ka < C::KATOMS; ++ka)
-                    ptx::tma_load_2d(ys + ka * C::ATOM, &tmY, ka * 64, int(base) + c0, full(s));
-                issued = it + 1;
-                if (!ptx::mbar_wait(bempty(bs), ((it / C::NB) & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(bfull(bs), C::BN * 4);
-                ptx::bulk_load(ptx::smem_u32(sm + C::OFF_BIAS + bs * C::BN * 4), a.colbias2 + base + c0, C::BN * 4,
-                               bfull(bs));
-                bissued = it + 1;
+                    ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(it.base) + it.r0, qfull(qb));
+                ++qi;
+                const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+                for (int t = it.t_lo; t <= it.t_hi; ++t) {
+                    if (!tile_bit(bits, t)) continue;
+                    const int c0 = t * C::BN;
+                    const int s = g % C::NS, bs = g % C::NB;
+                    if (!ptx::mbar_wait(empty(s), ((g / C::NS) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ptx::mbar_expect_tx(full(s), C::YB);
+                    const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+                    for (int ka = 0; ka < C::KATOMS; ++ka)
+                        ptx::tma_load_2d(ys + ka * C::ATOM, &tmY, ka * 64, int(it.base) + c0, full(s));
+                    if (!ptx::mbar_wait(bempty(bs), ((g / C::NB) & 1) ^ 1, abort_flag, a.status)) { ++g; ok = false; break; }
+                    ptx::mbar_expect_tx(bfull(bs), C::BN * 4);
+                    ptx::bulk_load(ptx::smem_u32(sm + C::OFF_BIAS + bs * C::BN * 4), a.colbias2 + it.base + c0, C::BN * 4,
+                                   bfull(bs));
+                    ++g;
+                }
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA retires.
                 volatile int dummy = 0;
-                for (int it = max(0, issued - C::NS); it < issued; ++it)
-                    ptx::mbar_wait(full(it % C::NS), (it / C::NS) & 1, &dummy, a.status);
-                for (int it = max(0, bissued - C::NB); it < bissued; ++it)
-                    ptx::mbar_wait(bfull(it % C::NB), (it / C::NB) & 1, &dummy, a.status);
-                ptx::mbar_wait(xfull, 0, &dummy, a.status);
+                for (int i = max(0, g - C::NS); i < g; ++i) ptx::mbar_wait(full(i % C::NS), (i / C::NS) & 1, &dummy, a.status);
+                for (int i = max(0, g - C::NB); i < g; ++i) ptx::mbar_wait(bfull(i % C::NB), (i / C::NB) & 1, &dummy, a.status);
+                for (int i = max(0, qi - C::NQ); i < qi; ++i) ptx::mbar_wait(qfull(i % C::NQ), (i / C::NQ) & 1, &dummy, a.status);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            const uint32_t xs = ptx::smem_u32(sm);
-            int last = -1;
-            if (ptx::mbar_wait(xfull, 0, abort_flag, a.status)) {
-                for (int it = 0; it < n; ++it) {
-                    const int s = it % C::NS, bb = it & 1;
-                    if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) break;
-                    if (!ptx::mbar_wait(tempty(bb), ((it >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+            int g = 0, qi = 0;
+            bool ok = true;
+            for (int item = item0; item < item1 && ok; ++item) {
+                const LseItem it = decode(item);
+                const int n = it.rows_active ? count_tiles(it) : 0;
+                if (n == 0) continue;
+                const int qb = qi % C::NQ;
+                if (!ptx::mbar_wait(qfull(qb), (qi / C::NQ) & 1, abort_flag, a.status)) { ok = false; break; }
+                ++qi;
+                const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
+                for (int k = 0; k < n; ++k) {
+                    const int s = g % C::NS, tb = g % C::NT;
+                    if (!ptx::mbar_wait(full(s), (g / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
+                    if (!ptx::mbar_wait(tempty(tb), ((g / C::NT) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
-                    const uint32_t dt = tbase + uint32_t(bb * C::BN);
+                    const uint32_t dt = tbase + uint32_t(tb * C::BN);
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk) {
                         const uint32_t koff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
@@ -255,53 +285,75 @@ __global__ void __launch_bounds__(kLseThreads, 2)
                                       C::IDESC, kk > 0 ? 1u : 0u);
                     }
                     ptx::mma_commit(empty(s));
-                    ptx::mma_commit(tfull(bb));
-                    last = it;
+                    ptx::mma_commit(tfull(tb));
+                    ++g;
                 }
+                ptx::mma_commit(qempty(qb));   // row tile free once this item's products are done
             }
-            if (*abort_flag && last >= 0) {
+            if (*abort_flag && g > 0) {
                 volatile int dummy = 0;
-                ptx::mbar_wait(tfull(last & 1), (last >> 1) & 1, &dummy, a.status);
+                ptx::mbar_wait(tfull((g - 1) % C::NT), ((g - 1) / C::NT) & 1, &dummy, a.status);
             }
         }
     } else {
-        // ---------------- epilogue: 8 warps, two per TMEM lane quadrant ----------------
-        const int q = warp & 3;                  // lane quadrant
-        const int half = (warp - 2) >> 2;        // columns [64 half, 64 half + 64) of each tile
-        const int row = q * 32 + lane, r = r0 + row;
-        const float lm = logm[r];
-        const bool is_dustbin_row = (r == D) && lm != kNegInf;
-        const float st = ONLINE ? 0.f : a.stab[pb + r];
-        const float st2 = st * kLog2e;
-        float m_run = kNegInf;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums (no serial FADD chain)
+        // ---------------- epilogue: 16 warps; (lane quadrant, 32-column chunk) each ----------------
+        const int q = warp & 3;                  // TMEM lane quadrant this warp may access
+        const int chunk = (warp - 2) >> 2;       // columns [32 chunk, 32 chunk + 32) of each tile
+        const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
+        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
+        int g = 0, ep = 0;
         bool ok = true;
-        for (int it = 0; it < n && ok; ++it) {
-            const int bb = it & 1, bs = it % C::NB;
-            const int c0 = tiles[it] * C::BN;
-            const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
-            // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-            bool w1 = ptx::mbar_wait(bfull(bs), (it / C::NB) & 1, abort_flag, a.status);
-            bool w2 = w1 && ptx::mbar_wait(tfull(bb), (it >> 1) & 1, abort_flag, a.status);
-            if (!__all_sync(0xffffffffu, w2)) { ok = false; break; }
-            ptx::tc_fence_after();
-            const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN);
-            const uint32_t tcol = tbase + lane_base + uint32_t(bb * C::BN);
-            auto process = [&](const float (&v)[32], int ch) {
+        for (int item = item0; item < item1; ++item) {
+            const LseItem it = decode(item);
+            const int r = it.r0 + row;
+            const size_t pb = size_t(it.bh) * a.pstride;
+            const float* logm = a.logm + size_t(it.b) * L;
+            if (!it.rows_active) {
+                if (chunk == 0) {
+                    a.out[pb + r] = 0.f;
+                    a.out_bias2[it.base + r] = kNegInf;
+                }
+                continue;
+            }
+            const float lm = logm[r];
+            const float st = ONLINE ? 0.f : a.stab[pb + r];
+            const float st2 = st * kLog2e;
+            float m_run = kNegInf;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+            for (int t = it.t_lo; t <= it.t_hi; ++t) {
+                if (!tile_bit(bits, t)) continue;
+                const int c0 = t * C::BN;
+                const int tb = g % C::NT, bs = g % C::NB;
+                const int gg = g++;
+                if (!ok) continue;
+                const bool interior = (c0 + C::BN - 1 - it.r0 <= h) && (it.r0 + C::BM - 1 - c0 <= h);
+                // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
+                bool w1 = ptx::mbar_wait(bfull(bs), (gg / C::NB) & 1, abort_flag, a.status);
+                bool w2 = w1 && ptx::mbar_wait(tfull(tb), (gg / C::NT) & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
+                ptx::tc_fence_after();
+                float v[32];
+                ptx::tmem_ld32(tbase + lane_base + uint32_t(tb * C::BN + chunk * 32), v);
+                ptx::tmem_wait_ld(v);
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(tempty(tb));
+                const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN + chunk * 32);
                 if (ONLINE || !interior) {
                     // scalar path: running maximum (first half-step) or band-edge masking
                     float x[32];
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = bias4[ch * 8 + j4];
+                        const float4 bv = bias4[j4];
                         x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
                         x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
                         x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
                         x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
                     }
                     if (!interior) {
-                        const int dlt0 = c0 + ch * 32 - r;
+                        const int dlt0 = c0 + chunk * 32 - r;
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const int dl = dlt0 + j;
@@ -328,13 +380,12 @@ __global__ void __launch_bounds__(kLseThreads, 2)
                     }
                 } else {
                     // interior tile, shifted by the previous potential: packed fp32x2 math;
-                    // the first kFmaPairs pairs of exponentials go to the FMA pipe, the rest
-                    // to the MUFU pipe, so that the two pipes share the exp2 work.
+                    // the first kFmaPairs pairs of exponentials go to the FMA pipe
                     const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
                     uint64_t acc2[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = bias4[ch * 8 + j4];
+                        const float4 bv = bias4[j4];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int k = 2 * j4 + hh;
@@ -360,56 +411,47 @@ __global__ void __launch_bounds__(kLseThreads, 2)
                     acc[2] += s2;
                     acc[3] += s3;
                 }
-            };
-            // TMEM load of the second chunk runs while the first is processed.
-            float va[32], vb[32];
-            const int ch0 = 2 * half;
-            ptx::tmem_ld32(tcol + uint32_t(32 * ch0), va);
-            ptx::tmem_wait_ld(va);
-            ptx::tmem_ld32(tcol + uint32_t(32 * ch0 + 32), vb);
-            process(va, ch0);
-            ptx::tmem_wait_ld(vb);
-            // this warp's half of the accumulator buffer is read: hand it back to the MMA warp
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(tempty(bb));
-            process(vb, ch0 + 1);
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bempty(bs));
-        }
-        float sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        // The two column halves of each row meet in shared memory.
-        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
-        red[(half * 2 + 0) * 128 + row] = m_run;
-        red[(half * 2 + 1) * 128 + row] = sum;
-        ptx::named_bar_sync(1, 256);
-        ok = __all_sync(0xffffffffu, ok);
-        if (half != 0) ok = false;   // the first half writes the row
-        else if (ONLINE) lse2_merge(m_run, sum, red[2 * 128 + row], red[3 * 128 + row]);
-        else sum += red[3 * 128 + row];
-        if (ok && !*abort_flag && !is_dustbin_row) {
-            float outv = 0.f, ob = kNegInf;
-            if (lm != kNegInf) {
-                const bool d_act = D >= 0 && logm[D] != kNegInf;
-                if (ONLINE) {
-                    if (d_act) lse2_add(m_run, sum, (a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e);
-                    outv = lm - (m_run + log2f(sum)) * kLn2;
-                } else {
-                    if (d_act) sum += ptx::ex2((a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e + st2);
-                    outv = lm - log2f(sum) * kLn2 + st;
-                }
-                if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
-                ob = outv * kLog2e;
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bempty(bs));
             }
-            a.out[pb + r] = outv;
-            a.out_bias2[base + r] = ob;
+            // The four chunk partials of each row meet in shared memory (two parity slots so
+            // that the next item can proceed while the first chunk's warps read this one).
+            float* rd = red + (ep & 1) * (4 * 2 * 128);
+            rd[(chunk * 2 + 0) * 128 + row] = m_run;
+            rd[(chunk * 2 + 1) * 128 + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            ++ep;
+            ptx::named_bar_sync(1, 512);
+            const bool is_dustbin_row = (r == D) && lm != kNegInf;
+            if (chunk == 0 && ok && !*abort_flag && !is_dustbin_row) {
+                float mm = rd[0 * 128 + row], sum = rd[1 * 128 + row];
+#pragma unroll
+                for (int c = 1; c < 4; ++c) {
+                    if (ONLINE) lse2_merge(mm, sum, rd[(c * 2 + 0) * 128 + row], rd[(c * 2 + 1) * 128 + row]);
+                    else sum += rd[(c * 2 + 1) * 128 + row];
+                }
+                float outv = 0.f, ob = kNegInf;
+                if (lm != kNegInf) {
+                    const bool d_act = D >= 0 && logm[D] != kNegInf;
+                    if (ONLINE) {
+                        if (d_act) lse2_add(mm, sum, (a.sd_term[it.base + r] + a.colpot[pb + D]) * kLog2e);
+                        outv = lm - (mm + log2f(sum)) * kLn2;
+                    } else {
+                        if (d_act) sum += ptx::ex2((a.sd_term[it.base + r] + a.colpot[pb + D]) * kLog2e + st2);
+                        outv = lm - log2f(sum) * kLn2 + st;
+                    }
+                    if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+                    ob = outv * kLog2e;
+                }
+                a.out[pb + r] = outv;
+                a.out_bias2[it.base + r] = ob;
+            }
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tbase, 256);
+        ptx::tmem_dealloc(tbase, 512);
     }
 }
 
@@ -865,8 +907,28 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 bool tc_supported(const Geom& g) { return g.dtype == EOT_BF16 && (g.d == 64 || g.d == 128) && encode_fn() != nullptr; }
 
+int sm_count() {
+    static int n = [] {
+        int dev = 0, v = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+        return v;
+    }();
+    return n;
+}
+
+template <int DH, bool ONLINE>
+cudaError_t launch_lse_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const TcLseArgs& a, int grid,
+                               cudaStream_t st) {
+    constexpr size_t smem = LseCfg<DH>::SMEM;
+    cudaError_t e = set_smem(tc_lse_kernel<DH, ONLINE>, smem);
+    if (e != cudaSuccess) return e;
+    tc_lse_kernel<DH, ONLINE><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     const Geom& g = p.g;
+    if (!p.tile_bits) return cudaErrorInvalidValue;
     CUtensorMap tmX, tmY;
     const uint64_t rows = uint64_t(g.BH) * g.L;
     if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
@@ -877,6 +939,8 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     a.D = g.D;
     a.sl2 = g.scale * kLog2e;
     a.logm = p.logm;
+    a.tile_bits = p.tile_bits;
+    a.words = tile_words(g.L);
     a.colbias2 = p.colbias2;
     a.colpot = p.colpot;
     a.stab = p.stab;
@@ -885,29 +949,17 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     a.pstride = p.pstride;
     a.sd_term = p.sd_term;
     a.status = p.status;
-    const int mt = max_tiles_for(g.L, g.h, 128, 128);
-    dim3 grid(g.L / 128, g.BH);
+    a.n_items = g.BH * (g.L / 128);
+    const int grid = std::max(1, std::min(a.n_items, sm_count()));
+    a.items_per_cta = (a.n_items + grid - 1) / grid;
+    const int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
     cudaError_t e;
-    if (g.d == 128) {
-        const size_t smem = LseCfg<128>::smem_bytes(mt);
-        if (p.stab) {
-            if ((e = set_smem(tc_lse_kernel<128, false>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<128, false><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
-        } else {
-            if ((e = set_smem(tc_lse_kernel<128, true>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<128, true><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
-        }
-    } else {
-        const size_t smem = LseCfg<64>::smem_bytes(mt);
-        if (p.stab) {
-            if ((e = set_smem(tc_lse_kernel<64, false>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<64, false><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
-        } else {
-            if ((e = set_smem(tc_lse_kernel<64, true>, smem)) != cudaSuccess) return e;
-            tc_lse_kernel<64, true><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a, mt);
-        }
-    }
-    e = cudaGetLastError();
+    if (g.d == 128)
+        e = p.stab ? launch_lse_variant<128, false>(tmX, tmY, a, grid_used, st)
+                   : launch_lse_variant<128, true>(tmX, tmY, a, grid_used, st);
+    else
+        e = p.stab ? launch_lse_variant<64, false>(tmX, tmY, a, grid_used, st)
+                   : launch_lse_variant<64, true>(tmX, tmY, a, grid_used, st);
     if (e != cudaSuccess || g.D < 0) return e;
     return launch_dustbin_lse(p, st);
 }
