@@ -26,11 +26,10 @@ namespace eot {
 
 namespace {
 
-constexpr int kThreads = 192;
 constexpr float kNegInf = -__builtin_huge_valf();
 // Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
-// interior forward tiles (3 of 16 pairs; measured best on the long workload).
-constexpr int kFmaPairs = 3;
+// interior forward tiles (2 of 16 pairs: measured best, 0.2585 vs 0.262 ms with none on the long workload).
+constexpr int kFmaPairs = 2;
 
 // ---------------------------------------------------------------------------------------
 // Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
@@ -203,8 +202,8 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         *abort_flag = 0;
         for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 1); }
         for (int i = 0; i < C::NQ; ++i) { ptx::mbar_init(qfull(i), 1); ptx::mbar_init(qempty(i), 1); }
-        for (int i = 0; i < C::NT; ++i) { ptx::mbar_init(tfull(i), 1); ptx::mbar_init(tempty(i), 16); }
-        for (int i = 0; i < C::NB; ++i) { ptx::mbar_init(bfull(i), 1); ptx::mbar_init(bempty(i), 16); }
+        for (int i = 0; i < C::NT; ++i) { ptx::mbar_init(tfull(i), 1); ptx::mbar_init(tempty(i), 8); }
+        for (int i = 0; i < C::NB; ++i) { ptx::mbar_init(bfull(i), 1); ptx::mbar_init(bempty(i), 8); }
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
@@ -296,9 +295,14 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: 16 warps; (lane quadrant, 32-column chunk) each ----------------
-        const int q = warp & 3;                  // TMEM lane quadrant this warp may access
-        const int chunk = (warp - 2) >> 2;       // columns [32 chunk, 32 chunk + 32) of each tile
+        // ---------------- epilogue: 16 warps in two groups that take alternate tiles ----------------
+        // warp (quadrant q, group grp, half hf): TMEM lanes [32 q, 32 q + 32), tiles with running
+        // index g of parity grp, columns [64 hf, 64 hf + 64) of each such tile.
+        const int e = warp - 2;
+        const int q = warp & 3;
+        const int grp = (e >> 2) & 1;
+        const int hf = e >> 3;
+        const int part = grp * 2 + hf;           // which of the four row partials this warp owns
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             const size_t pb = size_t(it.bh) * a.pstride;
             const float* logm = a.logm + size_t(it.b) * L;
             if (!it.rows_active) {
-                if (chunk == 0) {
+                if (part == 0) {
                     a.out[pb + r] = 0.f;
                     a.out_bias2[it.base + r] = kNegInf;
                 }
@@ -322,27 +326,10 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             float m_run = kNegInf;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
-            for (int t = it.t_lo; t <= it.t_hi; ++t) {
-                if (!tile_bit(bits, t)) continue;
-                const int c0 = t * C::BN;
-                const int tb = g % C::NT, bs = g % C::NB;
-                const int gg = g++;
-                if (!ok) continue;
-                const bool interior = (c0 + C::BN - 1 - it.r0 <= h) && (it.r0 + C::BM - 1 - c0 <= h);
-                // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-                bool w1 = ptx::mbar_wait(bfull(bs), (gg / C::NB) & 1, abort_flag, a.status);
-                bool w2 = w1 && ptx::mbar_wait(tfull(tb), (gg / C::NT) & 1, abort_flag, a.status);
-                if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
-                ptx::tc_fence_after();
-                float v[32];
-                ptx::tmem_ld32(tbase + lane_base + uint32_t(tb * C::BN + chunk * 32), v);
-                ptx::tmem_wait_ld(v);
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(tempty(tb));
+            // one 32-column chunk: scores v -> partial sums
+            auto process = [&](const float (&v)[32], int c0, int chunk, int bs, bool interior) {
                 const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN + chunk * 32);
                 if (ONLINE || !interior) {
-                    // scalar path: running maximum (first half-step) or band-edge masking
                     float x[32];
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
@@ -353,12 +340,11 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                         x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
                     }
                     if (!interior) {
-                        const int dlt0 = c0 + chunk * 32 - r;
+                        // valid columns j of this chunk: r - h <= c0 + 32 chunk + j <= r + h
+                        const int lo = r - h - (c0 + chunk * 32), hi = r + h - (c0 + chunk * 32);
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int dl = dlt0 + j;
-                            if (dl < -h || dl > h) x[j] = kNegInf;
-                        }
+                        for (int j = 0; j < 32; ++j)
+                            if (j < lo || j > hi) x[j] = kNegInf;
                     }
                     if (ONLINE) {
                         float cm = kNegInf;
@@ -379,10 +365,8 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                         for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] + st2);
                     }
                 } else {
-                    // interior tile, shifted by the previous potential: packed fp32x2 math;
-                    // the first kFmaPairs pairs of exponentials go to the FMA pipe
+                    // interior tile, shifted by the previous potential: packed fp32x2 math
                     const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
-                    uint64_t acc2[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
                         const float4 bv = bias4[j4];
@@ -400,29 +384,53 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                                 e0 = ptx::ex2(x0);
                                 e1 = ptx::ex2(x1);
                             }
-                            acc2[k & 1] = ptx::fadd2(acc2[k & 1], ptx::f2(e0, e1));
+                            acc[(2 * k) & 3] += e0;
+                            acc[(2 * k + 1) & 3] += e1;
                         }
                     }
-                    float s0, s1, s2, s3;
-                    ptx::f2split(acc2[0], s0, s1);
-                    ptx::f2split(acc2[1], s2, s3);
-                    acc[0] += s0;
-                    acc[1] += s1;
-                    acc[2] += s2;
-                    acc[3] += s3;
+                }
+            };
+            for (int t = it.t_lo; t <= it.t_hi; ++t) {
+                if (!tile_bit(bits, t)) continue;
+                const int gg = g++;
+                if ((gg & 1) != grp || !ok) continue;
+                const int c0 = t * C::BN;
+                const int tb = gg % C::NT, bs = gg % C::NB;
+                const bool interior = (c0 + C::BN - 1 - it.r0 <= h) && (it.r0 + C::BM - 1 - c0 <= h);
+                // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
+                bool w1 = ptx::mbar_wait(bfull(bs), (gg / C::NB) & 1, abort_flag, a.status);
+                bool w2 = w1 && ptx::mbar_wait(tfull(tb), (gg / C::NT) & 1, abort_flag, a.status);
+                if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
+                ptx::tc_fence_after();
+                const uint32_t tcol = tbase + lane_base + uint32_t(tb * C::BN + hf * 64);
+                {
+                    float v[32];
+                    ptx::tmem_ld32(tcol, v);
+                    ptx::tmem_wait_ld(v);
+                    process(v, c0, 2 * hf, bs, interior);
+                }
+                {
+                    float v[32];
+                    ptx::tmem_ld32(tcol + 32, v);
+                    ptx::tmem_wait_ld(v);
+                    // this warp's part of the accumulator buffer is read: hand it back
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(tempty(tb));
+                    process(v, c0, 2 * hf + 1, bs, interior);
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bempty(bs));
             }
-            // The four chunk partials of each row meet in shared memory (two parity slots so
-            // that the next item can proceed while the first chunk's warps read this one).
+            // The four partials of each row meet in shared memory (two parity slots so that
+            // the next item can proceed while the first part's warps read this one).
             float* rd = red + (ep & 1) * (4 * 2 * 128);
-            rd[(chunk * 2 + 0) * 128 + row] = m_run;
-            rd[(chunk * 2 + 1) * 128 + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            rd[(part * 2 + 0) * 128 + row] = m_run;
+            rd[(part * 2 + 1) * 128 + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             ++ep;
             ptx::named_bar_sync(1, 512);
             const bool is_dustbin_row = (r == D) && lm != kNegInf;
-            if (chunk == 0 && ok && !*abort_flag && !is_dustbin_row) {
+            if (part == 0 && ok && !*abort_flag && !is_dustbin_row) {
                 float mm = rd[0 * 128 + row], sum = rd[1 * 128 + row];
 #pragma unroll
                 for (int c = 1; c < 4; ++c) {
@@ -771,8 +779,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     const uint64_t P2 = ptx::f2(v[2 * k], v[2 * k + 1]);
                     if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(w[2 * k], w[2 * k + 1]), s1a[k & 1]);
                     if (M::SM) {
-                        const float2 mv = reinterpret_cast<const float2*>(cv + VOFF_M * C::BN + cc0)[k];
-                        s2a[k & 1] = ptx::ffma2(P2, ptx::f2(mv.x, mv.y), s2a[k & 1]);
+                        const float4 mv = reinterpret_cast<const float4*>(cv + VOFF_M * C::BN + cc0)[k >> 1];
+                        s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
                     }
                 }
             }
@@ -780,16 +788,21 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
                 uint32_t pk[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    uint64_t cf = M::VDP ? ptx::f2(w[2 * k], w[2 * k + 1]) : ptx::f2(1.f, 1.f);
+                for (int k4 = 0; k4 < 8; ++k4) {
+                    uint64_t cf0 = M::VDP ? ptx::f2(w[4 * k4], w[4 * k4 + 1]) : ptx::f2(1.f, 1.f);
+                    uint64_t cf1 = M::VDP ? ptx::f2(w[4 * k4 + 2], w[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
 #pragma unroll
                     for (int mm = 0; mm < NMOD; ++mm) {
-                        const float2 yv = reinterpret_cast<const float2*>(cv + (VOFF_Y + mm) * C::BN + cc0)[k];
-                        cf = ptx::ffma2(ptx::f2(xr[mm], xr[mm]), ptx::f2(yv.x, yv.y), cf);
+                        const float4 yv = reinterpret_cast<const float4*>(cv + (VOFF_Y + mm) * C::BN + cc0)[k4];
+                        const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
+                        cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
+                        cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
                     }
-                    float c0f, c1f;
-                    ptx::f2split(cf, c0f, c1f);
-                    pk[k] = ptx::pack_bf16(v[2 * k] * c0f, v[2 * k + 1] * c1f);
+                    float c0f, c1f, c2f, c3f;
+                    ptx::f2split(cf0, c0f, c1f);
+                    ptx::f2split(cf1, c2f, c3f);
+                    pk[2 * k4] = ptx::pack_bf16(v[4 * k4] * c0f, v[4 * k4 + 1] * c1f);
+                    pk[2 * k4 + 1] = ptx::pack_bf16(v[4 * k4 + 2] * c2f, v[4 * k4 + 3] * c3f);
                 }
                 const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + crow;
 #pragma unroll
