@@ -256,14 +256,26 @@ def barrier(device=None):
             dist.barrier()
 
 
+LSE_BEGIN = "// Forward half-step (band log-sum-exp)"
+LSE_END = "// Output / backward sweep"
+
+
+def lse_source_text(read) -> bytes:
+    """The forward half-step kernel's source: its section of tc.cu plus the headers it uses."""
+    tc = read("tc.cu").decode()
+    i, j = tc.index(LSE_BEGIN), tc.index(LSE_END)
+    return (tc[i:j] + read("ptx.cuh").decode() + read("common.cuh").decode()).encode()
+
+
 def source_hash() -> str:
-    h = hashlib.sha256()
+    """Hash of the forward half-step kernel's sources (identifies the code an ncu summary covers)."""
     csrc = os.path.join(ROOT, "entropic_ot_attention_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode())
-            h.update(fh.read())
-    return h.hexdigest()[:16]
+
+    def read(name):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            return fh.read()
+
+    return hashlib.sha256(lse_source_text(read)).hexdigest()[:16]
 
 
 def load_traffic(workload: str):

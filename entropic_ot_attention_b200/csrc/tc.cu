@@ -507,7 +507,7 @@ struct TcVecArgs {
     uint32_t* status;
 };
 
-constexpr int kSweepThreads = 320;   // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kSweepThreads = 352;   // TMA warp, score-MMA warp, 8 epilogue warps, product-MMA warp
 
 template <int DH, int NV>
 struct SweepCfg {
@@ -654,27 +654,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            // ---------------- MMA issuer ----------------
+            // ---------------- score MMA issuer: S (and dP) tiles ----------------
             const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
-            int vec_done = 0;
             bool ok = ptx::mbar_wait(xfull, 0, abort_flag, a.status);
-            auto do_vec = [&](int j) -> bool {
-                const int cb = j & 1;
-                if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) return false;
-                ptx::tc_fence_after();
-                const int s = j % C::NS;
-                const uint32_t zs = ptx::smem_u32(sm + (M::ZW2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
-                const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
-#pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + kk * 32, 16, 1024),
-                                  ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
-                                  (j > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(cempty(cb));
-                ptx::mma_commit(empty(s));
-                vec_done = j + 1;
-                return true;
-            };
             int issued = 0;
             for (int it = 0; it < n && ok; ++it) {
                 const int s = it % C::NS, bb = it & 1;
@@ -700,20 +682,45 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     }
                 }
                 ptx::mma_commit(tfull(bb));
-                if (!M::VEC) ptx::mma_commit(empty(s));
+                if (!M::VEC) ptx::mma_commit(empty(s));   // vector passes free the stage after the product
                 issued = it + 1;
-                if (M::VEC && it >= 1 && !do_vec(it - 1)) { ok = false; break; }
             }
-            if (M::VEC && ok && n > 0 && do_vec(n - 1)) ptx::mma_commit(accfull);
-            if (*abort_flag) {
+            if (*abort_flag && issued > 0) {
                 volatile int dummy = 0;
-                if (issued > 0) ptx::mbar_wait(tfull((issued - 1) & 1), ((issued - 1) >> 1) & 1, &dummy, a.status);
-                if (vec_done > 0)
-                    ptx::mbar_wait(cempty((vec_done - 1) & 1), ((vec_done - 1) >> 1) & 1, &dummy, a.status);
+                ptx::mbar_wait(tfull((issued - 1) & 1), ((issued - 1) >> 1) & 1, &dummy, a.status);
+            }
+        }
+    } else if (warp == 10) {
+        if (M::VEC && lane == 0) {
+            // ---------------- product MMA issuer: acc += coef(j) * Z(j) ----------------
+            // A thread of its own, so that score tiles are never queued behind a product
+            // that waits for the epilogue (tcgen05.commit tracks the issuing thread's MMAs).
+            int done = 0;
+            bool ok = true;
+            for (int j = 0; j < n && ok; ++j) {
+                const int cb = j & 1;
+                if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const int s = j % C::NS;
+                const uint32_t zs = ptx::smem_u32(sm + (M::ZW2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
+                const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + kk * 32, 16, 1024),
+                                  ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(cempty(cb));
+                ptx::mma_commit(empty(s));
+                done = j + 1;
+            }
+            if (ok && n > 0) ptx::mma_commit(accfull);
+            if (*abort_flag && done > 0) {
+                volatile int dummy = 0;
+                ptx::mbar_wait(cempty((done - 1) & 1), ((done - 1) >> 1) & 1, &dummy, a.status);
             }
         }
     } else {
-        // ---------------- epilogue: 8 warps, two per TMEM lane quadrant ----------------
+        // ---------------- epilogue: warps 2..9, two per TMEM lane quadrant ----------------
         const int q = warp & 3;                  // lane quadrant
         const int half = (warp - 2) >> 2;        // which 32 columns of each 64-column tile
         const int row = q * 32 + lane, r = r0 + row;
