@@ -418,13 +418,13 @@ def main():
     # backward sweeps are counted with their own MMA work per launch
     if dom == "fwd_sweep":
         dom_flops = 2 * d * omega
-        dom_name = "tc_lse_kernel (forward half-step band log-sum-exp)"
+        dom_name = "tc_band_kernel (forward half-step band log-sum-exp)"
     elif dom == "fwd_output":
         dom_flops = 2 * 2 * d * omega
-        dom_name = "tc_vec_kernel (forward output P V)"
+        dom_name = "tc_sweep_kernel (forward output P V)"
     else:
         dom_flops = fl_bwd / max(dom_n, 1)
-        dom_name = "tc_vec_kernel (backward sweeps)"
+        dom_name = "tc_sweep_kernel + tc_band_kernel (backward sweeps)"
     achieved = dom_flops / (per_launch_ms * 1e-3) / 1e12
     traffic = load_traffic(args.workload)
     # exp-unit context: one exp2 per band entry per launch for the forward half-step

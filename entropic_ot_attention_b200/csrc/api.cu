@@ -298,6 +298,9 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.dp_dense = e2;
     rowp.zero_vec = at<float>(ws, w.zero);
     rowp.status = status;
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
+    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
+    rowp.tile_bits = tbits;
     EOT_TRY(cudaMemsetAsync(at<float>(ws, w.zero), 0, vecn * sizeof(float), st));
     BwdPass colp = rowp;
     colp.X = K;

@@ -85,6 +85,7 @@ struct BwdPass {
     const float* dp_term;   // <A_r, Bm_D>
     const float* dp_dense;  // <A_D, Bm_c>
     const float* zero_vec;  // [BH, L] zeros (padding of the modifier list), or nullptr
+    const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
     uint32_t* status;
 };
 
@@ -93,7 +94,7 @@ struct WsLayout {
     size_t status, logm, sd_row, sd_col, e1, e2;
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
-    size_t tbits;           // forward: active-tile bitmask [B][tile_words(L)]
+    size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
     size_t zero;            // backward: a vector of zeros
     size_t pr, pc, f, hv, m;
@@ -123,8 +124,8 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.opcm = o; o += vec;
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
-        w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     }
+    w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     if (bwd) {
         w.pr = o; o += vec;
         w.pc = o; o += vec;

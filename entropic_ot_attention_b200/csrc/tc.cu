@@ -11,10 +11,12 @@
 // §2.2: the backward sweeps re-form the one reference plan P(R,R) per tile from S and the
 // stored potentials, and apply the per-row / per-column orbit factors in registers.
 //
-// Roles in a CTA of 192 threads:
-//   warp 0      TMA producer (one elected lane): row tile once, column tiles into a ring
-//   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..5  epilogue: thread t of warp w owns TMEM lane / row 32 (w % 4) + t
+// Two kernels:
+//   tc_band_kernel   persistent, 128 x 128 score tiles, row reductions only (forward
+//                    half-steps and the staircase sums of the backward pass)
+//   tc_sweep_kernel  one CTA per 128-row tile, 128 x 64 score tiles, row reductions and a
+//                    second MMA that multiplies coefficient tiles into d-wide outputs
+//                    (forward output, dV, dQ, dK)
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -95,74 +97,111 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ---------------------------------------------------------------------------------------
-// Forward half-step (band log-sum-exp): persistent kernel, 128 x 128 tiles
+// Forward half-step (band log-sum-exp) and weighted band row sums: persistent kernel
 // ---------------------------------------------------------------------------------------
-// One CTA per SM walks a contiguous range of (unit, row-tile) work items.  Barriers and TMEM
-// are set up once; the TMA warp runs ahead across item boundaries (two row-tile buffers,
-// NS column-tile stages, a bias ring), the MMA warp keeps up to four score tiles in flight
-// in TMEM (4 x 128 columns), and 16 epilogue warps (four per TMEM lane quadrant, one per
-// 32-column chunk of a tile) turn each tile into row partial sums.  All three roles walk
-// the same item / tile sequence, so ring indices and mbarrier phases follow from one
-// running tile counter.
-struct TcLseArgs {
-    int H, L, h, D, n_items, items_per_cta;
-    float sl2;              // scale * log2(e)
+// One CTA per SM walks a contiguous range of work items.  An item is a pair of adjacent
+// 128-row tiles of one unit, rows [256 p, 256 p + 256); both halves share every 128-column
+// tile that their bands touch, so each column tile comes into shared memory once and feeds
+// two MMAs.  Roles:
+//   warp 0       TMA producer (one lane): row halves into a small ring, column tiles into
+//                NS stages, and per half the tile's column vectors (log2 bias, weights)
+//   warp 1       TMEM allocator and MMA issuer (one lane): two 128-column fp32 score
+//                accumulators per half (4 x 128 TMEM columns)
+//   warps 2..9   epilogue of the first half, warps 10..17 of the second: warp (q, hf) reads
+//                TMEM lanes [32 q, 32 q + 32) and columns [64 hf, 64 hf + 64) of each tile
+// The two warps that share a row meet once per item on a 64-thread named barrier; the
+// halves are coupled only through the column-tile stages.  All roles walk the same item /
+// tile sequence, so ring slots and mbarrier phases follow from running counters.
+//
+// Reductions (KIND), for the rows r of a half and the band columns c of each row:
+//   online  out_r = logm_r - LSE_c (S_rc + colpot_c), with a running maximum (first step)
+//   shift   the same sum shifted by the previous potential st_r: after a completed
+//           half-step every term exp(S + st + colpot) is at most 1, so no maximum is kept
+//   wsum    out_r = f_r hv_r sum_c exp(S_rc + st_r + colpot_c) w_c  (staircase sums of the
+//           tail adjoint, with st = the row orbit bias and w = the column weights)
+enum BandKind { kBandOnline = 0, kBandShift = 1, kBandWsum = 2 };
+
+struct TcBandArgs {
+    int H, L, h, D, n_items, items_per_cta, pairs_per_unit;
+    float sl2;                  // scale * log2(e)
     const float* logm;
     const uint32_t* tile_bits;  // [B][words]: bit t = positions [128 t, 128 t + 128) hold an active non-dustbin token
     int words;
-    const float* colbias2;  // [BH, L] masked log2 column bias
-    const float* colpot;    // natural column potential (pstride), read at D
-    const float* stab;      // natural previous row potential (pstride) or nullptr
-    float* out;             // natural (pstride)
-    float* out_bias2;       // [BH, L]
+    const float* colbias2;      // [BH, L] masked log2 column bias
+    const float* colw;          // [BH, L] column weights (wsum)
+    const float* colpot;        // natural column potential (pstride), read at D
+    const float* stab;          // natural row shift (pstride); unused by online
+    float* out;                 // natural (pstride)
+    float* out_bias2;           // [BH, L] masked log2 copy of out (log-sum-exp kinds)
+    const float* f;             // [BH, L] row factors (wsum)
+    const float* hv;            // [BH, L] (wsum)
     size_t pstride;
     const float* sd_term;
     uint32_t* status;
 };
 
-template <int DH>
-struct LseCfg {
+template <int DH, int KIND>
+struct BandCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
-    static constexpr int NS = DH == 128 ? 4 : 8;   // column-tile stages
-    static constexpr int NQ = 2;                   // row-tile buffers
-    static constexpr int NT = 4;                   // TMEM accumulator buffers (4 x 128 columns)
-    static constexpr int NB = 8;                   // bias ring slots
-    static constexpr uint32_t XB = BM * DH * 2;    // row tile bytes
+    static constexpr int NQ = DH == 128 ? 3 : 6;   // row half-tile slots
+    static constexpr int NS = DH == 128 ? 3 : 6;   // column-tile stages
+    static constexpr int NV = 4;                   // column-vector slots per half
+    static constexpr int NVEC = KIND == kBandWsum ? 2 : 1;
+    static constexpr uint32_t XB = BM * DH * 2;    // row half-tile bytes
     static constexpr uint32_t YB = BN * DH * 2;    // column tile bytes
     static constexpr uint32_t ATOM = 128 * 128;    // one 64-element-wide atom column of 128 rows
+    static constexpr uint32_t VB = NVEC * BN * 4;  // column vectors of one tile
     static constexpr uint32_t OFF_Y = NQ * XB;
-    static constexpr uint32_t OFF_BIAS = OFF_Y + NS * YB;
-    static constexpr uint32_t OFF_RED = OFF_BIAS + NB * BN * 4;   // [2 parity][4 chunks][m, s][128 rows]
-    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 2 * 128 * 4;
-    // full[NS] empty[NS] qfull[NQ] qempty[NQ] tfull[NT] tempty[NT] bfull[NB] bempty[NB]
-    static constexpr uint32_t NBARS = 2 * NS + 2 * NQ + 2 * NT + 2 * NB;
+    static constexpr uint32_t OFF_V = OFF_Y + NS * YB;         // [half][NV][VB]
+    static constexpr uint32_t OFF_RED = OFF_V + 2 * NV * VB;    // [half][parity][m, s][128 rows]
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 2 * 128 * 4;
+    // full[NS] empty[NS] qfull[NQ] qempty[NQ], then per half: tfull[2] tempty[2] vfull[NV] vempty[NV]
+    static constexpr uint32_t HB0 = 2 * NS + 2 * NQ;
+    static constexpr uint32_t HBN = 4 + 2 * NV;
+    static constexpr uint32_t NBARS = HB0 + 2 * HBN;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr size_t SMEM = 1024 + OFF_MISC + 64;
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
-constexpr int kLseThreads = 576;   // TMA warp, MMA warp, 16 epilogue warps
+constexpr int kBandThreads = 576;   // TMA warp, MMA warp, 16 epilogue warps
 
-// Decoded work item: the 128-row tile I of unit bh and its band of column tiles.
-struct LseItem {
-    int bh, b, r0, t_lo, t_hi;
-    bool rows_active;
+// Decoded work item: rows [r0, r0 + 256) of unit bh as two halves with their column-tile bands.
+struct BandItem {
+    int bh, b, r0;
     size_t base;
+    bool exists[2], active[2];
+    int t_lo[2], t_hi[2];
 };
 
 __device__ __forceinline__ bool tile_bit(const uint32_t* bits, int t) { return (bits[t >> 5] >> (t & 31)) & 1u; }
 
-template <int DH, bool ONLINE>
-__global__ void __launch_bounds__(kLseThreads, 1)
-    tc_lse_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-                  const TcLseArgs a) {
-    using C = LseCfg<DH>;
+// Tile bits of one batch row, the current 32-bit word held in a register.
+struct TileBits {
+    const uint32_t* w;
+    int idx;
+    uint32_t word;
+    __device__ explicit TileBits(const uint32_t* p) : w(p), idx(-1), word(0u) {}
+    __device__ bool operator()(int t) {
+        if ((t >> 5) != idx) {
+            idx = t >> 5;
+            word = w[idx];
+        }
+        return (word >> (t & 31)) & 1u;
+    }
+};
+
+template <int DH, int KIND>
+__global__ void __launch_bounds__(kBandThreads, 1)
+    tc_band_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                   const TcBandArgs a) {
+    using C = BandCfg<DH, KIND>;
+    constexpr bool ONLINE = KIND == kBandOnline, WSUM = KIND == kBandWsum;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = a.L, h = a.h, D = a.D;
-    const int tiles_per_unit = L / C::BM;
     const int item0 = blockIdx.x * a.items_per_cta;
     const int item1 = min(a.n_items, item0 + a.items_per_cta);
 
@@ -172,38 +211,41 @@ __global__ void __launch_bounds__(kLseThreads, 1)
     auto empty = [&](int i) { return bar0 + 8u * (C::NS + i); };
     auto qfull = [&](int i) { return bar0 + 8u * (2 * C::NS + i); };
     auto qempty = [&](int i) { return bar0 + 8u * (2 * C::NS + C::NQ + i); };
-    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + i); };
-    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + C::NT + i); };
-    auto bfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + 2 * C::NT + i); };
-    auto bempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 2 * C::NQ + 2 * C::NT + C::NB + i); };
+    auto tfull = [&](int G, int i) { return bar0 + 8u * (C::HB0 + G * C::HBN + i); };
+    auto tempty = [&](int G, int i) { return bar0 + 8u * (C::HB0 + G * C::HBN + 2 + i); };
+    auto vfull = [&](int G, int i) { return bar0 + 8u * (C::HB0 + G * C::HBN + 4 + i); };
+    auto vempty = [&](int G, int i) { return bar0 + 8u * (C::HB0 + G * C::HBN + 4 + C::NV + i); };
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-    const float* bias_s = reinterpret_cast<const float*>(sm + C::OFF_BIAS);
 
     auto decode = [&](int item) {
-        LseItem it;
-        it.bh = item / tiles_per_unit;
+        BandItem it;
+        it.bh = item / a.pairs_per_unit;
         it.b = it.bh / a.H;
-        it.r0 = (item - it.bh * tiles_per_unit) * C::BM;
+        it.r0 = (item - it.bh * a.pairs_per_unit) * 2 * C::BM;
         it.base = size_t(it.bh) * L;
-        it.t_lo = max(0, it.r0 - h) / C::BN;
-        it.t_hi = min(L - 1, it.r0 + C::BM - 1 + h) / C::BN;
-        it.rows_active = tile_bit(a.tile_bits + size_t(it.b) * a.words, it.r0 / C::BM);
+        const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+#pragma unroll
+        for (int G = 0; G < 2; ++G) {
+            const int rg = it.r0 + G * C::BM;
+            it.exists[G] = rg < L;
+            it.active[G] = it.exists[G] && tile_bit(bits, rg / C::BM);
+            it.t_lo[G] = max(0, rg - h) / C::BN;
+            it.t_hi[G] = min(L - 1, rg + C::BM - 1 + h) / C::BN;
+        }
         return it;
     };
-    auto count_tiles = [&](const LseItem& it) {
-        const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
-        int n = 0;
-        for (int t = it.t_lo; t <= it.t_hi; ++t) n += tile_bit(bits, t);
-        return n;
-    };
+    // Column tiles that half G multiplies: inside its band and holding an active column.
+    auto uses = [&](const BandItem& it, int G, int t) { return it.active[G] && t >= it.t_lo[G] && t <= it.t_hi[G]; };
 
     if (tid == 0) {
         *abort_flag = 0;
         for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 1); }
         for (int i = 0; i < C::NQ; ++i) { ptx::mbar_init(qfull(i), 1); ptx::mbar_init(qempty(i), 1); }
-        for (int i = 0; i < C::NT; ++i) { ptx::mbar_init(tfull(i), 1); ptx::mbar_init(tempty(i), 8); }
-        for (int i = 0; i < C::NB; ++i) { ptx::mbar_init(bfull(i), 1); ptx::mbar_init(bempty(i), 8); }
+        for (int G = 0; G < 2; ++G) {
+            for (int i = 0; i < 2; ++i) { ptx::mbar_init(tfull(G, i), 1); ptx::mbar_init(tempty(G, i), 8); }
+            for (int i = 0; i < C::NV; ++i) { ptx::mbar_init(vfull(G, i), 1); ptx::mbar_init(vempty(G, i), 8); }
+        }
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
@@ -221,39 +263,61 @@ __global__ void __launch_bounds__(kLseThreads, 1)
             ptx::prefetch_tmap(&tmX);
             ptx::prefetch_tmap(&tmY);
             int g = 0, qi = 0;
+            int gv[2] = {0, 0};
             bool ok = true;
             for (int item = item0; item < item1 && ok; ++item) {
-                const LseItem it = decode(item);
-                if (!it.rows_active || count_tiles(it) == 0) continue;
-                const int qb = qi % C::NQ;
-                if (!ptx::mbar_wait(qempty(qb), ((qi / C::NQ) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-                ptx::mbar_expect_tx(qfull(qb), C::XB);
-                const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
-                for (int ka = 0; ka < C::KATOMS; ++ka)
-                    ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(it.base) + it.r0, qfull(qb));
-                ++qi;
-                const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
-                for (int t = it.t_lo; t <= it.t_hi; ++t) {
-                    if (!tile_bit(bits, t)) continue;
+                const BandItem it = decode(item);
+                if (!it.active[0] && !it.active[1]) continue;
+#pragma unroll
+                for (int G = 0; G < 2; ++G) {
+                    if (!it.active[G]) continue;
+                    const int qb = qi % C::NQ;
+                    if (!ptx::mbar_wait(qempty(qb), ((qi / C::NQ) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ptx::mbar_expect_tx(qfull(qb), C::XB);
+                    const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
+                    for (int ka = 0; ka < C::KATOMS; ++ka)
+                        ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(it.base) + it.r0 + G * C::BM, qfull(qb));
+                    ++qi;
+                }
+                if (!ok) break;
+                TileBits bits(a.tile_bits + size_t(it.b) * a.words);
+                const int u_lo = it.active[0] ? it.t_lo[0] : it.t_lo[1];
+                const int u_hi = it.active[1] ? it.t_hi[1] : it.t_hi[0];
+                for (int t = u_lo; t <= u_hi && ok; ++t) {
+                    if (!bits(t)) continue;
+                    const bool use0 = uses(it, 0, t), use1 = uses(it, 1, t);
+                    if (!use0 && !use1) continue;
                     const int c0 = t * C::BN;
-                    const int s = g % C::NS, bs = g % C::NB;
+                    const int s = g % C::NS;
                     if (!ptx::mbar_wait(empty(s), ((g / C::NS) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                     ptx::mbar_expect_tx(full(s), C::YB);
                     const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
                     for (int ka = 0; ka < C::KATOMS; ++ka)
                         ptx::tma_load_2d(ys + ka * C::ATOM, &tmY, ka * 64, int(it.base) + c0, full(s));
-                    if (!ptx::mbar_wait(bempty(bs), ((g / C::NB) & 1) ^ 1, abort_flag, a.status)) { ++g; ok = false; break; }
-                    ptx::mbar_expect_tx(bfull(bs), C::BN * 4);
-                    ptx::bulk_load(ptx::smem_u32(sm + C::OFF_BIAS + bs * C::BN * 4), a.colbias2 + it.base + c0, C::BN * 4,
-                                   bfull(bs));
                     ++g;
+#pragma unroll
+                    for (int G = 0; G < 2; ++G) {
+                        if (!(G ? use1 : use0)) continue;
+                        const int vs = gv[G] % C::NV;
+                        if (!ptx::mbar_wait(vempty(G, vs), ((gv[G] / C::NV) & 1) ^ 1, abort_flag, a.status)) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::mbar_expect_tx(vfull(G, vs), C::VB);
+                        const uint32_t vd = ptx::smem_u32(sm + C::OFF_V + (G * C::NV + vs) * C::VB);
+                        ptx::bulk_load(vd, a.colbias2 + it.base + c0, C::BN * 4, vfull(G, vs));
+                        if (WSUM) ptx::bulk_load(vd + C::BN * 4, a.colw + it.base + c0, C::BN * 4, vfull(G, vs));
+                        ++gv[G];
+                    }
                 }
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA retires.
                 volatile int dummy = 0;
                 for (int i = max(0, g - C::NS); i < g; ++i) ptx::mbar_wait(full(i % C::NS), (i / C::NS) & 1, &dummy, a.status);
-                for (int i = max(0, g - C::NB); i < g; ++i) ptx::mbar_wait(bfull(i % C::NB), (i / C::NB) & 1, &dummy, a.status);
+                for (int G = 0; G < 2; ++G)
+                    for (int i = max(0, gv[G] - C::NV); i < gv[G]; ++i)
+                        ptx::mbar_wait(vfull(G, i % C::NV), (i / C::NV) & 1, &dummy, a.status);
                 for (int i = max(0, qi - C::NQ); i < qi; ++i) ptx::mbar_wait(qfull(i % C::NQ), (i / C::NQ) & 1, &dummy, a.status);
             }
         }
@@ -261,74 +325,110 @@ __global__ void __launch_bounds__(kLseThreads, 1)
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
             int g = 0, qi = 0;
+            int gt[2] = {0, 0};
             bool ok = true;
             for (int item = item0; item < item1 && ok; ++item) {
-                const LseItem it = decode(item);
-                const int n = it.rows_active ? count_tiles(it) : 0;
-                if (n == 0) continue;
-                const int qb = qi % C::NQ;
-                if (!ptx::mbar_wait(qfull(qb), (qi / C::NQ) & 1, abort_flag, a.status)) { ok = false; break; }
-                ++qi;
-                const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
-                for (int k = 0; k < n; ++k) {
-                    const int s = g % C::NS, tb = g % C::NT;
-                    if (!ptx::mbar_wait(full(s), (g / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
-                    if (!ptx::mbar_wait(tempty(tb), ((g / C::NT) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
-                    const uint32_t dt = tbase + uint32_t(tb * C::BN);
+                const BandItem it = decode(item);
+                if (!it.active[0] && !it.active[1]) continue;
+                TileBits bits(a.tile_bits + size_t(it.b) * a.words);
+                int qslot[2] = {0, 0}, qpar[2] = {0, 0}, n[2] = {0, 0}, done[2] = {0, 0};
+                bool xready[2] = {false, false};
 #pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
-                        ptx::mma_bf16(dt, ptx::smem_desc(xs + koff, 16, 1024), ptx::smem_desc(ys + koff, 16, 1024),
-                                      C::IDESC, kk > 0 ? 1u : 0u);
+                for (int G = 0; G < 2; ++G) {
+                    if (!it.active[G]) continue;
+                    qslot[G] = qi % C::NQ;
+                    qpar[G] = (qi / C::NQ) & 1;
+                    ++qi;
+                    for (int t = it.t_lo[G]; t <= it.t_hi[G]; ++t) n[G] += bits(t);
+                }
+                const int u_lo = it.active[0] ? it.t_lo[0] : it.t_lo[1];
+                const int u_hi = it.active[1] ? it.t_hi[1] : it.t_hi[0];
+                for (int t = u_lo; t <= u_hi && ok; ++t) {
+                    if (!bits(t)) continue;
+                    const bool use0 = uses(it, 0, t), use1 = uses(it, 1, t);
+                    if (!use0 && !use1) continue;
+                    const int s = g % C::NS;
+                    if (!ptx::mbar_wait(full(s), (g / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
+                    const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
+#pragma unroll
+                    for (int G = 0; G < 2; ++G) {
+                        if (!(G ? use1 : use0)) continue;
+                        if (!xready[G]) {
+                            if (!ptx::mbar_wait(qfull(qslot[G]), qpar[G], abort_flag, a.status)) { ok = false; break; }
+                            xready[G] = true;
+                        }
+                        const int tb = gt[G] & 1;
+                        if (!ptx::mbar_wait(tempty(G, tb), ((gt[G] >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        const uint32_t xs = ptx::smem_u32(sm + qslot[G] * C::XB);
+                        const uint32_t dt = tbase + uint32_t((G * 2 + tb) * C::BN);
+#pragma unroll
+                        for (int kk = 0; kk < DH / 16; ++kk) {
+                            const uint32_t koff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
+                            ptx::mma_bf16(dt, ptx::smem_desc(xs + koff, 16, 1024), ptx::smem_desc(ys + koff, 16, 1024),
+                                          C::IDESC, kk > 0 ? 1u : 0u);
+                        }
+                        ptx::mma_commit(tfull(G, tb));
+                        ++gt[G];
+                        if (++done[G] == n[G]) ptx::mma_commit(qempty(qslot[G]));   // row half free once its products are done
                     }
+                    if (!ok) break;
                     ptx::mma_commit(empty(s));
-                    ptx::mma_commit(tfull(tb));
                     ++g;
                 }
-                ptx::mma_commit(qempty(qb));   // row tile free once this item's products are done
+                // (a half with no column tile cannot occur: an active row tile holds its own diagonal tile)
+                for (int G = 0; G < 2 && ok; ++G) {
+                    if (!it.active[G] || n[G] != 0) continue;
+                    if (!ptx::mbar_wait(qfull(qslot[G]), qpar[G], abort_flag, a.status)) { ok = false; break; }
+                    ptx::mma_commit(qempty(qslot[G]));
+                }
             }
-            if (*abort_flag && g > 0) {
+            if (*abort_flag) {
                 volatile int dummy = 0;
-                ptx::mbar_wait(tfull((g - 1) % C::NT), ((g - 1) / C::NT) & 1, &dummy, a.status);
+                for (int G = 0; G < 2; ++G)
+                    if (gt[G] > 0) ptx::mbar_wait(tfull(G, (gt[G] - 1) & 1), ((gt[G] - 1) >> 1) & 1, &dummy, a.status);
             }
         }
     } else {
-        // ---------------- epilogue: 16 warps in two groups that take alternate tiles ----------------
-        // warp (quadrant q, group grp, half hf): TMEM lanes [32 q, 32 q + 32), tiles with running
-        // index g of parity grp, columns [64 hf, 64 hf + 64) of each such tile.
+        // ---------------- epilogue: 8 warps per half ----------------
         const int e = warp - 2;
-        const int q = warp & 3;
-        const int grp = (e >> 2) & 1;
-        const int hf = e >> 3;
-        const int part = grp * 2 + hf;           // which of the four row partials this warp owns
+        const int G = e >> 3;                 // row half
+        const int hf = (e >> 2) & 1;          // column half of each tile
+        const int q = warp & 3;               // TMEM lane quadrant (fixed by the warp's rank)
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
-        int g = 0, ep = 0;
+        float* red = reinterpret_cast<float*>(sm + C::OFF_RED) + G * (2 * 2 * 128);
+        const float* vbase = reinterpret_cast<const float*>(sm + C::OFF_V + G * C::NV * C::VB);
+        int gt = 0, ep = 0;
         bool ok = true;
         for (int item = item0; item < item1; ++item) {
-            const LseItem it = decode(item);
-            const int r = it.r0 + row;
-            const size_t pb = size_t(it.bh) * a.pstride;
-            const float* logm = a.logm + size_t(it.b) * L;
-            if (!it.rows_active) {
-                if (part == 0) {
+            // this half of the item (no per-half arrays: G is not a compile-time index here)
+            const int bh = item / a.pairs_per_unit, b = bh / a.H;
+            const int rg = (item - bh * a.pairs_per_unit) * 2 * C::BM + G * C::BM;
+            if (rg >= L) continue;
+            const size_t base = size_t(bh) * L;
+            const int r = rg + row;
+            const size_t pb = size_t(bh) * a.pstride;
+            const uint32_t* bitp = a.tile_bits + size_t(b) * a.words;
+            if (!tile_bit(bitp, rg / C::BM)) {
+                if (hf == 0) {
                     a.out[pb + r] = 0.f;
-                    a.out_bias2[it.base + r] = kNegInf;
+                    if (!WSUM) a.out_bias2[base + r] = kNegInf;
                 }
                 continue;
             }
+            const int t_lo = max(0, rg - h) / C::BN, t_hi = min(L - 1, rg + C::BM - 1 + h) / C::BN;
+            const float* logm = a.logm + size_t(b) * L;
             const float lm = logm[r];
             const float st = ONLINE ? 0.f : a.stab[pb + r];
             const float st2 = st * kLog2e;
             float m_run = kNegInf;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+            TileBits bits(bitp);
             // one 32-column chunk: scores v -> partial sums
-            auto process = [&](const float (&v)[32], int c0, int chunk, int bs, bool interior) {
-                const float4* bias4 = reinterpret_cast<const float4*>(bias_s + bs * C::BN + chunk * 32);
+            auto process = [&](const float (&v)[32], int c0, int chunk, const float* vec, bool interior) {
+                const float4* bias4 = reinterpret_cast<const float4*>(vec + chunk * 32);
+                const float4* w4 = reinterpret_cast<const float4*>(vec + C::BN + chunk * 32);
                 if (ONLINE || !interior) {
                     float x[32];
 #pragma unroll
@@ -360,16 +460,27 @@ __global__ void __launch_bounds__(kLseThreads, 1)
 #pragma unroll
                             for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] - m_run);
                         }
+                    } else if (WSUM) {
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 wv = w4[j4];
+                            acc[0] = fmaf(ptx::ex2(x[4 * j4 + 0] + st2), wv.x, acc[0]);
+                            acc[1] = fmaf(ptx::ex2(x[4 * j4 + 1] + st2), wv.y, acc[1]);
+                            acc[2] = fmaf(ptx::ex2(x[4 * j4 + 2] + st2), wv.z, acc[2]);
+                            acc[3] = fmaf(ptx::ex2(x[4 * j4 + 3] + st2), wv.w, acc[3]);
+                        }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] + st2);
                     }
                 } else {
-                    // interior tile, shifted by the previous potential: packed fp32x2 math
+                    // interior tile, shifted: packed fp32x2 math
                     const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
                         const float4 bv = bias4[j4];
+                        float4 wv;
+                        if (WSUM) wv = w4[j4];
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int k = 2 * j4 + hh;
@@ -384,74 +495,85 @@ __global__ void __launch_bounds__(kLseThreads, 1)
                                 e0 = ptx::ex2(x0);
                                 e1 = ptx::ex2(x1);
                             }
-                            acc[(2 * k) & 3] += e0;
-                            acc[(2 * k + 1) & 3] += e1;
+                            if (WSUM) {
+                                acc[(2 * k) & 3] = fmaf(e0, hh ? wv.z : wv.x, acc[(2 * k) & 3]);
+                                acc[(2 * k + 1) & 3] = fmaf(e1, hh ? wv.w : wv.y, acc[(2 * k + 1) & 3]);
+                            } else {
+                                acc[(2 * k) & 3] += e0;
+                                acc[(2 * k + 1) & 3] += e1;
+                            }
                         }
                     }
                 }
             };
-            for (int t = it.t_lo; t <= it.t_hi; ++t) {
-                if (!tile_bit(bits, t)) continue;
-                const int gg = g++;
-                if ((gg & 1) != grp || !ok) continue;
+            for (int t = t_lo; t <= t_hi; ++t) {
+                if (!bits(t)) continue;
+                const int gg = gt++;
+                if (!ok) continue;
                 const int c0 = t * C::BN;
-                const int tb = gg % C::NT, bs = gg % C::NB;
-                const bool interior = (c0 + C::BN - 1 - it.r0 <= h) && (it.r0 + C::BM - 1 - c0 <= h);
+                const int tb = gg & 1, vs = gg % C::NV;
+                const bool interior = (c0 + C::BN - 1 - rg <= h) && (rg + C::BM - 1 - c0 <= h);
                 // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-                bool w1 = ptx::mbar_wait(bfull(bs), (gg / C::NB) & 1, abort_flag, a.status);
-                bool w2 = w1 && ptx::mbar_wait(tfull(tb), (gg / C::NT) & 1, abort_flag, a.status);
+                bool w1 = ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
+                bool w2 = w1 && ptx::mbar_wait(tfull(G, tb), (gg >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
                 ptx::tc_fence_after();
-                const uint32_t tcol = tbase + lane_base + uint32_t(tb * C::BN + hf * 64);
+                const float* vec = vbase + vs * (C::VB / 4);
+                const uint32_t tcol = tbase + lane_base + uint32_t((G * 2 + tb) * C::BN + hf * 64);
                 {
                     float v[32];
                     ptx::tmem_ld32(tcol, v);
                     ptx::tmem_wait_ld(v);
-                    process(v, c0, 2 * hf, bs, interior);
+                    process(v, c0, 2 * hf, vec, interior);
                 }
                 {
                     float v[32];
                     ptx::tmem_ld32(tcol + 32, v);
                     ptx::tmem_wait_ld(v);
-                    // this warp's part of the accumulator buffer is read: hand it back
+                    // this warp's part of the accumulator is read: hand it back
                     ptx::tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(tempty(tb));
-                    process(v, c0, 2 * hf + 1, bs, interior);
+                    if (lane == 0) ptx::mbar_arrive(tempty(G, tb));
+                    process(v, c0, 2 * hf + 1, vec, interior);
                 }
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bempty(bs));
+                if (lane == 0) ptx::mbar_arrive(vempty(G, vs));
             }
-            // The four partials of each row meet in shared memory (two parity slots so that
-            // the next item can proceed while the first part's warps read this one).
-            float* rd = red + (ep & 1) * (4 * 2 * 128);
-            rd[(part * 2 + 0) * 128 + row] = m_run;
-            rd[(part * 2 + 1) * 128 + row] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            // The two column halves of each row meet in shared memory (two parity slots:
+            // the partner writes item e + 1 only after this warp has read item e).
+            float* rd = red + (ep & 1) * (2 * 128);
             ++ep;
-            ptx::named_bar_sync(1, 512);
+            const float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            if (hf == 1) {
+                rd[row] = m_run;
+                rd[128 + row] = part;
+            }
+            ptx::named_bar_sync(1 + G * 4 + q, 64);
             const bool is_dustbin_row = (r == D) && lm != kNegInf;
-            if (part == 0 && ok && !*abort_flag && !is_dustbin_row) {
-                float mm = rd[0 * 128 + row], sum = rd[1 * 128 + row];
-#pragma unroll
-                for (int c = 1; c < 4; ++c) {
-                    if (ONLINE) lse2_merge(mm, sum, rd[(c * 2 + 0) * 128 + row], rd[(c * 2 + 1) * 128 + row]);
-                    else sum += rd[(c * 2 + 1) * 128 + row];
-                }
+            if (hf == 0 && ok && !*abort_flag && !is_dustbin_row) {
+                float mm = m_run, sum = part;
+                if (ONLINE) lse2_merge(mm, sum, rd[row], rd[128 + row]);
+                else sum += rd[128 + row];
                 float outv = 0.f, ob = kNegInf;
                 if (lm != kNegInf) {
                     const bool d_act = D >= 0 && logm[D] != kNegInf;
                     if (ONLINE) {
-                        if (d_act) lse2_add(mm, sum, (a.sd_term[it.base + r] + a.colpot[pb + D]) * kLog2e);
+                        if (d_act) lse2_add(mm, sum, (a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e);
                         outv = lm - (mm + log2f(sum)) * kLn2;
                     } else {
-                        if (d_act) sum += ptx::ex2((a.sd_term[it.base + r] + a.colpot[pb + D]) * kLog2e + st2);
-                        outv = lm - log2f(sum) * kLn2 + st;
+                        const float dterm = d_act ? ptx::ex2((a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e + st2) : 0.f;
+                        if (WSUM) {
+                            if (d_act) sum = fmaf(dterm, a.colw[base + D], sum);
+                            outv = a.f[base + r] * a.hv[base + r] * sum;
+                        } else {
+                            outv = lm - log2f(sum + dterm) * kLn2 + st;
+                        }
                     }
                     if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
                     ob = outv * kLog2e;
                 }
                 a.out[pb + r] = outv;
-                a.out_bias2[it.base + r] = ob;
+                if (!WSUM) a.out_bias2[base + r] = ob;
             }
         }
     }
@@ -470,7 +592,7 @@ __global__ void __launch_bounds__(kLseThreads, 1)
 //   Out    O  = sum_c (P/a)_rc V_c                                   (forward output)
 //   C1     beta_R = sum_c Pt_rc dP_rc  and  dV = sum_c Pt_rc dO_c     (column sweep)
 //   R2     alpha_R = sum_c Pt dP + hv_r sum_c Pt m_c                  (row sweep)
-//   Stair  f_r * hv_r * sum_c P_rc m_c                                (staircase sweeps)
+//   Stair  f_r * hv_r * sum_c P_rc m_c   (staircase sweeps; run as weighted band sums by tc_band_kernel)
 //   Grad   dQ / dK = scale sum_c Pt_rc (dP_rc - sum_k xr_k yc_k) Y_c  (final sweeps)
 enum SweepMode { kModeOut = 0, kModeC1 = 1, kModeR2 = 2, kModeStair = 3, kModeGrad = 4 };
 
@@ -936,31 +1058,53 @@ int sm_count() {
     return n;
 }
 
-template <int DH, bool ONLINE>
-cudaError_t launch_lse_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const TcLseArgs& a, int grid,
-                               cudaStream_t st) {
-    constexpr size_t smem = LseCfg<DH>::SMEM;
-    cudaError_t e = set_smem(tc_lse_kernel<DH, ONLINE>, smem);
+template <int DH, int KIND>
+cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const TcBandArgs& a, int grid,
+                                cudaStream_t st) {
+    constexpr size_t smem = BandCfg<DH, KIND>::SMEM;
+    cudaError_t e = set_smem(tc_band_kernel<DH, KIND>, smem);
     if (e != cudaSuccess) return e;
-    tc_lse_kernel<DH, ONLINE><<<grid, kLseThreads, smem, st>>>(tmX, tmY, a);
+    tc_band_kernel<DH, KIND><<<grid, kBandThreads, smem, st>>>(tmX, tmY, a);
     return cudaGetLastError();
 }
 
-cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
-    const Geom& g = p.g;
-    if (!p.tile_bits) return cudaErrorInvalidValue;
+// Band row reduction over S = scale X Y^T (geometry, tile bits and the per-kind vectors in a).
+cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs a, int kind, cudaStream_t st) {
+    if (!a.tile_bits) return cudaErrorInvalidValue;
     CUtensorMap tmX, tmY;
     const uint64_t rows = uint64_t(g.BH) * g.L;
-    if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
-    TcLseArgs a{};
+    if (!make_map(&tmX, X, rows, g.d, 128) || !make_map(&tmY, Y, rows, g.d, 128)) return cudaErrorInvalidValue;
     a.H = g.H;
     a.L = g.L;
     a.h = g.h;
     a.D = g.D;
     a.sl2 = g.scale * kLog2e;
+    a.words = tile_words(g.L);
+    a.pairs_per_unit = (g.L / 128 + 1) / 2;
+    a.n_items = g.BH * a.pairs_per_unit;
+    const int grid = std::max(1, std::min(a.n_items, sm_count()));
+    a.items_per_cta = (a.n_items + grid - 1) / grid;
+    const int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
+    if (g.d == 128) {
+        switch (kind) {
+            case kBandOnline: return launch_band_variant<128, kBandOnline>(tmX, tmY, a, grid_used, st);
+            case kBandShift: return launch_band_variant<128, kBandShift>(tmX, tmY, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<128, kBandWsum>(tmX, tmY, a, grid_used, st);
+        }
+    } else {
+        switch (kind) {
+            case kBandOnline: return launch_band_variant<64, kBandOnline>(tmX, tmY, a, grid_used, st);
+            case kBandShift: return launch_band_variant<64, kBandShift>(tmX, tmY, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<64, kBandWsum>(tmX, tmY, a, grid_used, st);
+        }
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
+    TcBandArgs a{};
     a.logm = p.logm;
     a.tile_bits = p.tile_bits;
-    a.words = tile_words(g.L);
     a.colbias2 = p.colbias2;
     a.colpot = p.colpot;
     a.stab = p.stab;
@@ -969,18 +1113,8 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     a.pstride = p.pstride;
     a.sd_term = p.sd_term;
     a.status = p.status;
-    a.n_items = g.BH * (g.L / 128);
-    const int grid = std::max(1, std::min(a.n_items, sm_count()));
-    a.items_per_cta = (a.n_items + grid - 1) / grid;
-    const int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
-    cudaError_t e;
-    if (g.d == 128)
-        e = p.stab ? launch_lse_variant<128, false>(tmX, tmY, a, grid_used, st)
-                   : launch_lse_variant<128, true>(tmX, tmY, a, grid_used, st);
-    else
-        e = p.stab ? launch_lse_variant<64, false>(tmX, tmY, a, grid_used, st)
-                   : launch_lse_variant<64, true>(tmX, tmY, a, grid_used, st);
-    if (e != cudaSuccess || g.D < 0) return e;
+    cudaError_t e = launch_band(p.g, p.X, p.Y, a, p.stab ? kBandShift : kBandOnline, st);
+    if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
 }
 
@@ -1002,7 +1136,6 @@ cudaError_t launch_sweep_dh(int mode, int nmod, const CUtensorMap& tmX, const CU
         case kModeOut: return launch_sweep<DH, kModeOut, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
         case kModeC1: return launch_sweep<DH, kModeC1, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
         case kModeR2: return launch_sweep<DH, kModeR2, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-        case kModeStair: return launch_sweep<DH, kModeStair, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
         case kModeGrad:
             switch (nmod) {
                 case 0: return launch_sweep<DH, kModeGrad, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
@@ -1025,6 +1158,25 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     else if (!p.vout && p.sout && !p.s_dp && p.m) mode = kModeStair;
     else if (p.vout && !p.sout && p.v_dp && p.Z == p.Y) mode = kModeGrad;
     else return cudaErrorInvalidValue;
+    if (mode == kModeStair) {
+        // f_r hv_r sum_c Pt_rc m_c: a weighted band row sum with row shift pr and column bias pc
+        TcBandArgs a{};
+        a.logm = p.logm;
+        a.tile_bits = p.tile_bits;
+        a.colbias2 = p.pcm2;
+        a.colw = p.m;
+        a.colpot = p.pc;
+        a.stab = p.pr;
+        a.out = p.sout;
+        a.f = p.f;
+        a.hv = p.hv;
+        a.pstride = size_t(g.L);
+        a.sd_term = p.sd_term;
+        a.status = p.status;
+        cudaError_t e = launch_band(g, p.X, p.Y, a, kBandWsum, st);
+        if (e != cudaSuccess || g.D < 0) return e;
+        return launch_dustbin_bwd(p, st);
+    }
     // Modifier count rounded up to an instantiated one; the padding terms have xr = 0.
     int nmod = p.nmod;
     const int nmod_k = nmod == 0 ? 0 : nmod <= 2 ? 2 : nmod <= 4 ? 4 : nmod <= 8 ? 8 : 16;
