@@ -51,18 +51,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Bounded wait: true when the phase completed; false when the CTA is aborting or the
 // limit ran out (then the timeout bit is set and the abort flag raised).
+// The abort flag and the clock are looked at on every 8th failed attempt only, so that a
+// spinning warp takes few issue slots from the warps that do the work.
 constexpr uint64_t kWaitLimitNs = 100000000ull;  // 100 ms: far beyond any legitimate wait
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    while (true) {
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            atomicOr(status, kStatusTimeout);
-            return false;
+        if ((i & 7u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
         }
     }
 }
@@ -142,8 +146,8 @@ __device__ __forceinline__ void tmem_wait_ld(float (&v)[32]) {
         :
         : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld(float (&v)[32], float (&w)[32]) {
-    tmem_wait_ld(v);
+// Ties registers loaded before an earlier wait to that wait (emits no instruction).
+__device__ __forceinline__ void tmem_tie(float (&w)[32]) {
     uint32_t* r = reinterpret_cast<uint32_t*>(w);
     asm volatile(""
         : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
@@ -152,6 +156,10 @@ __device__ __forceinline__ void tmem_wait_ld(float (&v)[32], float (&w)[32]) {
           "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
         :
         : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(float (&v)[32], float (&w)[32]) {
+    tmem_wait_ld(v);
+    tmem_tie(w);
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 "version 1" layout).
@@ -235,6 +243,12 @@ __device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

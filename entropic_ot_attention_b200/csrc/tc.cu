@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
         float* red = reinterpret_cast<float*>(sm + C::OFF_RED) + G * (2 * 2 * 128);
-        const float* vbase = reinterpret_cast<const float*>(sm + C::OFF_V + G * C::NV * C::VB);
+        const uint32_t vsm = ptx::smem_u32(sm + C::OFF_V + G * C::NV * C::VB);
         int gt = 0, ep = 0;
         bool ok = true;
         for (int item = item0; item < item1; ++item) {
@@ -425,23 +425,23 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             float m_run = kNegInf;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             TileBits bits(bitp);
-            // one 32-column chunk: scores v -> partial sums
-            auto process = [&](const float (&v)[32], int c0, int chunk, const float* vec, bool interior) {
-                const float4* bias4 = reinterpret_cast<const float4*>(vec + chunk * 32);
-                const float4* w4 = reinterpret_cast<const float4*>(vec + C::BN + chunk * 32);
-                if (ONLINE || !interior) {
+            // One 32-column chunk starting at column cc: scores v -> partial sums.  The chunk's
+            // column bias (and weights) sit in shared memory at vaddr (and vaddr + 4 BN).
+            // masked: some entries of the chunk lie outside the band of their row.
+            auto process = [&](const float (&v)[32], int cc, uint32_t vaddr, bool masked) {
+                if (ONLINE || masked) {
                     float x[32];
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = bias4[j4];
+                        const float4 bv = ptx::ld_shared_f4(vaddr + 16u * j4);
                         x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
                         x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
                         x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
                         x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
                     }
-                    if (!interior) {
-                        // valid columns j of this chunk: r - h <= c0 + 32 chunk + j <= r + h
-                        const int lo = r - h - (c0 + chunk * 32), hi = r + h - (c0 + chunk * 32);
+                    if (masked) {
+                        // valid columns j of this chunk: r - h <= cc + j <= r + h
+                        const int lo = r - h - cc, hi = r + h - cc;
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
                             if (j < lo || j > hi) x[j] = kNegInf;
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     } else if (WSUM) {
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4) {
-                            const float4 wv = w4[j4];
+                            const float4 wv = ptx::ld_shared_f4(vaddr + 4u * C::BN + 16u * j4);
                             acc[0] = fmaf(ptx::ex2(x[4 * j4 + 0] + st2), wv.x, acc[0]);
                             acc[1] = fmaf(ptx::ex2(x[4 * j4 + 1] + st2), wv.y, acc[1]);
                             acc[2] = fmaf(ptx::ex2(x[4 * j4 + 2] + st2), wv.z, acc[2]);
@@ -474,13 +474,13 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                         for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] + st2);
                     }
                 } else {
-                    // interior tile, shifted: packed fp32x2 math
+                    // every entry inside the band, shifted: packed fp32x2 math
                     const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = bias4[j4];
+                        const float4 bv = ptx::ld_shared_f4(vaddr + 16u * j4);
                         float4 wv;
-                        if (WSUM) wv = w4[j4];
+                        if (WSUM) wv = ptx::ld_shared_f4(vaddr + 4u * C::BN + 16u * j4);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int k = 2 * j4 + hh;
@@ -506,35 +506,47 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     }
                 }
             };
+            // Band position of a 32 x 32 block (this warp's rows, one 32-column chunk): 0 =
+            // outside the band for every row (skipped: no TMEM read, no exponentials),
+            // 1 = inside for every entry, 2 = cut by the band edge (masked per entry).
+            const int rw = rg + q * 32;
+            auto block_class = [&](int cc) {
+                const int dmin = cc - (rw + 31), dmax = cc + 31 - rw;   // range of c - r
+                if (dmin > h || dmax < -h) return 0;
+                return (dmax <= h && dmin >= -h) ? 1 : 2;
+            };
             for (int t = t_lo; t <= t_hi; ++t) {
                 if (!bits(t)) continue;
                 const int gg = gt++;
                 if (!ok) continue;
                 const int c0 = t * C::BN;
                 const int tb = gg & 1, vs = gg % C::NV;
-                const bool interior = (c0 + C::BN - 1 - rg <= h) && (rg + C::BM - 1 - c0 <= h);
+                const int cc0 = c0 + hf * 64, cc1 = cc0 + 32;
+                const int k0 = block_class(cc0), k1 = block_class(cc1);
                 // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
                 bool w1 = ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
                 bool w2 = w1 && ptx::mbar_wait(tfull(G, tb), (gg >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
                 ptx::tc_fence_after();
-                const float* vec = vbase + vs * (C::VB / 4);
+                const uint32_t vaddr = vsm + uint32_t(vs) * C::VB + uint32_t(hf) * 256u;
                 const uint32_t tcol = tbase + lane_base + uint32_t((G * 2 + tb) * C::BN + hf * 64);
-                {
+                if (k0 != 0) {
                     float v[32];
                     ptx::tmem_ld32(tcol, v);
                     ptx::tmem_wait_ld(v);
-                    process(v, c0, 2 * hf, vec, interior);
+                    process(v, cc0, vaddr, k0 == 2);
                 }
                 {
                     float v[32];
-                    ptx::tmem_ld32(tcol + 32, v);
-                    ptx::tmem_wait_ld(v);
+                    if (k1 != 0) {
+                        ptx::tmem_ld32(tcol + 32, v);
+                        ptx::tmem_wait_ld(v);
+                    }
                     // this warp's part of the accumulator is read: hand it back
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(tempty(G, tb));
-                    process(v, c0, 2 * hf + 1, vec, interior);
+                    if (k1 != 0) process(v, cc1, vaddr + 128u, k1 == 2);
                 }
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(vempty(G, vs));
