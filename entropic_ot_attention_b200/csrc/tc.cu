@@ -882,7 +882,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
             if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
             ptx::tc_fence_after();
-            const float* cv = reinterpret_cast<const float*>(sm + C::OFF_V + s * C::VB);
+            // column vectors of this stage (explicit shared-memory loads: the aligned base
+            // pointer no longer carries the address space)
+            const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
+            auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
             float v[32], w[32];
             ptx::tmem_ld32(tbase + lane_base + C::TM_S + uint32_t(bb * C::BN + cc0), v);
             if (M::HASDP) {
@@ -895,10 +898,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty(bb));
             // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
-            const float4* pc4 = reinterpret_cast<const float4*>(cv + cc0);
 #pragma unroll
             for (int j4 = 0; j4 < 8; ++j4) {
-                const float4 b4 = pc4[j4];
+                const float4 b4 = cvec(0, cc0 + 4 * j4);
                 uint64_t x0 = ptx::ffma2(ptx::f2(v[4 * j4 + 0], v[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
                 uint64_t x1 = ptx::ffma2(ptx::f2(v[4 * j4 + 2], v[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
                 ptx::f2split(x0, v[4 * j4 + 0], v[4 * j4 + 1]);
@@ -920,7 +922,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     const uint64_t P2 = ptx::f2(v[2 * k], v[2 * k + 1]);
                     if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(w[2 * k], w[2 * k + 1]), s1a[k & 1]);
                     if (M::SM) {
-                        const float4 mv = reinterpret_cast<const float4*>(cv + VOFF_M * C::BN + cc0)[k >> 1];
+                        const float4 mv = cvec(VOFF_M, cc0 + 4 * (k >> 1));
                         s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
                     }
                 }
@@ -934,7 +936,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     uint64_t cf1 = M::VDP ? ptx::f2(w[4 * k4 + 2], w[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
 #pragma unroll
                     for (int mm = 0; mm < NMOD; ++mm) {
-                        const float4 yv = reinterpret_cast<const float4*>(cv + (VOFF_Y + mm) * C::BN + cc0)[k4];
+                        const float4 yv = cvec(VOFF_Y + mm, cc0 + 4 * k4);
                         const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
                         cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
                         cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
