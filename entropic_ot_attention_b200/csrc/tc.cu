@@ -661,14 +661,16 @@ struct SweepCfg {
     static constexpr uint32_t OFF_V = OFF_C + 2 * CB;
     static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2][2][128] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
-    // full[NS] empty[NS] xfull tfull[2] tempty[2] cfull[2] cempty[2] accfull
-    static constexpr uint32_t NBARS = 2 * NS + 1 + 8 + 1;
+    // full[NS] empty[NS] xfull tfull[2] tempty[2] cfull[2] cempty[2] accfull xtm
+    static constexpr uint32_t NBARS = 2 * NS + 1 + 8 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
     static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
     static constexpr uint32_t IDESC_S = ptx::idesc_bf16(128, 64, false, false);
     static constexpr uint32_t IDESC_O = ptx::idesc_bf16(128, DH, false, true);
-    static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256;
+    // TMEM columns: S and dP tiles (double-buffered), the d-wide accumulator, and the row
+    // tiles X and A as MMA A operands (one row per lane, two bf16 per column)
+    static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256, TM_X = 384, TM_A = 448;
 };
 
 template <int DH, int MODE, int NMOD>
@@ -698,6 +700,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
     auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 7 + i); };
     const uint32_t accfull = bar0 + 8u * (2 * C::NS + 9);
+    const uint32_t xtm = bar0 + 8u * (2 * C::NS + 10);   // row tiles copied into TMEM
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
@@ -730,6 +733,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::mbar_init(cempty(i), 1);
         }
         ptx::mbar_init(accfull, 1);
+        ptx::mbar_init(xtm, 8);
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
@@ -789,8 +793,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- score MMA issuer: S (and dP) tiles ----------------
-            const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
-            bool ok = ptx::mbar_wait(xfull, 0, abort_flag, a.status);
+            bool ok = ptx::mbar_wait(xtm, 0, abort_flag, a.status);
+            ptx::tc_fence_after();
             int issued = 0;
             for (int it = 0; it < n && ok; ++it) {
                 const int s = it % C::NS, bb = it & 1;
@@ -799,20 +803,19 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 ptx::tc_fence_after();
                 const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
                 const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
+                // A operands (row tiles) from TMEM: 8 columns per K step of 16
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk) {
-                    const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
                     const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                    ptx::mma_bf16(tbase + C::TM_S + bb * C::BN, ptx::smem_desc(xs + xo, 16, 1024),
-                                  ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+                    ptx::mma_bf16_ts(tbase + C::TM_S + bb * C::BN, tbase + C::TM_X + uint32_t(kk * 8),
+                                     ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 if (M::HASDP) {
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk) {
-                        const uint32_t xo = (kk >> 2) * C::XATOM + (kk & 3) * 32;
                         const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                        ptx::mma_bf16(tbase + C::TM_DP + bb * C::BN, ptx::smem_desc(as + xo, 16, 1024),
-                                      ptx::smem_desc(ws + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+                        ptx::mma_bf16_ts(tbase + C::TM_DP + bb * C::BN, tbase + C::TM_A + uint32_t(kk * 8),
+                                         ptx::smem_desc(ws + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
                     }
                 }
                 ptx::mma_commit(tfull(bb));
@@ -872,6 +875,35 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         bool ok = true;
         const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
         const int cc0 = half * 32;
+        {
+            // Row tiles into TMEM as MMA A operands: warp (q, half 0) copies X, (q, half 1) A,
+            // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
+            const bool copy = half == 0 || M::HASDP;
+            bool okx = !copy || ptx::mbar_wait(xfull, 0, abort_flag, a.status);
+            okx = __all_sync(0xffffffffu, okx);
+            if (okx && copy) {
+                const uint32_t src = ptx::smem_u32(sm + (half ? C::OFF_A : 0u)) + crow;
+                const uint32_t dst = tbase + lane_base + (half ? C::TM_A : C::TM_X);
+#pragma unroll
+                for (int ka = 0; ka < C::KATOMS; ++ka) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 u = ptx::ld_shared_u4(src + ka * C::XATOM + ((uint32_t(j) ^ uint32_t(row & 7)) << 4));
+                        w[4 * j] = u.x;
+                        w[4 * j + 1] = u.y;
+                        w[4 * j + 2] = u.z;
+                        w[4 * j + 3] = u.w;
+                    }
+                    ptx::tmem_st32(dst + uint32_t(ka * 32), w);
+                }
+                ptx::tmem_wait_st();
+            }
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(xtm);
+            if (!okx) ok = false;
+        }
         for (int it = 0; it < n; ++it) {
             const int s = it % C::NS, bb = it & 1, cb = it & 1;
             const int c0 = tiles[it] * C::BN;
