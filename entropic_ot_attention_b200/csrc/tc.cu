@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// Output / backward sweep, 128-row x 64-column tiles
+// Output / backward sweep, 128 x 128 tiles
 // ---------------------------------------------------------------------------------------
 // Pass kinds (compile-time, so that each variant carries only its own arithmetic):
 //   Out    O  = sum_c (P/a)_rc V_c                                   (forward output)
@@ -645,31 +645,34 @@ constexpr int kSweepThreads = 352;   // TMA warp, score-MMA warp, 8 epilogue war
 
 template <int DH, int NV>
 struct SweepCfg {
-    static constexpr int BM = 128, BN = 64;
+    static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
-    static constexpr int NS = 3;
+    static constexpr int NS = 2;
     static constexpr uint32_t XB = BM * DH * 2;          // row tile bytes
     static constexpr uint32_t YB = BN * DH * 2;          // column tile bytes
-    static constexpr uint32_t XATOM = BM * 128;          // 16 KB
-    static constexpr uint32_t YATOM = BN * 128;          // 8 KB
-    static constexpr uint32_t CB = BM * BN * 2;          // coefficient tile bytes (16 KB)
+    static constexpr uint32_t XATOM = BM * 128;          // one 64-element atom column of a row tile
+    static constexpr uint32_t YATOM = BN * 128;          // ... of a column tile
+    static constexpr uint32_t CB = BM * BN * 2;          // coefficient tile bytes (32 KB)
+    static constexpr uint32_t CATOM = BM * 128;          // one 64-column atom of a coefficient tile
     static constexpr uint32_t VB = NV * BN * 4;          // column vector bytes per stage
-    static constexpr uint32_t OFF_A = XB;
-    static constexpr uint32_t OFF_Y = 2 * XB;
+    // The row tiles X and A land (TMA) in the coefficient buffers and are moved into TMEM
+    // before the first coefficient is written.
+    static constexpr uint32_t OFF_C = 0;
+    static constexpr uint32_t OFF_Y = 2 * CB;
     static constexpr uint32_t OFF_W = OFF_Y + NS * YB;
-    static constexpr uint32_t OFF_C = OFF_W + NS * YB;
-    static constexpr uint32_t OFF_V = OFF_C + 2 * CB;
+    static constexpr uint32_t OFF_V = OFF_W + NS * YB;
     static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2][2][128] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
-    // full[NS] empty[NS] xfull tfull[2] tempty[2] cfull[2] cempty[2] accfull xtm
-    static constexpr uint32_t NBARS = 2 * NS + 1 + 8 + 1 + 1;
+    // full[NS] empty[NS] xfull tfull tempty cfull[2] cempty[2] accfull xtm
+    static constexpr uint32_t NBARS = 2 * NS + 1 + 2 + 4 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
     static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
-    static constexpr uint32_t IDESC_S = ptx::idesc_bf16(128, 64, false, false);
+    static constexpr uint32_t IDESC_S = ptx::idesc_bf16(128, BN, false, false);
     static constexpr uint32_t IDESC_O = ptx::idesc_bf16(128, DH, false, true);
-    // TMEM columns: S and dP tiles (double-buffered), the d-wide accumulator, and the row
-    // tiles X and A as MMA A operands (one row per lane, two bf16 per column)
+    // TMEM columns: the S and dP tiles (one buffer each: the epilogue reads a whole tile into
+    // registers before any arithmetic and hands it back at once), the d-wide accumulator, and
+    // the row tiles X and A as MMA A operands (one row per lane, two bf16 per column)
     static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256, TM_X = 384, TM_A = 448;
 };
 
@@ -695,12 +698,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (C::NS + s); };
     const uint32_t xfull = bar0 + 8u * (2 * C::NS);
-    auto tfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 1 + i); };
-    auto tempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
-    auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
-    auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 7 + i); };
-    const uint32_t accfull = bar0 + 8u * (2 * C::NS + 9);
-    const uint32_t xtm = bar0 + 8u * (2 * C::NS + 10);   // row tiles copied into TMEM
+    const uint32_t tfull = bar0 + 8u * (2 * C::NS + 1);
+    const uint32_t tempty = bar0 + 8u * (2 * C::NS + 2);
+    auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
+    auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
+    const uint32_t accfull = bar0 + 8u * (2 * C::NS + 7);
+    const uint32_t xtm = bar0 + 8u * (2 * C::NS + 8);   // row tiles copied into TMEM
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
@@ -726,9 +729,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::mbar_init(empty(s), 9);   // MMA commit + 8 epilogue warps
         }
         ptx::mbar_init(xfull, 1);
+        ptx::mbar_init(tfull, 1);
+        ptx::mbar_init(tempty, 8);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(tfull(i), 1);
-            ptx::mbar_init(tempty(i), 8);
             ptx::mbar_init(cfull(i), 8);
             ptx::mbar_init(cempty(i), 1);
         }
@@ -752,7 +755,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::prefetch_tmap(&tmY);
             if (M::HASDP) ptx::prefetch_tmap(&tmA);
             if (M::W2) ptx::prefetch_tmap(&tmW);
-            const uint32_t xs = ptx::smem_u32(sm), as = ptx::smem_u32(sm + C::OFF_A);
+            const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
             ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1));
             for (int ka = 0; ka < C::KATOMS; ++ka) {
                 ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
@@ -797,9 +800,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::tc_fence_after();
             int issued = 0;
             for (int it = 0; it < n && ok; ++it) {
-                const int s = it % C::NS, bb = it & 1;
+                const int s = it % C::NS;
                 if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
-                if (!ptx::mbar_wait(tempty(bb), ((it >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                if (!ptx::mbar_wait(tempty, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
                 const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
@@ -807,24 +810,24 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk) {
                     const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                    ptx::mma_bf16_ts(tbase + C::TM_S + bb * C::BN, tbase + C::TM_X + uint32_t(kk * 8),
+                    ptx::mma_bf16_ts(tbase + C::TM_S, tbase + C::TM_X + uint32_t(kk * 8),
                                      ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 if (M::HASDP) {
 #pragma unroll
                     for (int kk = 0; kk < DH / 16; ++kk) {
                         const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                        ptx::mma_bf16_ts(tbase + C::TM_DP + bb * C::BN, tbase + C::TM_A + uint32_t(kk * 8),
+                        ptx::mma_bf16_ts(tbase + C::TM_DP, tbase + C::TM_A + uint32_t(kk * 8),
                                          ptx::smem_desc(ws + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
                     }
                 }
-                ptx::mma_commit(tfull(bb));
+                ptx::mma_commit(tfull);
                 if (!M::VEC) ptx::mma_commit(empty(s));   // vector passes free the stage after the product
                 issued = it + 1;
             }
             if (*abort_flag && issued > 0) {
                 volatile int dummy = 0;
-                ptx::mbar_wait(tfull((issued - 1) & 1), ((issued - 1) >> 1) & 1, &dummy, a.status);
+                ptx::mbar_wait(tfull, (issued - 1) & 1, &dummy, a.status);
             }
         }
     } else if (warp == 10) {
@@ -843,7 +846,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
-                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + kk * 32, 16, 1024),
+                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + (kk >> 2) * C::CATOM + (kk & 3) * 32, 16, 1024),
                                   ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
                                   (j > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(cempty(cb));
@@ -859,7 +862,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     } else {
         // ---------------- epilogue: warps 2..9, two per TMEM lane quadrant ----------------
         const int q = warp & 3;                  // lane quadrant
-        const int half = (warp - 2) >> 2;        // which 32 columns of each 64-column tile
+        const int half = (warp - 2) >> 2;        // which 64 columns of each 128-column tile
         const int row = q * 32 + lane, r = r0 + row;
         const float lm = logm[r];
         const bool ract = lm != kNegInf;
@@ -874,7 +877,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         uint64_t s2a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
         bool ok = true;
         const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
-        const int cc0 = half * 32;
         {
             // Row tiles into TMEM as MMA A operands: warp (q, half 0) copies X, (q, half 1) A,
             // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
@@ -882,7 +884,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             bool okx = !copy || ptx::mbar_wait(xfull, 0, abort_flag, a.status);
             okx = __all_sync(0xffffffffu, okx);
             if (okx && copy) {
-                const uint32_t src = ptx::smem_u32(sm + (half ? C::OFF_A : 0u)) + crow;
+                const uint32_t src = ptx::smem_u32(sm + C::OFF_C + (half ? C::XB : 0u)) + crow;
                 const uint32_t dst = tbase + lane_base + (half ? C::TM_A : C::TM_X);
 #pragma unroll
                 for (int ka = 0; ka < C::KATOMS; ++ka) {
@@ -903,14 +905,16 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(xtm);
             if (!okx) ok = false;
+            // every warp has read its rows of X and A before any coefficient overwrites them
+            ptx::named_bar_sync(2, 256);
         }
         for (int it = 0; it < n; ++it) {
-            const int s = it % C::NS, bb = it & 1, cb = it & 1;
+            const int s = it % C::NS, cb = it & 1;
             const int c0 = tiles[it] * C::BN;
             const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
             // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
             bool w1 = ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status);
-            bool w2 = w1 && ptx::mbar_wait(tfull(bb), (it >> 1) & 1, abort_flag, a.status);
+            bool w2 = w1 && ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
             bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
             if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -918,76 +922,89 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             // pointer no longer carries the address space)
             const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
             auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
-            float v[32], w[32];
-            ptx::tmem_ld32(tbase + lane_base + C::TM_S + uint32_t(bb * C::BN + cc0), v);
+            // this warp's 64 columns of S (and dP), read whole; the buffer goes back at once
+            float v[2][32], w[2][32];
+            const uint32_t tl = tbase + lane_base + uint32_t(half * 64);
+            ptx::tmem_ld32(tl + C::TM_S, v[0]);
+            ptx::tmem_ld32(tl + C::TM_S + 32, v[1]);
             if (M::HASDP) {
-                ptx::tmem_ld32(tbase + lane_base + C::TM_DP + uint32_t(bb * C::BN + cc0), w);
-                ptx::tmem_wait_ld(v, w);
-            } else {
-                ptx::tmem_wait_ld(v);
+                ptx::tmem_ld32(tl + C::TM_DP, w[0]);
+                ptx::tmem_ld32(tl + C::TM_DP + 32, w[1]);
+            }
+            ptx::tmem_wait_ld(v[0], v[1]);
+            if (M::HASDP) {
+                ptx::tmem_tie(w[0]);
+                ptx::tmem_tie(w[1]);
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(tempty(bb));
-            // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
+            if (lane == 0) ptx::mbar_arrive(tempty);
+            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(half) * C::CATOM + crow;
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-                const float4 b4 = cvec(0, cc0 + 4 * j4);
-                uint64_t x0 = ptx::ffma2(ptx::f2(v[4 * j4 + 0], v[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
-                uint64_t x1 = ptx::ffma2(ptx::f2(v[4 * j4 + 2], v[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
-                ptx::f2split(x0, v[4 * j4 + 0], v[4 * j4 + 1]);
-                ptx::f2split(x1, v[4 * j4 + 2], v[4 * j4 + 3]);
-            }
-            if (!interior) {
-                const int dlt0 = c0 + cc0 - r;
+            for (int ch = 0; ch < 2; ++ch) {
+                const int cc0 = half * 64 + ch * 32;
+                float (&vc)[32] = v[ch];
+                float (&wc)[32] = w[ch];
+                // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int dl = dlt0 + j;
-                    if (dl < -h || dl > h) v[j] = kNegInf;
+                for (int j4 = 0; j4 < 8; ++j4) {
+                    const float4 b4 = cvec(0, cc0 + 4 * j4);
+                    uint64_t x0 = ptx::ffma2(ptx::f2(vc[4 * j4 + 0], vc[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
+                    uint64_t x1 = ptx::ffma2(ptx::f2(vc[4 * j4 + 2], vc[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
+                    ptx::f2split(x0, vc[4 * j4 + 0], vc[4 * j4 + 1]);
+                    ptx::f2split(x1, vc[4 * j4 + 2], vc[4 * j4 + 3]);
                 }
-            }
+                if (!interior) {
+                    const int dlt0 = c0 + cc0 - r;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = ptx::ex2(v[j]);
-            if (M::SCAL) {
+                    for (int j = 0; j < 32; ++j) {
+                        const int dl = dlt0 + j;
+                        if (dl < -h || dl > h) vc[j] = kNegInf;
+                    }
+                }
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const uint64_t P2 = ptx::f2(v[2 * k], v[2 * k + 1]);
-                    if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(w[2 * k], w[2 * k + 1]), s1a[k & 1]);
-                    if (M::SM) {
-                        const float4 mv = cvec(VOFF_M, cc0 + 4 * (k >> 1));
-                        s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
+                for (int j = 0; j < 32; ++j) vc[j] = ptx::ex2(vc[j]);
+                if (M::SCAL) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const uint64_t P2 = ptx::f2(vc[2 * k], vc[2 * k + 1]);
+                        if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(wc[2 * k], wc[2 * k + 1]), s1a[k & 1]);
+                        if (M::SM) {
+                            const float4 mv = cvec(VOFF_M, cc0 + 4 * (k >> 1));
+                            s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
+                        }
+                    }
+                }
+                if (M::VEC) {
+                    // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        uint64_t cf0 = M::VDP ? ptx::f2(wc[4 * k4], wc[4 * k4 + 1]) : ptx::f2(1.f, 1.f);
+                        uint64_t cf1 = M::VDP ? ptx::f2(wc[4 * k4 + 2], wc[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
+#pragma unroll
+                        for (int mm = 0; mm < NMOD; ++mm) {
+                            const float4 yv = cvec(VOFF_Y + mm, cc0 + 4 * k4);
+                            const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
+                            cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
+                            cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
+                        }
+                        float c0f, c1f, c2f, c3f;
+                        ptx::f2split(cf0, c0f, c1f);
+                        ptx::f2split(cf1, c2f, c3f);
+                        pk[2 * k4] = ptx::pack_bf16(vc[4 * k4] * c0f, vc[4 * k4 + 1] * c1f);
+                        pk[2 * k4 + 1] = ptx::pack_bf16(vc[4 * k4 + 2] * c2f, vc[4 * k4 + 3] * c3f);
+                    }
+                    // 128-byte-swizzled K-major tile: 16-byte unit u of a row at (u ^ (row & 7))
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t unit = uint32_t(ch * 4 + t);
+                        ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1],
+                                          pk[4 * t + 2], pk[4 * t + 3]);
                     }
                 }
             }
-            if (M::VEC) {
-                // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
-                uint32_t pk[16];
-#pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {
-                    uint64_t cf0 = M::VDP ? ptx::f2(w[4 * k4], w[4 * k4 + 1]) : ptx::f2(1.f, 1.f);
-                    uint64_t cf1 = M::VDP ? ptx::f2(w[4 * k4 + 2], w[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
-#pragma unroll
-                    for (int mm = 0; mm < NMOD; ++mm) {
-                        const float4 yv = cvec(VOFF_Y + mm, cc0 + 4 * k4);
-                        const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
-                        cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
-                        cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
-                    }
-                    float c0f, c1f, c2f, c3f;
-                    ptx::f2split(cf0, c0f, c1f);
-                    ptx::f2split(cf1, c2f, c3f);
-                    pk[2 * k4] = ptx::pack_bf16(v[4 * k4] * c0f, v[4 * k4 + 1] * c1f);
-                    pk[2 * k4 + 1] = ptx::pack_bf16(v[4 * k4 + 2] * c2f, v[4 * k4 + 3] * c3f);
-                }
-                const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + crow;
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const uint32_t unit = uint32_t(half * 4 + t);
-                    ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1], pk[4 * t + 2],
-                                      pk[4 * t + 3]);
-                }
-                ptx::fence_proxy_async_smem();
-            }
+            if (M::VEC) ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 ptx::mbar_arrive(empty(s));
@@ -1231,9 +1248,9 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     const void* w2 = has_dp ? p.Bm : (mode == kModeOut ? p.Z : nullptr);
     const uint64_t rows = uint64_t(g.BH) * g.L;
     CUtensorMap tmX, tmA, tmY, tmW;
-    if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
+    if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
     if (!make_map(&tmA, has_dp ? p.A : p.X, rows, g.d, 128)) return cudaErrorInvalidValue;
-    if (!make_map(&tmW, w2 ? w2 : p.Y, rows, g.d, 64)) return cudaErrorInvalidValue;
+    if (!make_map(&tmW, w2 ? w2 : p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
     TcVecArgs a{};
     a.H = g.H;
     a.L = g.L;
@@ -1258,7 +1275,7 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.sd_term = p.sd_term;
     a.dp_term = p.dp_term;
     a.status = p.status;
-    const int mt = max_tiles_for(g.L, g.h, 128, 64);
+    const int mt = max_tiles_for(g.L, g.h, 128, 128);
     dim3 grid(g.L / 128, g.BH);
     cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st)
                                : launch_sweep_dh<64>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st);
