@@ -64,6 +64,8 @@ int resolve_impl(const eot_problem& p) {
     Geom g{};
     g.d = p.d;
     g.dtype = p.dtype;
+    g.L = p.L;
+    g.h = p.W / 2;
     const bool tc = tensor_core_ok(p) && tc_supported(g);
     if (p.impl == EOT_IMPL_TCGEN05) return tc ? EOT_IMPL_TCGEN05 : -1;
     return tc ? EOT_IMPL_TCGEN05 : EOT_IMPL_SIMT;

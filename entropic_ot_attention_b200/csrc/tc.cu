@@ -1110,7 +1110,14 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 
 }  // namespace
 
-bool tc_supported(const Geom& g) { return g.dtype == EOT_BF16 && (g.d == 64 || g.d == 128) && encode_fn() != nullptr; }
+// The sweep kernel keeps its band's tile list in shared memory: very wide bands (W beyond
+// about 2e5) do not fit next to the tiles and run on the CUDA-core kernels instead.
+constexpr size_t kMaxSmem = 227 * 1024;
+bool tc_supported(const Geom& g) {
+    if (g.dtype != EOT_BF16 || (g.d != 64 && g.d != 128) || encode_fn() == nullptr) return false;
+    const int mt = max_tiles_for(g.L, g.h, 128, 128);
+    return SweepCfg<128, 1 + kMaxMods>::smem_bytes(mt) <= kMaxSmem;
+}
 
 int sm_count() {
     static int n = [] {

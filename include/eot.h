@@ -61,8 +61,10 @@ typedef enum {
 typedef enum { EOT_FP32 = 0, EOT_BF16 = 1 } eot_dtype;
 
 /* Kernel family.  AUTO picks the tensor-core (tcgen05/TMA) kernels for bf16 with d in
- * {64, 128} and the CUDA-core kernels otherwise (fp32 is always computed on CUDA cores,
- * in fp32, so that its scores keep full fp32 precision). */
+ * {64, 128} and a band that fits their shared-memory tile list (W below about 2e5), and the
+ * CUDA-core kernels otherwise (fp32 is always computed on CUDA cores, in fp32, so that its
+ * scores keep full fp32 precision).  TCGEN05 on a problem outside that range is
+ * EOT_ERR_UNSUPPORTED. */
 typedef enum { EOT_IMPL_AUTO = 0, EOT_IMPL_SIMT = 1, EOT_IMPL_TCGEN05 = 2 } eot_impl;
 
 typedef struct {

@@ -159,3 +159,17 @@ def test_workload_parity(name):
     case = eot_inputs.workload(name)
     units = None if name == "tiny" else WORKLOAD_UNITS[name]
     _check(case, "auto", units=units, banded=name != "tiny")
+
+
+def test_kernel_family_selection():
+    """bf16 with d in {64, 128} runs on the tensor-core kernels unless the band's tile list
+    would not fit in shared memory; then AUTO picks the CUDA-core kernels and an explicit
+    tensor-core request is refused before anything runs."""
+    import torch
+    from entropic_ot_attention_b200 import _abi, api
+    p = api.make_problem(1, 4, 131072, 128, 1024, 10, 2, torch.bfloat16, 0.0, None, 0.0)
+    assert _abi.eot_resolved_impl(p) == 2
+    wide = api.make_problem(1, 1, 1 << 20, 128, 500000, 1, 1, torch.bfloat16, 0.0, None, 0.0)
+    assert _abi.eot_resolved_impl(wide) == 1
+    wide_tc = api.make_problem(1, 1, 1 << 20, 128, 500000, 1, 1, torch.bfloat16, 0.0, None, 0.0, impl="tcgen05")
+    assert _abi.eot_validate(wide_tc) == 2   # EOT_ERR_UNSUPPORTED
