@@ -641,7 +641,8 @@ struct TcVecArgs {
     uint32_t* status;
 };
 
-constexpr int kSweepThreads = 352;   // TMA warp, score-MMA warp, 8 epilogue warps, product-MMA warp
+constexpr int kSweepEpi = 16;         // epilogue warps: four per TMEM lane quadrant, 32 columns each
+constexpr int kSweepThreads = 32 * (3 + kSweepEpi);   // TMA warp, score-MMA warp, epilogue warps, product-MMA warp
 
 template <int DH, int NV>
 struct SweepCfg {
@@ -661,8 +662,8 @@ struct SweepCfg {
     static constexpr uint32_t OFF_Y = 2 * CB;
     static constexpr uint32_t OFF_W = OFF_Y + NS * YB;
     static constexpr uint32_t OFF_V = OFF_W + NS * YB;
-    static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2][2][128] scalar partials
-    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 128 * 4;
+    static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2 sums][4 quarters][128 rows] scalar partials
+    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 128 * 4;
     // full[NS] empty[NS] xfull tfull tempty cfull[2] cempty[2] accfull xtm
     static constexpr uint32_t NBARS = 2 * NS + 1 + 2 + 4 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
@@ -726,17 +727,17 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::NS; ++s) {
             ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 9);   // MMA commit + 8 epilogue warps
+            ptx::mbar_init(empty(s), 1 + kSweepEpi);   // MMA commit + epilogue warps
         }
         ptx::mbar_init(xfull, 1);
         ptx::mbar_init(tfull, 1);
-        ptx::mbar_init(tempty, 8);
+        ptx::mbar_init(tempty, kSweepEpi);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(cfull(i), 8);
+            ptx::mbar_init(cfull(i), kSweepEpi);
             ptx::mbar_init(cempty(i), 1);
         }
         ptx::mbar_init(accfull, 1);
-        ptx::mbar_init(xtm, 8);
+        ptx::mbar_init(xtm, kSweepEpi);
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
@@ -830,7 +831,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 ptx::mbar_wait(tfull, (issued - 1) & 1, &dummy, a.status);
             }
         }
-    } else if (warp == 10) {
+    } else if (warp == 2 + kSweepEpi) {
         if (M::VEC && lane == 0) {
             // ---------------- product MMA issuer: acc += coef(j) * Z(j) ----------------
             // A thread of its own, so that score tiles are never queued behind a product
@@ -860,9 +861,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: warps 2..9, two per TMEM lane quadrant ----------------
+        // ---------------- epilogue: warps 2..17, four per TMEM lane quadrant ----------------
         const int q = warp & 3;                  // lane quadrant
-        const int half = (warp - 2) >> 2;        // which 64 columns of each 128-column tile
+        const int qt = (warp - 2) >> 2;          // which 32 columns of each 128-column tile
+        const int half = qt;                     // (quarters 0, 1 also read back the accumulator halves)
         const int row = q * 32 + lane, r = r0 + row;
         const float lm = logm[r];
         const bool ract = lm != kNegInf;
@@ -878,9 +880,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         bool ok = true;
         const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
         {
-            // Row tiles into TMEM as MMA A operands: warp (q, half 0) copies X, (q, half 1) A,
+            // Row tiles into TMEM as MMA A operands: warp (q, quarter 0) copies X, (q, quarter 1) A,
             // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
-            const bool copy = half == 0 || M::HASDP;
+            const bool copy = qt == 0 || (qt == 1 && M::HASDP);
             bool okx = !copy || ptx::mbar_wait(xfull, 0, abort_flag, a.status);
             okx = __all_sync(0xffffffffu, okx);
             if (okx && copy) {
@@ -906,7 +908,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             if (lane == 0) ptx::mbar_arrive(xtm);
             if (!okx) ok = false;
             // every warp has read its rows of X and A before any coefficient overwrites them
-            ptx::named_bar_sync(2, 256);
+            ptx::named_bar_sync(2, 32 * kSweepEpi);
         }
         for (int it = 0; it < n; ++it) {
             const int s = it % C::NS, cb = it & 1;
@@ -922,27 +924,20 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             // pointer no longer carries the address space)
             const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
             auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
-            // this warp's 64 columns of S (and dP), read whole; the buffer goes back at once
-            float v[2][32], w[2][32];
-            const uint32_t tl = tbase + lane_base + uint32_t(half * 64);
+            // this warp's 32 columns of S (and dP), read whole; the buffer goes back at once
+            float v[1][32], w[1][32];
+            const uint32_t tl = tbase + lane_base + uint32_t(qt * 32);
             ptx::tmem_ld32(tl + C::TM_S, v[0]);
-            ptx::tmem_ld32(tl + C::TM_S + 32, v[1]);
-            if (M::HASDP) {
-                ptx::tmem_ld32(tl + C::TM_DP, w[0]);
-                ptx::tmem_ld32(tl + C::TM_DP + 32, w[1]);
-            }
-            ptx::tmem_wait_ld(v[0], v[1]);
-            if (M::HASDP) {
-                ptx::tmem_tie(w[0]);
-                ptx::tmem_tie(w[1]);
-            }
+            if (M::HASDP) ptx::tmem_ld32(tl + C::TM_DP, w[0]);
+            ptx::tmem_wait_ld(v[0]);
+            if (M::HASDP) ptx::tmem_tie(w[0]);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty);
-            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(half) * C::CATOM + crow;
+            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(qt >> 1) * C::CATOM + crow;
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-                const int cc0 = half * 64 + ch * 32;
+            for (int ch = 0; ch < 1; ++ch) {
+                const int cc0 = qt * 32;
                 float (&vc)[32] = v[ch];
                 float (&wc)[32] = w[ch];
                 // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
@@ -998,7 +993,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     // 128-byte-swizzled K-major tile: 16-byte unit u of a row at (u ^ (row & 7))
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
-                        const uint32_t unit = uint32_t(ch * 4 + t);
+                        const uint32_t unit = uint32_t((qt & 1) * 4 + t);
                         ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1],
                                           pk[4 * t + 2], pk[4 * t + 3]);
                     }
@@ -1011,16 +1006,16 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 if (M::VEC) ptx::mbar_arrive(cfull(cb));
             }
         }
-        // Scalar partials of the two column halves meet in shared memory.
+        // Scalar partials of the four column quarters meet in shared memory.
         float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
         if (M::SCAL) {
             float a0, a1, b0, b1;
             ptx::f2split(ptx::fadd2(s1a[0], s1a[1]), a0, a1);
             ptx::f2split(ptx::fadd2(s2a[0], s2a[1]), b0, b1);
-            red[(0 * 2 + half) * 128 + row] = a0 + a1;
-            red[(1 * 2 + half) * 128 + row] = b0 + b1;
+            red[(0 * 4 + qt) * 128 + row] = a0 + a1;
+            red[(1 * 4 + qt) * 128 + row] = b0 + b1;
         }
-        ptx::named_bar_sync(1, 256);
+        ptx::named_bar_sync(1, 32 * kSweepEpi);
         ok = __all_sync(0xffffffffu, ok);
         // Dustbin link of this row (the dustbin column), then the writes.
         const bool d_act = D >= 0 && logm[D] != kNegInf;
@@ -1033,9 +1028,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             for (int k = 0; k < NMOD; ++k) mod += xr[k] * a.yc[k][base + D];
             coefd = Pd * mod;
         }
-        if (M::SCAL && ok && half == 0 && !is_dustbin_row) {
-            float s1 = red[0 * 128 + row] + red[1 * 128 + row];
-            float s2 = red[2 * 128 + row] + red[3 * 128 + row];
+        if (M::SCAL && ok && qt == 0 && !is_dustbin_row) {
+            float s1 = (red[0 * 128 + row] + red[1 * 128 + row]) + (red[2 * 128 + row] + red[3 * 128 + row]);
+            float s2 = (red[4 * 128 + row] + red[5 * 128 + row]) + (red[6 * 128 + row] + red[7 * 128 + row]);
             if (d_act && ract) {
                 if (M::SDP) s1 = fmaf(Pd, dpd, s1);
                 if (M::SM) s2 = fmaf(Pd, a.m[base + D], s2);
@@ -1049,7 +1044,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         }
         // The accumulator read is a warp-collective: every lane takes part; only the stores
         // are predicated (the dustbin row is written by the dense dustbin kernel).
-        if (M::VEC && ok) {
+        if (M::VEC && ok && qt < 2) {
             const bool have_acc = n > 0;
             bool wacc = !have_acc || ptx::mbar_wait(accfull, 0, abort_flag, a.status);
             ok = __all_sync(0xffffffffu, wacc);
