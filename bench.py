@@ -461,36 +461,43 @@ def main():
     }
 
     # ---------------- e2e: host buffers, copies inside the timed region ----------------
-    if not args.no_e2e:
+    # One step = copy Q, K, V, dO in from pinned host memory, forward + backward, copy O, dQ,
+    # dK, dV out, through HostStep: the independent (batch, head) units run in chunks on three
+    # streams so that copies overlap the kernels.
+    if not args.no_e2e and case.dustbin:
+        line["e2e"] = None
+    elif not args.no_e2e:
+        from entropic_ot_attention_b200.host_pipeline import HostStep
+        hs = HostStep(B, H, L, d, case.W, case.T, case.R, tdt, case.scale, mask=mask, heads_per_chunk=1,
+                      device=dev, impl=args.impl)
         hq, hk, hv, hdo = (torch.empty(q.shape, dtype=tdt, pin_memory=True) for _ in range(4))
         for h_, d_ in ((hq, q), (hk, k), (hv, v), (hdo, dO)):
             h_.copy_(d_)
         ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=tdt, pin_memory=True) for _ in range(4))
         h2d = 4 * q.numel() * q.element_size()
         d2h = 4 * q.numel() * q.element_size()
+        for _ in range(args.warmup):
+            hs.run(hq, hk, hv, hdo, ho, hdq, hdk, hdv)
         torch.cuda.synchronize(dev)
         barrier(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        e0.record(hs.s_in)
         for _ in range(args.steps):
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            dO.copy_(hdo, non_blocking=True)
-            fwd()
-            bwd()
-            ho.copy_(O, non_blocking=True)
-            hdq.copy_(dQ, non_blocking=True)
-            hdk.copy_(dK, non_blocking=True)
-            hdv.copy_(dV, non_blocking=True)
-        e1.record(stream)
+            hs.run(hq, hk, hv, hdo, ho, hdq, hdk, hdv)
+        hs.s_out.wait_stream(hs.s_in)
+        hs.s_out.wait_stream(hs.s_comp)
+        e1.record(hs.s_out)
         torch.cuda.synchronize(dev)
+        if hs.device_status() != 0:
+            raise RuntimeError("device status after the host-buffer steps is not OK")
+        if not (torch.equal(ho.to(dev), O) and torch.equal(hdq.to(dev), dQ)):
+            raise RuntimeError("host-buffer step results differ from the device-resident step")
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
         line["e2e"] = {"value": total_entries / (t_e2e * 1e-3), "unit": UNIT, "ms_per_step": t_e2e,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "api": "eot_sinkhorn_fwd + eot_sinkhorn_bwd with pinned host inputs/outputs copied "
-                              "in and out every step"}
+                       "api": "HostStep: eot_sinkhorn_fwd + eot_sinkhorn_bwd per (batch, head) chunk on "
+                              "three streams, pinned host inputs copied in and results copied out every step"}
 
     # ---------------- CPU baseline: the oracle on the host cores (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:
