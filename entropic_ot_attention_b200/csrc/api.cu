@@ -156,7 +156,12 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     float* sd_col = p->dustbin ? at<float>(ws, w.sd_col) : nullptr;
 
     EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
-    if (p->dustbin) EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st); }));
+    float* dpart = p->dustbin ? at<float>(ws, w.dpart) : nullptr;
+    uint32_t* dcnt = p->dustbin ? at<uint32_t>(ws, w.dcnt) : nullptr;
+    if (p->dustbin) {
+        EOT_TRY(cudaMemsetAsync(dcnt, 0, size_t(g.BH) * sizeof(uint32_t), st));
+        EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, Q, K, g.scale, sd_row, sd_col, st); }));
+    }
     const size_t tail_bytes = size_t(g.BH) * pstride * sizeof(float);
     EOT_TRY(cudaMemsetAsync(u_tail, 0, tail_bytes, st));
     EOT_TRY(cudaMemsetAsync(v_tail, 0, tail_bytes, st));
@@ -169,6 +174,8 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     row.pstride = pstride;
     row.sd_term = sd_row;
     row.sd_dense = sd_col;
+    row.dpart = dpart;
+    row.dcnt = dcnt;
     row.status = status;
     float* ub2 = at<float>(ws, w.ub2);
     float* vb2 = at<float>(ws, w.vb2);
@@ -234,6 +241,8 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     op.nmod = 0;
     op.sd_term = sd_row;
     op.sd_dense = sd_col;
+    op.dpart = dpart;
+    op.dcnt = dcnt;
     op.status = status;
     EOT_TRY(run_bwd(impl, op, st, kProfOut));
     return EOT_OK;
@@ -251,7 +260,10 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     float* logm = at<float>(ws, w.logm);
     float *sd_row = nullptr, *sd_col = nullptr, *e1 = nullptr, *e2 = nullptr;
     EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
+    float* dpart = p->dustbin ? at<float>(ws, w.dpart) : nullptr;
+    uint32_t* dcnt = p->dustbin ? at<uint32_t>(ws, w.dcnt) : nullptr;
     if (p->dustbin) {
+        EOT_TRY(cudaMemsetAsync(dcnt, 0, size_t(g.BH) * sizeof(uint32_t), st));
         sd_row = at<float>(ws, w.sd_row);
         sd_col = at<float>(ws, w.sd_col);
         e1 = at<float>(ws, w.e1);
@@ -298,6 +310,8 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.sd_dense = sd_col;
     rowp.dp_term = e1;
     rowp.dp_dense = e2;
+    rowp.dpart = dpart;
+    rowp.dcnt = dcnt;
     rowp.zero_vec = at<float>(ws, w.zero);
     rowp.status = status;
     uint32_t* tbits = at<uint32_t>(ws, w.tbits);

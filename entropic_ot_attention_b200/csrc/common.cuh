@@ -50,6 +50,8 @@ struct LsePass {
     const uint32_t* tile_bits;  // [B][tile_words(L)]: 128-position tiles holding an active non-dustbin token
     const float* sd_term;   // [BH, L] S between row r and the dustbin column (dustbin only)
     const float* sd_dense;  // [BH, L] S between the dustbin row and column c (dustbin only)
+    float* dpart;           // dense dustbin row: per-CTA partial sums (dustbin only)
+    uint32_t* dcnt;         // [BH] CTAs of the dense dustbin row done (zero between launches)
     uint32_t* status;
 };
 
@@ -86,12 +88,15 @@ struct BwdPass {
     const float* dp_dense;  // <A_D, Bm_c>
     const float* zero_vec;  // [BH, L] zeros (padding of the modifier list), or nullptr
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
+    float* dpart;           // as in LsePass
+    uint32_t* dcnt;
     uint32_t* status;
 };
 
 // Workspace layout.  Every region is 256-byte aligned; offsets in bytes.
 struct WsLayout {
     size_t status, logm, sd_row, sd_col, e1, e2;
+    size_t dpart, dcnt;     // dense dustbin row: per-CTA partials and completion counters
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
@@ -104,6 +109,9 @@ struct WsLayout {
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+// The dense dustbin row is split over CTAs of kDCols columns (plus the (D, D) entry).
+constexpr int kDCols = 1024;
+__host__ __device__ inline int dustbin_splits(int L) { return (L + 1 + kDCols - 1) / kDCols; }
 __host__ __device__ inline int tile_words(int L) { return (L / 128 + 31) / 32; }
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
@@ -117,6 +125,8 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.sd_row = o; o += vec;
         w.sd_col = o; o += vec;
         if (bwd) { w.e1 = o; o += vec; w.e2 = o; o += vec; }
+        w.dpart = o; o += align256(BH * size_t(dustbin_splits(p.L)) * size_t(p.d + 2) * sizeof(float));
+        w.dcnt = o; o += align256(BH * sizeof(uint32_t));
     }
     if (!bwd) {
         w.opr = o; o += vec;

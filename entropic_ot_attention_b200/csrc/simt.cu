@@ -164,18 +164,25 @@ __global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
 // Dense dustbin row of a half-step: out_D = logm_D - LSE_c (S_Dc + colpot_c) over every
 // active real c, plus (D, D) when it is in the support.  One CTA per unit.
 __global__ void __launch_bounds__(256) dustbin_lse_kernel(LsePass p) {
-    const int bh = blockIdx.x, b = bh / p.g.H, L = p.g.L, D = p.g.D;
+    // CTA (split, unit): columns [split * kDCols, ...) of the dense dustbin row (column L stands
+    // for the (D, D) entry); the last CTA of a unit to finish merges the partial sums.
+    const int split = blockIdx.x, ns = gridDim.x, bh = blockIdx.y, b = bh / p.g.H, L = p.g.L, D = p.g.D;
     const size_t base = size_t(bh) * L;
     const size_t pb = size_t(bh) * p.pstride;
     const float* logm = p.logm + size_t(b) * L;
     if (D < 0 || logm[D] == neg_inf()) return;
     float m = neg_inf(), s = 0.f;
-    for (int c = threadIdx.x; c < L; c += blockDim.x) {
+    const int c_end = min(L + 1, (split + 1) * kDCols);
+    for (int c = split * kDCols + threadIdx.x; c < c_end; c += blockDim.x) {
+        if (c == L) {
+            if (p.g.dself) lse2_add(m, s, (p.sd_term[base + D] + p.colpot[pb + D]) * kLog2e);
+            continue;
+        }
         if (c == D || logm[c] == neg_inf()) continue;
         lse2_add(m, s, (p.sd_dense[base + c] + p.colpot[pb + c]) * kLog2e);
     }
-    if (threadIdx.x == 0 && p.g.dself) lse2_add(m, s, (p.sd_term[base + D] + p.colpot[pb + D]) * kLog2e);
     __shared__ float sm_m[256], sm_s[256];
+    __shared__ int last;
     sm_m[threadIdx.x] = m;
     sm_s[threadIdx.x] = s;
     __syncthreads();
@@ -188,12 +195,23 @@ __global__ void __launch_bounds__(256) dustbin_lse_kernel(LsePass p) {
         }
         __syncthreads();
     }
+    float* part = p.dpart + size_t(bh) * ns * 2;
     if (threadIdx.x == 0) {
-        float outv = logm[D] - (sm_m[0] + log2f(sm_s[0])) * kLn2;
-        if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
-        p.out[pb + D] = outv;
-        p.out_bias2[base + D] = neg_inf();   // the dustbin never enters a band sum
+        part[2 * split] = sm_m[0];
+        part[2 * split + 1] = sm_s[0];
+        __threadfence();
+        last = atomicAdd(p.dcnt + bh, 1u) == unsigned(ns - 1);
     }
+    __syncthreads();
+    if (!last || threadIdx.x != 0) return;
+    __threadfence();
+    float mm = neg_inf(), ss = 0.f;
+    for (int i = 0; i < ns; ++i) lse2_merge(mm, ss, __ldcg(part + 2 * i), __ldcg(part + 2 * i + 1));
+    p.dcnt[bh] = 0u;   // ready for the next launch of this call
+    float outv = logm[D] - (mm + log2f(ss)) * kLn2;
+    if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+    p.out[pb + D] = outv;
+    p.out_bias2[base + D] = neg_inf();   // the dustbin never enters a band sum
 }
 
 // ---------------------------------------------------------------------------------------
@@ -350,34 +368,32 @@ __global__ void __launch_bounds__(kSNT) simt_bwd_kernel(BwdPass p) {
 }
 
 // Dense dustbin row of a backward sweep (row r = D over every active real column, plus
-// (D, D)).  One CTA per unit.
+// (D, D)).  CTA (split, unit) takes kDCols columns (column L stands for (D, D)); the last CTA
+// of a unit to finish adds up the partial sums and vectors and writes the row's outputs.
 template <typename T>
 __global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
-    const int bh = blockIdx.x, b = bh / p.g.H, L = p.g.L, D = p.g.D, d = p.g.d;
+    const int split = blockIdx.x, ns = gridDim.x, bh = blockIdx.y, b = bh / p.g.H;
+    const int L = p.g.L, D = p.g.D, d = p.g.d;
     const size_t base = size_t(bh) * L;
     const float* logm = p.logm + size_t(b) * L;
     if (D < 0 || logm[D] == neg_inf()) return;
     const int nm = p.nmod;
     const bool has_dp = (p.sout && p.s_dp) || (p.vout && p.v_dp);
     const float prD = p.pr[base + D];
-    __shared__ float cs[256];
+    const int c_begin = split * kDCols, c_end = min(L + 1, c_begin + kDCols);
+    __shared__ float cs[kDCols];
     __shared__ float red1[256], red2[256];
-    __shared__ float vacc[256];
+    __shared__ float vred[8][128];
+    __shared__ int last;
     float a1 = 0.f, a2 = 0.f;
-    const T* Z = p.vout ? static_cast<const T*>(p.Z) + base * d : nullptr;
-    const int groups = d > 0 ? 256 / d : 1;      // threads per output element split over c
-    const int zc = threadIdx.x % d, grp = threadIdx.x / d;
-    float vpart = 0.f;
-    for (int c0 = 0; c0 < L + 1; c0 += 256) {
-        const int c = c0 + threadIdx.x;
+    for (int c = c_begin + threadIdx.x; c < c_begin + kDCols; c += blockDim.x) {
         float coef = 0.f;
-        // c == L stands for the (D, D) entry
         const bool self = (c == L) && p.g.dself;
         const bool band = (c < L) && c != D && logm[c] != neg_inf();
-        if (band || self) {
+        if (c < c_end && (band || self)) {
             const int cc = self ? D : c;
-            const float s = self ? p.sd_term[base + D] : p.sd_dense[base + c];
-            const float P = expf(s + prD + p.pc[base + cc]);
+            const float sv = self ? p.sd_term[base + D] : p.sd_dense[base + c];
+            const float P = expf(sv + prD + p.pc[base + cc]);
             const float dp = has_dp ? (self ? p.dp_term[base + D] : p.dp_dense[base + c]) : 0.f;
             if (p.sout) {
                 if (p.s_dp) a1 = fmaf(P, dp, a1);
@@ -389,23 +405,10 @@ __global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
                 coef = P * mod;
             }
         }
-        if (p.vout) {
-            __syncthreads();
-            cs[threadIdx.x] = coef;
-            __syncthreads();
-            if (grp < groups) {
-                for (int j = grp; j < 256; j += groups) {
-                    const int cj = c0 + j;
-                    if (cj > L) break;
-                    const int row = (cj == L) ? D : cj;
-                    if (cs[j] != 0.f) vpart = fmaf(cs[j], to_f(Z[size_t(row) * d + zc]), vpart);
-                }
-            }
-        }
+        cs[c - c_begin] = coef;
     }
     red1[threadIdx.x] = a1;
     red2[threadIdx.x] = a2;
-    vacc[threadIdx.x] = (grp < groups) ? vpart : 0.f;
     __syncthreads();
     for (int st = 128; st > 0; st >>= 1) {
         if (threadIdx.x < st) {
@@ -414,16 +417,63 @@ __global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
         }
         __syncthreads();
     }
+    // vector part: warp w takes columns w, w + 8, ...; lane covers elements lane + 32 z of Z's row
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nz = (d + 31) / 32;
+    if (p.vout) {
+        const T* Z = static_cast<const T*>(p.Z) + base * d;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int j = warp; j < c_end - c_begin; j += 8) {
+            const float cf = cs[j];
+            if (cf == 0.f) continue;
+            const int cj = c_begin + j;
+            const T* zr = Z + size_t(cj == L ? D : cj) * d;
+#pragma unroll
+            for (int z = 0; z < 4; ++z)
+                if (z < nz && lane + 32 * z < d) acc[z] = fmaf(cf, to_f(zr[lane + 32 * z]), acc[z]);
+        }
+#pragma unroll
+        for (int z = 0; z < 4; ++z)
+            if (z < nz && lane + 32 * z < d) vred[warp][lane + 32 * z] = acc[z];
+    }
+    __syncthreads();
+    const int pw = d + 2;
+    float* part = p.dpart + size_t(bh) * ns * pw + size_t(split) * pw;
+    if (threadIdx.x == 0) {
+        part[0] = red1[0];
+        part[1] = red2[0];
+    }
+    if (p.vout && threadIdx.x < d) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += vred[w][threadIdx.x];
+        part[2 + threadIdx.x] = v;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(p.dcnt + bh, 1u) == unsigned(ns - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const float* parts = p.dpart + size_t(bh) * ns * pw;
     if (p.sout && threadIdx.x == 0) {
-        float outv = (p.f ? p.f[base + D] : 1.f) * (red1[0] + (p.hv ? p.hv[base + D] : 0.f) * red2[0]);
+        float s1 = 0.f, s2 = 0.f;
+        for (int i = 0; i < ns; ++i) {
+            s1 += __ldcg(parts + size_t(i) * pw);
+            s2 += __ldcg(parts + size_t(i) * pw + 1);
+        }
+        float outv = (p.f ? p.f[base + D] : 1.f) * (s1 + (p.hv ? p.hv[base + D] : 0.f) * s2);
         if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
         p.sout[base + D] = outv;
     }
     if (p.vout && threadIdx.x < d) {
         float a = 0.f;
-        for (int g2 = 0; g2 < groups; ++g2) a += vacc[g2 * d + threadIdx.x];
+        for (int i = 0; i < ns; ++i) a += __ldcg(parts + size_t(i) * pw + 2 + threadIdx.x);
         static_cast<T*>(p.vout)[(base + D) * d + threadIdx.x] = from_f<T>(p.vscale * a);
     }
+    __syncthreads();
+    if (threadIdx.x == 0) p.dcnt[bh] = 0u;   // ready for the next launch of this call
 }
 
 // ---------------------------------------------------------------------------------------
@@ -542,7 +592,8 @@ cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st) {
 }
 
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st) {
-    dustbin_lse_kernel<<<p.g.BH, 256, 0, st>>>(p);
+    if (!p.dpart || !p.dcnt) return cudaErrorInvalidValue;
+    dustbin_lse_kernel<<<dim3(dustbin_splits(p.g.L), p.g.BH), 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -565,10 +616,12 @@ cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st) {
 }
 
 cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st) {
+    if (!p.dpart || !p.dcnt || p.g.d > 128) return cudaErrorInvalidValue;
+    const dim3 grid(dustbin_splits(p.g.L), p.g.BH);
     if (p.g.dtype == EOT_BF16)
-        dustbin_bwd_kernel<__nv_bfloat16><<<p.g.BH, 256, 0, st>>>(p);
+        dustbin_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(p);
     else
-        dustbin_bwd_kernel<float><<<p.g.BH, 256, 0, st>>>(p);
+        dustbin_bwd_kernel<float><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
 }
 
