@@ -14,7 +14,7 @@
 // Two kernels:
 //   tc_band_kernel   persistent, 128 x 128 score tiles, row reductions only (forward
 //                    half-steps and the staircase sums of the backward pass)
-//   tc_sweep_kernel  one CTA per 128-row tile, 128 x 64 score tiles, row reductions and a
+//   tc_sweep_kernel  one CTA per 128-row tile, 128 x 128 score tiles, row reductions and a
 //                    second MMA that multiplies coefficient tiles into d-wide outputs
 //                    (forward output, dV, dQ, dK)
 #include <cudaTypedefs.h>
