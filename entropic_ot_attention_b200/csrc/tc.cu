@@ -155,7 +155,9 @@ struct BandCfg {
     static constexpr uint32_t OFF_Y = NQ * XB;
     static constexpr uint32_t OFF_V = OFF_Y + NS * YB;         // [half][NV][VB]
     static constexpr uint32_t OFF_RED = OFF_V + 2 * NV * VB;    // [half][parity][m, s][128 rows]
-    static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 2 * 2 * 128 * 4;
+    static constexpr uint32_t OFF_BITS = OFF_RED + 2 * 2 * 2 * 128 * 4;   // tile bits of the CTA's batch rows
+    static constexpr int BITS_WORDS = 512;
+    static constexpr uint32_t OFF_BAR = OFF_BITS + BITS_WORDS * 4;
     // full[NS] empty[NS] qfull[NQ] qempty[NQ], then per half: tfull[2] tempty[2] vfull[NV] vempty[NV]
     static constexpr uint32_t HB0 = 2 * NS + 2 * NQ;
     static constexpr uint32_t HBN = 4 + 2 * NV;
@@ -217,6 +219,17 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     auto vempty = [&](int G, int i) { return bar0 + 8u * (C::HB0 + G * C::HBN + 4 + C::NV + i); };
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    // The tile bits of the batch rows this CTA's items touch, copied into shared memory when
+    // they fit (every role reads them for every item and tile).
+    uint32_t* sbits = reinterpret_cast<uint32_t*>(sm + C::OFF_BITS);
+    const int b_first = item1 > item0 ? (item0 / a.pairs_per_unit) / a.H : 0;
+    const int b_last = item1 > item0 ? ((item1 - 1) / a.pairs_per_unit) / a.H : -1;
+    const int nbw = (b_last - b_first + 1) * a.words;
+    const bool bits_in_smem = nbw <= C::BITS_WORDS;
+    if (bits_in_smem)
+        for (int i = tid; i < nbw; i += blockDim.x) sbits[i] = a.tile_bits[size_t(b_first) * a.words + i];
+    const uint32_t* bits0 = bits_in_smem ? sbits : a.tile_bits + size_t(b_first) * a.words;
+    auto bits_of = [&](int b) -> const uint32_t* { return bits0 + (b - b_first) * a.words; };
 
     auto decode = [&](int item) {
         BandItem it;
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         it.b = it.bh / a.H;
         it.r0 = (item - it.bh * a.pairs_per_unit) * 2 * C::BM;
         it.base = size_t(it.bh) * L;
-        const uint32_t* bits = a.tile_bits + size_t(it.b) * a.words;
+        const uint32_t* bits = bits_of(it.b);
 #pragma unroll
         for (int G = 0; G < 2; ++G) {
             const int rg = it.r0 + G * C::BM;
@@ -280,7 +293,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     ++qi;
                 }
                 if (!ok) break;
-                TileBits bits(a.tile_bits + size_t(it.b) * a.words);
+                TileBits bits(bits_of(it.b));
                 const int u_lo = it.active[0] ? it.t_lo[0] : it.t_lo[1];
                 const int u_hi = it.active[1] ? it.t_hi[1] : it.t_hi[0];
                 for (int t = u_lo; t <= u_hi && ok; ++t) {
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             for (int item = item0; item < item1 && ok; ++item) {
                 const BandItem it = decode(item);
                 if (!it.active[0] && !it.active[1]) continue;
-                TileBits bits(a.tile_bits + size_t(it.b) * a.words);
+                TileBits bits(bits_of(it.b));
                 int qslot[2] = {0, 0}, qpar[2] = {0, 0}, n[2] = {0, 0}, done[2] = {0, 0};
                 bool xready[2] = {false, false};
 #pragma unroll
@@ -409,7 +422,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             const size_t base = size_t(bh) * L;
             const int r = rg + row;
             const size_t pb = size_t(bh) * a.pstride;
-            const uint32_t* bitp = a.tile_bits + size_t(b) * a.words;
+            const uint32_t* bitp = bits_of(b);
             if (!tile_bit(bitp, rg / C::BM)) {
                 if (hf == 0) {
                     a.out[pb + r] = 0.f;
