@@ -207,8 +207,41 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         col.out = v_tail + size_t(k_out) * L;
         return run_lse(impl, col, st);
     };
-    for (int t = 0; t < p->T; ++t) EOT_TRY(step(0, 0));                 // stopped base
-    for (int k = 1; k <= p->R; ++k) EOT_TRY(step(k - 1, k));            // differentiable tail
+    // Tensor-core path without a dustbin: the first half-step (running maximum) on its own, then
+    // every later half-step in one cooperative launch with grid-wide barriers between them.  If
+    // the device cannot hold the whole grid at once the half-steps run as separate launches.
+    const int n_half = 2 * (p->T + p->R);
+    bool fused = false;
+    if (impl == EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
+        EOT_TRY(run_lse(impl, [&] {
+            LsePass r0 = row;
+            r0.colpot = v_tail;
+            r0.stab = nullptr;
+            r0.out = u_tail + (p->T > 0 ? 0 : L);
+            return r0;
+        }(), st));
+        uint32_t* gbar = at<uint32_t>(ws, w.gbar);
+        EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
+        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar};
+        const cudaError_t e = tracked(kProfLse, 1, st, [&] { return launch_tc_lse_fused(row, f, st); });
+        if (e == cudaSuccess) fused = true;
+        else if (e == cudaErrorCooperativeLaunchTooLarge) (void)cudaGetLastError();
+        else return EOT_ERR_CUDA;
+        if (!fused) {
+            // finish the first iteration's column half-step, then the rest one launch each
+            first = false;
+            const int k_out = p->T > 0 ? 0 : 1;
+            col.colpot = u_tail + size_t(k_out) * L;
+            col.stab = v_tail;
+            col.out = v_tail + size_t(k_out) * L;
+            EOT_TRY(run_lse(impl, col, st));
+            for (int t = 1; t < p->T; ++t) EOT_TRY(step(0, 0));
+            for (int k = (p->T > 0 ? 1 : 2); k <= p->R; ++k) EOT_TRY(step(k - 1, k));
+        }
+    } else {
+        for (int t = 0; t < p->T; ++t) EOT_TRY(step(0, 0));                 // stopped base
+        for (int k = 1; k <= p->R; ++k) EOT_TRY(step(k - 1, k));            // differentiable tail
+    }
 
     // Output O = diag(1/a) P(R,R) V (a vector sweep with coefficients P / a_r).
     BwdVecArgs va{};

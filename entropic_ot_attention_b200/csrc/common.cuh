@@ -99,6 +99,7 @@ struct WsLayout {
     size_t dpart, dcnt;     // dense dustbin row: per-CTA partials and completion counters
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
+    size_t gbar;            // forward: grid-barrier counters of the fused half-steps [2 (T + R)]
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
     size_t zero;            // backward: a vector of zeros
@@ -134,6 +135,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.opcm = o; o += vec;
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
+        w.gbar = o; o += align256(size_t(2) * (size_t(p.T) + size_t(p.R)) * sizeof(uint32_t) + 4);
     }
     w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     if (bwd) {

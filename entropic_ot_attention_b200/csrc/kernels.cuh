@@ -34,6 +34,15 @@ cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 // Tensor-core (tcgen05 + TMA) kernels; return cudaErrorNotSupported when not built.
 bool tc_supported(const Geom& g);
 cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st);
+// Shifted half-steps hs0 .. hs0 + nhs - 1 of the forward schedule (even hs: row, odd: column;
+// iteration hs / 2 writes slot 0 for the first T iterations and slot hs / 2 - T + 1 after) in one
+// cooperative launch with grid-wide barriers (gbar[hs]: zeroed counters).  No dustbin.
+struct FusedSteps {
+    int hs0, nhs, T;
+    float *u_tail, *v_tail, *ub2, *vb2;
+    uint32_t* gbar;
+};
+cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
 
 }  // namespace eot

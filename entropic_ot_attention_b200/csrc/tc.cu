@@ -138,7 +138,37 @@ struct TcBandArgs {
     size_t pstride;
     const float* sd_term;
     uint32_t* status;
+    // Several half-steps in one (cooperative) launch: half-steps hs0 .. hs0 + nhs - 1 of the
+    // forward schedule (even: row, X = Q; odd: column, X = K; iteration hs / 2 updates slot 0
+    // for the first T iterations and slot k = hs / 2 - T + 1 after), separated by a grid-wide
+    // barrier (gbar[hs] counts the CTAs done with half-step hs).
+    int hs0, nhs, T;
+    float* u_tail;
+    float* v_tail;
+    float* ub2;
+    float* vb2;
+    uint32_t* gbar;
 };
+
+// Bounded wait until a grid-wide counter reaches target (acquire); false on abort or timeout.
+__device__ __forceinline__ bool grid_wait(const uint32_t* ctr, uint32_t target, volatile int* abort_flag,
+                                          uint32_t* status) {
+    const uint64_t t0 = ptx::globaltimer();
+    for (uint32_t i = 0;; ++i) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        if ((i & 15u) == 15u) {
+            if (*abort_flag) return false;
+            if (ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
+}
 
 template <int DH, int KIND>
 struct BandCfg {
@@ -194,12 +224,29 @@ struct TileBits {
     }
 };
 
-template <int DH, int KIND>
+template <int DH, int KIND, bool MULTI>
 __global__ void __launch_bounds__(kBandThreads, 1)
     tc_band_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                    const TcBandArgs a) {
     using C = BandCfg<DH, KIND>;
     constexpr bool ONLINE = KIND == kBandOnline, WSUM = KIND == kBandWsum;
+    static_assert(!MULTI || KIND == kBandShift, "fused half-steps are shifted log-sum-exp sweeps");
+    // Operands of half-step hs (a single launch uses the fixed pointers of a).
+    const int hs_end = a.hs0 + a.nhs;
+    auto slot_of = [&](int hs, bool out) {
+        const int it = hs >> 1;
+        return it < a.T ? 0 : (out ? it - a.T + 1 : it - a.T);
+    };
+    auto colbias_of = [&](int hs) -> const float* { return MULTI ? ((hs & 1) ? a.ub2 : a.vb2) : a.colbias2; };
+    auto stab_of = [&](int hs) -> const float* {
+        return MULTI ? ((hs & 1) ? a.v_tail : a.u_tail) + size_t(slot_of(hs, false)) * a.L : a.stab;
+    };
+    auto out_of = [&](int hs) -> float* {
+        return MULTI ? ((hs & 1) ? a.v_tail : a.u_tail) + size_t(slot_of(hs, true)) * a.L : a.out;
+    };
+    auto outb_of = [&](int hs) -> float* { return MULTI ? ((hs & 1) ? a.vb2 : a.ub2) : a.out_bias2; };
+    auto mapx_of = [&](int hs) { return (MULTI && (hs & 1)) ? &tmY : &tmX; };
+    auto mapy_of = [&](int hs) { return (MULTI && (hs & 1)) ? &tmX : &tmY; };
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -278,6 +325,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             int g = 0, qi = 0;
             int gv[2] = {0, 0};
             bool ok = true;
+            for (int hs = a.hs0; hs < hs_end && ok; ++hs) {
+            const CUtensorMap* mX = mapx_of(hs);
+            const CUtensorMap* mY = mapy_of(hs);
+            const float* cb2 = colbias_of(hs);
+            // the column biases of half-step hs are written by every CTA in half-step hs - 1
+            bool biases_ready = !MULTI || hs == a.hs0;
             for (int item = item0; item < item1 && ok; ++item) {
                 const BandItem it = decode(item);
                 if (!it.active[0] && !it.active[1]) continue;
@@ -289,7 +342,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     ptx::mbar_expect_tx(qfull(qb), C::XB);
                     const uint32_t xs = ptx::smem_u32(sm + qb * C::XB);
                     for (int ka = 0; ka < C::KATOMS; ++ka)
-                        ptx::tma_load_2d(xs + ka * C::ATOM, &tmX, ka * 64, int(it.base) + it.r0 + G * C::BM, qfull(qb));
+                        ptx::tma_load_2d(xs + ka * C::ATOM, mX, ka * 64, int(it.base) + it.r0 + G * C::BM, qfull(qb));
                     ++qi;
                 }
                 if (!ok) break;
@@ -306,8 +359,13 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     ptx::mbar_expect_tx(full(s), C::YB);
                     const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
                     for (int ka = 0; ka < C::KATOMS; ++ka)
-                        ptx::tma_load_2d(ys + ka * C::ATOM, &tmY, ka * 64, int(it.base) + c0, full(s));
+                        ptx::tma_load_2d(ys + ka * C::ATOM, mY, ka * 64, int(it.base) + c0, full(s));
                     ++g;
+                    if (!biases_ready) {
+                        if (!grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) { ok = false; break; }
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        biases_ready = true;
+                    }
 #pragma unroll
                     for (int G = 0; G < 2; ++G) {
                         if (!(G ? use1 : use0)) continue;
@@ -318,11 +376,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                         }
                         ptx::mbar_expect_tx(vfull(G, vs), C::VB);
                         const uint32_t vd = ptx::smem_u32(sm + C::OFF_V + (G * C::NV + vs) * C::VB);
-                        ptx::bulk_load(vd, a.colbias2 + it.base + c0, C::BN * 4, vfull(G, vs));
+                        ptx::bulk_load(vd, cb2 + it.base + c0, C::BN * 4, vfull(G, vs));
                         if (WSUM) ptx::bulk_load(vd + C::BN * 4, a.colw + it.base + c0, C::BN * 4, vfull(G, vs));
                         ++gv[G];
                     }
                 }
+            }
             }
             if (*abort_flag) {
                 // Let every copy already issued land before the CTA retires.
@@ -340,6 +399,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             int g = 0, qi = 0;
             int gt[2] = {0, 0};
             bool ok = true;
+            for (int hs = a.hs0; hs < hs_end && ok; ++hs)
             for (int item = item0; item < item1 && ok; ++item) {
                 const BandItem it = decode(item);
                 if (!it.active[0] && !it.active[1]) continue;
@@ -414,6 +474,16 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         const uint32_t vsm = ptx::smem_u32(sm + C::OFF_V + G * C::NV * C::VB);
         int gt = 0, ep = 0;
         bool ok = true;
+        for (int hs = a.hs0; hs < hs_end; ++hs) {
+        const float* stab_hs = stab_of(hs);
+        float* out_hs = out_of(hs);
+        float* outb_hs = outb_of(hs);
+        if (MULTI && hs > a.hs0) {
+            // every CTA has written half-step hs - 1 (the shifts and biases read below)
+            if (tid == 64 && ok && !grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) ok = false;
+            ptx::named_bar_sync(9, 512);
+            ok = ok && !*abort_flag;
+        }
         for (int item = item0; item < item1; ++item) {
             // this half of the item (no per-half arrays: G is not a compile-time index here)
             const int bh = item / a.pairs_per_unit, b = bh / a.H;
@@ -425,15 +495,15 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             const uint32_t* bitp = bits_of(b);
             if (!tile_bit(bitp, rg / C::BM)) {
                 if (hf == 0) {
-                    a.out[pb + r] = 0.f;
-                    if (!WSUM) a.out_bias2[base + r] = kNegInf;
+                    out_hs[pb + r] = 0.f;
+                    if (!WSUM) outb_hs[base + r] = kNegInf;
                 }
                 continue;
             }
             const int t_lo = max(0, rg - h) / C::BN, t_hi = min(L - 1, rg + C::BM - 1 + h) / C::BN;
             const float* logm = a.logm + size_t(b) * L;
             const float lm = logm[r];
-            const float st = ONLINE ? 0.f : a.stab[pb + r];
+            const float st = ONLINE ? 0.f : stab_hs[pb + r];
             const float st2 = st * kLog2e;
             float m_run = kNegInf;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -597,9 +667,19 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
                     ob = outv * kLog2e;
                 }
-                a.out[pb + r] = outv;
-                if (!WSUM) a.out_bias2[base + r] = ob;
+                out_hs[pb + r] = outv;
+                if (!WSUM) outb_hs[base + r] = ob;
             }
+        }
+        if (MULTI) {
+            // this CTA is done with half-step hs: count it on the grid-wide barrier
+            ptx::named_bar_sync(9, 512);
+            if (tid == 64) {
+                __threadfence();
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                atomicAdd(a.gbar + hs, 1u);
+            }
+        }
         }
     }
     ptx::tc_fence_before();
@@ -1136,18 +1216,27 @@ int sm_count() {
     return n;
 }
 
-template <int DH, int KIND>
+template <int DH, int KIND, bool MULTI>
 cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const TcBandArgs& a, int grid,
                                 cudaStream_t st) {
     constexpr size_t smem = BandCfg<DH, KIND>::SMEM;
-    cudaError_t e = set_smem(tc_band_kernel<DH, KIND>, smem);
+    auto kernel = tc_band_kernel<DH, KIND, MULTI>;
+    cudaError_t e = set_smem(kernel, smem);
     if (e != cudaSuccess) return e;
-    tc_band_kernel<DH, KIND><<<grid, kBandThreads, smem, st>>>(tmX, tmY, a);
-    return cudaGetLastError();
+    if (!MULTI) {
+        kernel<<<grid, kBandThreads, smem, st>>>(tmX, tmY, a);
+        return cudaGetLastError();
+    }
+    // fused half-steps meet at grid-wide barriers: every CTA must be resident at once
+    void* args[] = {const_cast<CUtensorMap*>(&tmX), const_cast<CUtensorMap*>(&tmY), const_cast<TcBandArgs*>(&a)};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid), dim3(kBandThreads), args,
+                                       smem, st);
 }
 
-// Band row reduction over S = scale X Y^T (geometry, tile bits and the per-kind vectors in a).
-cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs a, int kind, cudaStream_t st) {
+// Band row reduction over S = scale X Y^T (geometry, tile bits and the per-kind vectors in a);
+// multi: the fused shifted half-steps a.hs0 .. a.hs0 + a.nhs - 1 in one cooperative launch.
+cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs a, int kind, cudaStream_t st,
+                        bool multi = false) {
     if (!a.tile_bits) return cudaErrorInvalidValue;
     CUtensorMap tmX, tmY;
     const uint64_t rows = uint64_t(g.BH) * g.L;
@@ -1163,17 +1252,25 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     const int grid = std::max(1, std::min(a.n_items, sm_count()));
     a.items_per_cta = (a.n_items + grid - 1) / grid;
     const int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
+    if (!multi) {
+        a.hs0 = 0;
+        a.nhs = 1;
+    } else if (kind != kBandShift || g.D >= 0 || !a.gbar || a.nhs < 1) {
+        return cudaErrorInvalidValue;
+    }
     if (g.d == 128) {
+        if (multi) return launch_band_variant<128, kBandShift, true>(tmX, tmY, a, grid_used, st);
         switch (kind) {
-            case kBandOnline: return launch_band_variant<128, kBandOnline>(tmX, tmY, a, grid_used, st);
-            case kBandShift: return launch_band_variant<128, kBandShift>(tmX, tmY, a, grid_used, st);
-            case kBandWsum: return launch_band_variant<128, kBandWsum>(tmX, tmY, a, grid_used, st);
+            case kBandOnline: return launch_band_variant<128, kBandOnline, false>(tmX, tmY, a, grid_used, st);
+            case kBandShift: return launch_band_variant<128, kBandShift, false>(tmX, tmY, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<128, kBandWsum, false>(tmX, tmY, a, grid_used, st);
         }
     } else {
+        if (multi) return launch_band_variant<64, kBandShift, true>(tmX, tmY, a, grid_used, st);
         switch (kind) {
-            case kBandOnline: return launch_band_variant<64, kBandOnline>(tmX, tmY, a, grid_used, st);
-            case kBandShift: return launch_band_variant<64, kBandShift>(tmX, tmY, a, grid_used, st);
-            case kBandWsum: return launch_band_variant<64, kBandWsum>(tmX, tmY, a, grid_used, st);
+            case kBandOnline: return launch_band_variant<64, kBandOnline, false>(tmX, tmY, a, grid_used, st);
+            case kBandShift: return launch_band_variant<64, kBandShift, false>(tmX, tmY, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<64, kBandWsum, false>(tmX, tmY, a, grid_used, st);
         }
     }
     return cudaErrorInvalidValue;
@@ -1194,6 +1291,25 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     cudaError_t e = launch_band(p.g, p.X, p.Y, a, p.stab ? kBandShift : kBandOnline, st);
     if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
+}
+
+cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st) {
+    if (!row.tile_bits || row.g.D >= 0) return cudaErrorInvalidValue;
+    TcBandArgs a{};
+    a.logm = row.logm;
+    a.tile_bits = row.tile_bits;
+    a.pstride = row.pstride;
+    a.status = row.status;
+    a.hs0 = f.hs0;
+    a.nhs = f.nhs;
+    a.T = f.T;
+    a.u_tail = f.u_tail;
+    a.v_tail = f.v_tail;
+    a.ub2 = f.ub2;
+    a.vb2 = f.vb2;
+    a.gbar = f.gbar;
+    // row half-steps: X = Q (row.X), Y = K (row.Y); the kernel swaps them for column half-steps
+    return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
 
 template <int DH, int MODE, int NMOD>
