@@ -279,8 +279,8 @@ def source_hash() -> str:
 
 
 def load_traffic(workload: str):
-    """DRAM traffic per launch of the dominant kernel from a committed ncu summary, or None
-    when the summary is missing or was taken on different kernel sources."""
+    """DRAM traffic per unit of work (forward half-step) of the dominant kernel from a committed
+    ncu summary, or None when the summary is missing or was taken on different kernel sources."""
     p = os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
     if not os.path.exists(p):
         return None
@@ -288,7 +288,7 @@ def load_traffic(workload: str):
         d = json.load(f)
     if d.get("source_hash") != source_hash():
         return None
-    return d.get("bytes_per_launch")
+    return d.get("bytes_per_half_step")
 
 
 # ----------------------------------------------------------------------------------------
@@ -413,19 +413,22 @@ def main():
     # dominant kernel: the sweep kind with the largest total time
     dom = max(("fwd_sweep", "fwd_output", "bwd_sweep"), key=lambda n_: prof[n_][0])
     dom_ms, dom_n = prof[dom]
-    per_launch_ms = dom_ms / max(dom_n, 1)
-    # one S evaluation (2d flops per band entry) per forward half-step launch; the output and
-    # backward sweeps are counted with their own MMA work per launch
+    # Unit of work: a forward half-step (one S evaluation, 2d flops per band entry; the
+    # half-steps after the first run fused in one launch), else one launch with its own MMA work.
     if dom == "fwd_sweep":
+        n_units, unit_name = 2 * (case.T + case.R), "forward half-step"
         dom_flops = 2 * d * omega
         dom_name = "tc_band_kernel (forward half-step band log-sum-exp)"
     elif dom == "fwd_output":
+        n_units, unit_name = max(dom_n, 1), "launch"
         dom_flops = 2 * 2 * d * omega
         dom_name = "tc_sweep_kernel (forward output P V)"
     else:
-        dom_flops = fl_bwd / max(dom_n, 1)
+        n_units, unit_name = max(dom_n, 1), "launch"
+        dom_flops = fl_bwd / n_units
         dom_name = "tc_sweep_kernel + tc_band_kernel (backward sweeps)"
-    achieved = dom_flops / (per_launch_ms * 1e-3) / 1e12
+    per_unit_ms = dom_ms / n_units
+    achieved = dom_flops / (per_unit_ms * 1e-3) / 1e12
     traffic = load_traffic(args.workload)
     # exp-unit context: one exp2 per band entry per launch for the forward half-step
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -452,8 +455,9 @@ def main():
         "roofline": {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak_tf,
                      "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": traffic,
                      "peak_kind": f"bf16_tflops_sustained ({peaks['source']})",
-                     "launches_timed": dom_n, "ms_per_launch": per_launch_ms,
-                     "exp2_per_s": (omega / (per_launch_ms * 1e-3)) if dom == "fwd_sweep" else None,
+                     "unit_of_work": unit_name, "units_timed": n_units, "ms_per_unit": per_unit_ms,
+                     "launches_timed": dom_n,
+                     "exp2_per_s": (omega / (per_unit_ms * 1e-3)) if dom == "fwd_sweep" else None,
                      "exp2_peak_per_s_assumed": mufu_peak},
         "kernel_ms": {k_: {"total_ms": v_[0], "launches": v_[1]} for k_, v_ in prof.items()},
         "gpu_launches": launches,
