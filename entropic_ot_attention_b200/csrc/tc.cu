@@ -30,8 +30,9 @@ namespace {
 
 constexpr float kNegInf = -__builtin_huge_valf();
 // Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
-// interior forward tiles (2 of 16 pairs: measured best, 0.2585 vs 0.262 ms with none on the long workload).
-constexpr int kFmaPairs = 2;
+// interior tiles of the band kernel (measured per half-step on the long workload: 0 pairs
+// 0.2271 ms, 1 pair 0.2264, 2 pairs 0.2302, 3 pairs 0.2339).
+constexpr int kFmaPairs = 1;
 
 // ---------------------------------------------------------------------------------------
 // Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
