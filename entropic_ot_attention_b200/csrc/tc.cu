@@ -29,10 +29,6 @@ namespace eot {
 namespace {
 
 constexpr float kNegInf = -__builtin_huge_valf();
-// Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
-// interior tiles of the band kernel (measured per half-step on the long workload: 0 pairs
-// 0.2271 ms, 1 pair 0.2264, 2 pairs 0.2302, 3 pairs 0.2339).
-constexpr int kFmaPairs = 1;
 
 // ---------------------------------------------------------------------------------------
 // Host: TMA descriptors over a [rows, d] bf16 matrix, box {64 elements, box_rows}, 128B swizzle
@@ -121,6 +117,11 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 //   wsum    out_r = f_r hv_r sum_c exp(S_rc + st_r + colpot_c) w_c  (staircase sums of the
 //           tail adjoint, with st = the row orbit bias and w = the column weights)
 enum BandKind { kBandOnline = 0, kBandShift = 1, kBandWsum = 2 };
+
+// Pairs of exponentials per 32-column chunk evaluated on the FMA pipe instead of MUFU in
+// interior tiles of the band kernel (measured per half-step on the long workload: 0 pairs
+// 0.2271 ms, 1 pair 0.2264, 2 pairs 0.2302, 3 pairs 0.2339).
+constexpr int kFmaPairs = 1;
 
 struct TcBandArgs {
     int H, L, h, D, n_items, items_per_cta, pairs_per_unit;
