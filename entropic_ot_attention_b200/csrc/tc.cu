@@ -199,7 +199,8 @@ struct BandCfg {
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
-constexpr int kBandThreads = 576;   // TMA warp, MMA warp, 16 epilogue warps
+constexpr int kBandThreads = 608;   // TMA warp, MMA warp (half 0), 16 epilogue warps, MMA warp (half 1)
+constexpr int kBandIssuerB = 18;
 
 // Decoded work item: rows [r0, r0 + 256) of unit bh as two halves with their column-tile bands.
 struct BandItem {
@@ -302,7 +303,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
 
     if (tid == 0) {
         *abort_flag = 0;
-        for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 1); }
+        for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 2); }
         for (int i = 0; i < C::NQ; ++i) { ptx::mbar_init(qfull(i), 1); ptx::mbar_init(qempty(i), 1); }
         for (int G = 0; G < 2; ++G) {
             for (int i = 0; i < 2; ++i) { ptx::mbar_init(tfull(G, i), 1); ptx::mbar_init(tempty(G, i), 8); }
@@ -395,27 +396,32 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 for (int i = max(0, qi - C::NQ); i < qi; ++i) ptx::mbar_wait(qfull(i % C::NQ), (i / C::NQ) & 1, &dummy, a.status);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kBandIssuerB) {
         if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            int g = 0, qi = 0;
-            int gt[2] = {0, 0};
+            // ---------------- MMA issuers: warp 1 for row half 0, warp kBandIssuerB for half 1 ----------------
+            // Two issuing threads halve the per-instruction bookkeeping each one carries; both
+            // walk every column tile (a stage is free once both have committed it).
+            const int GI = warp == 1 ? 0 : 1;
+            int g = 0, qi = 0, gt = 0;
             bool ok = true;
             for (int hs = a.hs0; hs < hs_end && ok; ++hs)
             for (int item = item0; item < item1 && ok; ++item) {
                 const BandItem it = decode(item);
                 if (!it.active[0] && !it.active[1]) continue;
                 TileBits bits(bits_of(it.b));
-                int qslot[2] = {0, 0}, qpar[2] = {0, 0}, n[2] = {0, 0}, done[2] = {0, 0};
-                bool xready[2] = {false, false};
+                int qslot = 0, qpar = 0, n = 0, done = 0;
+                bool xready = false;
 #pragma unroll
                 for (int G = 0; G < 2; ++G) {
                     if (!it.active[G]) continue;
-                    qslot[G] = qi % C::NQ;
-                    qpar[G] = (qi / C::NQ) & 1;
+                    if (G == GI) {
+                        qslot = qi % C::NQ;
+                        qpar = (qi / C::NQ) & 1;
+                        for (int t = it.t_lo[G]; t <= it.t_hi[G]; ++t) n += bits(t);
+                    }
                     ++qi;
-                    for (int t = it.t_lo[G]; t <= it.t_hi[G]; ++t) n[G] += bits(t);
                 }
+                const bool mine = it.active[GI];
                 const int u_lo = it.active[0] ? it.t_lo[0] : it.t_lo[1];
                 const int u_hi = it.active[1] ? it.t_hi[1] : it.t_hi[0];
                 for (int t = u_lo; t <= u_hi && ok; ++t) {
@@ -423,45 +429,41 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     const bool use0 = uses(it, 0, t), use1 = uses(it, 1, t);
                     if (!use0 && !use1) continue;
                     const int s = g % C::NS;
+                    // the stage's current fill must have landed before this thread's commit on it counts
                     if (!ptx::mbar_wait(full(s), (g / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
-                    const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
-#pragma unroll
-                    for (int G = 0; G < 2; ++G) {
-                        if (!(G ? use1 : use0)) continue;
-                        if (!xready[G]) {
-                            if (!ptx::mbar_wait(qfull(qslot[G]), qpar[G], abort_flag, a.status)) { ok = false; break; }
-                            xready[G] = true;
+                    if (GI ? use1 : use0) {
+                        if (!xready) {
+                            if (!ptx::mbar_wait(qfull(qslot), qpar, abort_flag, a.status)) { ok = false; break; }
+                            xready = true;
                         }
-                        const int tb = gt[G] & 1;
-                        if (!ptx::mbar_wait(tempty(G, tb), ((gt[G] >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                        const int tb = gt & 1;
+                        if (!ptx::mbar_wait(tempty(GI, tb), ((gt >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                         ptx::tc_fence_after();
-                        const uint32_t xs = ptx::smem_u32(sm + qslot[G] * C::XB);
-                        const uint32_t dt = tbase + uint32_t((G * 2 + tb) * C::BN);
+                        // descriptor start addresses advance in 16-byte units within one field
+                        const uint64_t xd = ptx::smem_desc(ptx::smem_u32(sm + qslot * C::XB), 16, 1024);
+                        const uint64_t yd = ptx::smem_desc(ptx::smem_u32(sm + C::OFF_Y + s * C::YB), 16, 1024);
+                        const uint32_t dt = tbase + uint32_t((GI * 2 + tb) * C::BN);
 #pragma unroll
                         for (int kk = 0; kk < DH / 16; ++kk) {
-                            const uint32_t koff = (kk >> 2) * C::ATOM + (kk & 3) * 32;
-                            ptx::mma_bf16(dt, ptx::smem_desc(xs + koff, 16, 1024), ptx::smem_desc(ys + koff, 16, 1024),
-                                          C::IDESC, kk > 0 ? 1u : 0u);
+                            const uint64_t koff = uint64_t(((kk >> 2) * C::ATOM + (kk & 3) * 32) >> 4);
+                            ptx::mma_bf16(dt, xd + koff, yd + koff, C::IDESC, kk > 0 ? 1u : 0u);
                         }
-                        ptx::mma_commit(tfull(G, tb));
-                        ++gt[G];
-                        if (++done[G] == n[G]) ptx::mma_commit(qempty(qslot[G]));   // row half free once its products are done
+                        ptx::mma_commit(tfull(GI, tb));
+                        ++gt;
+                        if (++done == n) ptx::mma_commit(qempty(qslot));   // row half free once its products are done
                     }
-                    if (!ok) break;
                     ptx::mma_commit(empty(s));
                     ++g;
                 }
                 // (a half with no column tile cannot occur: an active row tile holds its own diagonal tile)
-                for (int G = 0; G < 2 && ok; ++G) {
-                    if (!it.active[G] || n[G] != 0) continue;
-                    if (!ptx::mbar_wait(qfull(qslot[G]), qpar[G], abort_flag, a.status)) { ok = false; break; }
-                    ptx::mma_commit(qempty(qslot[G]));
+                if (ok && mine && n == 0) {
+                    if (!ptx::mbar_wait(qfull(qslot), qpar, abort_flag, a.status)) ok = false;
+                    else ptx::mma_commit(qempty(qslot));
                 }
             }
-            if (*abort_flag) {
+            if (*abort_flag && gt > 0) {
                 volatile int dummy = 0;
-                for (int G = 0; G < 2; ++G)
-                    if (gt[G] > 0) ptx::mbar_wait(tfull(G, (gt[G] - 1) & 1), ((gt[G] - 1) >> 1) & 1, &dummy, a.status);
+                ptx::mbar_wait(tfull(GI, (gt - 1) & 1), ((gt - 1) >> 1) & 1, &dummy, a.status);
             }
         }
     } else {
