@@ -739,7 +739,8 @@ struct TcVecArgs {
 };
 
 constexpr int kSweepEpi = 16;         // epilogue warps: four per TMEM lane quadrant, 32 columns each
-constexpr int kSweepThreads = 32 * (3 + kSweepEpi);   // TMA warp, score-MMA warp, epilogue warps, product-MMA warp
+constexpr int kSweepThreads = 32 * (4 + kSweepEpi);   // TMA warp, S-MMA warp, epilogue warps, product-MMA warp, dP-MMA warp
+constexpr int kSweepDpWarp = 3 + kSweepEpi;
 
 template <int DH, int NV>
 struct SweepCfg {
@@ -824,10 +825,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < C::NS; ++s) {
             ptx::mbar_init(full(s), 1);
-            ptx::mbar_init(empty(s), 1 + kSweepEpi);   // MMA commit + epilogue warps
+            // MMA commits (the product, or the S and dP issuers of a pass without one) + epilogue warps
+            ptx::mbar_init(empty(s), (M::VEC ? 1 : (M::HASDP ? 2 : 1)) + kSweepEpi);
         }
         ptx::mbar_init(xfull, 1);
-        ptx::mbar_init(tfull, 1);
+        ptx::mbar_init(tfull, M::HASDP ? 2 : 1);   // the S issuer and the dP issuer
         ptx::mbar_init(tempty, kSweepEpi);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(cfull(i), kSweepEpi);
@@ -891,33 +893,28 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 ptx::mbar_wait(xfull, 0, &dummy, a.status);
             }
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------- score MMA issuer: S (and dP) tiles ----------------
+    } else if (warp == 1 || warp == kSweepDpWarp) {
+        // ---------------- score MMA issuers: S (warp 1) and dP (warp kSweepDpWarp) tiles ----------------
+        // One thread each, so that neither product waits behind the other's instruction stream.
+        const bool is_dp = warp == kSweepDpWarp;
+        if (lane == 0 && (!is_dp || M::HASDP)) {
             bool ok = ptx::mbar_wait(xtm, 0, abort_flag, a.status);
             ptx::tc_fence_after();
             int issued = 0;
+            const uint32_t dtm = tbase + (is_dp ? C::TM_DP : C::TM_S);
+            const uint32_t atm = tbase + (is_dp ? C::TM_A : C::TM_X);
             for (int it = 0; it < n && ok; ++it) {
                 const int s = it % C::NS;
                 if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
                 if (!ptx::mbar_wait(tempty, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
-                const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
-                // A operands (row tiles) from TMEM: 8 columns per K step of 16
+                // B operand: the column tile of S (Y) or of dP (W); A operand (row tile) from TMEM,
+                // 8 columns per K step of 16
+                const uint64_t bd = ptx::smem_desc(ptx::smem_u32(sm + (is_dp ? C::OFF_W : C::OFF_Y) + s * C::YB), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk) {
-                    const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                    ptx::mma_bf16_ts(tbase + C::TM_S, tbase + C::TM_X + uint32_t(kk * 8),
-                                     ptx::smem_desc(ys + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
-                }
-                if (M::HASDP) {
-#pragma unroll
-                    for (int kk = 0; kk < DH / 16; ++kk) {
-                        const uint32_t yo = (kk >> 2) * C::YATOM + (kk & 3) * 32;
-                        ptx::mma_bf16_ts(tbase + C::TM_DP, tbase + C::TM_A + uint32_t(kk * 8),
-                                         ptx::smem_desc(ws + yo, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
-                    }
+                    const uint64_t bo = uint64_t(((kk >> 2) * C::YATOM + (kk & 3) * 32) >> 4);
+                    ptx::mma_bf16_ts(dtm, atm + uint32_t(kk * 8), bd + bo, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(tfull);
                 if (!M::VEC) ptx::mma_commit(empty(s));   // vector passes free the stage after the product
