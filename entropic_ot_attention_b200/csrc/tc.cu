@@ -582,13 +582,13 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                                 e0 = ptx::ex2(x0);
                                 e1 = ptx::ex2(x1);
                             }
-                            if (WSUM) {
-                                acc[(2 * k) & 3] = fmaf(e0, hh ? wv.z : wv.x, acc[(2 * k) & 3]);
-                                acc[(2 * k + 1) & 3] = fmaf(e1, hh ? wv.w : wv.y, acc[(2 * k + 1) & 3]);
-                            } else {
-                                acc[(2 * k) & 3] += e0;
-                                acc[(2 * k + 1) & 3] += e1;
-                            }
+                            // the pair's two fp32 sums in one packed instruction
+                            float* ap = acc + 2 * hh;
+                            if (WSUM)
+                                ptx::f2split(ptx::ffma2(ptx::f2(e0, e1), hh ? ptx::f2(wv.z, wv.w) : ptx::f2(wv.x, wv.y),
+                                                        ptx::f2(ap[0], ap[1])), ap[0], ap[1]);
+                            else
+                                ptx::f2split(ptx::fadd2(ptx::f2(ap[0], ap[1]), ptx::f2(e0, e1)), ap[0], ap[1]);
                         }
                     }
                 }
