@@ -746,7 +746,11 @@ template <int DH, int NV>
 struct SweepCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
-    static constexpr int NS = 2;
+    // Column tiles ride two rings.  The late ring holds the tile the product MMA reads (or, in
+    // a pass without one, the dP operand) together with the column vectors the epilogue reads;
+    // a slot comes back only after the product, so it gets three.  The early ring holds the
+    // other tile, which is free as soon as its score MMA completes: one slot suffices.
+    static constexpr int NL = 3, NE = 1;
     static constexpr uint32_t XB = BM * DH * 2;          // row tile bytes
     static constexpr uint32_t YB = BN * DH * 2;          // column tile bytes
     static constexpr uint32_t XATOM = BM * 128;          // one 64-element atom column of a row tile
@@ -757,13 +761,13 @@ struct SweepCfg {
     // The row tiles X and A land (TMA) in the coefficient buffers and are moved into TMEM
     // before the first coefficient is written.
     static constexpr uint32_t OFF_C = 0;
-    static constexpr uint32_t OFF_Y = 2 * CB;
-    static constexpr uint32_t OFF_W = OFF_Y + NS * YB;
-    static constexpr uint32_t OFF_V = OFF_W + NS * YB;
-    static constexpr uint32_t OFF_RED = OFF_V + NS * VB;  // [2 sums][4 quarters][128 rows] scalar partials
+    static constexpr uint32_t OFF_L = 2 * CB;
+    static constexpr uint32_t OFF_E = OFF_L + NL * YB;
+    static constexpr uint32_t OFF_V = OFF_E + NE * YB;
+    static constexpr uint32_t OFF_RED = OFF_V + NL * VB;  // [2 sums][4 quarters][128 rows] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 128 * 4;
-    // full[NS] empty[NS] xfull tfull tempty cfull[2] cempty[2] accfull xtm
-    static constexpr uint32_t NBARS = 2 * NS + 1 + 2 + 4 + 1 + 1;
+    // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm
+    static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
     static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
@@ -784,6 +788,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     constexpr int NV = 1 + (M::SM ? 1 : 0) + NMOD;   // column vectors per stage: pcm2, m, yc...
     using C = SweepCfg<DH, NV>;
     constexpr int VOFF_M = 1, VOFF_Y = 1 + (M::SM ? 1 : 0);
+    // W rides the late ring when the product reads it or when there is no product (R2); Y when
+    // the product reads Y (dQ / dK).
+    constexpr bool LATE_W = !M::VEC || M::ZW2;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -794,40 +801,32 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     const uint32_t bar0 = ptx::smem_u32(bars);
-    auto full = [&](int s) { return bar0 + 8u * s; };
-    auto empty = [&](int s) { return bar0 + 8u * (C::NS + s); };
-    const uint32_t xfull = bar0 + 8u * (2 * C::NS);
-    const uint32_t tfull = bar0 + 8u * (2 * C::NS + 1);
-    const uint32_t tempty = bar0 + 8u * (2 * C::NS + 2);
-    auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NS + 3 + i); };
-    auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NS + 5 + i); };
-    const uint32_t accfull = bar0 + 8u * (2 * C::NS + 7);
-    const uint32_t xtm = bar0 + 8u * (2 * C::NS + 8);   // row tiles copied into TMEM
+    auto full_l = [&](int s) { return bar0 + 8u * s; };
+    auto empty_l = [&](int s) { return bar0 + 8u * (C::NL + s); };
+    const uint32_t full_e = bar0 + 8u * (2 * C::NL);
+    const uint32_t empty_e = bar0 + 8u * (2 * C::NL + 1);
+    const uint32_t xfull = bar0 + 8u * (2 * C::NL + 2);
+    const uint32_t tfull = bar0 + 8u * (2 * C::NL + 3);
+    const uint32_t tempty = bar0 + 8u * (2 * C::NL + 4);
+    auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NL + 5 + i); };
+    auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NL + 7 + i); };
+    const uint32_t accfull = bar0 + 8u * (2 * C::NL + 9);
+    const uint32_t xtm = bar0 + 8u * (2 * C::NL + 10);   // row tiles copied into TMEM
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
     int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
     int* flags = tiles + max_tiles;
 
-    if (tid == 0) *abort_flag = 0;
-    bool any_row;
-    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
-                                                 reinterpret_cast<int*>(misc + 2), &any_row);
-    if (!any_row) {
-        if (M::SCAL)
-            for (int r = tid; r < C::BM; r += kSweepThreads) a.sout[base + r0 + r] = 0.f;
-        if (M::VEC) {
-            __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
-            for (int e = tid; e < C::BM * DH / 8; e += kSweepThreads)
-                reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
-        }
-        return;
-    }
     if (tid == 0) {
-        for (int s = 0; s < C::NS; ++s) {
-            ptx::mbar_init(full(s), 1);
-            // MMA commits (the product, or the S and dP issuers of a pass without one) + epilogue warps
-            ptx::mbar_init(empty(s), (M::VEC ? 1 : (M::HASDP ? 2 : 1)) + kSweepEpi);
+        *abort_flag = 0;
+        for (int s = 0; s < C::NL; ++s) {
+            ptx::mbar_init(full_l(s), 1);
+            // the epilogue warps (column vectors) + the product's commit, or in a pass without
+            // one the dP issuer's
+            ptx::mbar_init(empty_l(s), 1 + kSweepEpi);
         }
+        ptx::mbar_init(full_e, 1);
+        ptx::mbar_init(empty_e, 1);                 // the commit of the score MMA that reads it
         ptx::mbar_init(xfull, 1);
         ptx::mbar_init(tfull, M::HASDP ? 2 : 1);   // the S issuer and the dP issuer
         ptx::mbar_init(tempty, kSweepEpi);
@@ -838,6 +837,34 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         ptx::mbar_init(accfull, 1);
         ptx::mbar_init(xtm, kSweepEpi);
         ptx::mbar_fence_init();
+        // The row tiles do not depend on the band's tile list: their copies start first and
+        // overlap the scan below.
+        ptx::prefetch_tmap(&tmX);
+        if (M::HASDP) ptx::prefetch_tmap(&tmA);
+        const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
+        ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1));
+        for (int ka = 0; ka < C::KATOMS; ++ka) {
+            ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
+            if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
+        }
+    }
+    bool any_row;
+    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
+                                                 reinterpret_cast<int*>(misc + 2), &any_row);
+    if (!any_row) {
+        if (tid == 0) {
+            // no copy may still be writing this CTA's shared memory when it exits
+            volatile int dummy = 0;
+            ptx::mbar_wait(xfull, 0, &dummy, a.status);
+        }
+        if (M::SCAL)
+            for (int r = tid; r < C::BM; r += kSweepThreads) a.sout[base + r0 + r] = 0.f;
+        if (M::VEC) {
+            __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
+            for (int e = tid; e < C::BM * DH / 8; e += kSweepThreads)
+                reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
+        }
+        return;
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_u32(misc), 512);
@@ -850,17 +877,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            ptx::prefetch_tmap(&tmX);
+            // ---------------- TMA producer (the row tiles are already on their way) ----------------
+            static_assert(M::W2, "every sweep pass reads two column-side tensors");
             ptx::prefetch_tmap(&tmY);
-            if (M::HASDP) ptx::prefetch_tmap(&tmA);
-            if (M::W2) ptx::prefetch_tmap(&tmW);
-            const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
-            ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1));
-            for (int ka = 0; ka < C::KATOMS; ++ka) {
-                ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
-                if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
-            }
+            ptx::prefetch_tmap(&tmW);
+            const CUtensorMap* tm_late = LATE_W ? &tmW : &tmY;
+            const CUtensorMap* tm_early = LATE_W ? &tmY : &tmW;
             const float* vsrc[NV];
             {
                 int k = 0;
@@ -868,28 +890,36 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 if (M::SM) vsrc[k++] = a.m;
                 for (int i = 0; i < NMOD; ++i) vsrc[k++] = a.yc[i];
             }
-            constexpr uint32_t stage_bytes = C::YB * (M::W2 ? 2 : 1) + uint32_t(NV) * C::BN * 4;
-            int issued = 0;
+            constexpr uint32_t late_bytes = C::YB + uint32_t(NV) * C::BN * 4;
+            int issued_l = 0, issued_e = 0;
             for (int it = 0; it < n; ++it) {
-                const int s = it % C::NS;
+                const int sl = it % C::NL;
                 const int c0 = tiles[it] * C::BN;
-                if (!ptx::mbar_wait(empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(full(s), stage_bytes);
-                const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
-                const uint32_t ws = ptx::smem_u32(sm + C::OFF_W + s * C::YB);
-                for (int ka = 0; ka < C::KATOMS; ++ka) {
-                    ptx::tma_load_2d(ys + ka * C::YATOM, &tmY, ka * 64, int(base) + c0, full(s));
-                    if (M::W2) ptx::tma_load_2d(ws + ka * C::YATOM, &tmW, ka * 64, int(base) + c0, full(s));
-                }
-                const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
+                // late ring: column tile + column vectors
+                if (!ptx::mbar_wait(empty_l(sl), ((it / C::NL) & 1) ^ 1, abort_flag, a.status)) break;
+                ptx::mbar_expect_tx(full_l(sl), late_bytes);
+                const uint32_t ls = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);
+                for (int ka = 0; ka < C::KATOMS; ++ka)
+                    ptx::tma_load_2d(ls + ka * C::YATOM, tm_late, ka * 64, int(base) + c0, full_l(sl));
+                const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
 #pragma unroll
-                for (int i = 0; i < NV; ++i) ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full(s));
-                issued = it + 1;
+                for (int i = 0; i < NV; ++i)
+                    ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full_l(sl));
+                issued_l = it + 1;
+                // early ring: the other column tile
+                if (!ptx::mbar_wait(empty_e, (it & 1) ^ 1, abort_flag, a.status)) break;
+                ptx::mbar_expect_tx(full_e, C::YB);
+                const uint32_t es = ptx::smem_u32(sm + C::OFF_E);
+                for (int ka = 0; ka < C::KATOMS; ++ka)
+                    ptx::tma_load_2d(es + ka * C::YATOM, tm_early, ka * 64, int(base) + c0, full_e);
+                issued_e = it + 1;
             }
             if (*abort_flag) {
+                // let every copy still in flight land before the CTA can exit
                 volatile int dummy = 0;
-                for (int it = max(0, issued - C::NS); it < issued; ++it)
-                    ptx::mbar_wait(full(it % C::NS), (it / C::NS) & 1, &dummy, a.status);
+                for (int it = max(0, issued_l - C::NL); it < issued_l; ++it)
+                    ptx::mbar_wait(full_l(it % C::NL), (it / C::NL) & 1, &dummy, a.status);
+                if (issued_e > 0) ptx::mbar_wait(full_e, (issued_e - 1) & 1, &dummy, a.status);
                 ptx::mbar_wait(xfull, 0, &dummy, a.status);
             }
         }
@@ -903,21 +933,28 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             int issued = 0;
             const uint32_t dtm = tbase + (is_dp ? C::TM_DP : C::TM_S);
             const uint32_t atm = tbase + (is_dp ? C::TM_A : C::TM_X);
+            const bool late = is_dp == LATE_W;   // this issuer's column tile (W for dP, Y for S) rides the late ring
             for (int it = 0; it < n && ok; ++it) {
-                const int s = it % C::NS;
-                if (!ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status)) { ok = false; break; }
+                const int sl = it % C::NL;
+                const bool got = late ? ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status)
+                                      : ptx::mbar_wait(full_e, it & 1, abort_flag, a.status);
+                if (!got) { ok = false; break; }
                 if (!ptx::mbar_wait(tempty, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
                 ptx::tc_fence_after();
                 // B operand: the column tile of S (Y) or of dP (W); A operand (row tile) from TMEM,
                 // 8 columns per K step of 16
-                const uint64_t bd = ptx::smem_desc(ptx::smem_u32(sm + (is_dp ? C::OFF_W : C::OFF_Y) + s * C::YB), 16, 1024);
+                const uint32_t boff = late ? C::OFF_L + uint32_t(sl) * C::YB : C::OFF_E;
+                const uint64_t bd = ptx::smem_desc(ptx::smem_u32(sm + boff), 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < DH / 16; ++kk) {
                     const uint64_t bo = uint64_t(((kk >> 2) * C::YATOM + (kk & 3) * 32) >> 4);
                     ptx::mma_bf16_ts(dtm, atm + uint32_t(kk * 8), bd + bo, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(tfull);
-                if (!M::VEC) ptx::mma_commit(empty(s));   // vector passes free the stage after the product
+                // the early tile is free once this product completes; a late slot normally comes
+                // back after the product MMA, or here in a pass without one
+                if (!late) ptx::mma_commit(empty_e);
+                else if (!M::VEC) ptx::mma_commit(empty_l(sl));
                 issued = it + 1;
             }
             if (*abort_flag && issued > 0) {
@@ -936,8 +973,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 const int cb = j & 1;
                 if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const int s = j % C::NS;
-                const uint32_t zs = ptx::smem_u32(sm + (M::ZW2 ? C::OFF_W : C::OFF_Y) + s * C::YB);
+                const int sl = j % C::NL;
+                const uint32_t zs = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);   // Z rides the late ring
                 const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 16; ++kk)
@@ -945,7 +982,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                                   ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
                                   (j > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(cempty(cb));
-                ptx::mma_commit(empty(s));
+                ptx::mma_commit(empty_l(sl));
                 done = j + 1;
             }
             if (ok && n > 0) ptx::mma_commit(accfull);
@@ -1005,18 +1042,18 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::named_bar_sync(2, 32 * kSweepEpi);
         }
         for (int it = 0; it < n; ++it) {
-            const int s = it % C::NS, cb = it & 1;
+            const int sl = it % C::NL, cb = it & 1;
             const int c0 = tiles[it] * C::BN;
             const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
             // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-            bool w1 = ptx::mbar_wait(full(s), (it / C::NS) & 1, abort_flag, a.status);
+            bool w1 = ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status);   // column vectors
             bool w2 = w1 && ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
             bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
             if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
             ptx::tc_fence_after();
             // column vectors of this stage (explicit shared-memory loads: the aligned base
             // pointer no longer carries the address space)
-            const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + s * C::VB);
+            const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
             auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
             // this warp's 32 columns of S (and dP), read whole; the buffer goes back at once
             float v[1][32], w[1][32];
@@ -1096,7 +1133,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             if (M::VEC) ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                ptx::mbar_arrive(empty(s));
+                ptx::mbar_arrive(empty_l(sl));
                 if (M::VEC) ptx::mbar_arrive(cfull(cb));
             }
         }
