@@ -1237,7 +1237,8 @@ cudaError_t set_smem(K kernel, size_t bytes) {
 }  // namespace
 
 // The sweep kernel keeps its band's tile list in shared memory: very wide bands (W beyond
-// about 2e5) do not fit next to the tiles and run on the CUDA-core kernels instead.
+// about 7e4, with L longer than that) do not fit next to the tiles and run on the CUDA-core
+// kernels instead.
 constexpr size_t kMaxSmem = 227 * 1024;
 bool tc_supported(const Geom& g) {
     if (g.dtype != EOT_BF16 || (g.d != 64 && g.d != 128) || encode_fn() == nullptr) return false;

@@ -61,7 +61,8 @@ typedef enum {
 typedef enum { EOT_FP32 = 0, EOT_BF16 = 1 } eot_dtype;
 
 /* Kernel family.  AUTO picks the tensor-core (tcgen05/TMA) kernels for bf16 with d in
- * {64, 128} and a band that fits their shared-memory tile list (W below about 2e5), and the
+ * {64, 128} and a band that fits their shared-memory tile list (W up to about 7e4 when L is
+ * longer than that; any W for shorter L), and the
  * CUDA-core kernels otherwise (fp32 is always computed on CUDA cores, in fp32, so that its
  * scores keep full fp32 precision).  TCGEN05 on a problem outside that range is
  * EOT_ERR_UNSUPPORTED. */
