@@ -466,14 +466,12 @@ def main():
 
     # ---------------- e2e: host buffers, copies inside the timed region ----------------
     # One step = copy Q, K, V, dO in from pinned host memory, forward + backward, copy O, dQ,
-    # dK, dV out, through HostStep: the independent (batch, head) units run in chunks on three
-    # streams so that copies overlap the kernels.
-    if not args.no_e2e and case.dustbin:
-        line["e2e"] = None
-    elif not args.no_e2e:
+    # dK, dV out, through HostStep: the independent (batch, head) units run in chunks (whole batch
+    # rows, or heads of one row) on three streams so that copies overlap the kernels.
+    if not args.no_e2e:
         from entropic_ot_attention_b200.host_pipeline import HostStep
-        hs = HostStep(B, H, L, d, case.W, case.T, case.R, tdt, case.scale, mask=mask, heads_per_chunk=1,
-                      device=dev, impl=args.impl)
+        hs = HostStep(B, H, L, d, case.W, case.T, case.R, tdt, case.scale, mask=mask, device=dev, impl=args.impl,
+                      dustbin_index=dbi, dustbin_mass=case.dustbin_mass)
         hq, hk, hv, hdo = (torch.empty(q.shape, dtype=tdt, pin_memory=True) for _ in range(4))
         for h_, d_ in ((hq, q), (hk, k), (hv, v), (hdo, dO)):
             h_.copy_(d_)
@@ -500,8 +498,9 @@ def main():
         t_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
         line["e2e"] = {"value": total_entries / (t_e2e * 1e-3), "unit": UNIT, "ms_per_step": t_e2e,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "api": "HostStep: eot_sinkhorn_fwd + eot_sinkhorn_bwd per (batch, head) chunk on "
-                              "three streams, pinned host inputs copied in and results copied out every step"}
+                       "api": f"HostStep: eot_sinkhorn_fwd + eot_sinkhorn_bwd per chunk ({len(hs.chunks())} chunks "
+                              f"of {'%d batch rows' % hs.rows if hs.rows else '%d head(s) of one row' % hs.hc}) "
+                              "on three streams, pinned host inputs copied in and results copied out every step"}
 
     # ---------------- CPU baseline: the oracle on the host cores (rank 0, N = 1) ----------------
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -75,3 +75,33 @@ def test_long_workload_support_size_closed_form():
     c.Q = np.zeros((1, 4, 131072, 1), np.float32)
     c.W, c.mask, c.dustbin, c.dustbin_index, c.dustbin_mass = 1024, None, False, -1, 0.0
     assert bench.band_support_size(c) == 4 * (131072 * 1025 - 512 * 513)
+
+
+@pytest.mark.parametrize("B,H,kw,n_want", [
+    (1, 4, {}, 4),                       # long context: one head per chunk
+    (4, 8, {}, 4),                       # whole rows
+    (32, 4, {}, 4),                      # many short units: 8 rows per chunk
+    (5, 2, {}, 3),                       # ragged last chunk of rows
+    (2, 3, {}, 6),                       # too few rows: heads of one row
+    (3, 2, {"rows_per_chunk": 2}, 2),
+    (3, 2, {"heads_per_chunk": 2}, 3),
+])
+def test_host_step_chunk_plans(B, H, kw, n_want):
+    """Every (batch, head) unit of a host-memory step lands in exactly one chunk, in order, and
+    the automatic plan keeps many short units together instead of one call per unit."""
+    from entropic_ot_attention_b200.host_pipeline import chunk_list, plan_chunks
+    rows, hc = plan_chunks(B, H, **kw)
+    chunks = chunk_list(B, H, rows, hc)
+    assert len(chunks) == n_want
+    seen = [(b, h) for b0, b1, h0, h1 in chunks for b in range(b0, b1) for h in range(h0, h1)]
+    assert seen == [(b, h) for b in range(B) for h in range(H)]
+
+
+def test_host_step_chunk_plan_errors():
+    from entropic_ot_attention_b200.host_pipeline import plan_chunks
+    with pytest.raises(ValueError):
+        plan_chunks(2, 4, heads_per_chunk=3)
+    with pytest.raises(ValueError):
+        plan_chunks(2, 4, rows_per_chunk=3)
+    with pytest.raises(ValueError):
+        plan_chunks(2, 4, heads_per_chunk=1, rows_per_chunk=1)

@@ -175,12 +175,15 @@ def test_kernel_family_selection():
     assert _abi.eot_validate(wide_tc) == 2   # EOT_ERR_UNSUPPORTED
 
 
-def test_host_step_matches_device_calls():
-    """HostStep (chunks of heads on three streams, host buffers) gives bit-identical results to
-    one device-resident forward + backward over the whole batch: the units are independent."""
+@pytest.mark.parametrize("plan", [{"heads_per_chunk": 1}, {"rows_per_chunk": 1}, {"rows_per_chunk": 2}, {}],
+                         ids=["heads1", "rows1", "rows2_ragged", "auto"])
+def test_host_step_matches_device_calls(plan):
+    """HostStep (chunks of heads of one row, or of whole rows, on three streams, host buffers)
+    gives bit-identical results to one device-resident forward + backward over the whole batch:
+    the units are independent.  rows_per_chunk=2 over B=3 leaves a smaller last chunk."""
     import torch
     from entropic_ot_attention_b200 import HostStep, sinkhorn_bwd, sinkhorn_fwd
-    case = eot_inputs.dense_case(2, 3, 384, 64, 96, 4, 2, "bf16", seed=21, mask=_ragged_mask(2, 384, 21),
+    case = eot_inputs.dense_case(3, 2, 384, 64, 96, 4, 2, "bf16", seed=21, mask=_ragged_mask(3, 384, 21),
                                  name="host_step")
     dt = torch.bfloat16
     q, k, v, dO = (torch.from_numpy(x).to(dt) for x in (case.Q, case.K, case.V, case.dO))
@@ -189,7 +192,7 @@ def test_host_step_matches_device_calls():
     dQ, dK, dV = sinkhorn_bwd(q.cuda(), k.cuda(), v.cuda(), ut, vt, dO.cuda(), case.W, mask=mask.cuda(),
                               scale=case.scale)
     B, H, L, d = q.shape
-    hs = HostStep(B, H, L, d, case.W, case.T, case.R, dt, case.scale, mask=mask, heads_per_chunk=1)
+    hs = HostStep(B, H, L, d, case.W, case.T, case.R, dt, case.scale, mask=mask, **plan)
     host = [t.pin_memory() for t in (q, k, v, dO)]
     outs = [torch.empty_like(q).pin_memory() for _ in range(4)]
     for _ in range(2):   # slots reused across steps
