@@ -102,8 +102,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // two MMAs.  Roles:
 //   warp 0       TMA producer (one lane): row halves into a small ring, column tiles into
 //                NS stages, and per half the tile's column vectors (log2 bias, weights)
-//   warp 1       TMEM allocator and MMA issuer (one lane): two 128-column fp32 score
-//                accumulators per half (4 x 128 TMEM columns)
+//   warp 1       TMEM allocator and MMA issuer of the first half (one lane); warp 18 issues
+//                the second half's MMAs: two 128-column fp32 score accumulators per half
+//                (4 x 128 TMEM columns).  One issue thread per half, because one thread's
+//                per-MMA bookkeeping for both halves was slower than the tensor core.
 //   warps 2..9   epilogue of the first half, warps 10..17 of the second: warp (q, hf) reads
 //                TMEM lanes [32 q, 32 q + 32) and columns [64 hf, 64 hf + 64) of each tile
 // The two warps that share a row meet once per item on a 64-thread named barrier; the
