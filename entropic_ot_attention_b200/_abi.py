@@ -70,6 +70,8 @@ lib.eot_last_device_status.argtypes = [_vp, _vp]
 lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
 lib.eot_device_status_bits.restype = ctypes.c_int
+lib.eot_sq_norms.argtypes = [_vp, _vp, _sz, ctypes.c_int, _vp, _vp]
+lib.eot_sq_norms.restype = ctypes.c_int
 
 lib.eot_sinkhorn_fwd_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.eot_sinkhorn_fwd_static.restype = ctypes.c_int
@@ -163,3 +165,9 @@ def eot_device_status_bits(workspace: int, stream: int) -> int:
     bits = ctypes.c_uint32(0)
     _check(lib.eot_device_status_bits(workspace, stream, ctypes.byref(bits)), "eot_device_status_bits")
     return int(bits.value)
+
+
+def eot_sq_norms(a: int, b: int, n: int, dtype: int, out: int, stream: int) -> None:
+    """out[0] = sum (a - b)^2, out[1] = sum a^2 over n elements (raw device addresses; out is a
+    device array of two float64), enqueued on ``stream``."""
+    _check(lib.eot_sq_norms(a, b, n, dtype, out, stream), "eot_sq_norms")

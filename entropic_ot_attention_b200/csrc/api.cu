@@ -527,6 +527,15 @@ eot_status eot_device_status_bits(void* workspace, void* stream, uint32_t* bits)
     return EOT_OK;
 }
 
+eot_status eot_sq_norms(const void* a, const void* b, size_t n, eot_dtype dtype, double* out, void* stream) {
+    if (!out || (n > 0 && (!a || !b)) || (dtype != EOT_FP32 && dtype != EOT_BF16)) return EOT_ERR_INVALID_ARGUMENT;
+    int dev = 0, n_sm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = aux(st, [&] { return eot::launch_sq_norms(a, b, n, int(dtype), out, n_sm, st); });
+    return e == cudaSuccess ? EOT_OK : EOT_ERR_CUDA;
+}
+
 eot_status eot_last_device_status(void* workspace, void* stream) {
     uint32_t bits = 0;
     eot_status s = eot_device_status_bits(workspace, stream, &bits);

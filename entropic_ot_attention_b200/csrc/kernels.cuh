@@ -28,6 +28,8 @@ cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
 cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
 cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st);
 cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st);
+cudaError_t launch_sq_norms(const void* a, const void* b, size_t n, int dtype, double* out, int n_sm,
+                            cudaStream_t st);
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st);
 cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 

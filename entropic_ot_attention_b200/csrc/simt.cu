@@ -12,6 +12,8 @@
 // owns column l of the current tile.  Row-side operands stay in shared memory for the
 // whole sweep, column-side operands are staged per tile.  Scores are exact fp32 dot
 // products (FFMA), which keeps fp32 inputs at fp32 accuracy.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace eot {
@@ -654,6 +656,57 @@ __global__ void __launch_bounds__(1024) tile_bits_kernel(Geom g, const float* lo
     if (lane == 0 && vote) atomicOr(&acc, 1u << warp);
     __syncthreads();
     if (threadIdx.x == 0) bits[blockIdx.x] = acc;
+}
+
+// Squared norms for the tail's bias certificate: out[0] += sum (a - b)^2, out[1] += sum a^2,
+// accumulated in float64 (grid-stride loop, warp shuffles, one pair of atomics per block).
+template <typename T>
+__global__ void sq_norms_kernel(const T* __restrict__ a, const T* __restrict__ b, size_t n, double* out) {
+    double sd = 0.0, sa = 0.0;
+    for (size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += size_t(gridDim.x) * blockDim.x) {
+        const double x = to_f(a[i]), y = to_f(b[i]);
+        sd = fma(x - y, x - y, sd);
+        sa = fma(x, x, sa);
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        sd += __shfl_down_sync(0xffffffffu, sd, o);
+        sa += __shfl_down_sync(0xffffffffu, sa, o);
+    }
+    __shared__ double part[2][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    if (lane == 0) {
+        part[0][warp] = sd;
+        part[1][warp] = sa;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        sd = lane < nw ? part[0][lane] : 0.0;
+        sa = lane < nw ? part[1][lane] : 0.0;
+        for (int o = 16; o > 0; o >>= 1) {
+            sd += __shfl_down_sync(0xffffffffu, sd, o);
+            sa += __shfl_down_sync(0xffffffffu, sa, o);
+        }
+        if (lane == 0) {
+            atomicAdd(out, sd);
+            atomicAdd(out + 1, sa);
+        }
+    }
+}
+
+cudaError_t launch_sq_norms(const void* a, const void* b, size_t n, int dtype, double* out, int n_sm,
+                            cudaStream_t st) {
+    cudaError_t e = cudaMemsetAsync(out, 0, 2 * sizeof(double), st);
+    if (e != cudaSuccess || n == 0) return e;
+    const int threads = 256;
+    const size_t want = (n + threads - 1) / threads;
+    const int blocks = int(std::min<size_t>(want, size_t(4) * size_t(n_sm)));
+    if (dtype == EOT_BF16)
+        sq_norms_kernel<<<blocks, threads, 0, st>>>(static_cast<const __nv_bfloat16*>(a),
+                                                    static_cast<const __nv_bfloat16*>(b), n, out);
+    else
+        sq_norms_kernel<<<blocks, threads, 0, st>>>(static_cast<const float*>(a), static_cast<const float*>(b), n,
+                                                    out);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st) {

@@ -174,6 +174,17 @@ eot_status eot_sinkhorn_fwd_static(const eot_problem* p, const void* Q, const vo
  * the problem is invalid or unsupported. */
 int eot_resolved_impl(const eot_problem* p);
 
+/* Norms for the a-posteriori bias certificate of the tail ("Blockwise Differentiable Sinkhorn
+ * Attention" §2.4, third certificate: measure how far the tail gradient is from the gradient
+ * through the whole solve, and choose the tail depth from it).  Accumulates, in float64,
+ *     out[0] = sum_i (a_i - b_i)^2,    out[1] = sum_i a_i^2
+ * over the n elements of the device arrays a and b (element type ``dtype``, e.g. two tail
+ * gradients).  ``out`` is a device array of two doubles, overwritten.  Stream-ordered and
+ * asynchronous; the summation order varies between runs (float64 atomics), so the last bits
+ * may too.  Null pointers (a, b with n > 0) or an unknown dtype return
+ * EOT_ERR_INVALID_ARGUMENT before anything is enqueued; a launch failure EOT_ERR_CUDA. */
+eot_status eot_sq_norms(const void* a, const void* b, size_t n, eot_dtype dtype, double* out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,6 +9,10 @@ CPU: the full-gradient oracle (``oracle.bptt``, torch autodiff) is pinned agains
 hand-written tail adjoint of ``oracle.eot_oracle`` (independent code) for every base / tail
 split of a fixed step count, and against central differences of the forward.  GPU: the kernels'
 tail gradients for R = 0, 1, 2, 4 give the same bias curve as the oracle's.
+
+BDSA §2.4 (third certificate): the a-posteriori certificate (``entropic_ot_attention_b200.
+certificate``) is checked against the true residual on the CPU and, on the GPU, computed by
+the library and compared with the same quantities from oracle gradients.
 """
 import math
 
@@ -121,3 +125,89 @@ def test_tail_bias_curve_matches_oracle():
             assert abs(gpu_bias - curve[R]) <= 2e-4 + 1e-2 * curve[R]
     for curve in rows:
         assert curve[0] > curve[1] > curve[2] > curve[4]
+
+
+# ----------------------------------------------------------------------------------------
+# A-posteriori certificate (BDSA §2.4, third certificate; §4.1)
+# ----------------------------------------------------------------------------------------
+def test_geometric_estimate_closed_forms():
+    from entropic_ot_attention_b200.certificate import geometric_estimate
+    assert geometric_estimate(0.3, 0.5, 0) == 0.0
+    assert geometric_estimate(0.3, None, 1) == 0.3
+    assert geometric_estimate(0.3, 0.5, 3) == pytest.approx(0.3 + 0.15 + 0.075)
+    assert geometric_estimate(0.3, 1.0, 3) == math.inf
+    assert geometric_estimate(0.3, None, 2) == math.inf
+
+
+def _oracle_tails(q, k, v, dO, W, N, **kw):
+    """Stacked (dq, dk, dv) of every tail depth 0..N from the oracle (depth N: nothing stopped)."""
+    return {R: np.concatenate([g.ravel() for g in bptt.gradient_unit(q, k, v, dO, W, N, N - R, **kw)])
+            for R in range(N + 1)}
+
+
+def _oracle_certificates(tails, N):
+    """eta_R, rho_R and the certificate eta_hat_R from oracle tail gradients, with the same
+    reading as the library's (the formula under test is the library's geometric_estimate)."""
+    from entropic_ot_attention_b200.certificate import geometric_estimate
+    eta = {R: np.linalg.norm(tails[R + 1] - tails[R]) / np.linalg.norm(tails[R]) for R in range(N)}
+    out = {}
+    for R in range(N):
+        rho = eta[R + 1] / eta[R] if R + 1 < N else None
+        out[R] = (eta[R], rho, geometric_estimate(eta[R], rho, N - R))
+    return out
+
+
+def test_certificate_tracks_the_true_residual():
+    """On a banded, masked unit the certificate stays within a factor 2 of the true residual
+    |g(N) - g(R)| / |g(N)| from full backpropagation (the pages: it reconstructs the residual),
+    or declines (+inf) where the increments stop shrinking: the first steps from v = 0 move the
+    gradient more than the geometric model allows, so with two increments left it has none."""
+    L, d, W, N = 96, 16, 24, 12
+    mask = np.ones(L, np.uint8)
+    mask[[10, 50, 51, 90]] = 0
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((L, d)) for _ in range(3))
+    dO = rng.standard_normal((L, d))
+    tails = _oracle_tails(q, k, v, dO, W, N, mask_row=mask)
+    certs = _oracle_certificates(tails, N)
+    for R in range(N):
+        true = np.linalg.norm(tails[N] - tails[R]) / np.linalg.norm(tails[N])
+        est = certs[R][2]
+        if R <= N - 3:
+            assert math.isfinite(est), R
+        assert est == math.inf or 0.5 * true <= est <= 2.0 * true, (R, true, est)
+
+
+@pytest.mark.gpu
+def test_bias_certificate_matches_oracle():
+    """The library's certificate (tail gradients and norms on the GPU, fp32) equals the oracle's
+    at every depth, its exact residual equals full backpropagation's, and choose_tail_depth
+    picks the oracle's depth for tolerances away from the certificate values."""
+    import torch
+    from entropic_ot_attention_b200 import bias_certificate, choose_tail_depth
+    B, H, L, d, W, N = 1, 2, 256, 32, 32, 8
+    case = eot_inputs.dense_case(B, H, L, d, W, 0, N, "fp32", seed=78, name="certificate")
+    dev = torch.device("cuda:0")
+    q, k, v, dO = (torch.from_numpy(x).to(dev).contiguous() for x in (case.Q, case.K, case.V, case.dO))
+    per_head = [_oracle_tails(*(x[0, h].astype(np.float64) for x in (case.Q, case.K, case.V, case.dO)), W, N)
+                for h in range(H)]
+    tails = {R: np.concatenate([t[R] for t in per_head]) for R in range(N + 1)}   # both units, as the GPU
+    certs = _oracle_certificates(tails, N)
+    for R in range(N - 1):
+        c = bias_certificate(q, k, v, dO, W, N, R, exact=True)
+        eta, rho, est = certs[R]
+        true = np.linalg.norm(tails[N] - tails[R]) / np.linalg.norm(tails[N])
+        print(f"R={R}: eta {c['eta']:.4e} (oracle {eta:.4e})  rho {c['rho']:.4f}  "
+              f"estimate {c['estimate']:.4e} (oracle {est:.4e})  exact {c['exact']:.4e} (oracle {true:.4e})")
+        # eta is a difference of two nearly equal fp32 gradients (1e-3 of their size at the
+        # deeper tails), so a gradient error of ~1e-6 becomes ~1e-3 of eta
+        assert c["eta"] == pytest.approx(eta, rel=1e-2, abs=1e-6)
+        assert c["estimate"] == pytest.approx(est, rel=1e-2, abs=1e-6)
+        assert c["exact"] == pytest.approx(true, rel=5e-3, abs=1e-6)
+    ests = [certs[R][2] for R in range(N - 1)]
+    for tau in (0.1, 0.03, 0.008, 0.003):
+        if any(abs(e - tau) <= 0.05 * tau for e in ests):
+            continue   # too close to a certificate value to compare the choice
+        want = next((R for R, e in enumerate(ests) if e <= tau), None)
+        got, _ = choose_tail_depth(q, k, v, dO, W, N, tau=tau, R_max=N - 2)
+        assert got == want, (tau, got, want)
