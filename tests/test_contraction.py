@@ -1,0 +1,71 @@
+"""Projective contraction certificate of the band's strictly positive blocks (BDSA §2.4, second
+certificate: Hilbert's projective metric shows the strictly positive active blocks of the
+Sinkhorn map contract).
+
+CPU: the oracle's diameter (``oracle.contraction``) against its definition by brute force,
+closed forms, the Birkhoff-Hopf bound itself on random positive vectors, and the symmetry of
+the diameter under transposition.  GPU: the library's per-tile ratios against the oracle's.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import eot_inputs
+from oracle import contraction as oc
+
+
+@pytest.mark.parametrize("shape,seed", [((3, 4), 0), ((5, 5), 1), ((4, 2), 2), ((6, 3), 3)])
+def test_diameter_equals_its_definition(shape, seed):
+    B = np.random.default_rng(seed).standard_normal(shape) * 2.0
+    assert oc.block_diameter(B) == pytest.approx(oc.block_diameter_brute(B), rel=1e-13, abs=1e-13)
+
+
+def test_rank_one_and_two_by_two_closed_forms():
+    rng = np.random.default_rng(4)
+    a, b = rng.standard_normal(7), rng.standard_normal(5)
+    assert oc.block_diameter(a[:, None] + b[None, :]) == pytest.approx(0.0, abs=1e-12)   # one ray
+    for x in (0.3, -1.7, 5.0):
+        assert oc.block_diameter(np.array([[0.0, 0.0], [0.0, x]])) == pytest.approx(abs(x))
+    assert oc.block_diameter(np.ones((1, 6))) == 0.0 and oc.block_diameter(np.ones((6, 1))) == 0.0
+
+
+@pytest.mark.parametrize("seed", [5, 6, 7])
+def test_birkhoff_hopf_bound_holds(seed):
+    """d_H(K x, K y) <= tanh(Delta / 4) d_H(x, y) for K = exp(B) and positive x, y."""
+    rng = np.random.default_rng(seed)
+    B = rng.standard_normal((8, 6))
+    K = np.exp(B)
+    kappa = math.tanh(oc.block_diameter(B) / 4.0)
+    assert 0.0 < kappa < 1.0
+    worst = 0.0
+    for _ in range(2000):
+        x, y = np.exp(rng.standard_normal(6) * 2), np.exp(rng.standard_normal(6) * 2)
+        ratio = oc.hilbert_distance(K @ x, K @ y) / oc.hilbert_distance(x, y)
+        assert ratio <= kappa + 1e-12
+        worst = max(worst, ratio)
+    assert worst > 0.2 * kappa   # the bound is not vacuous on this block
+
+
+def test_tiles_transpose_symmetry_and_edges():
+    """Delta(B) = Delta(B^T): tile (I, I + o) of (q, k) equals tile (I + o, I) of (k, q).  Tiles
+    out of range and tiles without active tokens are -1; a band narrower than a tile has none."""
+    rng = np.random.default_rng(8)
+    L, d, W, t = 40, 3, 24, 4                      # tile 4: m = (12 - 3) // 4 = 2
+    q, k = rng.standard_normal((L, d)), rng.standard_normal((L, d))
+    mask = np.ones(L, np.uint8)
+    mask[8:12] = 0                                 # tile 2 wholly inactive
+    a = oc.contraction_tiles(q, k, W, mask_row=mask, tile=t)
+    b = oc.contraction_tiles(k, q, W, mask_row=mask, tile=t)
+    m = oc.offsets(W, t)
+    assert m == 2 and a.shape == (10, 5)
+    for I in range(10):
+        for o in range(-m, m + 1):
+            J = I + o
+            if 0 <= J < 10:
+                assert a[I, o + m] == pytest.approx(b[J, -o + m], abs=1e-13)
+            else:
+                assert a[I, o + m] == -1.0
+    assert np.all(a[2] == -1.0) and a[0, 2 + m] == -1.0   # rows of tile 2, columns of tile 2
+    assert ((a == -1.0) | ((a >= 0.0) & (a < 1.0))).all()
+    assert oc.contraction_tiles(q, k, 4, tile=t).shape == (10, 0)   # W // 2 = 2 < t - 1
