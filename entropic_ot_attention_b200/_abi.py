@@ -72,6 +72,10 @@ lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)
 lib.eot_device_status_bits.restype = ctypes.c_int
 lib.eot_sq_norms.argtypes = [_vp, _vp, _sz, ctypes.c_int, _vp, _vp]
 lib.eot_sq_norms.restype = ctypes.c_int
+lib.eot_contraction_offsets.argtypes = [_P]
+lib.eot_contraction_offsets.restype = ctypes.c_int
+lib.eot_contraction.argtypes = [_P, _vp, _vp, _vp, _vp, _vp]
+lib.eot_contraction.restype = ctypes.c_int
 
 lib.eot_sinkhorn_fwd_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.eot_sinkhorn_fwd_static.restype = ctypes.c_int
@@ -171,3 +175,12 @@ def eot_sq_norms(a: int, b: int, n: int, dtype: int, out: int, stream: int) -> N
     """out[0] = sum (a - b)^2, out[1] = sum a^2 over n elements (raw device addresses; out is a
     device array of two float64), enqueued on ``stream``."""
     _check(lib.eot_sq_norms(a, b, n, dtype, out, stream), "eot_sq_norms")
+
+
+def eot_contraction_offsets(p: eot_problem) -> int:
+    return int(lib.eot_contraction_offsets(ctypes.byref(p)))
+
+
+def eot_contraction(p: eot_problem, Q: int, K: int, mask: int | None, kappa: int, stream: int) -> None:
+    """Per-tile Birkhoff-Hopf ratios into kappa (raw device addresses; mask may be None)."""
+    _check(lib.eot_contraction(ctypes.byref(p), Q, K, mask, kappa, stream), "eot_contraction")

@@ -141,3 +141,26 @@ def choose_tail_depth(q, k, v, dO, W: int, N: int, tau: float = 1e-5, R_max: int
         if c["estimate"] <= tau:
             return R, certs
     return None, certs
+
+
+def contraction_certificate(q, k, W: int, mask=None, scale=None, dustbin_index=None, stream=None):
+    """Projective contraction certificate of the band's strictly positive blocks
+    ("Blockwise Differentiable Sinkhorn Attention" §2.4, second certificate): for every pair of
+    128-position tiles (I, I + o) that lies wholly inside the band, the Birkhoff-Hopf ratio
+    tanh(Delta / 4) < 1 of exp(S) on the block's active real tokens (eot_contraction).
+
+    Returns a float32 tensor [B, H, ceil(L / 128), 2 m + 1] (offset o at index o + m, -1 where
+    the pair is out of range or has no active token), empty in its last dimension when the
+    band is narrower than a tile."""
+    from .api import _check_inputs, _stream, make_problem
+    _check_inputs(q, k, k, mask)
+    B, H, L, d = q.shape
+    p = make_problem(B, H, L, d, W, 0, 0, q.dtype, scale, dustbin_index, 0.1 if dustbin_index is not None else 0.0)
+    n = _abi.eot_contraction_offsets(p)
+    if n < 0:
+        raise ValueError(f"problem rejected: {_abi.eot_status_string(_abi.eot_validate(p))}")
+    kappa = torch.empty((B, H, (L + 127) // 128, n), dtype=torch.float32, device=q.device)
+    if n > 0 and kappa.numel() > 0:
+        m = None if mask is None else mask.view(torch.uint8).data_ptr()
+        _abi.eot_contraction(p, q.data_ptr(), k.data_ptr(), m, kappa.data_ptr(), _stream(stream))
+    return kappa

@@ -536,6 +536,37 @@ eot_status eot_sq_norms(const void* a, const void* b, size_t n, eot_dtype dtype,
     return e == cudaSuccess ? EOT_OK : EOT_ERR_CUDA;
 }
 
+int eot_contraction_offsets(const eot_problem* p) {
+    if (validate(p) != EOT_OK) return -1;
+    const int h = p->W / 2;
+    return h >= 127 ? 2 * ((h - 127) / 128) + 1 : 0;
+}
+
+eot_status eot_contraction(const eot_problem* p, const void* Q, const void* K, const uint8_t* mask, float* kappa,
+                           void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (empty(*p)) return EOT_OK;
+    if (!Q || !K || !kappa) return EOT_ERR_INVALID_ARGUMENT;
+    const int n_off = eot_contraction_offsets(p);
+    if (n_off == 0) return EOT_OK;
+    eot::ContractArgs a{};
+    a.Q = Q;
+    a.K = K;
+    a.mask = mask;
+    a.H = p->H;
+    a.L = p->L;
+    a.d = p->d;
+    a.nT = (p->L + 127) / 128;
+    a.m = (n_off - 1) / 2;
+    a.D = p->dustbin ? p->dustbin_index : -1;
+    a.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(float(p->d));
+    a.kappa = kappa;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = aux(st, [&] { return eot::launch_contraction(a, int(p->dtype), p->B * p->H, st); });
+    return e == cudaSuccess ? EOT_OK : EOT_ERR_CUDA;
+}
+
 eot_status eot_last_device_status(void* workspace, void* stream) {
     uint32_t bits = 0;
     eot_status s = eot_device_status_bits(workspace, stream, &bits);

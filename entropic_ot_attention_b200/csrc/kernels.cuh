@@ -30,6 +30,21 @@ cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cu
 cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st);
 cudaError_t launch_sq_norms(const void* a, const void* b, size_t n, int dtype, double* out, int n_sm,
                             cudaStream_t st);
+
+// Projective contraction certificate: per tile pair wholly inside the band, tanh(Delta / 4) of
+// exp(S) on the block's active real tokens (CUDA cores, scores in fp32).
+struct ContractArgs {
+    const void* Q;
+    const void* K;
+    const uint8_t* mask;   // [B, L] or null (every position real and active)
+    int H, L, d;
+    int nT;                // 128-position tiles, ceil(L / 128)
+    int m;                 // offsets -m..m (m >= 0)
+    int D;                 // dustbin index: positions >= D are left out; -1 without a dustbin
+    float scale;
+    float* kappa;          // [B H, nT, 2 m + 1]
+};
+cudaError_t launch_contraction(const ContractArgs& a, int dtype, int BH, cudaStream_t st);
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st);
 cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 

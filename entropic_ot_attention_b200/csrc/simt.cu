@@ -709,6 +709,140 @@ cudaError_t launch_sq_norms(const void* a, const void* b, size_t n, int dtype, d
     return cudaGetLastError();
 }
 
+// Projective contraction certificate of the band's strictly positive blocks (the summary's
+// §2.4, second certificate: with Hilbert's projective metric the strictly positive active
+// blocks of the Sinkhorn map contract).  For a positive block K = exp(S) the Birkhoff-Hopf
+// ratio is tanh(Delta / 4), Delta = max over rows i, i' and columns j, j' of
+// S_ij + S_i'j' - S_ij' - S_i'j = max over row pairs of the range over j of S_ij - S_i'j.
+// One CTA per tile pair (I, J = I + o), |o| <= m (pairs wholly inside the band); the block is
+// restricted to its active real tokens.  The 128 x 128 score block is formed in fp32 in shared
+// memory (rows padded to 129 floats: the pair loop reads 32 different rows per warp).
+constexpr int kCT = 128, kCThreads = 256, kCChunk = 32;
+
+size_t contraction_smem() {
+    return (size_t(kCT) * (kCT + 1) + 2 * size_t(kCT) * (kCChunk + 1)) * sizeof(float) + 2 * kCT * sizeof(int);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kCThreads) contraction_kernel(ContractArgs a) {
+    extern __shared__ float csm[];
+    float* S = csm;                                  // [128][129]
+    float* Qs = S + kCT * (kCT + 1);                 // [128][33]: one 32-column chunk of the row tile
+    float* Ks = Qs + kCT * (kCChunk + 1);            // [128][33]: ... of the column tile
+    int* ract = reinterpret_cast<int*>(Ks + kCT * (kCChunk + 1));
+    int* cact = ract + kCT;
+    __shared__ float wmax[kCThreads / 32];
+    __shared__ int nact[2];
+    const int I = blockIdx.x, oi = blockIdx.y, bh = blockIdx.z, b = bh / a.H;
+    const int J = I + oi - a.m;
+    const int tid = threadIdx.x;
+    float* outp = a.kappa + (size_t(bh) * a.nT + I) * size_t(2 * a.m + 1) + oi;
+    if (J < 0 || J >= a.nT) {
+        if (tid == 0) *outp = -1.f;
+        return;
+    }
+    const int r0 = I * kCT, c0 = J * kCT;
+    if (tid < 2) nact[tid] = 0;
+    __syncthreads();
+    auto active = [&](int pos) -> int {
+        if (pos >= a.L || (a.D >= 0 && pos >= a.D)) return 0;
+        return a.mask == nullptr || a.mask[size_t(b) * a.L + pos] != 0;
+    };
+    {
+        const int t = tid & (kCT - 1);
+        const int f = active((tid < kCT ? r0 : c0) + t);
+        (tid < kCT ? ract : cact)[t] = f;
+        if (f) atomicAdd(&nact[tid < kCT ? 0 : 1], 1);
+    }
+    // S = scale Q_I K_J^T; thread (ty, tx) owns rows 8 ty .. 8 ty + 7 and columns tx + 16 j
+    const T* Qg = static_cast<const T*>(a.Q) + size_t(bh) * a.L * a.d;
+    const T* Kg = static_cast<const T*>(a.K) + size_t(bh) * a.L * a.d;
+    const int ty = tid >> 4, tx = tid & 15;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int k0 = 0; k0 < a.d; k0 += kCChunk) {
+        __syncthreads();   // the previous chunk has been read
+        for (int e = tid; e < kCT * kCChunk; e += kCThreads) {
+            const int r = e / kCChunk, c = e % kCChunk, col = k0 + c;
+            float qv = 0.f, kv = 0.f;
+            if (col < a.d) {
+                if (r0 + r < a.L) qv = to_f(Qg[size_t(r0 + r) * a.d + col]);
+                if (c0 + r < a.L) kv = to_f(Kg[size_t(c0 + r) * a.d + col]);
+            }
+            Qs[r * (kCChunk + 1) + c] = qv;
+            Ks[r * (kCChunk + 1) + c] = kv;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int c = 0; c < kCChunk; ++c) {
+            float qr[8], kc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) qr[i] = Qs[(8 * ty + i) * (kCChunk + 1) + c];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) kc[j] = Ks[(tx + 16 * j) * (kCChunk + 1) + c];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(qr[i], kc[j], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) S[(8 * ty + i) * (kCT + 1) + tx + 16 * j] = a.scale * acc[i][j];
+    __syncthreads();
+    if (nact[0] == 0 || nact[1] == 0) {   // no block on this tile pair
+        if (tid == 0) *outp = -1.f;
+        return;
+    }
+    // Delta: warp w takes the partner rows i' = w, w + 8, ...; lane l the rows l + 32 s
+    const int warp = tid >> 5, lane = tid & 31;
+    float best = 0.f;
+    for (int ip = warp; ip < kCT; ip += kCThreads / 32) {
+        if (!ract[ip]) continue;
+        for (int s = 0; s < kCT / 32; ++s) {
+            const int i = lane + 32 * s;
+            float mx = -INFINITY, mn = INFINITY;
+            for (int j = 0; j < kCT; ++j) {
+                if (!cact[j]) continue;
+                const float dl = S[i * (kCT + 1) + j] - S[ip * (kCT + 1) + j];
+                mx = fmaxf(mx, dl);
+                mn = fminf(mn, dl);
+            }
+            if (ract[i]) best = fmaxf(best, mx - mn);
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (lane == 0) wmax[warp] = best;
+    __syncthreads();
+    if (tid == 0) {
+        float v = 0.f;
+        for (int w = 0; w < kCThreads / 32; ++w) v = fmaxf(v, wmax[w]);
+        *outp = tanhf(0.25f * v);
+    }
+}
+
+cudaError_t launch_contraction(const ContractArgs& a, int dtype, int BH, cudaStream_t st) {
+    if (a.m < 0 || a.nT == 0 || BH == 0) return cudaSuccess;
+    const size_t smem = contraction_smem();
+    const dim3 grid(a.nT, 2 * a.m + 1, BH);
+    if (dtype == EOT_BF16) {
+        cudaError_t e = cudaFuncSetAttribute(contraction_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        contraction_kernel<__nv_bfloat16><<<grid, kCThreads, smem, st>>>(a);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(contraction_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
+        if (e != cudaSuccess) return e;
+        contraction_kernel<float><<<grid, kCThreads, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st) {
     tile_bits_kernel<<<g.B * tile_words(g.L), 1024, 0, st>>>(g, logm, bits);
     return cudaGetLastError();

@@ -185,6 +185,25 @@ int eot_resolved_impl(const eot_problem* p);
  * EOT_ERR_INVALID_ARGUMENT before anything is enqueued; a launch failure EOT_ERR_CUDA. */
 eot_status eot_sq_norms(const void* a, const void* b, size_t n, eot_dtype dtype, double* out, void* stream);
 
+/* Projective contraction certificate ("Blockwise Differentiable Sinkhorn Attention" §2.4, second
+ * certificate: with Hilbert's projective metric, the strictly positive active blocks of the
+ * Sinkhorn map are contractions).  For every pair of 128-position tiles I (positions
+ * [128 I, 128 I + 128)) and J = I + o that lies wholly inside the band, |o| * 128 + 127 <= W / 2,
+ * the Birkhoff-Hopf ratio of the block exp(S) on its active real tokens:
+ *     kappa = tanh(Delta / 4),  Delta = max over rows i, i' and columns j, j' of
+ *                                       S_ij + S_i'j' - S_ij' - S_i'j,
+ * S = scale Q K^T formed in float32.  kappa is a caller-owned device float32 array
+ * [B, H, ceil(L / 128), n] with n = eot_contraction_offsets(p) = 2 m + 1 entries per tile
+ * (offset o at index o + m), -1 where J is out of range or the block has no active row or
+ * column.  Q, K and mask are those of eot_sinkhorn_fwd (p->dtype; the dustbin and the fillers
+ * after it are left out of every block); T and R are not used.  No workspace; stream-ordered and
+ * asynchronous.  eot_contraction_offsets returns 0 when no tile pair fits in the band (then
+ * eot_contraction writes nothing) and -1 for an invalid problem; eot_contraction reports
+ * argument errors as eot_sinkhorn_fwd does, before anything is enqueued. */
+int eot_contraction_offsets(const eot_problem* p);
+eot_status eot_contraction(const eot_problem* p, const void* Q, const void* K, const uint8_t* mask, float* kappa,
+                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif

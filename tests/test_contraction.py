@@ -69,3 +69,67 @@ def test_tiles_transpose_symmetry_and_edges():
     assert np.all(a[2] == -1.0) and a[0, 2 + m] == -1.0   # rows of tile 2, columns of tile 2
     assert ((a == -1.0) | ((a >= 0.0) & (a < 1.0))).all()
     assert oc.contraction_tiles(q, k, 4, tile=t).shape == (10, 0)   # W // 2 = 2 < t - 1
+
+
+def _ragged(B, L, seed):
+    rng = np.random.default_rng(seed)
+    m = np.zeros((B, L), np.uint8)
+    for b in range(B):
+        n = int(rng.integers(L // 2, L + 1))
+        m[b, :n] = 1
+        m[b, rng.choice(n, size=max(1, n // 40), replace=False)] = 0
+    return m
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kind", ["fp32_d40_masked", "bf16_d64_W1024", "bf16_dustbin_masked", "narrow_band"])
+def test_contraction_matches_oracle(kind):
+    """eot_contraction's per-tile ratios equal the oracle's (float64 scores from the same
+    inputs); the -1 entries (pairs out of range or without active tokens) match exactly."""
+    import torch
+    from entropic_ot_attention_b200 import contraction_certificate
+    D = None
+    if kind == "fp32_d40_masked":
+        case = eot_inputs.dense_case(2, 2, 640, 40, 700, 1, 1, "fp32", seed=31, mask=_ragged(2, 640, 31))
+    elif kind == "bf16_d64_W1024":
+        case = eot_inputs.dense_case(2, 1, 768, 64, 1024, 1, 1, "bf16", seed=32)
+    elif kind == "bf16_dustbin_masked":
+        case = eot_inputs.dustbin_case(1, 2, 500, 32, 600, 1, 1, "bf16", seed=33, mask=_ragged(1, 500, 33)[0:1])
+        D = case.dustbin_index
+    else:
+        case = eot_inputs.dense_case(1, 1, 256, 32, 200, 1, 1, "fp32", seed=34)
+    dev = torch.device("cuda:0")
+    tdt = torch.float32 if case.dtype == "fp32" else torch.bfloat16
+    q, k = (torch.from_numpy(x).to(dev).to(tdt).contiguous() for x in (case.Q, case.K))
+    mask = None if case.mask is None else torch.from_numpy(case.mask).to(dev)
+    kappa = contraction_certificate(q, k, case.W, mask=mask, scale=case.scale, dustbin_index=D)
+    torch.cuda.synchronize()
+    got = kappa.cpu().numpy()
+    B, H = case.Q.shape[:2]
+    for b in range(B):
+        for h in range(H):
+            want = oc.contraction_tiles(case.Q[b, h].astype(np.float64), case.K[b, h].astype(np.float64), case.W,
+                                        case.scale, None if case.mask is None else case.mask[b],
+                                        -1 if D is None else D)
+            assert got[b, h].shape == want.shape
+            assert np.array_equal(got[b, h] == -1.0, want == -1.0)
+            np.testing.assert_allclose(got[b, h], want, atol=1e-4, rtol=0)
+    if kind == "narrow_band":
+        assert got.shape[-1] == 0
+    else:
+        assert (got > 0.0).any()
+
+
+def test_offsets_and_argument_errors():
+    """eot_contraction_offsets follows |o| 128 + 127 <= W / 2; null tensors are refused before
+    anything is launched (no GPU needed)."""
+    import torch
+    from entropic_ot_attention_b200 import _abi, api
+    for W, n in ((1024, 7), (254, 1), (253, 0), (0, 0), (700, 3)):
+        p = api.make_problem(1, 2, 1024, 64, W, 1, 1, torch.bfloat16)
+        assert _abi.eot_contraction_offsets(p) == n == max(2 * oc.offsets(W) + 1, 0)
+    bad = api.make_problem(1, 2, 1000, 64, 512, 1, 1, torch.bfloat16)   # L not a multiple of 128
+    assert _abi.eot_contraction_offsets(bad) == -1
+    p = api.make_problem(1, 2, 1024, 64, 1024, 1, 1, torch.bfloat16)
+    assert _abi.lib.eot_contraction(__import__("ctypes").byref(p), None, None, None, None, None) == \
+        _abi.EOT_ERR_INVALID_ARGUMENT
