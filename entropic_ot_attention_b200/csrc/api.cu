@@ -448,7 +448,7 @@ const char* eot_status_string(eot_status s) {
     switch (s) {
         case EOT_OK: return "ok";
         case EOT_ERR_INVALID_ARGUMENT: return "invalid argument";
-        case EOT_ERR_UNSUPPORTED: return "unsupported problem for this build";
+        case EOT_ERR_UNSUPPORTED: return "unsupported problem for this library";
         case EOT_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
         case EOT_ERR_CUDA: return "CUDA error";
         case EOT_ERR_NONFINITE: return "non-finite potential produced on the device";

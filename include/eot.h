@@ -51,7 +51,7 @@ extern "C" {
 typedef enum {
     EOT_OK = 0,
     EOT_ERR_INVALID_ARGUMENT = 1,   /* bad size, pointer or flag; nothing was launched */
-    EOT_ERR_UNSUPPORTED = 2,        /* valid problem this build cannot run (e.g. impl/dtype) */
+    EOT_ERR_UNSUPPORTED = 2,        /* valid problem this library cannot run (e.g. impl/dtype) */
     EOT_ERR_WORKSPACE_TOO_SMALL = 3,
     EOT_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
     EOT_ERR_NONFINITE = 5,          /* device status: a non-finite potential was produced */

@@ -19,7 +19,7 @@ Italian).  Section numbers are that page's:
   to Q/K/V and the same balanced solver runs on the extended state space.
 
 The pages state the method in words; the concrete equations below are the plainest
-reading of them (each reading is listed in the design doc):
+reading of them:
 
 * score      S_ij = scale * <q_i, k_j>, scale = 1/sqrt(d) by default (temperature absorbed)
 * support    Omega = {(i, j) : i, j active, |i - j| <= W // 2}; with a dustbin D also
