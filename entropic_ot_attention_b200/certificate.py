@@ -22,6 +22,11 @@ With one increment left (R = N - 1) eta_hat = eta; with none (R = N) it is 0.  W
 library's largest tail depth reaches N the exact residual |g(N) - g(R)| / |g(N)| can be measured
 too.  Every norm is computed by the library (eot_sq_norms, float64 accumulation) from the
 library's gradients; this module orders the calls and combines float64 scalars.
+
+Precision: eta is a difference of two nearly equal gradients.  With float32 tensors the
+gradients' own error (~1e-6 relative) is far below the increments; bfloat16 gradients are
+rounded to ~4e-3 relative, which swamps the increments of all but the first depths, so run the
+certificate on float32 copies of the inputs.
 """
 from __future__ import annotations
 
