@@ -211,3 +211,53 @@ def test_bias_certificate_matches_oracle():
         want = next((R for R, e in enumerate(ests) if e <= tau), None)
         got, _ = choose_tail_depth(q, k, v, dO, W, N, tau=tau, R_max=N - 2)
         assert got == want, (tau, got, want)
+
+
+def test_choose_tail_depth_control_flow(monkeypatch):
+    """The depth search on the host, with the library calls replaced by a synthetic gradient
+    sequence whose increments shrink by 1/2 per step (g(N) - g(R) known in closed form): each
+    depth is computed once, the first depth whose certificate is <= tau is returned, and the
+    certificate equals the geometric sum exactly when the increments are geometric."""
+    import numpy as np
+    from entropic_ot_attention_b200 import certificate as cm
+    N = 8
+    base = np.ones(4)
+    step = np.array([1.0, -2.0, 0.5, 3.0])
+
+    def g(R):   # g(R) = base + sum_{j < R} step * 0.5^(N - 1 - j): increments grow toward the full gradient
+        return base + sum(step * 0.5 ** (N - 1 - j) for j in range(R))
+
+    calls = []
+
+    def fake_tail(q, k, v, dO, W, N_, R, **kw):
+        calls.append(R)
+        return (g(R),)
+
+    def fake_norms(ga, gb, stream=None):
+        a, b = ga[0], gb[0]
+        return float(np.sum((a - b) ** 2)), float(np.sum(a ** 2))
+
+    monkeypatch.setattr(cm, "tail_gradients", fake_tail)
+    monkeypatch.setattr(cm, "_norms", fake_norms)
+    R, certs = cm.choose_tail_depth(None, None, None, None, 0, N, tau=1e-9)
+    assert R is None and len(calls) == len(set(calls))          # every depth computed once
+    # increments double with R here (rho = 2): no certificate except with one step left
+    assert all(c["estimate"] == math.inf for c in certs[:-1])
+    c = cm.bias_certificate(None, None, None, None, 0, N, N - 1)
+    assert c["estimate"] == pytest.approx(np.linalg.norm(g(N) - g(N - 1)) / np.linalg.norm(g(N - 1)))
+
+    # reversed: increments halve with R (rho = 1/2), the certificate is the exact geometric sum
+    def g2(R):
+        return base + sum(step * 0.5 ** j for j in range(R))
+
+    monkeypatch.setattr(cm, "tail_gradients", lambda q, k, v, dO, W, N_, R, **kw: (g2(R),))
+    R2 = 3
+    c = cm.bias_certificate(None, None, None, None, 0, N, R2)
+    eta = np.linalg.norm(g2(R2 + 1) - g2(R2)) / np.linalg.norm(g2(R2))
+    eta1 = np.linalg.norm(g2(R2 + 2) - g2(R2 + 1)) / np.linalg.norm(g2(R2 + 1))
+    assert c["eta"] == pytest.approx(eta) and c["rho"] == pytest.approx(eta1 / eta)
+    assert c["estimate"] == pytest.approx(eta * (1 - (eta1 / eta) ** (N - R2)) / (1 - eta1 / eta))
+    tau = c["estimate"] * 1.01
+    R, certs = cm.choose_tail_depth(None, None, None, None, 0, N, tau=tau)
+    assert R is not None and R <= R2 and certs[-1]["estimate"] <= tau
+    assert all(cc["estimate"] > tau for cc in certs[:-1])
