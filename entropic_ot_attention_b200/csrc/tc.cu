@@ -759,7 +759,7 @@ struct SweepCfg {
     static constexpr uint32_t YATOM = BN * 128;          // ... of a column tile
     static constexpr uint32_t CB = BM * BN * 2;          // coefficient tile bytes (32 KB)
     static constexpr uint32_t CATOM = BM * 128;          // one 64-column atom of a coefficient tile
-    static constexpr uint32_t VB = NV * BN * 4;          // column vector bytes per stage
+    static constexpr uint32_t VB = NV * BN * 4;          // column vector bytes per late-ring slot
     // The row tiles X and A land (TMA) in the coefficient buffers and are moved into TMEM
     // before the first coefficient is written.
     static constexpr uint32_t OFF_C = 0;
@@ -787,7 +787,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
                     const TcVecArgs a, int max_tiles) {
     using M = ModeT<MODE>;
-    constexpr int NV = 1 + (M::SM ? 1 : 0) + NMOD;   // column vectors per stage: pcm2, m, yc...
+    constexpr int NV = 1 + (M::SM ? 1 : 0) + NMOD;   // column vectors per column tile: pcm2, m, yc...
     using C = SweepCfg<DH, NV>;
     constexpr int VOFF_M = 1, VOFF_Y = 1 + (M::SM ? 1 : 0);
     // W rides the late ring when the product reads it or when there is no product (R2); Y when
@@ -1053,7 +1053,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
             if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
             ptx::tc_fence_after();
-            // column vectors of this stage (explicit shared-memory loads: the aligned base
+            // column vectors of this tile's late-ring slot (explicit shared-memory loads: the aligned base
             // pointer no longer carries the address space)
             const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
             auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
