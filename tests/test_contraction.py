@@ -133,3 +133,19 @@ def test_offsets_and_argument_errors():
     p = api.make_problem(1, 2, 1024, 64, 1024, 1, 1, torch.bfloat16)
     assert _abi.lib.eot_contraction(__import__("ctypes").byref(p), None, None, None, None, None) == \
         _abi.EOT_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("W,t", [(24, 4), (23, 4), (30, 5), (1024, 128)])
+def test_reported_pairs_are_exactly_the_wholly_supported_ones(W, t):
+    """The tile pairs the certificate reports (|o| <= m) are those on which the band support of
+    eot_oracle.unit_structure is complete, so exp(S) is strictly positive there; at |o| = m + 1
+    some entry of the pair lies outside the band."""
+    from oracle import eot_oracle as eo
+    L = 12 * t
+    sup = eo.unit_structure(L, W).support
+    m = oc.offsets(W, t)
+    I = 5
+    for o in range(0, m + 2):
+        J = I + o
+        full = bool(sup[I * t:(I + 1) * t, J * t:(J + 1) * t].all())
+        assert full == (o <= m), (o, m)
