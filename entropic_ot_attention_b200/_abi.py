@@ -81,6 +81,8 @@ lib.eot_sinkhorn_fwd_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _
 lib.eot_sinkhorn_fwd_static.restype = ctypes.c_int
 EOT_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 lib.eot_kernel_launches.restype = ctypes.c_longlong
+lib.eot_solve_exp_passes.argtypes = [_P]
+lib.eot_solve_exp_passes.restype = ctypes.c_int
 lib.eot_profile_begin.restype = None
 lib.eot_profile_end.argtypes = [_vp]
 lib.eot_profile_end.restype = ctypes.c_int
@@ -91,13 +93,17 @@ lib.eot_profile_read.restype = ctypes.c_int
 EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sinkhorn_bwd",
             "eot_last_device_status", "eot_device_status_bits", "eot_status_string",
             "eot_abi_version", "eot_resolved_impl", "eot_kernel_launches", "eot_profile_begin",
-            "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static")
+            "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static", "eot_solve_exp_passes")
 
 PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3}
 
 
 def eot_kernel_launches() -> int:
     return int(lib.eot_kernel_launches())
+
+
+def eot_solve_exp_passes(p: eot_problem) -> int:
+    return int(lib.eot_solve_exp_passes(ctypes.byref(p)))
 
 
 def eot_profile_begin() -> None:

@@ -483,6 +483,12 @@ eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, 
                          static_cast<cudaStream_t>(stream));
 }
 
+int eot_solve_exp_passes(const eot_problem* p) {
+    if (validate(p) != EOT_OK) return -1;
+    // every half-step evaluates one exponential per band entry
+    return 2 * (p->T + p->R);
+}
+
 long long eot_kernel_launches(void) { return g_launches.load(); }
 
 void eot_profile_begin(void) {

@@ -144,6 +144,11 @@ int eot_abi_version(void);
  * 2 = backward sweeps, 3 = auxiliary kernels (marginals, vectors, dustbin links); returns
  * the summed milliseconds and the number of bracketed launches of that kind. */
 long long eot_kernel_launches(void);
+/* Exponentials per band entry that the forward solve (base and tail, not the output sweep)
+ * evaluates for problem *p with the kernels this library picks for it: 2 (T + R) when every
+ * half-step forms its own plan entries, T + R + 1 when each iteration forms them once; -1 for an
+ * invalid problem.  Benchmark support: the exponential-unit bound of the solve. */
+int eot_solve_exp_passes(const eot_problem* p);
 void eot_profile_begin(void);
 eot_status eot_profile_end(void* stream);
 eot_status eot_profile_read(int kind, double* total_ms, long long* launches);

@@ -105,3 +105,58 @@ def test_host_step_chunk_plan_errors():
         plan_chunks(2, 4, rows_per_chunk=3)
     with pytest.raises(ValueError):
         plan_chunks(2, 4, heads_per_chunk=1, rows_per_chunk=1)
+
+
+# Algorithmic work of one call (the workload table of the measurement plan): MMA flops
+# (T+R+2) 2d |Omega| forward and 5 2d |Omega| backward, roofline max(flops / 1630 TFLOP/s,
+# bytes / 6547.2 GB/s) per pass.
+@pytest.mark.parametrize("shape,omega,fwd_flops,bwd_flops,fwd_ms,bwd_ms,bounds", [
+    # medium: B=4 H=8 L=4096 d=64 W=256 T=20 R=2; |Omega| = 32 (4096*257 - 128*129)
+    ((4, 8, 4096, 64, 20, 2), 32 * (4096 * 257 - 128 * 129), 1.019e11, 2.12e10, 0.0625, 0.0191, ("tensor", "hbm")),
+    # long: B=1 H=4 L=131072 d=128 W=1024 T=10 R=2; |Omega| = 4 (131072*1025 - 512*513)
+    ((1, 4, 131072, 128, 10, 2), 4 * (131072 * 1025 - 512 * 513), 1.922e12, 6.87e11, 1.179, 0.421,
+     ("tensor", "tensor")),
+])
+def test_algorithmic_work_and_roofline(shape, omega, fwd_flops, bwd_flops, fwd_ms, bwd_ms, bounds):
+    B, H, L, d, T, R = shape
+    w = bench.algorithmic_work(B, H, L, d, T, R, omega, 2)
+    assert w["fwd_flops"] == pytest.approx(fwd_flops, rel=2e-3)
+    assert w["bwd_flops"] == pytest.approx(bwd_flops, rel=2e-3)
+    assert w["solve_flops"] == (T + R) * 2 * d * omega
+    assert w["solve_flops"] + w["output_flops"] == w["fwd_flops"]
+    tf, bf = bench.roofline_ms(w["fwd_flops"], w["fwd_bytes"], 1630.0, 6547.2)
+    tb, bb = bench.roofline_ms(w["bwd_flops"], w["bwd_bytes"], 1630.0, 6547.2)
+    assert tf == pytest.approx(fwd_ms, rel=5e-3) and bf == bounds[0]
+    assert tb == pytest.approx(bwd_ms, rel=5e-3) and bb == bounds[1]
+
+
+def test_dominant_kernel_counts_one_score_evaluation_per_iteration():
+    """The forward solve of the long workload, timed at 4.893 ms per call, does 12 iterations of
+    2d |Omega| flops: 337 TFLOP/s, 0.207 of the 1630 TFLOP/s burst peak."""
+    omega = 4 * (131072 * 1025 - 512 * 513)
+    w = bench.algorithmic_work(1, 4, 131072, 128, 10, 2, omega, 2)
+    prof = {"fwd_sweep": (4.893, 2), "fwd_output": (0.498, 1), "bwd_sweep": (2.760, 6), "aux": (0.24, 12)}
+    r = bench.dominant_kernel(prof, w, 10, 2, 1630.0, "measured", exp_passes=24, omega=omega, mufu_peak=4.65e12)
+    assert r["kind"] == "fwd_sweep" and r["units_timed"] == 12
+    assert r["achieved"] == pytest.approx(337.0, rel=2e-3)
+    assert r["frac"] == pytest.approx(0.207, abs=1e-3)
+    assert r["exp2_per_s"] == pytest.approx(24 * omega / 4.893e-3, rel=1e-9)
+    prof["bwd_sweep"] = (6.0, 6)
+    r = bench.dominant_kernel(prof, w, 10, 2, 1630.0, "measured", exp_passes=24, omega=omega, mufu_peak=4.65e12)
+    assert r["kind"] == "bwd_sweep" and r["achieved"] == pytest.approx(w["bwd_flops"] / 6.0e-3 / 1e12)
+
+
+def test_gpus_flag_spawns_that_many_ranks():
+    """--gpus 2 without a launcher re-runs bench.py as two ranks; rank 0 alone prints one line
+    whose n_gpus is 2 (host plumbing only: gloo, no GPU)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    res = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--dry-run"],
+                         capture_output=True, text=True, timeout=300, env=env, cwd=root)
+    assert res.returncode == 0, res.stderr
+    lines = [json.loads(x) for x in res.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["ranks_reporting"] == 2.0 and lines[0]["ms_per_step"] == 2.0
