@@ -79,7 +79,15 @@ lib.eot_contraction.restype = ctypes.c_int
 
 lib.eot_sinkhorn_fwd_static.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
 lib.eot_sinkhorn_fwd_static.restype = ctypes.c_int
-EOT_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
+lib.eot_static_last_device_status.argtypes = [_vp]
+lib.eot_static_last_device_status.restype = ctypes.c_int
+lib.eot_static_scratch_bytes.restype = _sz
+EOT_STATIC_SCRATCH_BYTES = int(lib.eot_static_scratch_bytes())
+lib.eot_wait_selftest.argtypes = [ctypes.c_int, ctypes.c_uint64, _vp, _vp]
+lib.eot_wait_selftest.restype = ctypes.c_int
+EOT_SELFTEST_MBARRIER = 0
+EOT_SELFTEST_GRID = 1
+EOT_SELFTEST_CONTROL = 2
 lib.eot_kernel_launches.restype = ctypes.c_longlong
 lib.eot_solve_exp_passes.argtypes = [_P]
 lib.eot_solve_exp_passes.restype = ctypes.c_int
@@ -93,7 +101,8 @@ lib.eot_profile_read.restype = ctypes.c_int
 EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sinkhorn_bwd",
             "eot_last_device_status", "eot_device_status_bits", "eot_status_string",
             "eot_abi_version", "eot_resolved_impl", "eot_kernel_launches", "eot_profile_begin",
-            "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static", "eot_solve_exp_passes")
+            "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static", "eot_solve_exp_passes",
+            "eot_static_last_device_status", "eot_static_scratch_bytes", "eot_wait_selftest")
 
 PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3}
 
@@ -165,6 +174,16 @@ def eot_sinkhorn_fwd_static(p: eot_problem, Q: int, K: int, V: int, mask: int | 
                             v_tail: int, stream: int) -> int:
     """Forward with the library's static scratch (no workspace); returns the raw status."""
     return lib.eot_sinkhorn_fwd_static(ctypes.byref(p), Q, K, V, mask, O, u_tail, v_tail, stream)
+
+
+def eot_static_last_device_status(stream: int) -> int:
+    """Status of the last eot_sinkhorn_fwd_static call(s) in this context (syncs ``stream``)."""
+    return lib.eot_static_last_device_status(stream)
+
+
+def eot_wait_selftest(which: int, limit_ns: int, scratch: int, stream: int) -> None:
+    """Launch the bounded-wait self-test (raw device address of a 256-byte scratch buffer)."""
+    _check(lib.eot_wait_selftest(int(which), int(limit_ns), scratch, stream), "eot_wait_selftest")
 
 
 def eot_last_device_status(workspace: int, stream: int) -> int:

@@ -32,6 +32,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     cmd = [NVCC, "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-I", INCLUDE, "-o", LIB + ".tmp", *sources()]
+    if os.environ.get("EOT_NVTX", "0") == "1":   # NVTX ranges around the passes (timeline profiling)
+        cmd[1:1] = ["-DEOT_NVTX"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -14,6 +14,25 @@
 
 #include "kernels.cuh"
 
+// NVTX ranges around the passes of a call (host-side enqueue ranges that a timeline profiler
+// pairs with the kernels they launch), compiled in only with -DEOT_NVTX.
+#ifdef EOT_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace {
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+}  // namespace
+#define EOT_CAT2(a, b) a##b
+#define EOT_CAT(a, b) EOT_CAT2(a, b)
+#define EOT_RANGE(name) NvtxRange EOT_CAT(eot_nvtx_, __LINE__)(name)
+#else
+#define EOT_RANGE(name) ((void)0)
+#endif
+
 using namespace eot;
 
 namespace {
@@ -145,6 +164,7 @@ eot_status validate_problem(const eot_problem* p) { return validate(p); }
 
 eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
                         void* O, float* u_tail, float* v_tail, void* ws, cudaStream_t st) {
+    EOT_RANGE("eot forward");
     const Geom g = make_geom(*p);
     const int impl = resolve_impl(*p);
     const WsLayout w = ws_layout(*p, false);
@@ -195,6 +215,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
 
     bool first = true;
     auto step = [&](int k_in, int k_out) -> cudaError_t {
+        EOT_RANGE("eot iteration (row + column half-step)");
         // row half-step: u(k_out) from v(k_in); column half-step: v(k_out) from u(k_out)
         row.colpot = v_tail + size_t(k_in) * L;
         row.stab = first ? nullptr : u_tail + size_t(k_in) * L;
@@ -244,6 +265,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     }
 
     // Output O = diag(1/a) P(R,R) V (a vector sweep with coefficients P / a_r).
+    EOT_RANGE("eot output sweep");
     BwdVecArgs va{};
     va.kind = kPassOut;
     va.R = p->R;
@@ -284,6 +306,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
 eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
                          const float* u_tail, const float* v_tail, const void* dO, void* dQ, void* dK, void* dV,
                          void* ws, cudaStream_t st) {
+    EOT_RANGE("eot backward");
     const Geom g = make_geom(*p);
     const int impl = resolve_impl(*p);
     const WsLayout w = ws_layout(*p, true);
@@ -378,6 +401,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     // C1: beta_R = colsum(P(R,R) * dP) and dV = P(R,R)^T (dO / a)   (one column sweep)
     EOT_TRY(vec(kPassC1, 0));
     {
+        EOT_RANGE("eot backward: beta_R, dV");
         BwdPass bp = colp;
         if (R > 0) {
             bp.sout = beta + size_t(R) * vecn;
@@ -395,6 +419,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     }
     if (R > 0) {
         // R2: alpha_R = rowsum(P(R,R) * dP) - P(R,R) (beta_R / b)
+        EOT_RANGE("eot backward: staircase vectors");
         EOT_TRY(vec(kPassR2, 0));
         EOT_TRY(scalar_pass(rowp, alpha + size_t(R) * vecn, true));
         for (int k = R - 1; k >= 1; --k) {
@@ -407,6 +432,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     }
     // dQ = scale dS K (row sweep), dK = scale dS^T Q (column sweep); dS = P(R,R) (dP - sum x y^T)
     for (int orient = 0; orient < 2; ++orient) {
+        EOT_RANGE(orient == 0 ? "eot backward: dQ" : "eot backward: dK");
         EOT_TRY(vec(orient == 0 ? kPassRF : kPassCF, 0));
         BwdPass bp = orient == 0 ? rowp : colp;
         bp.vout = orient == 0 ? dQ : dK;

@@ -52,22 +52,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait: true when the phase completed; false when the CTA is aborting or the
 // limit ran out (then the timeout bit is set and the abort flag raised).
 // The abort flag and the clock are looked at on every 8th failed attempt only, so that a
-// spinning warp takes few issue slots from the warps that do the work.
+// spinning warp takes few issue slots from the warps that do the work.  The limit is an
+// argument (the kernels pass the default; the wait self-test passes about a millisecond).
 constexpr uint64_t kWaitLimitNs = 100000000ull;  // 100 ms: far beyond any legitimate wait
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 7u) == 0u) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicOr(status, kStatusTimeout);
                 return false;
             }
         }
+    }
+}
+
+// Bounded wait until a grid-wide counter reaches target (acquire); false on abort or timeout
+// (then, as for mbar_wait, the timeout bit is set and the abort flag raised).
+__device__ __forceinline__ bool grid_wait(const uint32_t* ctr, uint32_t target, volatile int* abort_flag,
+                                          uint32_t* status, uint64_t limit_ns = kWaitLimitNs) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 0;; ++i) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) return true;
+        if ((i & 15u) == 15u) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                *abort_flag = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+        __nanosleep(64);
     }
 }
 

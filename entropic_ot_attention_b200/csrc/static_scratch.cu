@@ -7,12 +7,13 @@
 // start-up because those calls can synchronise the device and stall other streams.  Such a
 // caller still provides Q, K, V, the mask and the outputs; only the scratch comes from here.
 //
-// The array is a file-scope __device__ object, so every GPU that loads this library holds
-// EOT_STATIC_SCRATCH_BYTES of it until the process exits.  In host code its name is only a
-// host-side stand-in: the device address is obtained once per device with
-// cudaGetSymbolAddress (with that device current) and cached.
-#include <mutex>
-
+// The array is a file-scope __device__ object, so every context that loads this library's
+// kernels holds EOT_STATIC_SCRATCH_BYTES of it until the module is unloaded (normally process
+// exit).  In host code its name is only a host-side stand-in: the device address is looked up
+// with cudaGetSymbolAddress, in the context that is current, on every call.  The lookup is a
+// host-side query that allocates nothing; keeping no cached address means a caller that makes
+// its own driver context current, or one that resets the device, always gets the address of the
+// array in the context it is using.
 #include "kernels.cuh"
 
 namespace eot {
@@ -25,21 +26,11 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[EOT_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
-
-// Device address of g_static_scratch on the current device (looked up once per device).
+// Device address of g_static_scratch in the current context.
 eot_status scratch_address(void** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EOT_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return EOT_ERR_CUDA;
-        g_addr[dev] = ptr;
-    }
-    *out = g_addr[dev];
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return EOT_ERR_CUDA;
+    *out = ptr;
     return EOT_OK;
 }
 
@@ -60,3 +51,12 @@ extern "C" eot_status eot_sinkhorn_fwd_static(const eot_problem* p, const void* 
     // kernel of every forward call.
     return eot::forward_impl(p, Q, K, V, mask, O, u_tail, v_tail, ws, static_cast<cudaStream_t>(stream));
 }
+
+extern "C" eot_status eot_static_last_device_status(void* stream) {
+    void* ws = nullptr;
+    const eot_status s = scratch_address(&ws);
+    if (s != EOT_OK) return s;
+    return eot_last_device_status(ws, stream);
+}
+
+extern "C" size_t eot_static_scratch_bytes(void) { return size_t(EOT_STATIC_SCRATCH_BYTES); }

@@ -154,26 +154,6 @@ struct TcBandArgs {
     uint32_t* gbar;
 };
 
-// Bounded wait until a grid-wide counter reaches target (acquire); false on abort or timeout.
-__device__ __forceinline__ bool grid_wait(const uint32_t* ctr, uint32_t target, volatile int* abort_flag,
-                                          uint32_t* status) {
-    const uint64_t t0 = ptx::globaltimer();
-    for (uint32_t i = 0;; ++i) {
-        uint32_t v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-        if (v >= target) return true;
-        if ((i & 15u) == 15u) {
-            if (*abort_flag) return false;
-            if (ptx::globaltimer() - t0 > ptx::kWaitLimitNs) {
-                *abort_flag = 1;
-                atomicOr(status, kStatusTimeout);
-                return false;
-            }
-        }
-        __nanosleep(64);
-    }
-}
-
 template <int DH, int KIND>
 struct BandCfg {
     static constexpr int BM = 128, BN = 128;
@@ -367,7 +347,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                         ptx::tma_load_2d(ys + ka * C::ATOM, mY, ka * 64, int(it.base) + c0, full(s));
                     ++g;
                     if (!biases_ready) {
-                        if (!grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) { ok = false; break; }
+                        if (!ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) { ok = false; break; }
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                         biases_ready = true;
                     }
@@ -486,7 +466,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         float* outb_hs = outb_of(hs);
         if (MULTI && hs > a.hs0) {
             // every CTA has written half-step hs - 1 (the shifts and biases read below)
-            if (tid == 64 && ok && !grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) ok = false;
+            if (tid == 64 && ok && !ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) ok = false;
             ptx::named_bar_sync(9, 512);
             ok = ok && !*abort_flag;
         }

@@ -158,22 +158,48 @@ eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
  * memory where they run it (a plug-in inside a host that owns all device memory and gives it
  * no allocator; a serving loop that forbids cudaMalloc/cudaFree after start-up because those
  * calls can synchronise the device).  Arguments and results are those of eot_sinkhorn_fwd;
- * the scratch is a fixed array of EOT_STATIC_SCRATCH_BYTES in this library's device memory,
- * held on every GPU that loads the library until the process exits.
- *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current); make that first call before any stream capture.
+ * the scratch is a fixed array of EOT_STATIC_SCRATCH_BYTES in this library's device memory.
+ *   - The array belongs to each context that loads this library's kernels and is held until
+ *     the module is unloaded (normally process exit).  Every call looks up its address in the
+ *     context current at that moment (cudaGetSymbolAddress, a host-side query that allocates
+ *     nothing), so callers that switch contexts or reset the device stay correct.
+ *   - The first call in a context loads the library's kernels there (CUDA lazy module loading),
+ *     which may allocate device memory for the module and is not allowed during stream capture:
+ *     make one call before any capture and before the phase in which nothing may allocate.
+ *     Later calls allocate nothing.
  *   - Problems whose forward scratch, eot_workspace_bytes(p, 0), exceeds
  *     EOT_STATIC_SCRATCH_BYTES are rejected with EOT_ERR_WORKSPACE_TOO_SMALL before anything
  *     is launched.
- *   - Every call on a device shares the one array and leaves its contents behind (the first
+ *   - Every call in a context shares the one array and leaves its contents behind (the first
  *     kernel of each call clears what must start at zero).  Calls that overlap on the GPU
  *     (other streams, other host threads) race on it and corrupt each other: serialise them.
- *   - The device status word of these calls lives in the shared array and is not readable
- *     through eot_last_device_status. */
+ *   - The device status word of these calls lives in the shared array: read (and clear) it
+ *     with eot_static_last_device_status, which syncs ``stream`` like eot_last_device_status.
+ * eot_static_scratch_bytes returns EOT_STATIC_SCRATCH_BYTES as built into the library. */
 #define EOT_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 eot_status eot_sinkhorn_fwd_static(const eot_problem* p, const void* Q, const void* K, const void* V,
                                    const uint8_t* mask, void* O, float* u_tail, float* v_tail,
                                    void* stream);
+eot_status eot_static_last_device_status(void* stream);
+size_t eot_static_scratch_bytes(void);
+
+/* Self-test of the bounded device waits (failure detection; the paper has no counterpart).
+ * Every wait inside this library's kernels (on an mbarrier, or on a grid-wide counter between
+ * fused half-steps) gives up after a time limit, sets the timeout bit of the status word and
+ * ends the kernel instead of spinning forever.  This call runs one tiny kernel whose single
+ * wait, with limit ``limit_ns`` (1 ns .. 1 s), is made so that nothing completes it:
+ *   EOT_SELFTEST_MBARRIER  an mbarrier expecting two arrivals receives one;
+ *   EOT_SELFTEST_GRID      a grid-wide counter waits for one CTA more than the grid holds;
+ *   EOT_SELFTEST_CONTROL   the mbarrier receives both arrivals (the wait completes at once).
+ * ``scratch`` is a caller-owned device buffer of at least 256 bytes, 256-byte aligned: word 0
+ * is the status word (read it with eot_last_device_status(scratch, stream): EOT_ERR_TIMEOUT for
+ * the first two cases, EOT_OK for the control), word 2 is 2 when the wait gave up and 1 when it
+ * completed.  Asynchronous on ``stream``; invalid arguments return EOT_ERR_INVALID_ARGUMENT
+ * before anything is enqueued. */
+#define EOT_SELFTEST_MBARRIER 0
+#define EOT_SELFTEST_GRID 1
+#define EOT_SELFTEST_CONTROL 2
+eot_status eot_wait_selftest(int which, uint64_t limit_ns, void* scratch, void* stream);
 
 /* Kernel family that ``p`` would run with (EOT_IMPL_SIMT or EOT_IMPL_TCGEN05), or -1 if
  * the problem is invalid or unsupported. */

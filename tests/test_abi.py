@@ -122,3 +122,23 @@ def test_status_strings(abi):
     for s in range(7):
         assert abi.eot_status_string(s)
     assert "unknown" in abi.eot_status_string(99)
+
+
+def test_static_scratch_size_matches_header(abi):
+    """The size the library was built with equals the header's EOT_STATIC_SCRATCH_BYTES."""
+    src = open(os.path.join(ROOT, "include", "eot.h")).read()
+    m = re.search(r"#define\s+EOT_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*\*\s*(\d+)u\s*\*\s*(\d+)u\)", src)
+    assert m, "EOT_STATIC_SCRATCH_BYTES not found in the header"
+    want = int(m.group(1)) * int(m.group(2)) * int(m.group(3))
+    assert abi.lib.eot_static_scratch_bytes() == want == abi.EOT_STATIC_SCRATCH_BYTES
+
+
+def test_nvtx_build_flag_compiles(tmp_path):
+    """The NVTX ranges around the passes (EOT_NVTX=1 builds) compile for sm_100a."""
+    import subprocess
+    src = os.path.join(ROOT, "entropic_ot_attention_b200", "csrc", "api.cu")
+    nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+    res = subprocess.run([nvcc, "-DEOT_NVTX", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                          "-I", os.path.join(ROOT, "include"), "-c", src, "-o", str(tmp_path / "api_nvtx.o")],
+                         capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
