@@ -1,0 +1,145 @@
+"""Sequence sharding of one (batch, head) unit over ranks: contiguous row ranges, with the band
+neighbours' potentials exchanged after every half-step.
+
+"Blockwise Differentiable Sinkhorn Attention" §2.1 keeps the extra state of the solve at O(L)
+potentials because the support is a fixed band: position i is coupled only with |i - j| <= h,
+h = W // 2.  A rank that owns positions [r0, r1) therefore needs, for its row half-steps, the
+scores of its rows against the columns [r0 - h, r1 + h) and the column potentials over that
+range; for its column half-steps the same with rows and columns swapped.  The Q and K rows of
+that halo are copied to the rank once; after every half-step each rank sends the potentials its
+neighbours' halos cover (at most h values to each side) and receives theirs, point to point.
+Shards are at least h positions long, so only the two adjacent ranks exchange.
+
+With a dustbin (§2.3) the dustbin row and column are dense: their log-sum-exp is a sum over all
+positions, formed per rank as a (max, sum) partial and merged with one all-reduce of the maxima
+and one of the rescaled sums per half-step (``allreduce_lse``).
+
+Every rank takes the same collective steps in the same order.  The per-rank half-step is a
+callable, so the same driver runs a rank's part of the solve wherever its scores live.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Callable
+
+import torch
+import torch.distributed as dist
+
+
+@dataclass(frozen=True)
+class Shard:
+    """Positions [r0, r1) owned by ``rank``; [c0, c1) = [max(0, r0 - h), min(L, r1 + h)) is the
+    range its band reaches (its rows' columns, and its columns' rows)."""
+
+    rank: int
+    r0: int
+    r1: int
+    c0: int
+    c1: int
+
+    @property
+    def n(self) -> int:
+        return self.r1 - self.r0
+
+    @property
+    def owned(self) -> slice:
+        """The owned positions inside the halo range."""
+        return slice(self.r0 - self.c0, self.r1 - self.c0)
+
+
+def shard_plan(L: int, W: int, world: int, align: int = 128) -> list[Shard]:
+    """Split L positions into ``world`` contiguous ranges of whole ``align``-position tiles (the
+    first ranks take one tile more when the tiles do not divide evenly).  Raises ValueError when
+    a range would be shorter than the band's half-width h = W // 2 (then a rank's halo would
+    reach past its neighbour) or empty."""
+    if world < 1 or L <= 0 or L % align != 0 or W < 0:
+        raise ValueError("need world >= 1, L > 0 a multiple of align, W >= 0")
+    h = W // 2
+    tiles = L // align
+    if tiles < world:
+        raise ValueError(f"{tiles} tiles cannot be shared by {world} ranks")
+    base, extra = divmod(tiles, world)
+    out, r0 = [], 0
+    for r in range(world):
+        n = (base + (1 if r < extra else 0)) * align
+        r1 = r0 + n
+        if world > 1 and n < h:
+            raise ValueError(f"rank {r} owns {n} positions, fewer than the band half-width {h}")
+        out.append(Shard(r, r0, r1, max(0, r0 - h), min(L, r1 + h)))
+        r0 = r1
+    return out
+
+
+def halo_exchange(x_owned: torch.Tensor, plan: list[Shard], rank: int, group=None) -> torch.Tensor:
+    """Potentials over this rank's halo range [c0, c1): its own values in the middle, the left
+    neighbour's last values and the right neighbour's first values on the sides.  Sends this
+    rank's first and last values to the neighbours whose halos reach them (send / recv pairs
+    batched into one exchange)."""
+    sh = plan[rank]
+    out = torch.zeros(sh.c1 - sh.c0, dtype=x_owned.dtype, device=x_owned.device)
+    out[sh.owned] = x_owned
+    ops, recv = [], []
+    if rank > 0:
+        left = plan[rank - 1]
+        # the left neighbour's halo reaches [left.r1, left.c1) = the first values of this rank
+        n_send = left.c1 - left.r1
+        if n_send > 0:
+            ops.append(dist.P2POp(dist.isend, x_owned[:n_send].contiguous(), rank - 1, group))
+        n_recv = sh.r0 - sh.c0
+        if n_recv > 0:
+            buf = torch.empty(n_recv, dtype=x_owned.dtype, device=x_owned.device)
+            ops.append(dist.P2POp(dist.irecv, buf, rank - 1, group))
+            recv.append((slice(0, n_recv), buf))
+    if rank < len(plan) - 1:
+        right = plan[rank + 1]
+        n_send = right.r0 - right.c0
+        if n_send > 0:
+            ops.append(dist.P2POp(dist.isend, x_owned[sh.n - n_send:].contiguous(), rank + 1, group))
+        n_recv = sh.c1 - sh.r1
+        if n_recv > 0:
+            buf = torch.empty(n_recv, dtype=x_owned.dtype, device=x_owned.device)
+            ops.append(dist.P2POp(dist.irecv, buf, rank + 1, group))
+            recv.append((slice(sh.r1 - sh.c0, sh.c1 - sh.c0), buf))
+    if ops:
+        for req in dist.batch_isend_irecv(ops):
+            req.wait()
+    for sl, buf in recv:
+        out[sl] = buf
+    return out
+
+
+def allreduce_lse(m: torch.Tensor, s: torch.Tensor, group=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Merge per-rank log-sum-exp partials: sum_r s_r exp(m_r - M) with M = max_r m_r (one
+    all-reduce of the maxima, one of the rescaled sums).  Returns (M, total); an all -inf
+    partial set gives (-inf, 0)."""
+    M = m.clone()
+    dist.all_reduce(M, op=dist.ReduceOp.MAX, group=group)
+    finite = torch.isfinite(M)
+    scaled = torch.where(finite & torch.isfinite(m), s * torch.exp(m - torch.where(finite, M, torch.zeros_like(M))),
+                         torch.zeros_like(s))
+    dist.all_reduce(scaled, op=dist.ReduceOp.SUM, group=group)
+    return M, scaled
+
+
+def sharded_solve(plan: list[Shard], rank: int, T: int, R: int,
+                  row_step: Callable[[torch.Tensor], torch.Tensor],
+                  col_step: Callable[[torch.Tensor], torch.Tensor],
+                  group=None, dtype=torch.float64, device=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """This rank's part of the T stopped + R tail iterations (§2.1).
+
+    ``row_step(v_halo)`` returns the owned rows' u from the column potentials over [c0, c1);
+    ``col_step(u_halo)`` returns the owned columns' v from the row potentials over [c0, c1).
+    Returns (u_tail, v_tail), each [R + 1, r1 - r0], in the slot layout of eot_sinkhorn_fwd:
+    slot 0 the stopped base (u after T steps, 0 when T = 0; v0), slot k tail step k."""
+    sh = plan[rank]
+    u_tail = torch.zeros(R + 1, sh.n, dtype=dtype, device=device)
+    v_tail = torch.zeros(R + 1, sh.n, dtype=dtype, device=device)
+    v_halo = torch.zeros(sh.c1 - sh.c0, dtype=dtype, device=device)
+    for k in range(T + R):
+        u = row_step(v_halo)
+        v = col_step(halo_exchange(u, plan, rank, group))
+        v_halo = halo_exchange(v, plan, rank, group)
+        slot = 0 if k < T else k - T + 1
+        u_tail[slot] = u
+        v_tail[slot] = v
+    return u_tail, v_tail
