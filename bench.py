@@ -410,6 +410,8 @@ def main():
     ap.add_argument("--L", type=int, default=0, help="override the sequence length (profiling captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--schedule", default="auto", choices=["auto", "half_steps", "one_exp"],
+                    help="forward schedule (eot_set_forward_schedule); auto picks per problem")
     ap.add_argument("--dry-run", action="store_true", dest="dry_run",
                     help="launch and aggregate over ranks without a GPU (host plumbing check)")
     args = ap.parse_args()
@@ -447,6 +449,8 @@ def main():
     dbi = case.dustbin_index if case.dustbin else None
     p = api.make_problem(B, H, L, d, case.W, case.T, case.R, tdt, case.scale, dbi, case.dustbin_mass,
                          impl=args.impl)
+    _abi.eot_set_forward_schedule({"auto": _abi.SCHEDULE_AUTO, "half_steps": _abi.SCHEDULE_HALF_STEPS,
+                                   "one_exp": _abi.SCHEDULE_ONE_EXP}[args.schedule])
     impl_used = {1: "simt", 2: "tcgen05"}.get(_abi.eot_resolved_impl(p), "unsupported")
     ws_f = api.workspace(p, False, dev)
     ws_b = api.workspace(p, True, dev)
@@ -533,6 +537,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16" if case.dtype == "bf16" else "fp32",
         "data": "synthetic, seeded (eot_inputs); no dataset",
         "config": dict(workload_config(args.workload, case), impl=impl_used,
+                       forward_exp_per_band_entry_per_call=_abi.eot_solve_exp_passes(p),
                        parallelism=f"{world} independent replica(s), no data-path collective",
                        l2="inputs larger than L2: Q, K, V, dO are 134 MB each" if args.workload == "long"
                        else "inputs resident; see workload sizes",

@@ -34,6 +34,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
            "-I", INCLUDE, "-o", LIB + ".tmp", *sources()]
     if os.environ.get("EOT_NVTX", "0") == "1":   # NVTX ranges around the passes (timeline profiling)
         cmd[1:1] = ["-DEOT_NVTX"]
+    if os.environ.get("EOT_ITER_PREFETCH"):      # next tile's TMEM scores loaded during this tile (tuning)
+        cmd[1:1] = [f"-DEOT_ITER_PREFETCH={int(os.environ['EOT_ITER_PREFETCH'])}"]
+    if os.environ.get("EOT_ITER_FMA_PAIRS"):     # exponential pairs per 32 columns on the FMA pipe (tuning)
+        cmd[1:1] = [f"-DEOT_ITER_FMA_PAIRS={int(os.environ['EOT_ITER_FMA_PAIRS'])}"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -76,6 +76,11 @@ cudaError_t tracked(int kind, int nkernels, cudaStream_t st, F&& f) {
     return e;
 }
 
+// Forward schedule (process-wide; benchmark and test support): 0 and 1 run the half-step
+// schedule (measured faster on every workload), 2 the one-exponential-per-iteration kernel in one
+// cooperative launch, 3 that kernel with one launch per iteration.
+std::atomic<int> g_fwd_schedule{0};
+
 bool tensor_core_ok(const eot_problem& p) { return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128); }
 
 int resolve_impl(const eot_problem& p) {
@@ -229,11 +234,45 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         return run_lse(impl, col, st);
     };
     // Tensor-core path without a dustbin: the first half-step (running maximum) on its own, then
-    // every later half-step in one cooperative launch with grid-wide barriers between them.  If
-    // the device cannot hold the whole grid at once the half-steps run as separate launches.
+    // either every iteration with one exponential per band entry (iter.cu: the first row
+    // half-step's u is the row stabiliser of iteration 1, which recomputes it), or every later
+    // half-step in one cooperative launch with grid-wide barriers between them.  If the device
+    // cannot hold the whole grid at once the iterations / half-steps run as separate launches.
     const int n_half = 2 * (p->T + p->R);
     bool fused = false;
-    if (impl == EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
+    const int sched = g_fwd_schedule.load();
+    const bool use_iter = impl == EOT_IMPL_TCGEN05 && sched >= 2 && iter_schedule_possible(*p) && iter_split(g) > 0;
+    if (sched >= 2 && !use_iter) return EOT_ERR_UNSUPPORTED;
+    if (use_iter) {
+        EOT_TRY(run_lse(impl, [&] {
+            LsePass r0 = row;
+            r0.colpot = v_tail;
+            r0.stab = nullptr;
+            r0.out = u_tail;
+            return r0;
+        }(), st));
+        uint32_t* gbar = at<uint32_t>(ws, w.gbar);
+        EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
+        IterLaunch il{};
+        il.g = g;
+        il.Q = Q;
+        il.K = K;
+        il.logm = logm;
+        il.tile_bits = tbits;
+        il.u_tail = u_tail;
+        il.v_tail = v_tail;
+        il.pstride = pstride;
+        il.vb2 = vb2;
+        il.part = at<float>(ws, w.part);
+        il.gbar = gbar;
+        il.status = status;
+        il.T = p->T;
+        il.R = p->R;
+        il.fused = sched == 2 ? 2 : sched == 3 ? 0 : 1;
+        int launched = 0;
+        EOT_TRY(tracked(kProfLse, 0, st, [&] { return launch_tc_iter(il, st, &launched); }));
+        g_launches += launched;
+    } else if (impl == EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
         EOT_TRY(run_lse(impl, [&] {
             LsePass r0 = row;
             r0.colpot = v_tail;
@@ -511,8 +550,18 @@ eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, 
 
 int eot_solve_exp_passes(const eot_problem* p) {
     if (validate(p) != EOT_OK) return -1;
+    const Geom g = make_geom(*p);
+    if (resolve_impl(*p) == EOT_IMPL_TCGEN05 && g_fwd_schedule.load() >= 2 && iter_schedule_possible(*p) &&
+        iter_split(g) > 0)
+        return p->T + p->R + 1;   // the first row half-step, then one per iteration
     // every half-step evaluates one exponential per band entry
     return 2 * (p->T + p->R);
+}
+
+eot_status eot_set_forward_schedule(int schedule) {
+    if (schedule < 0 || schedule > 3) return EOT_ERR_INVALID_ARGUMENT;
+    g_fwd_schedule.store(schedule);
+    return EOT_OK;
 }
 
 long long eot_kernel_launches(void) { return g_launches.load(); }

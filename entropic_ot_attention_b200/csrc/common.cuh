@@ -100,6 +100,7 @@ struct WsLayout {
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t gbar;            // forward: grid-barrier counters of the fused half-steps [2 (T + R)]
+    size_t part;            // forward, one exponential per iteration: column partial sums [BH][L/128][window][128]
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
     size_t zero;            // backward: a vector of zeros
@@ -114,6 +115,19 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int kDCols = 1024;
 __host__ __device__ inline int dustbin_splits(int L) { return (L + 1 + kDCols - 1) / kDCols; }
 __host__ __device__ inline int tile_words(int L) { return (L / 128 + 31) / 32; }
+
+// Window of a 128-row strip: the 128-column tiles that meet the band of its rows,
+// [128 s - h, 128 s + 127 + h]; the most any strip has (L / 128 at most).
+inline int iter_window_tiles(int L, int h) {
+    const long n = 1L + (long(h) + 127) / 128 + (long(h) + 127) / 128;
+    return int(n < L / 128 ? n : L / 128);
+}
+// Problems the one-exponential-per-iteration forward can run (tensor cores, bf16, no dustbin, a
+// stopped base, a window of at most nine tiles); they get its column-partial workspace.
+inline bool iter_schedule_possible(const eot_problem& p) {
+    return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin && p.T >= 1 && p.impl != EOT_IMPL_SIMT &&
+           p.L >= 128 && iter_window_tiles(p.L, p.W / 2) <= 9;
+}
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     WsLayout w{};
@@ -136,6 +150,10 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
         w.gbar = o; o += align256(size_t(2) * (size_t(p.T) + size_t(p.R)) * sizeof(uint32_t) + 4);
+        if (iter_schedule_possible(p)) {
+            w.part = o;
+            o += align256(BH * size_t(p.L / 128) * size_t(iter_window_tiles(p.L, p.W / 2)) * 128 * sizeof(float));
+        }
     }
     w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     if (bwd) {

@@ -1,6 +1,8 @@
 // Kernel launchers shared between the C-ABI layer (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace eot {
@@ -50,6 +52,9 @@ cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 
 // Tensor-core (tcgen05 + TMA) kernels; return cudaErrorNotSupported when not built.
 bool tc_supported(const Geom& g);
+// 2-D TMA descriptor over a [rows, d] bf16 matrix, boxes of 64 elements x box_rows, 128-byte swizzle.
+bool tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows);
+int sm_count();
 cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st);
 // Shifted half-steps hs0 .. hs0 + nhs - 1 of the forward schedule (even hs: row, odd: column;
 // iteration hs / 2 writes slot 0 for the first T iterations and slot hs / 2 - T + 1 after) in one
@@ -61,5 +66,31 @@ struct FusedSteps {
 };
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
+
+// Forward iterations 1 .. T + R with one exponential per band entry per iteration (row sums and
+// the plan entries of a 128-row strip on chip, column sums on the tensor core from the stored
+// entries).  Iteration 1 starts from the row potential already in u_tail slot 0 (any finite row
+// stabiliser, normally the first row half-step) and v = 0 in vb2.  No dustbin; T >= 1.
+struct IterLaunch {
+    Geom g;
+    const void* Q;
+    const void* K;
+    const float* logm;
+    const uint32_t* tile_bits;
+    float* u_tail;
+    float* v_tail;
+    size_t pstride;           // (R + 1) L
+    float* vb2;               // [BH, L] masked log2 v (initialised to v = 0)
+    float* part;              // column partial sums (workspace region ``part``)
+    uint32_t* gbar;           // 2 (T + R) zeroed grid-barrier counters
+    uint32_t* status;
+    int T, R;
+    int fused;                // 0: one launch per iteration; 1: one cooperative launch, per-iteration
+                              // launches if the device refuses it; 2: the cooperative launch only
+};
+// 0 when the problem does not fit the kernel, else 1 (one CTA per strip) or 2 (a CTA pair).
+int iter_split(const Geom& g);
+// *launched: kernels enqueued (1 cooperative launch, or 2 per iteration).
+cudaError_t launch_tc_iter(const IterLaunch& p, cudaStream_t st, int* launched);
 
 }  // namespace eot

@@ -1228,6 +1228,10 @@ bool tc_supported(const Geom& g) {
     return SweepCfg<128, 1 + kMaxMods>::smem_bytes(mt) <= kMaxSmem;
 }
 
+bool tma_map_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_rows) {
+    return make_map(m, base, rows, d, box_rows);
+}
+
 int sm_count() {
     static int n = [] {
         int dev = 0, v = 148;

@@ -145,10 +145,25 @@ int eot_abi_version(void);
  * the summed milliseconds and the number of bracketed launches of that kind. */
 long long eot_kernel_launches(void);
 /* Exponentials per band entry that the forward solve (base and tail, not the output sweep)
- * evaluates for problem *p with the kernels this library picks for it: 2 (T + R) when every
- * half-step forms its own plan entries, T + R + 1 when each iteration forms them once; -1 for an
- * invalid problem.  Benchmark support: the exponential-unit bound of the solve. */
+ * evaluates for problem *p under the current forward schedule: 2 (T + R) when every half-step
+ * forms its own plan entries, T + R + 1 when each iteration forms them once; -1 for an invalid
+ * problem.  Benchmark support: the exponential-unit bound of the solve. */
 int eot_solve_exp_passes(const eot_problem* p);
+/* Forward schedule for every later call in this process (benchmark and test support):
+ *   0, 1  the half-step schedule: every half-step forms the plan entries of its band once (two
+ *         exponentials per band entry per iteration).  0 is the default; it is the faster schedule
+ *         on every workload measured (a B200 at 1965 MHz: the long workload's solve 5.05 ms against
+ *         8.25 ms, the medium 1.12 against 1.85 ms, the protein-like 2.45 against 3.97 ms);
+ *   2     one exponential per band entry per iteration (row sums in registers, column sums on the
+ *         tensor core from the entries kept on chip) for bf16 problems without a dustbin, T >= 1,
+ *         d in {64, 128} and a band whose 128-row strips meet at most nine 128-column tiles (W up
+ *         to 1024), in one cooperative launch; a forward it cannot run returns EOT_ERR_UNSUPPORTED
+ *         (EOT_ERR_CUDA if the device refuses the launch);
+ *   3     the same with one launch per iteration (what 2 falls back to when the device refuses
+ *         the cooperative launch).
+ * Both schedules compute the same iterates; results differ by floating-point rounding only.
+ * Returns EOT_ERR_INVALID_ARGUMENT for any other value. */
+eot_status eot_set_forward_schedule(int schedule);
 void eot_profile_begin(void);
 eot_status eot_profile_end(void* stream);
 eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
@@ -176,7 +191,7 @@ eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
  *   - The device status word of these calls lives in the shared array: read (and clear) it
  *     with eot_static_last_device_status, which syncs ``stream`` like eot_last_device_status.
  * eot_static_scratch_bytes returns EOT_STATIC_SCRATCH_BYTES as built into the library. */
-#define EOT_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+#define EOT_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
 eot_status eot_sinkhorn_fwd_static(const eot_problem* p, const void* Q, const void* K, const void* V,
                                    const uint8_t* mask, void* O, float* u_tail, float* v_tail,
                                    void* stream);

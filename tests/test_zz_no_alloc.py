@@ -143,8 +143,8 @@ def test_static_scratch_call_allocates_no_device_memory():
 def test_static_scratch_rejects_oversized_problem():
     import torch
     from entropic_ot_attention_b200 import _abi, api
-    # forward scratch of B=8, H=16, L=8192 is ~21 MB > 16 MiB; nothing is launched
-    p = api.make_problem(8, 16, 8192, 64, 64, 2, 2, torch.bfloat16)
+    # forward scratch of B=8, H=16, L=16384 is ~42 MB, more than the static array; nothing is launched
+    p = api.make_problem(8, 16, 16384, 64, 64, 2, 2, torch.bfloat16)
     assert _abi.eot_workspace_bytes(p, False) > _abi.EOT_STATIC_SCRATCH_BYTES
     fake = 1 << 20
     st = _abi.eot_sinkhorn_fwd_static(p, fake, fake, fake, None, fake, fake, fake, 0)
