@@ -412,6 +412,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--schedule", default="auto", choices=["auto", "half_steps", "one_exp"],
                     help="forward schedule (eot_set_forward_schedule); auto picks per problem")
+    ap.add_argument("--bwd-schedule", default="recompute", choices=["recompute", "cached"], dest="bwd_schedule",
+                    help="backward: recompute the reference plan per sweep, or cache it for the staircase sweeps")
     ap.add_argument("--dry-run", action="store_true", dest="dry_run",
                     help="launch and aggregate over ranks without a GPU (host plumbing check)")
     args = ap.parse_args()
@@ -451,6 +453,7 @@ def main():
                          impl=args.impl)
     _abi.eot_set_forward_schedule({"auto": _abi.SCHEDULE_AUTO, "half_steps": _abi.SCHEDULE_HALF_STEPS,
                                    "one_exp": _abi.SCHEDULE_ONE_EXP}[args.schedule])
+    _abi.eot_set_backward_schedule(1 if args.bwd_schedule == "cached" else 0)
     impl_used = {1: "simt", 2: "tcgen05"}.get(_abi.eot_resolved_impl(p), "unsupported")
     ws_f = api.workspace(p, False, dev)
     ws_b = api.workspace(p, True, dev)
@@ -526,7 +529,11 @@ def main():
     roof_bwd_ms, bound_bwd = roofline_ms(work["bwd_flops"], work["bwd_bytes"], peak_tf, hbm)
     sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
     clk = clocks.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    dominant = dominant_kernel(prof, work, case.T, case.R, peak_tf, peaks["source"],
+    # the backward's sweeps are the staircase ones plus the others
+    prof_dom = dict(prof)
+    stair = prof.get("bwd_staircase", (0.0, 0))
+    prof_dom["bwd_sweep"] = (prof["bwd_sweep"][0] + stair[0], prof["bwd_sweep"][1] + stair[1])
+    dominant = dominant_kernel(prof_dom, work, case.T, case.R, peak_tf, peaks["source"],
                                exp_passes=_abi.eot_solve_exp_passes(p), omega=omega,
                                mufu_peak=sm_count * 16 * clk * 1e6)
     dominant["traffic"] = load_traffic(args.workload) if dominant["kind"] == "fwd_sweep" else None
@@ -538,6 +545,7 @@ def main():
         "data": "synthetic, seeded (eot_inputs); no dataset",
         "config": dict(workload_config(args.workload, case), impl=impl_used,
                        forward_exp_per_band_entry_per_call=_abi.eot_solve_exp_passes(p),
+                       forward_schedule=args.schedule, backward_schedule=args.bwd_schedule,
                        parallelism=f"{world} independent replica(s), no data-path collective",
                        l2="inputs larger than L2: Q, K, V, dO are 134 MB each" if args.workload == "long"
                        else "inputs resident; see workload sizes",

@@ -91,6 +91,8 @@ EOT_SELFTEST_CONTROL = 2
 lib.eot_kernel_launches.restype = ctypes.c_longlong
 lib.eot_solve_exp_passes.argtypes = [_P]
 lib.eot_solve_exp_passes.restype = ctypes.c_int
+lib.eot_set_backward_schedule.argtypes = [ctypes.c_int]
+lib.eot_set_backward_schedule.restype = ctypes.c_int
 lib.eot_set_forward_schedule.argtypes = [ctypes.c_int]
 lib.eot_set_forward_schedule.restype = ctypes.c_int
 SCHEDULE_AUTO, SCHEDULE_HALF_STEPS, SCHEDULE_ONE_EXP, SCHEDULE_ONE_EXP_PER_ITERATION = 0, 1, 2, 3
@@ -106,9 +108,9 @@ EXPORTED = ("eot_workspace_bytes", "eot_validate", "eot_sinkhorn_fwd", "eot_sink
             "eot_abi_version", "eot_resolved_impl", "eot_kernel_launches", "eot_profile_begin",
             "eot_profile_end", "eot_profile_read", "eot_sinkhorn_fwd_static", "eot_solve_exp_passes",
             "eot_static_last_device_status", "eot_static_scratch_bytes", "eot_wait_selftest",
-            "eot_set_forward_schedule")
+            "eot_set_forward_schedule", "eot_set_backward_schedule")
 
-PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3}
+PROF_KINDS = {"fwd_sweep": 0, "fwd_output": 1, "bwd_sweep": 2, "aux": 3, "bwd_staircase": 4}
 
 
 def eot_kernel_launches() -> int:
@@ -117,6 +119,10 @@ def eot_kernel_launches() -> int:
 
 def eot_solve_exp_passes(p: eot_problem) -> int:
     return int(lib.eot_solve_exp_passes(ctypes.byref(p)))
+
+
+def eot_set_backward_schedule(schedule: int) -> None:
+    _check(lib.eot_set_backward_schedule(int(schedule)), "eot_set_backward_schedule")
 
 
 def eot_set_forward_schedule(schedule: int) -> None:

@@ -40,7 +40,7 @@ namespace {
 // ---------------------------------------------------------------------------------------
 // Launch accounting and optional per-kind CUDA-event timing (benchmark support)
 // ---------------------------------------------------------------------------------------
-enum ProfKind { kProfLse = 0, kProfOut = 1, kProfBwd = 2, kProfAux = 3, kProfKinds = 4 };
+enum ProfKind { kProfLse = 0, kProfOut = 1, kProfBwd = 2, kProfAux = 3, kProfStair = 4, kProfKinds = 5 };
 
 struct Profiler {
     bool on = false;
@@ -80,6 +80,9 @@ cudaError_t tracked(int kind, int nkernels, cudaStream_t st, F&& f) {
 // schedule (measured faster on every workload), 2 the one-exponential-per-iteration kernel in one
 // cooperative launch, 3 that kernel with one launch per iteration.
 std::atomic<int> g_fwd_schedule{0};
+// Backward schedule (process-wide; measurement support): 0 recomputes the reference plan in every
+// sweep, 1 caches it (bf16 band store written by the alpha_R sweep) for the staircase sweeps.
+std::atomic<int> g_bwd_schedule{0};
 
 bool tensor_core_ok(const eot_problem& p) { return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128); }
 
@@ -164,6 +167,8 @@ cudaError_t aux(cudaStream_t st, F&& f) { return tracked(kProfAux, 1, st, f); }
 // Forward/backward bodies that take the workspace as an already-resolved device address.
 // (Also used by entry points that supply their own scratch.)
 namespace eot {
+
+int backward_schedule() { return g_bwd_schedule.load(); }
 
 eot_status validate_problem(const eot_problem* p) { return validate(p); }
 
@@ -459,14 +464,56 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     if (R > 0) {
         // R2: alpha_R = rowsum(P(R,R) * dP) - P(R,R) (beta_R / b)
         EOT_RANGE("eot backward: staircase vectors");
+        // With the cached schedule this sweep also stores its plan entries for the staircase.
+        const bool cached = impl == EOT_IMPL_TCGEN05 && cache_plan_possible(*p) && cached_sweeps_supported(g);
+        __nv_bfloat16* pcache = cached ? at<__nv_bfloat16>(ws, w.pcache) : nullptr;
         EOT_TRY(vec(kPassR2, 0));
-        EOT_TRY(scalar_pass(rowp, alpha + size_t(R) * vecn, true));
+        {
+            BwdPass bp = rowp;
+            bp.pcache = pcache;
+            EOT_TRY(scalar_pass(bp, alpha + size_t(R) * vecn, true));
+        }
+        CachedSweep cs{};
+        cs.H = g.H;
+        cs.L = g.L;
+        cs.h = g.h;
+        cs.BH = g.BH;
+        cs.cpitch = 2 * g.h + 128;
+        cs.logm = logm;
+        cs.tile_bits = tbits;
+        cs.P = pcache;
+        cs.f = va.f;
+        cs.hv = va.hv;
+        cs.m = va.m;
+        cs.status = status;
         for (int k = R - 1; k >= 1; --k) {
             // beta_k = -P(k+1,k)^T (alpha_{k+1} / a), alpha_k = -P(k,k) (beta_k / b)
             EOT_TRY(vec(kPassCk, k));
-            EOT_TRY(scalar_pass(colp, beta + size_t(k) * vecn, false));
+            if (cached) {
+                cs.out = beta + size_t(k) * vecn;
+                EOT_TRY(tracked(kProfStair, 1, st, [&] { return launch_cached_sweep(cs, true, st); }));
+            } else {
+                BwdPass bp = colp;
+                bp.sout = beta + size_t(k) * vecn;
+                bp.f = va.f;
+                bp.hv = va.hv;
+                bp.m = va.m;
+                bp.s_dp = 0;
+                EOT_TRY(run_bwd(impl, bp, st, kProfStair));
+            }
             EOT_TRY(vec(kPassRk, k));
-            EOT_TRY(scalar_pass(rowp, alpha + size_t(k) * vecn, false));
+            if (cached) {
+                cs.out = alpha + size_t(k) * vecn;
+                EOT_TRY(tracked(kProfStair, 1, st, [&] { return launch_cached_sweep(cs, false, st); }));
+            } else {
+                BwdPass bp = rowp;
+                bp.sout = alpha + size_t(k) * vecn;
+                bp.f = va.f;
+                bp.hv = va.hv;
+                bp.m = va.m;
+                bp.s_dp = 0;
+                EOT_TRY(run_bwd(impl, bp, st, kProfStair));
+            }
         }
     }
     // dQ = scale dS K (row sweep), dK = scale dS^T Q (column sweep); dS = P(R,R) (dP - sum x y^T)
@@ -556,6 +603,12 @@ int eot_solve_exp_passes(const eot_problem* p) {
         return p->T + p->R + 1;   // the first row half-step, then one per iteration
     // every half-step evaluates one exponential per band entry
     return 2 * (p->T + p->R);
+}
+
+eot_status eot_set_backward_schedule(int schedule) {
+    if (schedule < 0 || schedule > 1) return EOT_ERR_INVALID_ARGUMENT;
+    g_bwd_schedule.store(schedule);
+    return EOT_OK;
 }
 
 eot_status eot_set_forward_schedule(int schedule) {

@@ -87,6 +87,7 @@ struct BwdPass {
     const float* dp_term;   // <A_r, Bm_D>
     const float* dp_dense;  // <A_D, Bm_c>
     const float* zero_vec;  // [BH, L] zeros (padding of the modifier list), or nullptr
+    __nv_bfloat16* pcache;  // row sweep (alpha_R): cache its plan tiles here (tensor-core kernels), or nullptr
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
     float* dpart;           // as in LsePass
     uint32_t* dcnt;
@@ -107,6 +108,7 @@ struct WsLayout {
     size_t pr, pc, f, hv, m;
     size_t xr, yc;          // kMaxMods vectors each, [BH, L]
     size_t alpha, beta;     // (R + 1) vectors each, [BH, L]
+    size_t pcache;          // backward with the cached reference plan: bf16 band store [BH, L, 2 h + 128]
     size_t total;
 };
 
@@ -127,6 +129,15 @@ inline int iter_window_tiles(int L, int h) {
 inline bool iter_schedule_possible(const eot_problem& p) {
     return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin && p.T >= 1 && p.impl != EOT_IMPL_SIMT &&
            p.L >= 128 && iter_window_tiles(p.L, p.W / 2) <= 9;
+}
+
+// The backward caches its reference plan (a bf16 band store of 2 h + 128 entries a row) only
+// when asked to (eot_set_backward_schedule) and for tensor-core problems without a dustbin whose
+// half-width h is a multiple of 128 and whose tail has a staircase (R >= 2).
+int backward_schedule();
+inline bool cache_plan_possible(const eot_problem& p) {
+    return backward_schedule() == 1 && p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin &&
+           p.impl != EOT_IMPL_SIMT && (p.W / 2) % 128 == 0 && p.R >= 2;
 }
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
@@ -168,6 +179,10 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.yc = o; o += vec * 2 * p.R;
         w.alpha = o; o += vec * (p.R + 1);
         w.beta = o; o += vec * (p.R + 1);
+        if (cache_plan_possible(p)) {
+            w.pcache = o;
+            o += align256(BH * L * size_t(p.W / 2 * 2 + 128) * 2);
+        }
     }
     w.total = o;
     return w;

@@ -67,6 +67,23 @@ struct FusedSteps {
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
 
+// Staircase sweeps from the cached reference plan (cache.cu): out = f hv sum P m over the band, by
+// rows (P a_r Pt) or by columns; P is the bf16 tile-relative band store written by the alpha_R row
+// sweep (pcache).  Tensor-core bf16 problems without a dustbin and with h a multiple of 128.
+struct CachedSweep {
+    int H, L, h, BH, cpitch;
+    const float* logm;
+    const uint32_t* tile_bits;
+    const __nv_bfloat16* P;
+    const float* f;
+    const float* hv;
+    const float* m;
+    float* out;
+    uint32_t* status;
+};
+bool cached_sweeps_supported(const Geom& g);
+cudaError_t launch_cached_sweep(const CachedSweep& a, bool column, cudaStream_t st);
+
 // Forward iterations 1 .. T + R with one exponential per band entry per iteration (row sums and
 // the plan entries of a 128-row strip on chip, column sums on the tensor core from the stored
 // entries).  Iteration 1 starts from the row potential already in u_tail slot 0 (any finite row

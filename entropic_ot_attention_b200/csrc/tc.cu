@@ -718,6 +718,10 @@ struct TcVecArgs {
     const float* sd_term;
     const float* dp_term;
     uint32_t* status;
+    // Row sweep only: the plan entries Pt of every band tile, bf16, in a tile-relative band store
+    // (row r of row tile I at pcache[r * cpitch + (c - 128 I + h)], cpitch = 2 h + 128), or null.
+    __nv_bfloat16* pcache;
+    int cpitch;
 };
 
 constexpr int kSweepEpi = 16;         // epilogue warps: four per TMEM lane quadrant, 32 columns each
@@ -1072,6 +1076,14 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 }
 #pragma unroll
                 for (int j = 0; j < 32; ++j) vc[j] = ptx::ex2(vc[j]);
+                if (MODE == kModeR2 && a.pcache) {
+                    // cache this chunk of the plan: 32 entries of row r, 16-byte aligned (h % 8 == 0)
+                    uint4* dst = reinterpret_cast<uint4*>(a.pcache + (base + r) * size_t(a.cpitch) + (c0 + cc0 - r0 + h));
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        dst[t] = make_uint4(ptx::pack_bf16(vc[8 * t], vc[8 * t + 1]), ptx::pack_bf16(vc[8 * t + 2], vc[8 * t + 3]),
+                                            ptx::pack_bf16(vc[8 * t + 4], vc[8 * t + 5]), ptx::pack_bf16(vc[8 * t + 6], vc[8 * t + 7]));
+                }
                 if (M::SCAL) {
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
@@ -1431,6 +1443,8 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.sd_term = p.sd_term;
     a.dp_term = p.dp_term;
     a.status = p.status;
+    a.pcache = mode == kModeR2 ? p.pcache : nullptr;
+    a.cpitch = 2 * g.h + 128;
     const int mt = max_tiles_for(g.L, g.h, 128, 128);
     dim3 grid(g.L / 128, g.BH);
     cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st)

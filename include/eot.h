@@ -141,7 +141,8 @@ int eot_abi_version(void);
  * enqueue is bracketed by a pair of CUDA events recorded on the call's stream;
  * eot_profile_end synchronises ``stream`` and totals the elapsed times per kind.
  * eot_profile_read(kind, ...): kind 0 = forward half-step sweeps, 1 = forward output sweep,
- * 2 = backward sweeps, 3 = auxiliary kernels (marginals, vectors, dustbin links); returns
+ * 2 = backward sweeps other than the staircase, 3 = auxiliary kernels (marginals, vectors,
+ * dustbin links), 4 = the staircase sweeps of the backward (R >= 2); returns
  * the summed milliseconds and the number of bracketed launches of that kind. */
 long long eot_kernel_launches(void);
 /* Exponentials per band entry that the forward solve (base and tail, not the output sweep)
@@ -164,6 +165,17 @@ int eot_solve_exp_passes(const eot_problem* p);
  * Both schedules compute the same iterates; results differ by floating-point rounding only.
  * Returns EOT_ERR_INVALID_ARGUMENT for any other value. */
 eot_status eot_set_forward_schedule(int schedule);
+/* Backward schedule for every later workspace query and backward call in this process
+ * (measurement support):
+ *   0  every sweep recomputes the reference plan P(R,R) from S on the tensor cores (default; the
+ *      extra memory stays O(L));
+ *   1  the alpha_R row sweep also stores its plan entries as bf16 in a band store of
+ *      B H L (2 (W/2) + 128) entries inside the workspace, and the staircase sweeps (R >= 2) stream
+ *      it on CUDA cores instead of recomputing it: for tensor-core problems without a dustbin
+ *      whose half-width W/2 is a multiple of 128; others run schedule 0.
+ * eot_workspace_bytes(p, 1) includes the band store only under schedule 1.  Returns
+ * EOT_ERR_INVALID_ARGUMENT for any other value. */
+eot_status eot_set_backward_schedule(int schedule);
 void eot_profile_begin(void);
 eot_status eot_profile_end(void* stream);
 eot_status eot_profile_read(int kind, double* total_ms, long long* launches);
