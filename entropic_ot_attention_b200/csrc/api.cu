@@ -238,11 +238,12 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         col.out = v_tail + size_t(k_out) * L;
         return run_lse(impl, col, st);
     };
-    // Tensor-core path without a dustbin: the first half-step (running maximum) on its own, then
-    // either every iteration with one exponential per band entry (iter.cu: the first row
+    // Tensor-core path: the first half-step (running maximum) on its own, then either every
+    // iteration with one exponential per band entry (iter.cu, no dustbin: the first row
     // half-step's u is the row stabiliser of iteration 1, which recomputes it), or every later
-    // half-step in one cooperative launch with grid-wide barriers between them.  If the device
-    // cannot hold the whole grid at once the iterations / half-steps run as separate launches.
+    // half-step in one cooperative launch with grid-wide barriers between them (with a dustbin
+    // that launch also sums each half-step's dense dustbin row).  If the device cannot hold the
+    // whole grid at once the iterations / half-steps run as separate launches.
     const int n_half = 2 * (p->T + p->R);
     bool fused = false;
     const int sched = g_fwd_schedule.load();
@@ -277,7 +278,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         int launched = 0;
         EOT_TRY(tracked(kProfLse, 0, st, [&] { return launch_tc_iter(il, st, &launched); }));
         g_launches += launched;
-    } else if (impl == EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
+    } else if (impl == EOT_IMPL_TCGEN05 && n_half >= 2) {
         EOT_TRY(run_lse(impl, [&] {
             LsePass r0 = row;
             r0.colpot = v_tail;
@@ -290,7 +291,10 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar};
         const cudaError_t e = tracked(kProfLse, 1, st, [&] { return launch_tc_lse_fused(row, f, st); });
         if (e == cudaSuccess) fused = true;
-        else if (e == cudaErrorCooperativeLaunchTooLarge) (void)cudaGetLastError();
+        else if (e == cudaErrorCooperativeLaunchTooLarge) {
+            (void)cudaGetLastError();
+            g_launches -= 1;   // the refused launch
+        }
         else return EOT_ERR_CUDA;
         if (!fused) {
             // finish the first iteration's column half-step, then the rest one launch each
@@ -302,6 +306,22 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
             EOT_TRY(run_lse(impl, col, st));
             for (int t = 1; t < p->T; ++t) EOT_TRY(step(0, 0));
             for (int k = (p->T > 0 ? 1 : 2); k <= p->R; ++k) EOT_TRY(step(k - 1, k));
+        }
+    } else if (impl != EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
+        // CUDA-core path without a dustbin: every half-step in one cooperative launch (the kernel
+        // keeps no running stabiliser, so the first half-step needs no separate launch).
+        uint32_t* gbar = at<uint32_t>(ws, w.gbar);
+        EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
+        const cudaError_t e = tracked(kProfLse, 1, st, [&] {
+            return launch_simt_lse_fused(row, Q, K, u_tail, v_tail, ub2, vb2, p->T, p->R, gbar, st);
+        });
+        if (e == cudaErrorCooperativeLaunchTooLarge) {
+            (void)cudaGetLastError();
+            g_launches -= 1;   // the refused launch
+            for (int t = 0; t < p->T; ++t) EOT_TRY(step(0, 0));
+            for (int k = 1; k <= p->R; ++k) EOT_TRY(step(k - 1, k));
+        } else if (e != cudaSuccess) {
+            return EOT_ERR_CUDA;
         }
     } else {
         for (int t = 0; t < p->T; ++t) EOT_TRY(step(0, 0));                 // stopped base

@@ -26,6 +26,10 @@ cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbi
 cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
                                 cudaStream_t st);
 cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st);
+// Every half-step of a forward without a dustbin on CUDA cores in one cooperative launch (row
+// half-step template `row`; slots as in FusedSteps; gbar: 2 (T + R) zeroed counters).
+cudaError_t launch_simt_lse_fused(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail,
+                                  float* ub2, float* vb2, int T, int R, uint32_t* gbar, cudaStream_t st);
 cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
 cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
 cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st);

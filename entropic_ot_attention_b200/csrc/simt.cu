@@ -15,6 +15,7 @@
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace eot {
 
@@ -82,15 +83,15 @@ __global__ void __launch_bounds__(256) prep_dustbin_dots_kernel(Geom g, const T*
 // ---------------------------------------------------------------------------------------
 // Forward half-step on CUDA cores (online max; fp32 scores)
 // ---------------------------------------------------------------------------------------
+// Rows [32 rblk, 32 rblk + 32) of unit bh (the whole CTA takes part).
 template <typename T>
-__global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
-    extern __shared__ float sm[];
+__device__ void simt_lse_item(const LsePass& p, int rblk, int bh, float* sm) {
     const int d = p.g.d, ld = d + 1, L = p.g.L, h = p.g.h, D = p.g.D;
     float* Xs = sm;
     float* Ys = Xs + kSB * ld;
     float* bs = Ys + kSB * ld;
-    const int bh = blockIdx.y, b = bh / p.g.H;
-    const int r0 = blockIdx.x * kSB;
+    const int b = bh / p.g.H;
+    const int r0 = rblk * kSB;
     const size_t base = size_t(bh) * L;
     const size_t pb = size_t(bh) * p.pstride;
     const T* X = static_cast<const T*>(p.X) + base * d;
@@ -160,6 +161,61 @@ __global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
         }
         p.out[pb + r] = outv;
         p.out_bias2[base + r] = ob;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kSNT) simt_lse_kernel(LsePass p) {
+    extern __shared__ float sm[];
+    simt_lse_item<T>(p, blockIdx.x, blockIdx.y, sm);
+}
+
+// Every half-step of a forward without a dustbin in one cooperative launch: half-step hs
+// (row when even: X = Q, Y = K; column when odd: X = K, Y = Q) of iteration it = hs / 2 reads and
+// writes potential slot 0 for the first T iterations and slot it - T + 1 after (the column
+// potential of a row half-step comes from the previous iteration's slot); a grid-wide barrier
+// (gbar[hs]: CTAs done with half-step hs) separates consecutive half-steps.
+template <typename T>
+__global__ void __launch_bounds__(kSNT) simt_lse_fused_kernel(LsePass row, const void* Qp, const void* Kp, float* u_tail,
+                                                              float* v_tail, float* ub2, float* vb2, int nhs, int Tb,
+                                                              uint32_t* gbar) {
+    extern __shared__ float sm[];
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) abort_flag = 0;
+    __syncthreads();
+    const int L = row.g.L, items = (L / kSB) * row.g.BH;
+    for (int hs = 0; hs < nhs; ++hs) {
+        if (hs > 0) {
+            // every CTA is done with half-step hs - 1
+            if (threadIdx.x == 0) ptx::grid_wait(gbar + hs - 1, gridDim.x, &abort_flag, row.status);
+            __syncthreads();
+            if (abort_flag) return;
+        }
+        const int it = hs >> 1;
+        const int sout = it < Tb ? 0 : it - Tb + 1, sin = it < Tb ? 0 : it - Tb;
+        LsePass p = row;
+        if ((hs & 1) == 0) {
+            p.X = Qp;
+            p.Y = Kp;
+            p.colpot = v_tail + size_t(sin) * L;
+            p.out = u_tail + size_t(sout) * L;
+            p.out_bias2 = ub2;
+        } else {
+            p.X = Kp;
+            p.Y = Qp;
+            p.colpot = u_tail + size_t(sout) * L;
+            p.out = v_tail + size_t(sout) * L;
+            p.out_bias2 = vb2;
+        }
+        for (int item = blockIdx.x; item < items; item += gridDim.x) {
+            __syncthreads();   // the previous item's tiles are no longer read
+            simt_lse_item<T>(p, item % (L / kSB), item / (L / kSB), sm);
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atomicAdd(gbar + hs, 1u);
+        }
     }
 }
 
@@ -591,6 +647,28 @@ cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
+}
+
+cudaError_t launch_simt_lse_fused(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail,
+                                  float* ub2, float* vb2, int T, int R, uint32_t* gbar, cudaStream_t st) {
+    if (row.g.D >= 0 || !gbar) return cudaErrorInvalidValue;
+    const size_t smem = simt_lse_smem(row.g.d);
+    const int items = (row.g.L / kSB) * row.g.BH;
+    int nhs = 2 * (T + R);
+    auto launch = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        int per_sm = 0, dev = 0, n_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kSNT, smem);
+        if (e != cudaSuccess) return e;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        const int grid = std::max(1, std::min(items, per_sm * n_sm));
+        LsePass r = row;
+        void* args[] = {&r, const_cast<void**>(&Q), const_cast<void**>(&K), &u_tail, &v_tail, &ub2, &vb2, &nhs, &T, &gbar};
+        return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid), dim3(kSNT), args, smem, st);
+    };
+    return row.g.dtype == EOT_BF16 ? launch(simt_lse_fused_kernel<__nv_bfloat16>) : launch(simt_lse_fused_kernel<float>);
 }
 
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st) {

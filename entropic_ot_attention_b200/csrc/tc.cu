@@ -152,6 +152,15 @@ struct TcBandArgs {
     float* ub2;
     float* vb2;
     uint32_t* gbar;
+    // Fused half-steps with a dustbin: the dustbin links of the rows (sd_row: S between row r
+    // and the dustbin column) and of the columns (sd_col: S between the dustbin row and column
+    // c); the dense dustbin row of every half-step is summed per item ((max, sum) partials in
+    // dpart[bh][pair]) and merged by the last item of the unit (dcnt[bh], zero at launch).
+    const float* sd_row;
+    const float* sd_col;
+    float* dpart;
+    uint32_t* dcnt;
+    int dself;                  // (D, D) in the support
 };
 
 template <int DH, int KIND>
@@ -230,6 +239,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         return MULTI ? ((hs & 1) ? a.v_tail : a.u_tail) + size_t(slot_of(hs, true)) * a.L : a.out;
     };
     auto outb_of = [&](int hs) -> float* { return MULTI ? ((hs & 1) ? a.vb2 : a.ub2) : a.out_bias2; };
+    // natural column potential (read at the dustbin) and the rows' dustbin links
+    auto colpot_of = [&](int hs) -> const float* {
+        return MULTI ? ((hs & 1) ? a.u_tail + size_t(slot_of(hs, true)) * a.L : a.v_tail + size_t(slot_of(hs, false)) * a.L)
+                     : a.colpot;
+    };
+    auto sdterm_of = [&](int hs) -> const float* { return MULTI ? ((hs & 1) ? a.sd_col : a.sd_row) : a.sd_term; };
     auto mapx_of = [&](int hs) { return (MULTI && (hs & 1)) ? &tmY : &tmX; };
     auto mapy_of = [&](int hs) { return (MULTI && (hs & 1)) ? &tmX : &tmY; };
     extern __shared__ uint8_t smraw[];
@@ -480,7 +495,9 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             const size_t pb = size_t(bh) * a.pstride;
             const uint32_t* bitp = bits_of(b);
             if (!tile_bit(bitp, rg / C::BM)) {
-                if (hf == 0) {
+                // (fused half-steps: an active dustbin's row is written by the dense dustbin row;
+                // a single half-step's dense dustbin kernel runs after this one)
+                if (hf == 0 && !(MULTI && r == D && a.logm[size_t(b) * L + D] != kNegInf)) {
                     out_hs[pb + r] = 0.f;
                     if (!WSUM) outb_hs[base + r] = kNegInf;
                 }
@@ -639,10 +656,11 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 if (lm != kNegInf) {
                     const bool d_act = D >= 0 && logm[D] != kNegInf;
                     if (ONLINE) {
-                        if (d_act) lse2_add(mm, sum, (a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e);
+                        if (d_act) lse2_add(mm, sum, (sdterm_of(hs)[base + r] + colpot_of(hs)[pb + D]) * kLog2e);
                         outv = lm - (mm + log2f(sum)) * kLn2;
                     } else {
-                        const float dterm = d_act ? ptx::ex2((a.sd_term[base + r] + a.colpot[pb + D]) * kLog2e + st2) : 0.f;
+                        const float dterm =
+                            d_act ? ptx::ex2((sdterm_of(hs)[base + r] + colpot_of(hs)[pb + D]) * kLog2e + st2) : 0.f;
                         if (WSUM) {
                             if (d_act) sum = fmaf(dterm, a.colw[base + D], sum);
                             outv = a.f[base + r] * a.hv[base + r] * sum;
@@ -655,6 +673,59 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 }
                 out_hs[pb + r] = outv;
                 if (!WSUM) outb_hs[base + r] = ob;
+            }
+        }
+        if (MULTI && D >= 0 && __all_sync(0xffffffffu, ok && !*abort_flag)) {
+            // Dense dustbin row of half-step hs: out_D = logm_D - LSE_c (S_Dc + colpot_c) over
+            // every active real column c (plus (D, D) when it is in the support).  Epilogue warp e
+            // sums the columns of this CTA's items e, e + 16, ... (the item's 256 positions); the
+            // last item of a unit to finish merges the unit's partials.
+            const float* colpot_hs = colpot_of(hs);
+            const float* sdterm_hs = sdterm_of(hs);
+            for (int item = item0 + e; item < item1; item += 16) {
+                const int bh = item / a.pairs_per_unit, b = bh / a.H, pi = item - bh * a.pairs_per_unit;
+                const float* logm = a.logm + size_t(b) * L;
+                if (logm[D] == kNegInf) continue;
+                const size_t base = size_t(bh) * L, pb = size_t(bh) * a.pstride;
+                const float* sdense = (hs & 1) ? a.sd_row : a.sd_col;
+                float m = kNegInf, s = 0.f;
+                const int c_end = min(L, pi * 2 * C::BM + 2 * C::BM);
+                for (int c = pi * 2 * C::BM + lane; c < c_end; c += 32) {
+                    if (c == D) {
+                        if (a.dself) lse2_add(m, s, (sdterm_hs[base + D] + colpot_hs[pb + D]) * kLog2e);
+                    } else if (logm[c] != kNegInf) {
+                        lse2_add(m, s, (sdense[base + c] + colpot_hs[pb + c]) * kLog2e);
+                    }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float m2 = __shfl_xor_sync(0xffffffffu, m, off), s2 = __shfl_xor_sync(0xffffffffu, s, off);
+                    lse2_merge(m, s, m2, s2);
+                }
+                float* part = a.dpart + size_t(bh) * 2 * a.pairs_per_unit;
+                uint32_t last = 0;
+                if (lane == 0) {
+                    part[2 * pi] = m;
+                    part[2 * pi + 1] = s;
+                    __threadfence();
+                    last = atomicAdd(a.dcnt + bh, 1u) == uint32_t(a.pairs_per_unit - 1);
+                }
+                if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+                __threadfence();
+                float mm = kNegInf, ss = 0.f;
+                for (int i = lane; i < a.pairs_per_unit; i += 32) lse2_merge(mm, ss, __ldcg(part + 2 * i), __ldcg(part + 2 * i + 1));
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float m2 = __shfl_xor_sync(0xffffffffu, mm, off), s2 = __shfl_xor_sync(0xffffffffu, ss, off);
+                    lse2_merge(mm, ss, m2, s2);
+                }
+                if (lane == 0) {
+                    const float outv = logm[D] - (mm + log2f(ss)) * kLn2;
+                    if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+                    out_hs[pb + D] = outv;
+                    outb_hs[base + D] = kNegInf;   // the dustbin never enters a band sum
+                    a.dcnt[bh] = 0u;                 // ready for the next half-step
+                }
             }
         }
         if (MULTI) {
@@ -1282,6 +1353,7 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     a.L = g.L;
     a.h = g.h;
     a.D = g.D;
+    a.dself = g.dself;
     a.sl2 = g.scale * kLog2e;
     a.words = tile_words(g.L);
     a.pairs_per_unit = (g.L / 128 + 1) / 2;
@@ -1292,7 +1364,9 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     if (!multi) {
         a.hs0 = 0;
         a.nhs = 1;
-    } else if (kind != kBandShift || g.D >= 0 || !a.gbar || a.nhs < 1) {
+    } else if (kind != kBandShift || !a.gbar || a.nhs < 1 ||
+               (g.D >= 0 && (!a.sd_row || !a.sd_col || !a.dpart || !a.dcnt ||
+                             2 * size_t(a.pairs_per_unit) > size_t(dustbin_splits(g.L)) * size_t(g.d + 2)))) {
         return cudaErrorInvalidValue;
     }
     if (g.d == 128) {
@@ -1331,7 +1405,7 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
 }
 
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st) {
-    if (!row.tile_bits || row.g.D >= 0) return cudaErrorInvalidValue;
+    if (!row.tile_bits) return cudaErrorInvalidValue;
     TcBandArgs a{};
     a.logm = row.logm;
     a.tile_bits = row.tile_bits;
@@ -1345,6 +1419,10 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     a.ub2 = f.ub2;
     a.vb2 = f.vb2;
     a.gbar = f.gbar;
+    a.sd_row = row.sd_term;
+    a.sd_col = row.sd_dense;
+    a.dpart = row.dpart;
+    a.dcnt = row.dcnt;
     // row half-steps: X = Q (row.X), Y = K (row.Y); the kernel swaps them for column half-steps
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
