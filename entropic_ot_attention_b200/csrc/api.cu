@@ -307,6 +307,9 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
             for (int t = 1; t < p->T; ++t) EOT_TRY(step(0, 0));
             for (int k = (p->T > 0 ? 1 : 2); k <= p->R; ++k) EOT_TRY(step(k - 1, k));
         }
+    } else if (impl != EOT_IMPL_TCGEN05 && n_half >= 2 && simt_resident_possible(g)) {
+        // CUDA-core path, small units: the whole solve of each unit in one CTA, scores formed once
+        EOT_TRY(tracked(kProfLse, 1, st, [&] { return launch_simt_resident(row, Q, K, u_tail, v_tail, p->T, p->R, st); }));
     } else if (impl != EOT_IMPL_TCGEN05 && g.D < 0 && n_half >= 2) {
         // CUDA-core path without a dustbin: every half-step in one cooperative launch (the kernel
         // keeps no running stabiliser, so the first half-step needs no separate launch).
@@ -462,6 +465,14 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
         return run_bwd(impl, bp, st);
     };
 
+    // With the split alpha_R sweep (tensor-core kernels), the column sweep C1 also leaves the
+    // partial row sums of Pt dP in s1part, and alpha_R becomes a staircase-form band sum plus them.
+    const bool split = R > 0 && impl == EOT_IMPL_TCGEN05 && w.s1split;
+    float* s1part = split ? at<float>(ws, w.s1part) : nullptr;
+    const int s1E = s1_reach(p->W);
+    const int s1slots = int(s1_slots(p->W));
+    if (split) EOT_TRY(cudaMemsetAsync(s1part, 0, size_t(s1slots) * vecn * sizeof(float), st));
+
     // C1: beta_R = colsum(P(R,R) * dP) and dV = P(R,R)^T (dO / a)   (one column sweep)
     EOT_TRY(vec(kPassC1, 0));
     {
@@ -473,6 +484,9 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
             bp.hv = va.hv;
             bp.m = nullptr;
             bp.s_dp = 1;
+            bp.s1part = s1part;
+            bp.s1stride = vecn;
+            bp.s1E = s1E;
         }
         bp.vout = dV;
         bp.Z = dO;
@@ -487,8 +501,26 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
         // With the cached schedule this sweep also stores its plan entries for the staircase.
         const bool cached = impl == EOT_IMPL_TCGEN05 && cache_plan_possible(*p) && cached_sweeps_supported(g);
         __nv_bfloat16* pcache = cached ? at<__nv_bfloat16>(ws, w.pcache) : nullptr;
+        if (split) {
+            va.s1part = s1part;
+            va.s1slots = s1slots;
+            va.s1stride = vecn;
+            va.sadd = at<float>(ws, w.sadd);
+        }
         EOT_TRY(vec(kPassR2, 0));
-        {
+        va.s1part = nullptr;
+        va.sadd = nullptr;
+        if (split) {
+            // alpha_R = (row sums of Pt dP from C1) + hv_r sum_c Pt_rc m_c: a staircase-form sum
+            BwdPass bp = rowp;
+            bp.sout = alpha + size_t(R) * vecn;
+            bp.f = va.f;
+            bp.hv = va.hv;
+            bp.m = va.m;
+            bp.s_dp = 0;
+            bp.sadd = at<float>(ws, w.sadd);
+            EOT_TRY(run_bwd(impl, bp, st, kProfStair));
+        } else {
             BwdPass bp = rowp;
             bp.pcache = pcache;
             EOT_TRY(scalar_pass(bp, alpha + size_t(R) * vecn, true));

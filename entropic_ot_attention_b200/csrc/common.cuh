@@ -88,6 +88,13 @@ struct BwdPass {
     const float* dp_dense;  // <A_D, Bm_c>
     const float* zero_vec;  // [BH, L] zeros (padding of the modifier list), or nullptr
     __nv_bfloat16* pcache;  // row sweep (alpha_R): cache its plan tiles here (tensor-core kernels), or nullptr
+    // Column sweep beta_R (tensor-core kernels): also write, per column position c, partial sums
+    // of Pt_rc dP_rc over the 32 rows r of each (row tile, TMEM lane quadrant q) into
+    // s1part[(o * 4 + q) s1stride + bh L + c], o = column tile - row tile + s1E; or nullptr.
+    float* s1part;
+    size_t s1stride;
+    int s1E;
+    const float* sadd;      // staircase-form sweeps: out_r = f_r (hv_r sum_c ... + sadd_r), or nullptr
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
     float* dpart;           // as in LsePass
     uint32_t* dcnt;
@@ -109,6 +116,8 @@ struct WsLayout {
     size_t xr, yc;          // kMaxMods vectors each, [BH, L]
     size_t alpha, beta;     // (R + 1) vectors each, [BH, L]
     size_t pcache;          // backward with the cached reference plan: bf16 band store [BH, L, 2 h + 128]
+    size_t s1part, sadd;    // backward, split alpha_R sweep: partial sums [4 (2 E + 1)][BH, L] and their total
+    bool s1split;
     size_t total;
 };
 
@@ -139,6 +148,17 @@ inline bool cache_plan_possible(const eot_problem& p) {
     return backward_schedule() == 1 && p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin &&
            p.impl != EOT_IMPL_SIMT && (p.W / 2) % 128 == 0 && p.R >= 2;
 }
+
+// The alpha_R sweep of the backward is split (the column sweep beta_R also writes the partial row
+// sums of Pt dP, and alpha_R becomes a staircase-form band sum) for tensor-core problems without
+// a dustbin whose band reaches at most E = ceil(h / 128) <= 7 tiles to each side, unless the
+// cached-plan schedule is selected (its alpha_R sweep stores the plan).
+inline int s1_reach(int W) { return (W / 2 + 127) / 128; }
+inline bool s1_split_possible(const eot_problem& p) {
+    return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin && p.impl != EOT_IMPL_SIMT && p.R >= 1 &&
+           p.L % 128 == 0 && s1_reach(p.W) <= 7 && !cache_plan_possible(p);
+}
+inline size_t s1_slots(int W) { return size_t(4) * size_t(2 * s1_reach(W) + 1); }
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     WsLayout w{};
@@ -182,6 +202,11 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         if (cache_plan_possible(p)) {
             w.pcache = o;
             o += align256(BH * L * size_t(p.W / 2 * 2 + 128) * 2);
+        }
+        if (s1_split_possible(p)) {
+            w.s1split = true;
+            w.s1part = o; o += s1_slots(p.W) * vec;
+            w.sadd = o; o += vec;
         }
     }
     w.total = o;

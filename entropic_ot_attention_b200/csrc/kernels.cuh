@@ -19,6 +19,12 @@ struct BwdVecArgs {
     const float* beta;      // [R+1][BH*L]
     float *pr, *pc, *pcm2, *f, *hv, *m;
     float *xr, *yc;         // [2R][BH*L]
+    // kPassR2 of the split alpha_R sweep: sadd = sum of the s1slots partial sums in s1part
+    // (slot stride s1stride), the Pt dP row sums the column sweep beta_R left there
+    const float* s1part;
+    int s1slots;
+    size_t s1stride;
+    float* sadd;
 };
 
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
@@ -30,6 +36,11 @@ cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st);
 // half-step template `row`; slots as in FusedSteps; gbar: 2 (T + R) zeroed counters).
 cudaError_t launch_simt_lse_fused(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail,
                                   float* ub2, float* vb2, int T, int R, uint32_t* gbar, cudaStream_t st);
+// The whole forward solve (every half-step, no dustbin) of each unit in one CTA, with the
+// unit's band scores formed once into shared memory; when they fit (simt_resident_possible).
+bool simt_resident_possible(const Geom& g);
+cudaError_t launch_simt_resident(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail, int T,
+                                 int R, cudaStream_t st);
 cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
 cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
 cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st);

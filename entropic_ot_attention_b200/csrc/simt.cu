@@ -59,12 +59,14 @@ __global__ void __launch_bounds__(256) prep_marginals_kernel(Geom g, const uint8
 }
 
 // Dustbin link vectors: out_term[r] = s1 * <P_r, Q_D>, out_dense[r] = s1 * <P_D, Q_r> for
-// every position r of every unit (used for S and, in the backward, for dP).
+// every position r of every unit (used for S and, in the backward, for dP).  One warp per row:
+// lane l takes elements l, l + 32, ... (coalesced), the two dots meet by shuffles.
 template <typename T>
 __global__ void __launch_bounds__(256) prep_dustbin_dots_kernel(Geom g, const T* P, const T* Qm, float s1,
                                                                 float* out_term, float* out_dense) {
-    const int bh = blockIdx.y;
-    const int r = blockIdx.x * blockDim.x + threadIdx.x;
+    const int bh = blockIdx.y, lane = threadIdx.x & 31;
+    const int rows_per_block = blockDim.x >> 5;
+    const int r = blockIdx.x * rows_per_block + (threadIdx.x >> 5);
     if (r >= g.L) return;
     const size_t base = size_t(bh) * g.L;
     const T* pr = P + (base + r) * g.d;
@@ -72,12 +74,19 @@ __global__ void __launch_bounds__(256) prep_dustbin_dots_kernel(Geom g, const T*
     const T* qr = Qm + (base + r) * g.d;
     const T* qD = Qm + (base + g.D) * g.d;
     float a = 0.f, b = 0.f;
-    for (int k = 0; k < g.d; ++k) {
+    for (int k = lane; k < g.d; k += 32) {
         a = fmaf(to_f(pr[k]), to_f(qD[k]), a);
         b = fmaf(to_f(pD[k]), to_f(qr[k]), b);
     }
-    out_term[base + r] = s1 * a;
-    out_dense[base + r] = s1 * b;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, off);
+        b += __shfl_xor_sync(0xffffffffu, b, off);
+    }
+    if (lane == 0) {
+        out_term[base + r] = s1 * a;
+        out_dense[base + r] = s1 * b;
+    }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -599,6 +608,12 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
     if (a.f) a.f[idx] = f;
     if (a.hv) a.hv[idx] = hv;
     if (a.m) a.m[idx] = m;
+    if (a.kind == kPassR2 && a.s1part && a.sadd) {
+        float t = 0.f;
+        if (act)
+            for (int sl = 0; sl < a.s1slots; ++sl) t += a.s1part[size_t(sl) * a.s1stride + idx];
+        a.sadd[idx] = t;
+    }
     for (int k = 0; k < nm; ++k) {
         a.xr[size_t(k) * a.BH * L + idx] = xr[k];
         a.yc[size_t(k) * a.BH * L + idx] = yc[k];
@@ -616,7 +631,7 @@ cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbi
 
 cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
                                 cudaStream_t st) {
-    dim3 grid((g.L + 255) / 256, g.BH);
+    dim3 grid((g.L + 7) / 8, g.BH);   // 8 rows (warps) per block
     if (g.dtype == EOT_BF16)
         prep_dustbin_dots_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
             g, static_cast<const __nv_bfloat16*>(P), static_cast<const __nv_bfloat16*>(Qm), s1, term, dense);
@@ -647,6 +662,141 @@ cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
+}
+
+// ---------------------------------------------------------------------------------------
+// Whole forward solve of one unit in one CTA (small problems on CUDA cores)
+// ---------------------------------------------------------------------------------------
+// The scores S_rc of the unit's band (|r - c| <= h) do not change between half-steps, so they
+// are formed once, in fp32 with the same products as simt_lse_item, and kept in shared memory
+// as sband[r * (2 h + 1) + (c - r + h)]; the log2 potential biases of both sides stay there too.
+// Every half-step is then a band log-sum-exp over shared memory (groups of G threads per row
+// or column, merged by shuffles), separated by __syncthreads() instead of a grid barrier.
+constexpr int kResThreads = 1024;
+constexpr int kResRB = 32;   // rows of Q per staging chunk while the scores are formed
+
+size_t simt_resident_smem(int L, int h, int d) {
+    const size_t stage = size_t(2 * kResRB + 2 * h) * size_t(d + 1);   // Q chunk + the K rows its band reaches
+    return (size_t(L) * size_t(2 * h + 1) + 3 * size_t(L) + stage) * sizeof(float);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kResThreads) simt_resident_kernel(LsePass g0, const void* Qp, const void* Kp,
+                                                                     float* u_tail, float* v_tail, int Tb, int R) {
+    extern __shared__ float sm[];
+    const int L = g0.g.L, h = g0.g.h, d = g0.g.d, ld = 2 * h + 1;
+    const int bh = blockIdx.x, b = bh / g0.g.H;
+    float* sband = sm;
+    float* lmb = sband + size_t(L) * ld;   // log marginals
+    float* ub2 = lmb + L;                  // log2 e * u, -inf for inactive rows
+    float* vb2 = ub2 + L;
+    float* Qs = vb2 + L;                     // [kResRB][d + 1]
+    float* Ks = Qs + kResRB * (d + 1);       // [kResRB + 2 h][d + 1]
+    const size_t base = size_t(bh) * L, pb = size_t(bh) * g0.pstride;
+    const T* Q = static_cast<const T*>(Qp) + base * d;
+    const T* K = static_cast<const T*>(Kp) + base * d;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+        const float lm = g0.logm[size_t(b) * L + i];
+        lmb[i] = lm;
+        vb2[i] = lm != neg_inf() ? 0.f : neg_inf();   // v = 0
+    }
+    // scores of rows [r0, r0 + kResRB): Q rows and the K rows [r0 - h, r0 + kResRB + h) staged
+    // in shared memory (row pitch d + 1: neighbouring columns fall in different banks)
+    for (int r0 = 0; r0 < L; r0 += kResRB) {
+        const int nr = min(kResRB, L - r0), k0 = r0 - h, nk = nr + 2 * h;
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * d; e += blockDim.x) {
+            const int i = e / d, k = e - i * d;
+            Qs[i * (d + 1) + k] = to_f(Q[size_t(r0 + i) * d + k]);
+        }
+        for (int e = threadIdx.x; e < nk * d; e += blockDim.x) {
+            const int i = e / d, k = e - i * d, c = k0 + i;
+            Ks[i * (d + 1) + k] = (c >= 0 && c < L) ? to_f(K[size_t(c) * d + k]) : 0.f;
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < nr * ld; e += blockDim.x) {
+            const int i = e / ld, j = e - i * ld;   // row r0 + i, column r0 + i - h + j = k0 + i + j
+            const float* qa = Qs + i * (d + 1);
+            const float* ka = Ks + (i + j) * (d + 1);
+            float acc = 0.f;
+            for (int k = 0; k < d; ++k) acc = fmaf(qa[k], ka[k], acc);
+            sband[size_t(r0) * ld + e] = acc;
+        }
+    }
+    __syncthreads();
+    // G threads per row (a power of two dividing 32), groups strided over the rows
+    int G = 1;
+    while (G < 32 && G * 2 * L <= int(blockDim.x)) G *= 2;
+    const int grp = threadIdx.x / G, gl = threadIdx.x % G, ngrp = blockDim.x / G;
+    const float sl2 = g0.g.scale * kLog2e;
+    for (int hs = 0; hs < 2 * (Tb + R); ++hs) {
+        const int it = hs >> 1;
+        const int slot = it < Tb ? 0 : it - Tb + 1;
+        const bool col = hs & 1;
+        const float* bias = col ? ub2 : vb2;   // the other side's log2 potential
+        float* outb = col ? vb2 : ub2;
+        float* out = (col ? v_tail : u_tail) + pb + size_t(slot) * L;
+        for (int r0 = 0; r0 < L; r0 += ngrp) {   // uniform trip count: the shuffles below see every lane
+            const int r = r0 + grp;
+            // this thread's band entries: the maximum first, then the shifted sum
+            float m = neg_inf(), s = 0.f;
+            auto term = [&](int j) {
+                const int c = r - h + j;
+                if (c < 0 || c >= L) return neg_inf();
+                const float bc = bias[c];
+                if (bc == neg_inf()) return neg_inf();
+                // S_rc for a row half-step, S_cr (the same product) for a column half-step
+                const float sv = col ? sband[size_t(c) * ld + (r - c + h)] : sband[size_t(r) * ld + j];
+                return fmaf(sv, sl2, bc);
+            };
+            if (r < L) {
+                for (int j = gl; j < ld; j += G) m = fmaxf(m, term(j));
+                if (m != neg_inf())
+                    for (int j = gl; j < ld; j += G) {
+                        const float x = term(j);
+                        if (x != neg_inf()) s += exp2f(x - m);
+                    }
+            }
+            for (int off = G / 2; off > 0; off >>= 1) {
+                const float m2 = __shfl_xor_sync(0xffffffffu, m, off), s2 = __shfl_xor_sync(0xffffffffu, s, off);
+                lse2_merge(m, s, m2, s2);
+            }
+            if (r < L && gl == 0) {
+                const float lm = lmb[r];
+                float outv = 0.f, ob = neg_inf();
+                if (lm != neg_inf()) {
+                    outv = lm - (m + log2f(s)) * kLn2;
+                    if (!isfinite(outv)) atomicOr(g0.status, kStatusNonFinite);
+                    ob = outv * kLog2e;
+                }
+                outb[r] = ob;
+                out[r] = outv;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+bool simt_resident_possible(const Geom& g) {
+    if (g.D >= 0 || g.L <= 0 || g.d <= 0) return false;
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return false;
+    return simt_resident_smem(g.L, g.h, g.d) <= size_t(optin);
+}
+
+cudaError_t launch_simt_resident(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail, int T,
+                                 int R, cudaStream_t st) {
+    if (!simt_resident_possible(row.g)) return cudaErrorInvalidValue;
+    const size_t smem = simt_resident_smem(row.g.L, row.g.h, row.g.d);
+    auto launch = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        if (e != cudaSuccess) return e;
+        kernel<<<row.g.BH, kResThreads, smem, st>>>(row, Q, K, u_tail, v_tail, T, R);
+        return cudaGetLastError();
+    };
+    return row.g.dtype == EOT_BF16 ? launch(simt_resident_kernel<__nv_bfloat16>) : launch(simt_resident_kernel<float>);
 }
 
 cudaError_t launch_simt_lse_fused(const LsePass& row, const void* Q, const void* K, float* u_tail, float* v_tail,

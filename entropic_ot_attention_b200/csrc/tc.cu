@@ -161,6 +161,7 @@ struct TcBandArgs {
     float* dpart;
     uint32_t* dcnt;
     int dself;                  // (D, D) in the support
+    const float* sadd;          // wsum: out_r = f_r (hv_r sum + sadd_r) when not null
 };
 
 template <int DH, int KIND>
@@ -663,7 +664,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                             d_act ? ptx::ex2((sdterm_of(hs)[base + r] + colpot_of(hs)[pb + D]) * kLog2e + st2) : 0.f;
                         if (WSUM) {
                             if (d_act) sum = fmaf(dterm, a.colw[base + D], sum);
-                            outv = a.f[base + r] * a.hv[base + r] * sum;
+                            outv = a.f[base + r] * (a.hv[base + r] * sum + (a.sadd ? a.sadd[base + r] : 0.f));
                         } else {
                             outv = lm - log2f(sum + dterm) * kLn2 + st;
                         }
@@ -793,6 +794,10 @@ struct TcVecArgs {
     // (row r of row tile I at pcache[r * cpitch + (c - 128 I + h)], cpitch = 2 h + 128), or null.
     __nv_bfloat16* pcache;
     int cpitch;
+    // Column sweep beta_R: partial row-side sums of Pt dP (see BwdPass::s1part), or null.
+    float* s1part;
+    size_t s1stride;
+    int s1E;
 };
 
 constexpr int kSweepEpi = 16;         // epilogue warps: four per TMEM lane quadrant, 32 columns each
@@ -1194,6 +1199,26 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                                           pk[4 * t + 2], pk[4 * t + 3]);
                     }
                 }
+                if (MODE == kModeC1 && a.s1part) {
+                    // Pt dP summed over this warp's 32 rows for each of its 32 columns: a transposing
+                    // butterfly (each step keeps half of the columns and adds the partner lane's copy
+                    // of them), after which lane l holds column cc0 + l.  wc is free by now.
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) wc[j] *= vc[j];
+                    const int lb = lane;
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1) {
+                        const bool up = (lb & off) != 0;
+#pragma unroll
+                        for (int i = 0; i < off; ++i) {
+                            const float send = up ? wc[i] : wc[i + off];
+                            const float keep = up ? wc[i + off] : wc[i];
+                            wc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                        }
+                    }
+                    const int slot = (tiles[it] - int(blockIdx.x) + a.s1E) * 4 + q;
+                    a.s1part[size_t(slot) * a.s1stride + base + size_t(c0 + cc0 + lane)] = wc[0];
+                }
             }
             if (M::VEC) ptx::fence_proxy_async_smem();
             __syncwarp();
@@ -1482,6 +1507,7 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
         a.pstride = size_t(g.L);
         a.sd_term = p.sd_term;
         a.status = p.status;
+        a.sadd = p.sadd;
         cudaError_t e = launch_band(g, p.X, p.Y, a, kBandWsum, st);
         if (e != cudaSuccess || g.D < 0) return e;
         return launch_dustbin_bwd(p, st);
@@ -1523,6 +1549,9 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.status = p.status;
     a.pcache = mode == kModeR2 ? p.pcache : nullptr;
     a.cpitch = 2 * g.h + 128;
+    a.s1part = mode == kModeC1 ? p.s1part : nullptr;
+    a.s1stride = p.s1stride;
+    a.s1E = p.s1E;
     const int mt = max_tiles_for(g.L, g.h, 128, 128);
     dim3 grid(g.L / 128, g.BH);
     cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st)
