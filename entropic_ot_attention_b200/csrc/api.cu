@@ -568,11 +568,20 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
             }
         }
     }
-    // dQ = scale dS K (row sweep), dK = scale dS^T Q (column sweep); dS = P(R,R) (dP - sum x y^T)
+    // dQ = scale dS K (row sweep), dK = scale dS^T Q (column sweep); dS = P(R,R) (dP - sum x y^T).
+    // Tensor-core problems without a dustbin take the modifier term out of the dP product.
+    const bool fold = impl == EOT_IMPL_TCGEN05 && w.fold && 2 * R <= kMaxFoldMods;
     for (int orient = 0; orient < 2; ++orient) {
         EOT_RANGE(orient == 0 ? "eot backward: dQ" : "eot backward: dK");
+        va.xext = fold ? at<__nv_bfloat16>(ws, w.xext) : nullptr;
+        va.yext = fold ? at<__nv_bfloat16>(ws, w.yext) : nullptr;
         EOT_TRY(vec(orient == 0 ? kPassRF : kPassCF, 0));
+        va.xext = va.yext = nullptr;
         BwdPass bp = orient == 0 ? rowp : colp;
+        if (fold) {
+            bp.xext = at<__nv_bfloat16>(ws, w.xext);
+            bp.yext = at<__nv_bfloat16>(ws, w.yext);
+        }
         bp.vout = orient == 0 ? dQ : dK;
         bp.Z = orient == 0 ? K : Q;
         bp.vscale = g.scale;

@@ -95,6 +95,10 @@ struct BwdPass {
     size_t s1stride;
     int s1E;
     const float* sadd;      // staircase-form sweeps: out_r = f_r (hv_r sum_c ... + sadd_r), or nullptr
+    // dQ / dK (tensor-core kernels, no dustbin): the modifiers as [BH L, 16] bf16 operand rows
+    // (xext row side, yext column side; see BwdVecArgs) to fold into the dP product, or nullptr
+    const __nv_bfloat16* xext;
+    const __nv_bfloat16* yext;
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
     float* dpart;           // as in LsePass
     uint32_t* dcnt;
@@ -118,6 +122,8 @@ struct WsLayout {
     size_t pcache;          // backward with the cached reference plan: bf16 band store [BH, L, 2 h + 128]
     size_t s1part, sadd;    // backward, split alpha_R sweep: partial sums [4 (2 E + 1)][BH, L] and their total
     bool s1split;
+    size_t xext, yext;      // backward, folded modifiers: [BH L, 16] bf16 each
+    bool fold;
     size_t total;
 };
 
@@ -159,6 +165,15 @@ inline bool s1_split_possible(const eot_problem& p) {
            p.L % 128 == 0 && s1_reach(p.W) <= 7 && !cache_plan_possible(p);
 }
 inline size_t s1_slots(int W) { return size_t(4) * size_t(2 * s1_reach(W) + 1); }
+
+// The rank-2R modifier term of the dQ / dK sweeps is folded into their dP product (three bf16
+// products per modifier, hi x hi + hi x lo + lo x hi, in one K = 16 step) for tensor-core
+// problems without a dustbin and with 2 R <= kMaxFoldMods.
+constexpr int kMaxFoldMods = 5;
+inline bool fold_possible(const eot_problem& p) {
+    return p.dtype == EOT_BF16 && (p.d == 64 || p.d == 128) && !p.dustbin && p.impl != EOT_IMPL_SIMT && p.R >= 1 &&
+           2 * p.R <= kMaxFoldMods && p.L % 128 == 0;
+}
 
 inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     WsLayout w{};
@@ -207,6 +222,11 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
             w.s1split = true;
             w.s1part = o; o += s1_slots(p.W) * vec;
             w.sadd = o; o += vec;
+        }
+        if (fold_possible(p)) {
+            w.fold = true;
+            w.xext = o; o += align256(BH * L * 32);
+            w.yext = o; o += align256(BH * L * 32);
         }
     }
     w.total = o;

@@ -25,6 +25,12 @@ struct BwdVecArgs {
     int s1slots;
     size_t s1stride;
     float* sadd;
+    // kPassRF / kPassCF with at most kMaxFoldMods modifiers: also the operand rows of the folded
+    // modifier product, 16 bf16 per position; modifier k takes entries 3k .. 3k + 2 as
+    // xext = (-x_hi, -x_hi, -x_lo), yext = (y_hi, y_lo, y_hi) with x = x_hi + x_lo, y = y_hi + y_lo
+    // (bf16 parts), so <xext_r, yext_c> = -sum_k xr_k[r] yc_k[c] up to the lo x lo products.
+    __nv_bfloat16* xext;
+    __nv_bfloat16* yext;
 };
 
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,

@@ -301,6 +301,18 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return d;
 }
 
+// K-major operand of 16 bf16 (32 bytes) a row with the 32-byte swizzle (the layout a TMA copy
+// with CU_TENSOR_MAP_SWIZZLE_32B writes): 8-row groups 256 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t addr) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);
+    d |= uint64_t(1) << 16;            // leading byte offset 16 (unused within one swizzle atom)
+    d |= uint64_t(256 >> 4) << 32;     // stride byte offset 256
+    d |= uint64_t(1) << 46;            // descriptor version (sm_100)
+    d |= uint64_t(6) << 61;            // SWIZZLE_32B
+    return d;
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                      // D format: f32

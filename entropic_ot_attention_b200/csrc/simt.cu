@@ -618,6 +618,27 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
         a.xr[size_t(k) * a.BH * L + idx] = xr[k];
         a.yc[size_t(k) * a.BH * L + idx] = yc[k];
     }
+    if ((a.kind == kPassRF || a.kind == kPassCF) && a.xext && a.yext && nm <= kMaxFoldMods) {
+        alignas(16) __nv_bfloat16 xe[16];
+        alignas(16) __nv_bfloat16 ye[16];
+        const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xe[j] = ye[j] = z;
+        for (int k = 0; k < nm; ++k) {
+            const float x = -xr[k], y = yc[k];
+            const __nv_bfloat16 xh = __float2bfloat16_rn(x), yh = __float2bfloat16_rn(y);
+            const __nv_bfloat16 xl = __float2bfloat16_rn(x - __bfloat162float(xh));
+            const __nv_bfloat16 yl = __float2bfloat16_rn(y - __bfloat162float(yh));
+            xe[3 * k] = xh; xe[3 * k + 1] = xh; xe[3 * k + 2] = xl;
+            ye[3 * k] = yh; ye[3 * k + 1] = yl; ye[3 * k + 2] = yh;
+        }
+        uint4* xo = reinterpret_cast<uint4*>(a.xext + idx * 16);
+        uint4* yo = reinterpret_cast<uint4*>(a.yext + idx * 16);
+        xo[0] = *reinterpret_cast<const uint4*>(xe);
+        xo[1] = *reinterpret_cast<const uint4*>(xe + 8);
+        yo[0] = *reinterpret_cast<const uint4*>(ye);
+        yo[1] = *reinterpret_cast<const uint4*>(ye + 8);
+    }
 }
 
 // ---------------------------------------------------------------------------------------

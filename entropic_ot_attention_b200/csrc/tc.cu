@@ -58,6 +58,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_ro
     return r == CUDA_SUCCESS;
 }
 
+// 2-D TMA descriptor over a [rows, 16] bf16 matrix (the folded modifier operands), boxes of
+// 16 x box_rows, 32-byte swizzle.
+bool make_map_ext(CUtensorMap* m, const void* base, uint64_t rows, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn || !base || (reinterpret_cast<uintptr_t>(base) & 15)) return false;
+    cuuint64_t dims[2] = {16u, cuuint64_t(rows)};
+    cuuint64_t strides[1] = {32u};
+    cuuint32_t box[2] = {16u, cuuint32_t(box_rows)};
+    cuuint32_t es[2] = {1u, 1u};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------------------
 // Device: band tile list shared by all roles of a CTA
 // ---------------------------------------------------------------------------------------
@@ -804,7 +819,7 @@ constexpr int kSweepEpi = 16;         // epilogue warps: four per TMEM lane quad
 constexpr int kSweepThreads = 32 * (4 + kSweepEpi);   // TMA warp, S-MMA warp, epilogue warps, product-MMA warp, dP-MMA warp
 constexpr int kSweepDpWarp = 3 + kSweepEpi;
 
-template <int DH, int NV>
+template <int DH, int NV, bool FOLD = false>
 struct SweepCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
@@ -826,7 +841,12 @@ struct SweepCfg {
     static constexpr uint32_t OFF_L = 2 * CB;
     static constexpr uint32_t OFF_E = OFF_L + NL * YB;
     static constexpr uint32_t OFF_V = OFF_E + NE * YB;
-    static constexpr uint32_t OFF_RED = OFF_V + NL * VB;  // [2 sums][4 quarters][128 rows] scalar partials
+    // Folded modifiers (dQ / dK): the row tile's and the early column tile's [128 x 16] bf16
+    // modifier operands, 32-byte swizzled
+    static constexpr uint32_t EXTB = 128 * 16 * 2;
+    static constexpr uint32_t OFF_XE = (OFF_V + NL * VB + 1023) / 1024 * 1024;
+    static constexpr uint32_t OFF_YE = OFF_XE + EXTB;
+    static constexpr uint32_t OFF_RED = FOLD ? OFF_YE + EXTB : OFF_V + NL * VB;  // [2 sums][4 quarters][128 rows] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 128 * 4;
     // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm
     static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1;
@@ -841,14 +861,20 @@ struct SweepCfg {
     static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_ACC = 256, TM_X = 384, TM_A = 448;
 };
 
-template <int DH, int MODE, int NMOD>
+// FOLD (dQ / dK without a dustbin): the rank-2R modifier term sum_k xr_k yc_k^T comes out of the
+// dP product itself, one more K = 16 step over [128 x 16] bf16 operand tiles XE (rows) and YE
+// (columns) that carry each modifier split into hi + lo bf16 parts (see bwd_vectors_kernel), so
+// the epilogue's coefficient is Pt * dP' with no per-entry modifier arithmetic.
+template <int DH, int MODE, int NMOD, bool FOLD>
 __global__ void __launch_bounds__(kSweepThreads, 1)
     tc_sweep_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
+                    const __grid_constant__ CUtensorMap tmXE, const __grid_constant__ CUtensorMap tmYE,
                     const TcVecArgs a, int max_tiles) {
     using M = ModeT<MODE>;
+    static_assert(!FOLD || (MODE == kModeGrad && NMOD == 0), "folded modifiers are a dQ / dK form");
     constexpr int NV = 1 + (M::SM ? 1 : 0) + NMOD;   // column vectors per column tile: pcm2, m, yc...
-    using C = SweepCfg<DH, NV>;
+    using C = SweepCfg<DH, NV, FOLD>;
     constexpr int VOFF_M = 1, VOFF_Y = 1 + (M::SM ? 1 : 0);
     // W rides the late ring when the product reads it or when there is no product (R2); Y when
     // the product reads Y (dQ / dK).
@@ -904,10 +930,14 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         ptx::prefetch_tmap(&tmX);
         if (M::HASDP) ptx::prefetch_tmap(&tmA);
         const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
-        ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1));
+        ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1) + (FOLD ? C::EXTB : 0u));
         for (int ka = 0; ka < C::KATOMS; ++ka) {
             ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
             if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
+        }
+        if (FOLD) {
+            ptx::prefetch_tmap(&tmXE);
+            ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_XE), &tmXE, 0, int(base) + r0, xfull);
         }
     }
     bool any_row;
@@ -943,6 +973,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             static_assert(M::W2, "every sweep pass reads two column-side tensors");
             ptx::prefetch_tmap(&tmY);
             ptx::prefetch_tmap(&tmW);
+            if (FOLD) ptx::prefetch_tmap(&tmYE);
             const CUtensorMap* tm_late = LATE_W ? &tmW : &tmY;
             const CUtensorMap* tm_early = LATE_W ? &tmY : &tmW;
             const float* vsrc[NV];
@@ -970,10 +1001,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 issued_l = it + 1;
                 // early ring: the other column tile
                 if (!ptx::mbar_wait(empty_e, (it & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(full_e, C::YB);
+                ptx::mbar_expect_tx(full_e, C::YB + (FOLD ? C::EXTB : 0u));
                 const uint32_t es = ptx::smem_u32(sm + C::OFF_E);
                 for (int ka = 0; ka < C::KATOMS; ++ka)
                     ptx::tma_load_2d(es + ka * C::YATOM, tm_early, ka * 64, int(base) + c0, full_e);
+                // (the dP operand rides the early ring in dQ / dK: its modifier tile goes with it)
+                if (FOLD) ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE), &tmYE, 0, int(base) + c0, full_e);
                 issued_e = it + 1;
             }
             if (*abort_flag) {
@@ -991,6 +1024,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         const bool is_dp = warp == kSweepDpWarp;
         if (lane == 0 && (!is_dp || M::HASDP)) {
             bool ok = ptx::mbar_wait(xtm, 0, abort_flag, a.status);
+            // (the row modifier tile XE is read from shared memory by the dP product)
+            if (FOLD && is_dp) ok = ok && ptx::mbar_wait(xfull, 0, abort_flag, a.status);
             ptx::tc_fence_after();
             int issued = 0;
             const uint32_t dtm = tbase + (is_dp ? C::TM_DP : C::TM_S);
@@ -1012,6 +1047,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     const uint64_t bo = uint64_t(((kk >> 2) * C::YATOM + (kk & 3) * 32) >> 4);
                     ptx::mma_bf16_ts(dtm, atm + uint32_t(kk * 8), bd + bo, C::IDESC_S, kk > 0 ? 1u : 0u);
                 }
+                // dP' = dP + XE YE^T = dP - sum_k xr_k yc_k^T
+                if (FOLD && is_dp)
+                    ptx::mma_bf16(dtm, ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_XE)),
+                                  ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_YE)), C::IDESC_S, 1u);
                 ptx::mma_commit(tfull);
                 // the early tile is free once this product completes; a late slot normally comes
                 // back after the product MMA, or here in a pass without one
@@ -1452,31 +1491,38 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
 
-template <int DH, int MODE, int NMOD>
+struct ExtMaps {
+    CUtensorMap xe, ye;
+};
+
+template <int DH, int MODE, int NMOD, bool FOLD = false>
 cudaError_t launch_sweep(const CUtensorMap& tmX, const CUtensorMap& tmA, const CUtensorMap& tmY, const CUtensorMap& tmW,
-                         const TcVecArgs& a, int mt, dim3 grid, cudaStream_t st) {
+                         const ExtMaps& ext, const TcVecArgs& a, int mt, dim3 grid, cudaStream_t st) {
     constexpr int NV = 1 + (ModeT<MODE>::SM ? 1 : 0) + NMOD;
-    const size_t smem = SweepCfg<DH, NV>::smem_bytes(mt);
-    cudaError_t e = set_smem(tc_sweep_kernel<DH, MODE, NMOD>, smem);
+    const size_t smem = SweepCfg<DH, NV, FOLD>::smem_bytes(mt);
+    cudaError_t e = set_smem(tc_sweep_kernel<DH, MODE, NMOD, FOLD>, smem);
     if (e != cudaSuccess) return e;
-    tc_sweep_kernel<DH, MODE, NMOD><<<grid, kSweepThreads, smem, st>>>(tmX, tmA, tmY, tmW, a, mt);
+    tc_sweep_kernel<DH, MODE, NMOD, FOLD><<<grid, kSweepThreads, smem, st>>>(tmX, tmA, tmY, tmW, ext.xe, ext.ye, a, mt);
     return cudaGetLastError();
 }
 
 template <int DH>
-cudaError_t launch_sweep_dh(int mode, int nmod, const CUtensorMap& tmX, const CUtensorMap& tmA, const CUtensorMap& tmY,
-                            const CUtensorMap& tmW, const TcVecArgs& a, int mt, dim3 grid, cudaStream_t st) {
+cudaError_t launch_sweep_dh(int mode, int nmod, bool fold, const CUtensorMap& tmX, const CUtensorMap& tmA,
+                            const CUtensorMap& tmY, const CUtensorMap& tmW, const ExtMaps& ext, const TcVecArgs& a,
+                            int mt, dim3 grid, cudaStream_t st) {
+    if (fold) return mode == kModeGrad ? launch_sweep<DH, kModeGrad, 0, true>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st)
+                                       : cudaErrorInvalidValue;
     switch (mode) {
-        case kModeOut: return launch_sweep<DH, kModeOut, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-        case kModeC1: return launch_sweep<DH, kModeC1, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-        case kModeR2: return launch_sweep<DH, kModeR2, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+        case kModeOut: return launch_sweep<DH, kModeOut, 0>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+        case kModeC1: return launch_sweep<DH, kModeC1, 0>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+        case kModeR2: return launch_sweep<DH, kModeR2, 0>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
         case kModeGrad:
             switch (nmod) {
-                case 0: return launch_sweep<DH, kModeGrad, 0>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-                case 2: return launch_sweep<DH, kModeGrad, 2>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-                case 4: return launch_sweep<DH, kModeGrad, 4>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-                case 8: return launch_sweep<DH, kModeGrad, 8>(tmX, tmA, tmY, tmW, a, mt, grid, st);
-                case 16: return launch_sweep<DH, kModeGrad, 16>(tmX, tmA, tmY, tmW, a, mt, grid, st);
+                case 0: return launch_sweep<DH, kModeGrad, 0>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+                case 2: return launch_sweep<DH, kModeGrad, 2>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+                case 4: return launch_sweep<DH, kModeGrad, 4>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+                case 8: return launch_sweep<DH, kModeGrad, 8>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
+                case 16: return launch_sweep<DH, kModeGrad, 16>(tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
             }
     }
     return cudaErrorInvalidValue;
@@ -1512,8 +1558,12 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
         if (e != cudaSuccess || g.D < 0) return e;
         return launch_dustbin_bwd(p, st);
     }
+    // dQ / dK without a dustbin, with the modifiers prepared as hi / lo bf16 operand rows: fold
+    // them into the dP product.
+    const bool fold = mode == kModeGrad && p.xext && p.yext && g.D < 0 && p.nmod <= kMaxFoldMods;
+    ExtMaps ext;
     // Modifier count rounded up to an instantiated one; the padding terms have xr = 0.
-    int nmod = p.nmod;
+    int nmod = fold ? 0 : p.nmod;
     const int nmod_k = nmod == 0 ? 0 : nmod <= 2 ? 2 : nmod <= 4 ? 4 : nmod <= 8 ? 8 : 16;
     if (nmod_k > nmod && !p.zero_vec) return cudaErrorInvalidValue;
     const bool has_dp = mode == kModeC1 || mode == kModeR2 || mode == kModeGrad;
@@ -1523,6 +1573,13 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     if (!make_map(&tmX, p.X, rows, g.d, 128) || !make_map(&tmY, p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
     if (!make_map(&tmA, has_dp ? p.A : p.X, rows, g.d, 128)) return cudaErrorInvalidValue;
     if (!make_map(&tmW, w2 ? w2 : p.Y, rows, g.d, 128)) return cudaErrorInvalidValue;
+    if (fold) {
+        if (!make_map_ext(&ext.xe, p.xext, rows, 128) || !make_map_ext(&ext.ye, p.yext, rows, 128))
+            return cudaErrorInvalidValue;
+    } else {
+        ext.xe = tmX;   // not read
+        ext.ye = tmX;
+    }
     TcVecArgs a{};
     a.H = g.H;
     a.L = g.L;
@@ -1554,8 +1611,8 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.s1E = p.s1E;
     const int mt = max_tiles_for(g.L, g.h, 128, 128);
     dim3 grid(g.L / 128, g.BH);
-    cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st)
-                               : launch_sweep_dh<64>(mode, nmod_k, tmX, tmA, tmY, tmW, a, mt, grid, st);
+    cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, fold, tmX, tmA, tmY, tmW, ext, a, mt, grid, st)
+                               : launch_sweep_dh<64>(mode, nmod_k, fold, tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
     if (e != cudaSuccess || g.D < 0) return e;
     return launch_dustbin_bwd(p, st);
 }

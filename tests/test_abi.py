@@ -87,8 +87,10 @@ def test_workspace_query(abi):
     assert fw > 0 and bw > fw
     assert abi.eot_workspace_bytes(_prob(abi, L=200), False) == 0
     assert abi.eot_workspace_bytes(_prob(abi, B=0), True) == 0
-    p4 = _prob(abi, R=4)
-    assert abi.eot_workspace_bytes(p4, True) > bw
+    # more tail steps keep more staircase and modifier vectors (R = 3 and 4 both leave the
+    # modifiers unfolded: 2 R > 5)
+    p3, p4 = _prob(abi, R=3), _prob(abi, R=4)
+    assert abi.eot_workspace_bytes(p4, True) > abi.eot_workspace_bytes(p3, True)
 
 
 def test_host_errors_launch_nothing(abi):
