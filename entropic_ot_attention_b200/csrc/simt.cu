@@ -28,32 +28,50 @@ constexpr int kSNT = 256;  // threads per CTA
 
 // Uniform marginals over the active real tokens (§2.1), dustbin mass (§2.3).  One CTA per
 // batch row.  logm[b, i] = log a_i, -inf for inactive positions.
-__global__ void __launch_bounds__(256) prep_marginals_kernel(Geom g, const uint8_t* mask, int dustbin,
-                                                             float mass, float* logm, uint32_t* status) {
+// One CTA of 1024 threads per batch row (L is a multiple of 128): count the real tokens (mask
+// bytes read 16 at a time when the mask is 16-byte aligned), then write the row's log marginals
+// 4 at a time.
+__global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint8_t* mask, int dustbin,
+                                                              float mass, float* logm, uint32_t* status) {
     const int b = blockIdx.x;
     const int L = g.L;
     const int D = dustbin ? g.D : L;
-    __shared__ int red[256];
+    const uint8_t* mrow = mask ? mask + size_t(b) * L : nullptr;
+    const bool vec = mrow && (reinterpret_cast<uintptr_t>(mask) & 15) == 0;
+    __shared__ int red[32];
     int cnt = 0;
-    for (int i = threadIdx.x; i < L; i += blockDim.x) {
-        int real = (mask ? (mask[size_t(b) * L + i] != 0) : 1) && (i < D);
-        cnt += real;
+    if (!mrow) {
+        cnt = threadIdx.x == 0 ? min(L, D) : 0;
+    } else if (vec) {
+        for (int i0 = threadIdx.x * 16; i0 < L; i0 += blockDim.x * 16) {
+            const uint4 w = *reinterpret_cast<const uint4*>(mrow + i0);
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 16; ++j) cnt += (((ww[j >> 2] >> (8 * (j & 3))) & 0xffu) != 0u) && (i0 + j < D);
+        }
+    } else {
+        for (int i = threadIdx.x; i < L; i += blockDim.x) cnt += (mrow[i] != 0) && (i < D);
     }
-    red[threadIdx.x] = cnt;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cnt;
     __syncthreads();
-    for (int s = 128; s > 0; s >>= 1) {
-        if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
-        __syncthreads();
-    }
-    const int n = red[0];
+    int n = 0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) n += red[w];
     const bool use_db = dustbin && n > 0 && mass > 0.f;
     const double real_mass = use_db ? (1.0 - double(mass)) : 1.0;
     const float lr = n > 0 ? float(log(real_mass / double(n))) : neg_inf();
-    for (int i = threadIdx.x; i < L; i += blockDim.x) {
-        int real = (mask ? (mask[size_t(b) * L + i] != 0) : 1) && (i < D);
-        float v = real ? lr : neg_inf();
-        if (dustbin && i == D) v = use_db ? float(log(double(mass))) : neg_inf();
-        logm[size_t(b) * L + i] = v;
+    const float ld = use_db ? float(log(double(mass))) : neg_inf();
+    for (int i0 = threadIdx.x * 4; i0 < L; i0 += blockDim.x * 4) {
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            const bool real = (mrow ? (mrow[i] != 0) : true) && (i < D);
+            v[j] = real ? lr : neg_inf();
+            if (dustbin && i == D) v[j] = ld;
+        }
+        *reinterpret_cast<float4*>(logm + size_t(b) * L + i0) = make_float4(v[0], v[1], v[2], v[3]);
     }
     if (b == 0 && threadIdx.x == 0 && status) *status = 0u;
 }
@@ -646,7 +664,7 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
 // ---------------------------------------------------------------------------------------
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
                                   uint32_t* status, cudaStream_t st) {
-    prep_marginals_kernel<<<g.B, 256, 0, st>>>(g, mask, dustbin, mass, logm, status);
+    prep_marginals_kernel<<<g.B, 1024, 0, st>>>(g, mask, dustbin, mass, logm, status);
     return cudaGetLastError();
 }
 

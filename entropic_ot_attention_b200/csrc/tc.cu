@@ -117,12 +117,17 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // two MMAs.  Roles:
 //   warp 0       TMA producer (one lane): row halves into a small ring, column tiles into
 //                NS stages, and per half the tile's column vectors (log2 bias, weights)
-//   warp 1       TMEM allocator and MMA issuer of the first half (one lane); warp 18 issues
+//   warp 1       TMEM allocator and MMA issuer of the first half (one lane); warp 2 issues
 //                the second half's MMAs: two 128-column fp32 score accumulators per half
 //                (4 x 128 TMEM columns).  One issue thread per half, because one thread's
 //                per-MMA bookkeeping for both halves was slower than the tensor core.
-//   warps 2..9   epilogue of the first half, warps 10..17 of the second: warp (q, hf) reads
+//   warp 3       idle (it completes the first warpgroup)
+//   warps 4..11  epilogue of the first half, warps 12..19 of the second: warp (q, hf) reads
 //                TMEM lanes [32 q, 32 q + 32) and columns [64 hf, 64 hf + 64) of each tile
+// Registers: the block is launched at 96 a thread; warpgroup 0 (warps 0-3) gives registers
+// back (setmaxnreg 48) and the four epilogue warpgroups take them (104), so the epilogue's
+// chain of score, exponential and sums keeps more values live (long workload, forward: 5.61 ->
+// 5.33 ms against 96 registers everywhere; control warps at 40 or 56 registers: 5.43 / 5.36).
 // The two warps that share a row meet once per item on a 64-thread named barrier; the
 // halves are coupled only through the column-tile stages.  All roles walk the same item /
 // tile sequence, so ring slots and mbarrier phases follow from running counters.
@@ -206,8 +211,10 @@ struct BandCfg {
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
-constexpr int kBandThreads = 608;   // TMA warp, MMA warp (half 0), 16 epilogue warps, MMA warp (half 1)
-constexpr int kBandIssuerB = 18;
+constexpr int kBandThreads = 640;   // TMA warp, MMA warps (halves 0, 1), an idle warp, 16 epilogue warps
+constexpr int kBandIssuerB = 2;
+constexpr int kBandEpi0 = 4;
+constexpr int kBandLaunchRegs = 96;
 
 // Decoded work item: rows [r0, r0 + 256) of unit bh as two halves with their column-tile bands.
 struct BandItem {
@@ -333,6 +340,8 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     ptx::tc_fence_after();
     const uint32_t tbase = misc[0];
 
+    if (warp < kBandEpi0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
@@ -479,9 +488,11 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 ptx::mbar_wait(tfull(GI, (gt - 1) & 1), ((gt - 1) >> 1) & 1, &dummy, a.status);
             }
         }
+    }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 104;");
         // ---------------- epilogue: 8 warps per half ----------------
-        const int e = warp - 2;
+        const int e = warp - kBandEpi0;
         const int G = e >> 3;                 // row half
         const int hf = (e >> 2) & 1;          // column half of each tile
         const int q = warp & 3;               // TMEM lane quadrant (fixed by the warp's rank)
@@ -497,7 +508,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         float* outb_hs = outb_of(hs);
         if (MULTI && hs > a.hs0) {
             // every CTA has written half-step hs - 1 (the shifts and biases read below)
-            if (tid == 64 && ok && !ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) ok = false;
+            if (tid == 32 * kBandEpi0 && ok && !ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) ok = false;
             ptx::named_bar_sync(9, 512);
             ok = ok && !*abort_flag;
         }
@@ -747,7 +758,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         if (MULTI) {
             // this CTA is done with half-step hs: count it on the grid-wide barrier
             ptx::named_bar_sync(9, 512);
-            if (tid == 64) {
+            if (tid == 32 * kBandEpi0) {
                 __threadfence();
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 atomicAdd(a.gbar + hs, 1u);
@@ -1395,6 +1406,10 @@ cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, 
     auto kernel = tc_band_kernel<DH, KIND, MULTI>;
     cudaError_t e = set_smem(kernel, smem);
     if (e != cudaSuccess) return e;
+    // the register split inside the kernel assumes this launch allocation
+    cudaFuncAttributes fa{};
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+    if (fa.numRegs != kBandLaunchRegs) return cudaErrorNotSupported;
     if (!MULTI) {
         kernel<<<grid, kBandThreads, smem, st>>>(tmX, tmY, a);
         return cudaGetLastError();
