@@ -279,16 +279,21 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         EOT_TRY(tracked(kProfLse, 0, st, [&] { return launch_tc_iter(il, st, &launched); }));
         g_launches += launched;
     } else if (impl == EOT_IMPL_TCGEN05 && n_half >= 2) {
+        // (the fused d = 128 half-steps of a band of W >= 512 take the column bias from these rows)
+        const bool bext = w.bext && g.h >= 256;
+        __nv_bfloat16* ue = bext ? at<__nv_bfloat16>(ws, w.ue) : nullptr;
+        __nv_bfloat16* ve = bext ? at<__nv_bfloat16>(ws, w.ve) : nullptr;
         EOT_TRY(run_lse(impl, [&] {
             LsePass r0 = row;
             r0.colpot = v_tail;
             r0.stab = nullptr;
             r0.out = u_tail + (p->T > 0 ? 0 : L);
+            r0.ext_out = ue;
             return r0;
         }(), st));
         uint32_t* gbar = at<uint32_t>(ws, w.gbar);
         EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
-        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar};
+        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar, ue, ve};
         const cudaError_t e = tracked(kProfLse, 1, st, [&] { return launch_tc_lse_fused(row, f, st); });
         if (e == cudaSuccess) fused = true;
         else if (e == cudaErrorCooperativeLaunchTooLarge) {

@@ -53,6 +53,9 @@ struct LsePass {
     float* dpart;           // dense dustbin row: per-CTA partial sums (dustbin only)
     uint32_t* dcnt;         // [BH] CTAs of the dense dustbin row done (zero between launches)
     uint32_t* status;
+    // tensor-core kernels: also write each output position's column-bias operand row here
+    // ([BH L, 16] bf16; read by the fused half-steps that follow), or nullptr
+    __nv_bfloat16* ext_out;
 };
 
 // One backward sweep (§2.2).  With Pt_rc = exp(S_rc + pr_r + pc_c) on the support:
@@ -124,6 +127,8 @@ struct WsLayout {
     bool s1split;
     size_t xext, yext;      // backward, folded modifiers: [BH L, 16] bf16 each
     bool fold;
+    size_t ue, ve;          // forward, fused d = 128 half-steps: column-bias operand rows [BH L, 16] bf16 of u and v
+    bool bext;
     size_t total;
 };
 
@@ -196,6 +201,11 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
         w.gbar = o; o += align256(size_t(2) * (size_t(p.T) + size_t(p.R)) * sizeof(uint32_t) + 4);
+        if (p.dtype == EOT_BF16 && p.d == 128 && p.impl != EOT_IMPL_SIMT && p.L % 128 == 0 && p.W / 2 >= 256) {
+            w.bext = true;
+            w.ue = o; o += align256(BH * L * 32);
+            w.ve = o; o += align256(BH * L * 32);
+        }
         if (iter_schedule_possible(p)) {
             w.part = o;
             o += align256(BH * size_t(p.L / 128) * size_t(iter_window_tiles(p.L, p.W / 2)) * 128 * sizeof(float));

@@ -84,6 +84,9 @@ struct FusedSteps {
     int hs0, nhs, T;
     float *u_tail, *v_tail, *ub2, *vb2;
     uint32_t* gbar;
+    // d = 128: the column-bias operand rows of u and v ([BH L, 16] bf16; the first half-step
+    // before this launch writes those of u)
+    __nv_bfloat16 *ue, *ve;
 };
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);

@@ -182,9 +182,42 @@ struct TcBandArgs {
     uint32_t* dcnt;
     int dself;                  // (D, D) in the support
     const float* sadd;          // wsum: out_r = f_r (hv_r sum + sadd_r) when not null
+    // Column-bias operand rows (see band_ext_row): written for every output position when not
+    // null (a single half-step), and, in fused d = 128 half-steps, written and read through ue
+    // (u side) and ve (v side), [BH L, 16] bf16 each.
+    __nv_bfloat16* ext_out;
+    __nv_bfloat16* ue;
+    __nv_bfloat16* ve;
 };
 
-template <int DH, int KIND>
+// The column bias enters the fused half-steps' score product (d = 128): one more K = 16 step
+// multiplies a constant row operand (1, 1, 1, 0, ...) with a column operand row
+// (y_hi, y_mid, y_lo, 0, ...) carrying y = b_c / (scale log2 e), b_c the column's masked log2
+// potential, as three bf16 parts (fp32 accuracy); the accumulator then holds S + y and the
+// epilogue forms the exponent with one packed FMA, acc * scale log2 e + st_r.  A column
+// that never enters a band sum (inactive, the dustbin) carries y = -2^100.
+__device__ __forceinline__ void band_ext_row(__nv_bfloat16* dst, float b2, float sl2) {
+    const float y = b2 == kNegInf ? -1.2676506e30f : b2 / sl2;   // -2^100
+    const __nv_bfloat16 hi = __float2bfloat16_rn(y);
+    const float r1 = y - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __nv_bfloat162 p0, p1;
+    p0.x = hi;
+    p0.y = mid;
+    p1.x = lo;
+    p1.y = __float2bfloat16_rn(0.f);
+    uint4 w0;
+    w0.x = *reinterpret_cast<const uint32_t*>(&p0);
+    w0.y = *reinterpret_cast<const uint32_t*>(&p1);
+    w0.z = 0u;
+    w0.w = 0u;
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = w0;
+    d[1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+template <int DH, int KIND, bool EXT = false>
 struct BandCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
@@ -201,7 +234,12 @@ struct BandCfg {
     static constexpr uint32_t OFF_RED = OFF_V + 2 * NV * VB;    // [half][parity][m, s][128 rows]
     static constexpr uint32_t OFF_BITS = OFF_RED + 2 * 2 * 2 * 128 * 4;   // tile bits of the CTA's batch rows
     static constexpr int BITS_WORDS = 512;
-    static constexpr uint32_t OFF_BAR = OFF_BITS + BITS_WORDS * 4;
+    // column-bias operands (EXT): the constant row operand and one column operand per stage,
+    // [128 x 16] bf16 each, 32-byte swizzled
+    static constexpr uint32_t EXTB = 128 * 16 * 2;
+    static constexpr uint32_t OFF_ONES = (OFF_BITS + BITS_WORDS * 4 + 1023) / 1024 * 1024;
+    static constexpr uint32_t OFF_YE = OFF_ONES + EXTB;
+    static constexpr uint32_t OFF_BAR = EXT ? OFF_YE + NS * EXTB : OFF_BITS + BITS_WORDS * 4;
     // full[NS] empty[NS] qfull[NQ] qempty[NQ], then per half: tfull[2] tempty[2] vfull[NV] vempty[NV]
     static constexpr uint32_t HB0 = 2 * NS + 2 * NQ;
     static constexpr uint32_t HBN = 4 + 2 * NV;
@@ -241,11 +279,18 @@ struct TileBits {
     }
 };
 
-template <int DH, int KIND, bool MULTI>
+// EXT (fused d = 128 half-steps of a wide band): the column bias comes out of the score product
+// (band_ext_row).  Its operand rows are written in the previous half-step, so the first product
+// of a half-step waits for the grid-wide barrier; with a short band (few tiles a row) that wait
+// costs more than the fold saves (protein-like workload, W = 128: 3.12 -> 3.28 ms per call), so
+// the launch selects it for W >= 512 only (long workload: 7.85 -> 7.70 ms).
+template <int DH, int KIND, bool MULTI, bool EXT>
 __global__ void __launch_bounds__(kBandThreads, 1)
     tc_band_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                   const __grid_constant__ CUtensorMap tmUE, const __grid_constant__ CUtensorMap tmVE,
                    const TcBandArgs a) {
-    using C = BandCfg<DH, KIND>;
+    static_assert(!EXT || (MULTI && DH == 128 && KIND == kBandShift), "the folded column bias is a fused d = 128 form");
+    using C = BandCfg<DH, KIND, EXT>;
     constexpr bool ONLINE = KIND == kBandOnline, WSUM = KIND == kBandWsum;
     static_assert(!MULTI || KIND == kBandShift, "fused half-steps are shifted log-sum-exp sweeps");
     // Operands of half-step hs (a single launch uses the fixed pointers of a).
@@ -262,6 +307,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         return MULTI ? ((hs & 1) ? a.v_tail : a.u_tail) + size_t(slot_of(hs, true)) * a.L : a.out;
     };
     auto outb_of = [&](int hs) -> float* { return MULTI ? ((hs & 1) ? a.vb2 : a.ub2) : a.out_bias2; };
+    // column-bias operand rows written by half-step hs (and, EXT, read by it: the other side's)
+    auto exto_of = [&](int hs) -> __nv_bfloat16* {
+        return MULTI ? (EXT ? ((hs & 1) ? a.ve : a.ue) : nullptr) : a.ext_out;
+    };
     // natural column potential (read at the dustbin) and the rows' dustbin links
     auto colpot_of = [&](int hs) -> const float* {
         return MULTI ? ((hs & 1) ? a.u_tail + size_t(slot_of(hs, true)) * a.L : a.v_tail + size_t(slot_of(hs, false)) * a.L)
@@ -321,6 +370,17 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     // Column tiles that half G multiplies: inside its band and holding an active column.
     auto uses = [&](const BandItem& it, int G, int t) { return it.active[G] && t >= it.t_lo[G] && t <= it.t_hi[G]; };
 
+    if (EXT) {
+        // constant row operand: logical 16-byte chunk 0 of every row is (1, 1, 1, 0, 0, 0, 0, 0),
+        // chunk 1 zeros; the 32-byte swizzle stores chunk c of row r at c ^ ((r >> 2) & 1)
+        uint32_t* ones = reinterpret_cast<uint32_t*>(sm + C::OFF_ONES);
+        for (int i = tid; i < 128 * 8; i += blockDim.x) {
+            const int r = i >> 3, pc = (i >> 2) & 1, w = i & 3;
+            const int lc = pc ^ ((r >> 2) & 1);
+            ones[i] = lc == 0 ? (w == 0 ? 0x3f803f80u : w == 1 ? 0x00003f80u : 0u) : 0u;
+        }
+        ptx::fence_proxy_async_smem();
+    }
     if (tid == 0) {
         *abort_flag = 0;
         for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 2); }
@@ -347,6 +407,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             // ---------------- TMA producer ----------------
             ptx::prefetch_tmap(&tmX);
             ptx::prefetch_tmap(&tmY);
+            if (EXT) {
+                ptx::prefetch_tmap(&tmUE);
+                ptx::prefetch_tmap(&tmVE);
+            }
             int g = 0, qi = 0;
             int gv[2] = {0, 0};
             bool ok = true;
@@ -381,16 +445,28 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     const int c0 = t * C::BN;
                     const int s = g % C::NS;
                     if (!ptx::mbar_wait(empty(s), ((g / C::NS) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-                    ptx::mbar_expect_tx(full(s), C::YB);
+                    ptx::mbar_expect_tx(full(s), C::YB + (EXT ? C::EXTB : 0u));
                     const uint32_t ys = ptx::smem_u32(sm + C::OFF_Y + s * C::YB);
                     for (int ka = 0; ka < C::KATOMS; ++ka)
                         ptx::tma_load_2d(ys + ka * C::ATOM, mY, ka * 64, int(it.base) + c0, full(s));
                     ++g;
                     if (!biases_ready) {
-                        if (!ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) { ok = false; break; }
+                        if (!ptx::grid_wait(a.gbar + hs - 1, gridDim.x, abort_flag, a.status)) {
+                            // the stage still expects its column-bias operand: fill it so that
+                            // no copy is left pending when the CTA retires
+                            if (EXT)
+                                ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (hs & 1) ? &tmUE : &tmVE, 0,
+                                                 int(it.base) + c0, full(s));
+                            ok = false;
+                            break;
+                        }
                         asm volatile("fence.proxy.async.global;" ::: "memory");
                         biases_ready = true;
                     }
+                    // the column-bias operand rows of half-step hs were written in half-step hs - 1
+                    if (EXT)
+                        ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (hs & 1) ? &tmUE : &tmVE, 0,
+                                         int(it.base) + c0, full(s));
 #pragma unroll
                     for (int G = 0; G < 2; ++G) {
                         if (!(G ? use1 : use0)) continue;
@@ -470,6 +546,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                             const uint64_t koff = uint64_t(((kk >> 2) * C::ATOM + (kk & 3) * 32) >> 4);
                             ptx::mma_bf16(dt, xd + koff, yd + koff, C::IDESC, kk > 0 ? 1u : 0u);
                         }
+                        // + the column bias b_c / (scale log2 e) (band_ext_row)
+                        if (EXT)
+                            ptx::mma_bf16(dt, ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_ONES)),
+                                          ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB)), C::IDESC, 1u);
                         ptx::mma_commit(tfull(GI, tb));
                         ++gt;
                         if (++done == n) ptx::mma_commit(qempty(qslot));   // row half free once its products are done
@@ -528,6 +608,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     out_hs[pb + r] = 0.f;
                     if (!WSUM) outb_hs[base + r] = kNegInf;
                 }
+                if (!WSUM && hf == 0 && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.sl2);
                 continue;
             }
             const int t_lo = max(0, rg - h) / C::BN, t_hi = min(L - 1, rg + C::BM - 1 + h) / C::BN;
@@ -544,13 +625,19 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             auto process = [&](const float (&v)[32], int cc, uint32_t vaddr, bool masked) {
                 if (ONLINE || masked) {
                     float x[32];
+                    if (EXT) {
+                        // the accumulator holds S + b_c / (scale log2 e): x = exponent incl. the shift
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = ptx::ld_shared_f4(vaddr + 16u * j4);
-                        x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
-                        x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
-                        x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
-                        x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
+                        for (int j = 0; j < 32; ++j) x[j] = fmaf(v[j], a.sl2, st2);
+                    } else {
+#pragma unroll
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 bv = ptx::ld_shared_f4(vaddr + 16u * j4);
+                            x[4 * j4 + 0] = fmaf(v[4 * j4 + 0], a.sl2, bv.x);
+                            x[4 * j4 + 1] = fmaf(v[4 * j4 + 1], a.sl2, bv.y);
+                            x[4 * j4 + 2] = fmaf(v[4 * j4 + 2], a.sl2, bv.z);
+                            x[4 * j4 + 3] = fmaf(v[4 * j4 + 3], a.sl2, bv.w);
+                        }
                     }
                     if (masked) {
                         // valid columns j of this chunk: r - h <= cc + j <= r + h
@@ -584,22 +671,29 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                         }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(x[j] + st2);
+                        for (int j = 0; j < 32; ++j) acc[j & 3] += ptx::ex2(EXT ? x[j] : x[j] + st2);
                     }
                 } else {
                     // every entry inside the band, shifted: packed fp32x2 math
                     const uint64_t SL2 = ptx::f2(a.sl2, a.sl2), ST2 = ptx::f2(st2, st2);
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 bv = ptx::ld_shared_f4(vaddr + 16u * j4);
+                        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (!EXT) bv = ptx::ld_shared_f4(vaddr + 16u * j4);
                         float4 wv;
                         if (WSUM) wv = ptx::ld_shared_f4(vaddr + 4u * C::BN + 16u * j4);
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             const int k = 2 * j4 + hh;
-                            uint64_t xx = ptx::ffma2(ptx::f2(v[2 * k], v[2 * k + 1]), SL2,
-                                                     hh ? ptx::f2(bv.z, bv.w) : ptx::f2(bv.x, bv.y));
-                            xx = ptx::fadd2(xx, ST2);
+                            uint64_t xx;
+                            if (EXT) {
+                                // bias already in the accumulator: one packed FMA with the row shift
+                                xx = ptx::ffma2(ptx::f2(v[2 * k], v[2 * k + 1]), SL2, ST2);
+                            } else {
+                                xx = ptx::ffma2(ptx::f2(v[2 * k], v[2 * k + 1]), SL2,
+                                                hh ? ptx::f2(bv.z, bv.w) : ptx::f2(bv.x, bv.y));
+                                xx = ptx::fadd2(xx, ST2);
+                            }
                             float x0, x1, e0, e1;
                             ptx::f2split(xx, x0, x1);
                             if (k < kFmaPairs) {
@@ -700,6 +794,9 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 }
                 out_hs[pb + r] = outv;
                 if (!WSUM) outb_hs[base + r] = ob;
+                if (!WSUM && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, ob, a.sl2);
+            } else if (!WSUM && hf == 0 && is_dustbin_row && exto_of(hs)) {
+                band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.sl2);   // the dustbin never enters a band sum
             }
         }
         if (MULTI && D >= 0 && __all_sync(0xffffffffu, ok && !*abort_flag)) {
@@ -1399,11 +1496,11 @@ int sm_count() {
     return n;
 }
 
-template <int DH, int KIND, bool MULTI>
-cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const TcBandArgs& a, int grid,
-                                cudaStream_t st) {
-    constexpr size_t smem = BandCfg<DH, KIND>::SMEM;
-    auto kernel = tc_band_kernel<DH, KIND, MULTI>;
+template <int DH, int KIND, bool MULTI, bool EXT = false>
+cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, const CUtensorMap& tmUE,
+                                const CUtensorMap& tmVE, const TcBandArgs& a, int grid, cudaStream_t st) {
+    constexpr size_t smem = BandCfg<DH, KIND, EXT>::SMEM;
+    auto kernel = tc_band_kernel<DH, KIND, MULTI, EXT>;
     cudaError_t e = set_smem(kernel, smem);
     if (e != cudaSuccess) return e;
     // the register split inside the kernel assumes this launch allocation
@@ -1411,11 +1508,12 @@ cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, 
     if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
     if (fa.numRegs != kBandLaunchRegs) return cudaErrorNotSupported;
     if (!MULTI) {
-        kernel<<<grid, kBandThreads, smem, st>>>(tmX, tmY, a);
+        kernel<<<grid, kBandThreads, smem, st>>>(tmX, tmY, tmUE, tmVE, a);
         return cudaGetLastError();
     }
     // fused half-steps meet at grid-wide barriers: every CTA must be resident at once
-    void* args[] = {const_cast<CUtensorMap*>(&tmX), const_cast<CUtensorMap*>(&tmY), const_cast<TcBandArgs*>(&a)};
+    void* args[] = {const_cast<CUtensorMap*>(&tmX), const_cast<CUtensorMap*>(&tmY), const_cast<CUtensorMap*>(&tmUE),
+                    const_cast<CUtensorMap*>(&tmVE), const_cast<TcBandArgs*>(&a)};
     return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3(grid), dim3(kBandThreads), args,
                                        smem, st);
 }
@@ -1428,6 +1526,14 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     CUtensorMap tmX, tmY;
     const uint64_t rows = uint64_t(g.BH) * g.L;
     if (!make_map(&tmX, X, rows, g.d, 128) || !make_map(&tmY, Y, rows, g.d, 128)) return cudaErrorInvalidValue;
+    // fused d = 128 half-steps read the column-bias operand rows of both sides
+    CUtensorMap tmUE = tmX, tmVE = tmX;
+    const bool ext = multi && g.d == 128 && g.h >= 256 && a.ue && a.ve;
+    if (ext) {
+        if (!make_map_ext(&tmUE, a.ue, rows, 128) || !make_map_ext(&tmVE, a.ve, rows, 128)) return cudaErrorInvalidValue;
+    } else if (multi) {
+        a.ue = a.ve = nullptr;   // (no operand rows written either)
+    }
     a.H = g.H;
     a.L = g.L;
     a.h = g.h;
@@ -1449,18 +1555,20 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
         return cudaErrorInvalidValue;
     }
     if (g.d == 128) {
-        if (multi) return launch_band_variant<128, kBandShift, true>(tmX, tmY, a, grid_used, st);
+        if (multi)
+            return ext ? launch_band_variant<128, kBandShift, true, true>(tmX, tmY, tmUE, tmVE, a, grid_used, st)
+                       : launch_band_variant<128, kBandShift, true, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
         switch (kind) {
-            case kBandOnline: return launch_band_variant<128, kBandOnline, false>(tmX, tmY, a, grid_used, st);
-            case kBandShift: return launch_band_variant<128, kBandShift, false>(tmX, tmY, a, grid_used, st);
-            case kBandWsum: return launch_band_variant<128, kBandWsum, false>(tmX, tmY, a, grid_used, st);
+            case kBandOnline: return launch_band_variant<128, kBandOnline, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
+            case kBandShift: return launch_band_variant<128, kBandShift, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<128, kBandWsum, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
         }
     } else {
-        if (multi) return launch_band_variant<64, kBandShift, true>(tmX, tmY, a, grid_used, st);
+        if (multi) return launch_band_variant<64, kBandShift, true>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
         switch (kind) {
-            case kBandOnline: return launch_band_variant<64, kBandOnline, false>(tmX, tmY, a, grid_used, st);
-            case kBandShift: return launch_band_variant<64, kBandShift, false>(tmX, tmY, a, grid_used, st);
-            case kBandWsum: return launch_band_variant<64, kBandWsum, false>(tmX, tmY, a, grid_used, st);
+            case kBandOnline: return launch_band_variant<64, kBandOnline, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
+            case kBandShift: return launch_band_variant<64, kBandShift, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
+            case kBandWsum: return launch_band_variant<64, kBandWsum, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
         }
     }
     return cudaErrorInvalidValue;
@@ -1478,6 +1586,7 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     a.pstride = p.pstride;
     a.sd_term = p.sd_term;
     a.status = p.status;
+    a.ext_out = p.ext_out;
     cudaError_t e = launch_band(p.g, p.X, p.Y, a, p.stab ? kBandShift : kBandOnline, st);
     if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
@@ -1502,6 +1611,8 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     a.sd_col = row.sd_dense;
     a.dpart = row.dpart;
     a.dcnt = row.dcnt;
+    a.ue = f.ue;
+    a.ve = f.ve;
     // row half-steps: X = Q (row.X), Y = K (row.Y); the kernel swaps them for column half-steps
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
