@@ -1253,7 +1253,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         for (int it = 0; it < n; ++it) {
             const int sl = it % C::NL, cb = it & 1;
             const int c0 = tiles[it] * C::BN;
-            const bool interior = (c0 + C::BN - 1 - r0 <= h) && (r0 + C::BM - 1 - c0 <= h);
+            // This warp's 32 x 32 block (rows r0 + 32 q .., columns c0 + 32 qt ..) against the band:
+            // 0 = outside for every entry (no TMEM read, no exponentials; zero coefficients),
+            // 1 = inside for every entry, 2 = cut by the band edge (masked per entry).
+            const int dmin = c0 + qt * 32 - (r0 + q * 32 + 31), dmax = c0 + qt * 32 + 31 - (r0 + q * 32);
+            const int cls = (dmin > h || dmax < -h) ? 0 : (dmax <= h && dmin >= -h) ? 1 : 2;
             // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
             bool w1 = ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status);   // column vectors
             bool w2 = w1 && ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
@@ -1264,6 +1268,21 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             // pointer no longer carries the address space)
             const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
             auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
+            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(qt >> 1) * C::CATOM + crow;
+            if (cls == 0) {
+                // nothing of this block is in the band: hand the scores back unread; the product
+                // reads zeros for it
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(tempty);
+                if (M::VEC) {
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t unit = uint32_t((qt & 1) * 4 + t);
+                        ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), 0u, 0u, 0u, 0u);
+                    }
+                }
+            } else {
             // this warp's 32 columns of S (and dP), read whole; the buffer goes back at once
             float v[1][32], w[1][32];
             const uint32_t tl = tbase + lane_base + uint32_t(qt * 32);
@@ -1274,7 +1293,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty);
-            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(qt >> 1) * C::CATOM + crow;
 #pragma unroll
             for (int ch = 0; ch < 1; ++ch) {
                 const int cc0 = qt * 32;
@@ -1289,7 +1307,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     ptx::f2split(x0, vc[4 * j4 + 0], vc[4 * j4 + 1]);
                     ptx::f2split(x1, vc[4 * j4 + 2], vc[4 * j4 + 3]);
                 }
-                if (!interior) {
+                if (cls == 2) {
                     const int dlt0 = c0 + cc0 - r;
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
@@ -1367,6 +1385,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     a.s1part[size_t(slot) * a.s1stride + base + size_t(c0 + cc0 + lane)] = wc[0];
                 }
             }
+            }   // cls != 0
             if (M::VEC) ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
