@@ -371,6 +371,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     op.dpart = dpart;
     op.dcnt = dcnt;
     op.status = status;
+    op.tile_bits = tbits;
     EOT_TRY(run_bwd(impl, op, st, kProfOut));
     return EOT_OK;
 }

@@ -895,7 +895,9 @@ struct ModeT {
 };
 
 struct TcVecArgs {
-    int H, L, h, D;
+    int H, L, h, D, BH;
+    const uint32_t* tile_bits;  // [B][words]: 128-position tiles holding an active non-dustbin token
+    int words;
     float sc2;              // scale * log2(e)
     const float* logm;
     const float* pr;        // natural row bias [BH, L]
@@ -956,8 +958,8 @@ struct SweepCfg {
     static constexpr uint32_t OFF_YE = OFF_XE + EXTB;
     static constexpr uint32_t OFF_RED = FOLD ? OFF_YE + EXTB : OFF_V + NL * VB;  // [2 sums][4 quarters][128 rows] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 128 * 4;
-    // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm
-    static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1;
+    // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm accempty
+    static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
     static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
@@ -990,10 +992,33 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.y, b = bh / a.H, L = a.L, h = a.h, D = a.D;
-    const int r0 = blockIdx.x * C::BM;
-    const size_t base = size_t(bh) * L;
-    const float* logm = a.logm + size_t(b) * L;
+    const int L = a.L, h = a.h, D = a.D;
+    (void)max_tiles;
+    // Persistent: CTA c takes the jobs c, c + gridDim.x, ... (job = one 128-row tile of one unit,
+    // BH L / 128 of them; neighbouring CTAs work on neighbouring row tiles at the same time, so
+    // the column tiles they share are read from L2).  Every role walks the same jobs and, inside
+    // a job, the same band tiles (those holding an active non-dustbin column, from the tile
+    // bits), so ring slots and barrier phases follow from running counters across jobs; a job
+    // whose row tile holds no active token only has its outputs zeroed.
+    const int nT = L / C::BM, n_jobs = a.BH * nT;
+    struct Job {
+        int bh, b, r0, t_lo, t_hi;
+        size_t base;
+        const uint32_t* bits;
+        bool act;
+    };
+    auto job_of = [&](int job) {
+        Job j;
+        j.bh = job / nT;
+        j.b = j.bh / a.H;
+        j.r0 = (job - j.bh * nT) * C::BM;
+        j.base = size_t(j.bh) * L;
+        j.bits = a.tile_bits + size_t(j.b) * a.words;
+        j.act = tile_bit(j.bits, j.r0 / C::BM);
+        j.t_lo = max(0, j.r0 - h) / C::BN;
+        j.t_hi = min(L - 1, j.r0 + C::BM - 1 + h) / C::BN;
+        return j;
+    };
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     const uint32_t bar0 = ptx::smem_u32(bars);
@@ -1007,11 +1032,10 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     auto cfull = [&](int i) { return bar0 + 8u * (2 * C::NL + 5 + i); };
     auto cempty = [&](int i) { return bar0 + 8u * (2 * C::NL + 7 + i); };
     const uint32_t accfull = bar0 + 8u * (2 * C::NL + 9);
-    const uint32_t xtm = bar0 + 8u * (2 * C::NL + 10);   // row tiles copied into TMEM
+    const uint32_t xtm = bar0 + 8u * (2 * C::NL + 10);       // row tiles copied into TMEM
+    const uint32_t accempty = bar0 + 8u * (2 * C::NL + 11);  // accumulator read back
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-    int* tiles = reinterpret_cast<int*>(sm + C::OFF_TILES);
-    int* flags = tiles + max_tiles;
 
     if (tid == 0) {
         *abort_flag = 0;
@@ -1032,39 +1056,8 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         }
         ptx::mbar_init(accfull, 1);
         ptx::mbar_init(xtm, kSweepEpi);
+        ptx::mbar_init(accempty, kSweepEpi / 2);   // the warps of column quarters 0 and 1
         ptx::mbar_fence_init();
-        // The row tiles do not depend on the band's tile list: their copies start first and
-        // overlap the scan below.
-        ptx::prefetch_tmap(&tmX);
-        if (M::HASDP) ptx::prefetch_tmap(&tmA);
-        const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
-        ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1) + (FOLD ? C::EXTB : 0u));
-        for (int ka = 0; ka < C::KATOMS; ++ka) {
-            ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(base) + r0, xfull);
-            if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(base) + r0, xfull);
-        }
-        if (FOLD) {
-            ptx::prefetch_tmap(&tmXE);
-            ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_XE), &tmXE, 0, int(base) + r0, xfull);
-        }
-    }
-    bool any_row;
-    const int n = build_tile_list<C::BM, C::BN>(logm, L, r0, h, D, tiles, flags,
-                                                 reinterpret_cast<int*>(misc + 2), &any_row);
-    if (!any_row) {
-        if (tid == 0) {
-            // no copy may still be writing this CTA's shared memory when it exits
-            volatile int dummy = 0;
-            ptx::mbar_wait(xfull, 0, &dummy, a.status);
-        }
-        if (M::SCAL)
-            for (int r = tid; r < C::BM; r += kSweepThreads) a.sout[base + r0 + r] = 0.f;
-        if (M::VEC) {
-            __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
-            for (int e = tid; e < C::BM * DH / 8; e += kSweepThreads)
-                reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
-        }
-        return;
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_u32(misc), 512);
@@ -1077,7 +1070,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------- TMA producer (the row tiles are already on their way) ----------------
+            // ---------------- TMA producer: the column tiles of every job ----------------
             static_assert(M::W2, "every sweep pass reads two column-side tensors");
             ptx::prefetch_tmap(&tmY);
             ptx::prefetch_tmap(&tmW);
@@ -1092,30 +1085,37 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 for (int i = 0; i < NMOD; ++i) vsrc[k++] = a.yc[i];
             }
             constexpr uint32_t late_bytes = C::YB + uint32_t(NV) * C::BN * 4;
-            int issued_l = 0, issued_e = 0;
-            for (int it = 0; it < n; ++it) {
-                const int sl = it % C::NL;
-                const int c0 = tiles[it] * C::BN;
-                // late ring: column tile + column vectors
-                if (!ptx::mbar_wait(empty_l(sl), ((it / C::NL) & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(full_l(sl), late_bytes);
-                const uint32_t ls = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);
-                for (int ka = 0; ka < C::KATOMS; ++ka)
-                    ptx::tma_load_2d(ls + ka * C::YATOM, tm_late, ka * 64, int(base) + c0, full_l(sl));
-                const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
+            int issued_l = 0, issued_e = 0, itg = 0;
+            bool ok = true;
+            for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
+                const Job jb = job_of(job);
+                if (!jb.act) continue;
+                for (int t = jb.t_lo; t <= jb.t_hi; ++t) {
+                    if (!tile_bit(jb.bits, t)) continue;
+                    const int it = itg++;
+                    const int sl = it % C::NL;
+                    const int c0 = t * C::BN;
+                    // late ring: column tile + column vectors
+                    if (!ptx::mbar_wait(empty_l(sl), ((it / C::NL) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ptx::mbar_expect_tx(full_l(sl), late_bytes);
+                    const uint32_t ls = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);
+                    for (int ka = 0; ka < C::KATOMS; ++ka)
+                        ptx::tma_load_2d(ls + ka * C::YATOM, tm_late, ka * 64, int(jb.base) + c0, full_l(sl));
+                    const uint32_t vs = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
 #pragma unroll
-                for (int i = 0; i < NV; ++i)
-                    ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + base + c0, C::BN * 4, full_l(sl));
-                issued_l = it + 1;
-                // early ring: the other column tile
-                if (!ptx::mbar_wait(empty_e, (it & 1) ^ 1, abort_flag, a.status)) break;
-                ptx::mbar_expect_tx(full_e, C::YB + (FOLD ? C::EXTB : 0u));
-                const uint32_t es = ptx::smem_u32(sm + C::OFF_E);
-                for (int ka = 0; ka < C::KATOMS; ++ka)
-                    ptx::tma_load_2d(es + ka * C::YATOM, tm_early, ka * 64, int(base) + c0, full_e);
-                // (the dP operand rides the early ring in dQ / dK: its modifier tile goes with it)
-                if (FOLD) ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE), &tmYE, 0, int(base) + c0, full_e);
-                issued_e = it + 1;
+                    for (int i = 0; i < NV; ++i)
+                        ptx::bulk_load(vs + i * C::BN * 4, vsrc[i] + jb.base + c0, C::BN * 4, full_l(sl));
+                    issued_l = it + 1;
+                    // early ring: the other column tile
+                    if (!ptx::mbar_wait(empty_e, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ptx::mbar_expect_tx(full_e, C::YB + (FOLD ? C::EXTB : 0u));
+                    const uint32_t es = ptx::smem_u32(sm + C::OFF_E);
+                    for (int ka = 0; ka < C::KATOMS; ++ka)
+                        ptx::tma_load_2d(es + ka * C::YATOM, tm_early, ka * 64, int(jb.base) + c0, full_e);
+                    // (the dP operand rides the early ring in dQ / dK: its modifier tile goes with it)
+                    if (FOLD) ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE), &tmYE, 0, int(jb.base) + c0, full_e);
+                    issued_e = it + 1;
+                }
             }
             if (*abort_flag) {
                 // let every copy still in flight land before the CTA can exit
@@ -1123,7 +1123,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 for (int it = max(0, issued_l - C::NL); it < issued_l; ++it)
                     ptx::mbar_wait(full_l(it % C::NL), (it / C::NL) & 1, &dummy, a.status);
                 if (issued_e > 0) ptx::mbar_wait(full_e, (issued_e - 1) & 1, &dummy, a.status);
-                ptx::mbar_wait(xfull, 0, &dummy, a.status);
             }
         }
     } else if (warp == 1 || warp == kSweepDpWarp) {
@@ -1131,40 +1130,50 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         // One thread each, so that neither product waits behind the other's instruction stream.
         const bool is_dp = warp == kSweepDpWarp;
         if (lane == 0 && (!is_dp || M::HASDP)) {
-            bool ok = ptx::mbar_wait(xtm, 0, abort_flag, a.status);
-            // (the row modifier tile XE is read from shared memory by the dP product)
-            if (FOLD && is_dp) ok = ok && ptx::mbar_wait(xfull, 0, abort_flag, a.status);
-            ptx::tc_fence_after();
-            int issued = 0;
+            int issued = 0, itg = 0, jc = 0;
+            bool ok = true;
             const uint32_t dtm = tbase + (is_dp ? C::TM_DP : C::TM_S);
             const uint32_t atm = tbase + (is_dp ? C::TM_A : C::TM_X);
             const bool late = is_dp == LATE_W;   // this issuer's column tile (W for dP, Y for S) rides the late ring
-            for (int it = 0; it < n && ok; ++it) {
-                const int sl = it % C::NL;
-                const bool got = late ? ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status)
-                                      : ptx::mbar_wait(full_e, it & 1, abort_flag, a.status);
-                if (!got) { ok = false; break; }
-                if (!ptx::mbar_wait(tempty, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+            for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
+                const Job jb = job_of(job);
+                if (!jb.act) continue;
+                // this job's row tiles are in TMEM (and its row modifier tile XE, read from shared
+                // memory by the dP product, has landed)
+                ok = ptx::mbar_wait(xtm, jc & 1, abort_flag, a.status);
+                if (FOLD && is_dp) ok = ok && ptx::mbar_wait(xfull, jc & 1, abort_flag, a.status);
+                ++jc;
+                if (!ok) break;
                 ptx::tc_fence_after();
-                // B operand: the column tile of S (Y) or of dP (W); A operand (row tile) from TMEM,
-                // 8 columns per K step of 16
-                const uint32_t boff = late ? C::OFF_L + uint32_t(sl) * C::YB : C::OFF_E;
-                const uint64_t bd = ptx::smem_desc(ptx::smem_u32(sm + boff), 16, 1024);
+                for (int t = jb.t_lo; t <= jb.t_hi && ok; ++t) {
+                    if (!tile_bit(jb.bits, t)) continue;
+                    const int it = itg++;
+                    const int sl = it % C::NL;
+                    const bool got = late ? ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status)
+                                          : ptx::mbar_wait(full_e, it & 1, abort_flag, a.status);
+                    if (!got) { ok = false; break; }
+                    if (!ptx::mbar_wait(tempty, (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    // B operand: the column tile of S (Y) or of dP (W); A operand (row tile) from TMEM,
+                    // 8 columns per K step of 16
+                    const uint32_t boff = late ? C::OFF_L + uint32_t(sl) * C::YB : C::OFF_E;
+                    const uint64_t bd = ptx::smem_desc(ptx::smem_u32(sm + boff), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < DH / 16; ++kk) {
-                    const uint64_t bo = uint64_t(((kk >> 2) * C::YATOM + (kk & 3) * 32) >> 4);
-                    ptx::mma_bf16_ts(dtm, atm + uint32_t(kk * 8), bd + bo, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < DH / 16; ++kk) {
+                        const uint64_t bo = uint64_t(((kk >> 2) * C::YATOM + (kk & 3) * 32) >> 4);
+                        ptx::mma_bf16_ts(dtm, atm + uint32_t(kk * 8), bd + bo, C::IDESC_S, kk > 0 ? 1u : 0u);
+                    }
+                    // dP' = dP + XE YE^T = dP - sum_k xr_k yc_k^T
+                    if (FOLD && is_dp)
+                        ptx::mma_bf16(dtm, ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_XE)),
+                                      ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_YE)), C::IDESC_S, 1u);
+                    ptx::mma_commit(tfull);
+                    // the early tile is free once this product completes; a late slot normally comes
+                    // back after the product MMA, or here in a pass without one
+                    if (!late) ptx::mma_commit(empty_e);
+                    else if (!M::VEC) ptx::mma_commit(empty_l(sl));
+                    issued = it + 1;
                 }
-                // dP' = dP + XE YE^T = dP - sum_k xr_k yc_k^T
-                if (FOLD && is_dp)
-                    ptx::mma_bf16(dtm, ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_XE)),
-                                  ptx::smem_desc_sw32(ptx::smem_u32(sm + C::OFF_YE)), C::IDESC_S, 1u);
-                ptx::mma_commit(tfull);
-                // the early tile is free once this product completes; a late slot normally comes
-                // back after the product MMA, or here in a pass without one
-                if (!late) ptx::mma_commit(empty_e);
-                else if (!M::VEC) ptx::mma_commit(empty_l(sl));
-                issued = it + 1;
             }
             if (*abort_flag && issued > 0) {
                 volatile int dummy = 0;
@@ -1172,32 +1181,68 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             }
         }
     } else if (warp == 2 + kSweepEpi) {
-        if (M::VEC && lane == 0) {
-            // ---------------- product MMA issuer: acc += coef(j) * Z(j) ----------------
-            // A thread of its own, so that score tiles are never queued behind a product
-            // that waits for the epilogue (tcgen05.commit tracks the issuing thread's MMAs).
-            int done = 0;
-            bool ok = true;
-            for (int j = 0; j < n && ok; ++j) {
-                const int cb = j & 1;
-                if (!ptx::mbar_wait(cfull(cb), (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                ptx::tc_fence_after();
-                const int sl = j % C::NL;
-                const uint32_t zs = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);   // Z rides the late ring
-                const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
+        if (lane == 0) {
+            // ---------------- row-tile loads and the product MMA issuer ----------------
+            // The row tiles of a job land in the coefficient buffers (copied from there into
+            // TMEM by the epilogue), so they are loaded here, once the previous job's products
+            // (or, in a pass without products, its copy into TMEM) are done.  The products
+            // acc += coef(j) * Z(j) have a thread of their own, so that score tiles are never
+            // queued behind a product that waits for the epilogue (tcgen05.commit tracks the
+            // issuing thread's MMAs).
+            ptx::prefetch_tmap(&tmX);
+            if (M::HASDP) ptx::prefetch_tmap(&tmA);
+            if (FOLD) ptx::prefetch_tmap(&tmXE);
+            int done = 0, itg = 0, jc = 0;
+            bool ok = true, xpending = false;
+            for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
+                const Job jb = job_of(job);
+                if (!jb.act) continue;
+                if (jc > 0) {
+                    ok = M::VEC ? ptx::mbar_wait(accfull, (jc - 1) & 1, abort_flag, a.status)
+                                : ptx::mbar_wait(xtm, (jc - 1) & 1, abort_flag, a.status);
+                    if (!ok) break;
+                }
+                const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
+                ptx::mbar_expect_tx(xfull, C::XB * (M::HASDP ? 2 : 1) + (FOLD ? C::EXTB : 0u));
+                for (int ka = 0; ka < C::KATOMS; ++ka) {
+                    ptx::tma_load_2d(xs + ka * C::XATOM, &tmX, ka * 64, int(jb.base) + jb.r0, xfull);
+                    if (M::HASDP) ptx::tma_load_2d(as + ka * C::XATOM, &tmA, ka * 64, int(jb.base) + jb.r0, xfull);
+                }
+                if (FOLD) ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_XE), &tmXE, 0, int(jb.base) + jb.r0, xfull);
+                xpending = true;
+                if (M::VEC) {
+                    // the previous job's accumulator has been read back
+                    if (jc > 0 && !ptx::mbar_wait(accempty, (jc - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                    int j = 0;
+                    for (int t = jb.t_lo; t <= jb.t_hi && ok; ++t) {
+                        if (!tile_bit(jb.bits, t)) continue;
+                        const int it = itg++;
+                        const int cb = it & 1;
+                        if (!ptx::mbar_wait(cfull(cb), (it >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                        xpending = false;   // (the epilogue has copied the row tiles)
+                        ptx::tc_fence_after();
+                        const int sl = it % C::NL;
+                        const uint32_t zs = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);   // Z rides the late ring
+                        const uint32_t cs = ptx::smem_u32(sm + C::OFF_C + cb * C::CB);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + (kk >> 2) * C::CATOM + (kk & 3) * 32, 16, 1024),
-                                  ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
-                                  (j > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(cempty(cb));
-                ptx::mma_commit(empty_l(sl));
-                done = j + 1;
+                        for (int kk = 0; kk < C::BN / 16; ++kk)
+                            ptx::mma_bf16(tbase + C::TM_ACC, ptx::smem_desc(cs + (kk >> 2) * C::CATOM + (kk & 3) * 32, 16, 1024),
+                                          ptx::smem_desc(zs + kk * 2048, C::YATOM, 1024), C::IDESC_O,
+                                          (j > 0 || kk > 0) ? 1u : 0u);
+                        ptx::mma_commit(cempty(cb));
+                        ptx::mma_commit(empty_l(sl));
+                        done = it + 1;
+                        ++j;
+                    }
+                    if (ok) ptx::mma_commit(accfull);
+                }
+                ++jc;
             }
-            if (ok && n > 0) ptx::mma_commit(accfull);
-            if (*abort_flag && done > 0) {
+            if (*abort_flag) {
                 volatile int dummy = 0;
-                ptx::mbar_wait(cempty((done - 1) & 1), ((done - 1) >> 1) & 1, &dummy, a.status);
+                if (M::VEC && done > 0) ptx::mbar_wait(cempty((done - 1) & 1), ((done - 1) >> 1) & 1, &dummy, a.status);
+                // no row-tile copy may still be writing this CTA's shared memory when it exits
+                if (xpending) ptx::mbar_wait(xfull, (jc - 1) & 1, &dummy, a.status);
             }
         }
     } else {
@@ -1205,44 +1250,64 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         const int q = warp & 3;                  // lane quadrant
         const int qt = (warp - 2) >> 2;          // which 32 columns of each 128-column tile
         const int half = qt;                     // (quarters 0, 1 also read back the accumulator halves)
-        const int row = q * 32 + lane, r = r0 + row;
+        const int row = q * 32 + lane;
+        const uint32_t lane_base = uint32_t(q * 32) << 16;
+        const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
+        const int etid = tid - 64;               // 0 .. 511
+        const uint64_t SC2 = ptx::f2(a.sc2, a.sc2);
+        int itg = 0, jc = 0;
+        bool ok = true;
+        for (int job = blockIdx.x; job < n_jobs; job += gridDim.x) {
+        const Job jb = job_of(job);
+        const int r0 = jb.r0;
+        const size_t base = jb.base;
+        if (!jb.act) {
+            // no active token in this row tile: zero outputs
+            if (M::SCAL)
+                for (int i = etid; i < C::BM; i += 32 * kSweepEpi) a.sout[base + r0 + i] = 0.f;
+            if (M::VEC) {
+                __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r0) * DH;
+                for (int e = etid; e < C::BM * DH / 8; e += 32 * kSweepEpi)
+                    reinterpret_cast<uint4*>(vo)[e] = make_uint4(0, 0, 0, 0);
+            }
+            continue;
+        }
+        const float* logm = a.logm + size_t(jb.b) * L;
+        const int r = r0 + row;
         const float lm = logm[r];
         const bool ract = lm != kNegInf;
         const bool is_dustbin_row = (r == D) && ract;
         const float pr2 = ract ? a.pr[base + r] * kLog2e : kNegInf;
-        const uint64_t PR2 = ptx::f2(pr2, pr2), SC2 = ptx::f2(a.sc2, a.sc2);
+        const uint64_t PR2 = ptx::f2(pr2, pr2);
         float xr[NMOD > 0 ? NMOD : 1];
 #pragma unroll
         for (int k = 0; k < NMOD; ++k) xr[k] = ract ? -a.xr[k][base + r] : 0.f;
-        const uint32_t lane_base = uint32_t(q * 32) << 16;
         uint64_t s1a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
         uint64_t s2a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
-        bool ok = true;
-        const uint32_t crow = uint32_t(row >> 3) * 1024u + uint32_t(row & 7) * 128u;
         {
-            // Row tiles into TMEM as MMA A operands: warp (q, quarter 0) copies X, (q, quarter 1) A,
-            // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
-            const bool copy = qt == 0 || (qt == 1 && M::HASDP);
-            bool okx = !copy || ptx::mbar_wait(xfull, 0, abort_flag, a.status);
-            okx = __all_sync(0xffffffffu, okx);
-            if (okx && copy) {
-                const uint32_t src = ptx::smem_u32(sm + C::OFF_C + (half ? C::XB : 0u)) + crow;
-                const uint32_t dst = tbase + lane_base + (half ? C::TM_A : C::TM_X);
+                // Row tiles into TMEM as MMA A operands: warp (q, quarter 0) copies X, (q, quarter 1) A,
+                // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
+                const bool copy = qt == 0 || (qt == 1 && M::HASDP);
+                bool okx = !copy || ptx::mbar_wait(xfull, jc & 1, abort_flag, a.status);
+                okx = __all_sync(0xffffffffu, okx);
+                if (okx && copy) {
+                    const uint32_t src = ptx::smem_u32(sm + C::OFF_C + (half ? C::XB : 0u)) + crow;
+                    const uint32_t dst = tbase + lane_base + (half ? C::TM_A : C::TM_X);
 #pragma unroll
-                for (int ka = 0; ka < C::KATOMS; ++ka) {
-                    uint32_t w[32];
+                    for (int ka = 0; ka < C::KATOMS; ++ka) {
+                        uint32_t w[32];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint4 u = ptx::ld_shared_u4(src + ka * C::XATOM + ((uint32_t(j) ^ uint32_t(row & 7)) << 4));
-                        w[4 * j] = u.x;
-                        w[4 * j + 1] = u.y;
-                        w[4 * j + 2] = u.z;
-                        w[4 * j + 3] = u.w;
+                        for (int j = 0; j < 8; ++j) {
+                            const uint4 u = ptx::ld_shared_u4(src + ka * C::XATOM + ((uint32_t(j) ^ uint32_t(row & 7)) << 4));
+                            w[4 * j] = u.x;
+                            w[4 * j + 1] = u.y;
+                            w[4 * j + 2] = u.z;
+                            w[4 * j + 3] = u.w;
+                        }
+                        ptx::tmem_st32(dst + uint32_t(ka * 32), w);
                     }
-                    ptx::tmem_st32(dst + uint32_t(ka * 32), w);
+                    ptx::tmem_wait_st();
                 }
-                ptx::tmem_wait_st();
-            }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(xtm);
@@ -1250,225 +1315,236 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             // every warp has read its rows of X and A before any coefficient overwrites them
             ptx::named_bar_sync(2, 32 * kSweepEpi);
         }
-        for (int it = 0; it < n; ++it) {
-            const int sl = it % C::NL, cb = it & 1;
-            const int c0 = tiles[it] * C::BN;
-            // This warp's 32 x 32 block (rows r0 + 32 q .., columns c0 + 32 qt ..) against the band:
-            // 0 = outside for every entry (no TMEM read, no exponentials; zero coefficients),
-            // 1 = inside for every entry, 2 = cut by the band edge (masked per entry).
-            const int dmin = c0 + qt * 32 - (r0 + q * 32 + 31), dmax = c0 + qt * 32 + 31 - (r0 + q * 32);
-            const int cls = (dmin > h || dmax < -h) ? 0 : (dmax <= h && dmin >= -h) ? 1 : 2;
-            // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-            bool w1 = ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status);   // column vectors
-            bool w2 = w1 && ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
-            bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
-            if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
-            ptx::tc_fence_after();
-            // column vectors of this tile's late-ring slot (explicit shared-memory loads: the aligned base
-            // pointer no longer carries the address space)
-            const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
-            auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
-            const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(qt >> 1) * C::CATOM + crow;
-            if (cls == 0) {
-                // nothing of this block is in the band: hand the scores back unread; the product
-                // reads zeros for it
+        for (int tcol = jb.t_lo; tcol <= jb.t_hi; ++tcol) {
+            if (!tile_bit(jb.bits, tcol)) continue;
+            const int it = itg++;
+            if (!ok) continue;
+                const int sl = it % C::NL, cb = it & 1;
+                const int c0 = tcol * C::BN;
+                // This warp's 32 x 32 block (rows r0 + 32 q .., columns c0 + 32 qt ..) against the band:
+                // 0 = outside for every entry (no TMEM read, no exponentials; zero coefficients),
+                // 1 = inside for every entry, 2 = cut by the band edge (masked per entry).
+                const int dmin = c0 + qt * 32 - (r0 + q * 32 + 31), dmax = c0 + qt * 32 + 31 - (r0 + q * 32);
+                const int cls = (dmin > h || dmax < -h) ? 0 : (dmax <= h && dmin >= -h) ? 1 : 2;
+                // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
+                bool w1 = ptx::mbar_wait(full_l(sl), (it / C::NL) & 1, abort_flag, a.status);   // column vectors
+                bool w2 = w1 && ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
+                bool w3 = w2 && (!M::VEC || ptx::mbar_wait(cempty(cb), ((it >> 1) & 1) ^ 1, abort_flag, a.status));
+                if (!__all_sync(0xffffffffu, w3)) { ok = false; break; }
+                ptx::tc_fence_after();
+                // column vectors of this tile's late-ring slot (explicit shared-memory loads: the aligned base
+                // pointer no longer carries the address space)
+                const uint32_t cva = ptx::smem_u32(sm + C::OFF_V + sl * C::VB);
+                auto cvec = [&](int vec, int col) { return ptx::ld_shared_f4(cva + uint32_t((vec * C::BN + col) * 4)); };
+                const uint32_t cbase = ptx::smem_u32(sm + C::OFF_C + cb * C::CB) + uint32_t(qt >> 1) * C::CATOM + crow;
+                if (cls == 0) {
+                    // nothing of this block is in the band: hand the scores back unread; the product
+                    // reads zeros for it
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(tempty);
+                    if (M::VEC) {
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const uint32_t unit = uint32_t((qt & 1) * 4 + t);
+                            ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), 0u, 0u, 0u, 0u);
+                        }
+                    }
+                } else {
+                // this warp's 32 columns of S (and dP), read whole; the buffer goes back at once
+                float v[1][32], w[1][32];
+                const uint32_t tl = tbase + lane_base + uint32_t(qt * 32);
+                ptx::tmem_ld32(tl + C::TM_S, v[0]);
+                if (M::HASDP) ptx::tmem_ld32(tl + C::TM_DP, w[0]);
+                ptx::tmem_wait_ld(v[0]);
+                if (M::HASDP) ptx::tmem_tie(w[0]);
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(tempty);
-                if (M::VEC) {
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint32_t unit = uint32_t((qt & 1) * 4 + t);
-                        ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), 0u, 0u, 0u, 0u);
+                for (int ch = 0; ch < 1; ++ch) {
+                    const int cc0 = qt * 32;
+                    float (&vc)[32] = v[ch];
+                    float (&wc)[32] = w[ch];
+                    // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 b4 = cvec(0, cc0 + 4 * j4);
+                        uint64_t x0 = ptx::ffma2(ptx::f2(vc[4 * j4 + 0], vc[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
+                        uint64_t x1 = ptx::ffma2(ptx::f2(vc[4 * j4 + 2], vc[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
+                        ptx::f2split(x0, vc[4 * j4 + 0], vc[4 * j4 + 1]);
+                        ptx::f2split(x1, vc[4 * j4 + 2], vc[4 * j4 + 3]);
                     }
-                }
-            } else {
-            // this warp's 32 columns of S (and dP), read whole; the buffer goes back at once
-            float v[1][32], w[1][32];
-            const uint32_t tl = tbase + lane_base + uint32_t(qt * 32);
-            ptx::tmem_ld32(tl + C::TM_S, v[0]);
-            if (M::HASDP) ptx::tmem_ld32(tl + C::TM_DP, w[0]);
-            ptx::tmem_wait_ld(v[0]);
-            if (M::HASDP) ptx::tmem_tie(w[0]);
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(tempty);
+                    if (cls == 2) {
+                        const int dlt0 = c0 + cc0 - r;
 #pragma unroll
-            for (int ch = 0; ch < 1; ++ch) {
-                const int cc0 = qt * 32;
-                float (&vc)[32] = v[ch];
-                float (&wc)[32] = w[ch];
-                // P~ = exp2(S * scale * log2e + row bias + column bias), pairs in fp32x2
-#pragma unroll
-                for (int j4 = 0; j4 < 8; ++j4) {
-                    const float4 b4 = cvec(0, cc0 + 4 * j4);
-                    uint64_t x0 = ptx::ffma2(ptx::f2(vc[4 * j4 + 0], vc[4 * j4 + 1]), SC2, ptx::fadd2(PR2, ptx::f2(b4.x, b4.y)));
-                    uint64_t x1 = ptx::ffma2(ptx::f2(vc[4 * j4 + 2], vc[4 * j4 + 3]), SC2, ptx::fadd2(PR2, ptx::f2(b4.z, b4.w)));
-                    ptx::f2split(x0, vc[4 * j4 + 0], vc[4 * j4 + 1]);
-                    ptx::f2split(x1, vc[4 * j4 + 2], vc[4 * j4 + 3]);
-                }
-                if (cls == 2) {
-                    const int dlt0 = c0 + cc0 - r;
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int dl = dlt0 + j;
-                        if (dl < -h || dl > h) vc[j] = kNegInf;
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 32; ++j) vc[j] = ptx::ex2(vc[j]);
-                if (MODE == kModeR2 && a.pcache) {
-                    // cache this chunk of the plan: 32 entries of row r, 16-byte aligned (h % 8 == 0)
-                    uint4* dst = reinterpret_cast<uint4*>(a.pcache + (base + r) * size_t(a.cpitch) + (c0 + cc0 - r0 + h));
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        dst[t] = make_uint4(ptx::pack_bf16(vc[8 * t], vc[8 * t + 1]), ptx::pack_bf16(vc[8 * t + 2], vc[8 * t + 3]),
-                                            ptx::pack_bf16(vc[8 * t + 4], vc[8 * t + 5]), ptx::pack_bf16(vc[8 * t + 6], vc[8 * t + 7]));
-                }
-                if (M::SCAL) {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const uint64_t P2 = ptx::f2(vc[2 * k], vc[2 * k + 1]);
-                        if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(wc[2 * k], wc[2 * k + 1]), s1a[k & 1]);
-                        if (M::SM) {
-                            const float4 mv = cvec(VOFF_M, cc0 + 4 * (k >> 1));
-                            s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
+                        for (int j = 0; j < 32; ++j) {
+                            const int dl = dlt0 + j;
+                            if (dl < -h || dl > h) vc[j] = kNegInf;
                         }
                     }
-                }
-                if (M::VEC) {
-                    // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
-                    uint32_t pk[16];
 #pragma unroll
-                    for (int k4 = 0; k4 < 8; ++k4) {
-                        uint64_t cf0 = M::VDP ? ptx::f2(wc[4 * k4], wc[4 * k4 + 1]) : ptx::f2(1.f, 1.f);
-                        uint64_t cf1 = M::VDP ? ptx::f2(wc[4 * k4 + 2], wc[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
-#pragma unroll
-                        for (int mm = 0; mm < NMOD; ++mm) {
-                            const float4 yv = cvec(VOFF_Y + mm, cc0 + 4 * k4);
-                            const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
-                            cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
-                            cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
-                        }
-                        float c0f, c1f, c2f, c3f;
-                        ptx::f2split(cf0, c0f, c1f);
-                        ptx::f2split(cf1, c2f, c3f);
-                        pk[2 * k4] = ptx::pack_bf16(vc[4 * k4] * c0f, vc[4 * k4 + 1] * c1f);
-                        pk[2 * k4 + 1] = ptx::pack_bf16(vc[4 * k4 + 2] * c2f, vc[4 * k4 + 3] * c3f);
-                    }
-                    // 128-byte-swizzled K-major tile: 16-byte unit u of a row at (u ^ (row & 7))
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint32_t unit = uint32_t((qt & 1) * 4 + t);
-                        ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1],
-                                          pk[4 * t + 2], pk[4 * t + 3]);
-                    }
-                }
-                if (MODE == kModeC1 && a.s1part) {
-                    // Pt dP summed over this warp's 32 rows for each of its 32 columns: a transposing
-                    // butterfly (each step keeps half of the columns and adds the partner lane's copy
-                    // of them), after which lane l holds column cc0 + l.  wc is free by now.
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) wc[j] *= vc[j];
-                    const int lb = lane;
-#pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1) {
-                        const bool up = (lb & off) != 0;
-#pragma unroll
-                        for (int i = 0; i < off; ++i) {
-                            const float send = up ? wc[i] : wc[i + off];
-                            const float keep = up ? wc[i + off] : wc[i];
-                            wc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                        }
-                    }
-                    const int slot = (tiles[it] - int(blockIdx.x) + a.s1E) * 4 + q;
-                    a.s1part[size_t(slot) * a.s1stride + base + size_t(c0 + cc0 + lane)] = wc[0];
-                }
-            }
-            }   // cls != 0
-            if (M::VEC) ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(empty_l(sl));
-                if (M::VEC) ptx::mbar_arrive(cfull(cb));
-            }
-        }
-        // Scalar partials of the four column quarters meet in shared memory.
-        float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
-        if (M::SCAL) {
-            float a0, a1, b0, b1;
-            ptx::f2split(ptx::fadd2(s1a[0], s1a[1]), a0, a1);
-            ptx::f2split(ptx::fadd2(s2a[0], s2a[1]), b0, b1);
-            red[(0 * 4 + qt) * 128 + row] = a0 + a1;
-            red[(1 * 4 + qt) * 128 + row] = b0 + b1;
-        }
-        ptx::named_bar_sync(1, 32 * kSweepEpi);
-        ok = __all_sync(0xffffffffu, ok);
-        // Dustbin link of this row (the dustbin column), then the writes.
-        const bool d_act = D >= 0 && logm[D] != kNegInf;
-        float Pd = 0.f, dpd = 0.f, coefd = 0.f;
-        if (ract && d_act && !is_dustbin_row) {
-            Pd = ptx::ex2((a.sd_term[base + r] + a.pr[base + r] + a.pc[base + D]) * kLog2e);
-            if (M::HASDP) dpd = a.dp_term[base + r];
-            float mod = M::VDP ? dpd : 1.f;
-#pragma unroll
-            for (int k = 0; k < NMOD; ++k) mod += xr[k] * a.yc[k][base + D];
-            coefd = Pd * mod;
-        }
-        if (M::SCAL && ok && qt == 0 && !is_dustbin_row) {
-            float s1 = (red[0 * 128 + row] + red[1 * 128 + row]) + (red[2 * 128 + row] + red[3 * 128 + row]);
-            float s2 = (red[4 * 128 + row] + red[5 * 128 + row]) + (red[6 * 128 + row] + red[7 * 128 + row]);
-            if (d_act && ract) {
-                if (M::SDP) s1 = fmaf(Pd, dpd, s1);
-                if (M::SM) s2 = fmaf(Pd, a.m[base + D], s2);
-            }
-            float outv = 0.f;
-            if (ract) {
-                outv = (a.f ? a.f[base + r] : 1.f) * (s1 + (a.hv ? a.hv[base + r] : 0.f) * s2);
-                if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
-            }
-            a.sout[base + r] = outv;
-        }
-        // The accumulator read is a warp-collective: every lane takes part; only the stores
-        // are predicated (the dustbin row is written by the dense dustbin kernel).
-        if (M::VEC && ok && qt < 2) {
-            const bool have_acc = n > 0;
-            bool wacc = !have_acc || ptx::mbar_wait(accfull, 0, abort_flag, a.status);
-            ok = __all_sync(0xffffffffu, wacc);
-            ptx::tc_fence_after();
-            if (ok) {
-                __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r) * DH;
-                const __nv_bfloat16* zD = d_act ? a.Zg + (base + D) * DH : nullptr;
-                const bool store = !is_dustbin_row;
-#pragma unroll
-                for (int chh = 0; chh < DH / 64; ++chh) {
-                    const int col = half * (DH / 2) + chh * 32;
-                    float v[32];
-                    if (have_acc) {
-                        ptx::tmem_ld32(tbase + lane_base + C::TM_ACC + uint32_t(col), v);
-                        ptx::tmem_wait_ld(v);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-                    }
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float lo = v[2 * j], hi = v[2 * j + 1];
-                        if (ract && d_act && store) {
-                            lo = fmaf(coefd, __bfloat162float(zD[col + 2 * j]), lo);
-                            hi = fmaf(coefd, __bfloat162float(zD[col + 2 * j + 1]), hi);
-                        }
-                        pk[j] = ract ? ptx::pack_bf16(a.vscale * lo, a.vscale * hi) : 0u;
-                    }
-                    if (store) {
-                        uint4* dst = reinterpret_cast<uint4*>(vo + col);
+                    for (int j = 0; j < 32; ++j) vc[j] = ptx::ex2(vc[j]);
+                    if (MODE == kModeR2 && a.pcache) {
+                        // cache this chunk of the plan: 32 entries of row r, 16-byte aligned (h % 8 == 0)
+                        uint4* dst = reinterpret_cast<uint4*>(a.pcache + (base + r) * size_t(a.cpitch) + (c0 + cc0 - r0 + h));
 #pragma unroll
                         for (int t = 0; t < 4; ++t)
-                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                            dst[t] = make_uint4(ptx::pack_bf16(vc[8 * t], vc[8 * t + 1]), ptx::pack_bf16(vc[8 * t + 2], vc[8 * t + 3]),
+                                                ptx::pack_bf16(vc[8 * t + 4], vc[8 * t + 5]), ptx::pack_bf16(vc[8 * t + 6], vc[8 * t + 7]));
+                    }
+                    if (M::SCAL) {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const uint64_t P2 = ptx::f2(vc[2 * k], vc[2 * k + 1]);
+                            if (M::SDP) s1a[k & 1] = ptx::ffma2(P2, ptx::f2(wc[2 * k], wc[2 * k + 1]), s1a[k & 1]);
+                            if (M::SM) {
+                                const float4 mv = cvec(VOFF_M, cc0 + 4 * (k >> 1));
+                                s2a[k & 1] = ptx::ffma2(P2, (k & 1) ? ptx::f2(mv.z, mv.w) : ptx::f2(mv.x, mv.y), s2a[k & 1]);
+                            }
+                        }
+                    }
+                    if (M::VEC) {
+                        // coefficient = P~ * (dP - sum_k xr_k yc_k)  (or P~ when the pass has no dP)
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int k4 = 0; k4 < 8; ++k4) {
+                            uint64_t cf0 = M::VDP ? ptx::f2(wc[4 * k4], wc[4 * k4 + 1]) : ptx::f2(1.f, 1.f);
+                            uint64_t cf1 = M::VDP ? ptx::f2(wc[4 * k4 + 2], wc[4 * k4 + 3]) : ptx::f2(1.f, 1.f);
+#pragma unroll
+                            for (int mm = 0; mm < NMOD; ++mm) {
+                                const float4 yv = cvec(VOFF_Y + mm, cc0 + 4 * k4);
+                                const uint64_t X2 = ptx::f2(xr[mm], xr[mm]);
+                                cf0 = ptx::ffma2(X2, ptx::f2(yv.x, yv.y), cf0);
+                                cf1 = ptx::ffma2(X2, ptx::f2(yv.z, yv.w), cf1);
+                            }
+                            float c0f, c1f, c2f, c3f;
+                            ptx::f2split(cf0, c0f, c1f);
+                            ptx::f2split(cf1, c2f, c3f);
+                            pk[2 * k4] = ptx::pack_bf16(vc[4 * k4] * c0f, vc[4 * k4 + 1] * c1f);
+                            pk[2 * k4 + 1] = ptx::pack_bf16(vc[4 * k4 + 2] * c2f, vc[4 * k4 + 3] * c3f);
+                        }
+                        // 128-byte-swizzled K-major tile: 16-byte unit u of a row at (u ^ (row & 7))
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const uint32_t unit = uint32_t((qt & 1) * 4 + t);
+                            ptx::st_shared_v4(cbase + ((unit ^ uint32_t(row & 7)) << 4), pk[4 * t], pk[4 * t + 1],
+                                              pk[4 * t + 2], pk[4 * t + 3]);
+                        }
+                    }
+                    if (MODE == kModeC1 && a.s1part) {
+                        // Pt dP summed over this warp's 32 rows for each of its 32 columns: a transposing
+                        // butterfly (each step keeps half of the columns and adds the partner lane's copy
+                        // of them), after which lane l holds column cc0 + l.  wc is free by now.
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) wc[j] *= vc[j];
+                        const int lb = lane;
+#pragma unroll
+                        for (int off = 16; off >= 1; off >>= 1) {
+                            const bool up = (lb & off) != 0;
+#pragma unroll
+                            for (int i = 0; i < off; ++i) {
+                                const float send = up ? wc[i] : wc[i + off];
+                                const float keep = up ? wc[i + off] : wc[i];
+                                wc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                            }
+                        }
+                        const int slot = (tcol - jb.r0 / C::BM + a.s1E) * 4 + q;
+                        a.s1part[size_t(slot) * a.s1stride + base + size_t(c0 + cc0 + lane)] = wc[0];
+                    }
+                }
+                }   // cls != 0
+                if (M::VEC) ptx::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::mbar_arrive(empty_l(sl));
+                    if (M::VEC) ptx::mbar_arrive(cfull(cb));
+                }
+        }
+            // Scalar partials of the four column quarters meet in shared memory.
+            float* red = reinterpret_cast<float*>(sm + C::OFF_RED);
+            if (M::SCAL) {
+                float a0, a1, b0, b1;
+                ptx::f2split(ptx::fadd2(s1a[0], s1a[1]), a0, a1);
+                ptx::f2split(ptx::fadd2(s2a[0], s2a[1]), b0, b1);
+                red[(0 * 4 + qt) * 128 + row] = a0 + a1;
+                red[(1 * 4 + qt) * 128 + row] = b0 + b1;
+            }
+            ptx::named_bar_sync(1, 32 * kSweepEpi);
+            ok = __all_sync(0xffffffffu, ok);
+            // Dustbin link of this row (the dustbin column), then the writes.
+            const bool d_act = D >= 0 && logm[D] != kNegInf;
+            float Pd = 0.f, dpd = 0.f, coefd = 0.f;
+            if (ract && d_act && !is_dustbin_row) {
+                Pd = ptx::ex2((a.sd_term[base + r] + a.pr[base + r] + a.pc[base + D]) * kLog2e);
+                if (M::HASDP) dpd = a.dp_term[base + r];
+                float mod = M::VDP ? dpd : 1.f;
+#pragma unroll
+                for (int k = 0; k < NMOD; ++k) mod += xr[k] * a.yc[k][base + D];
+                coefd = Pd * mod;
+            }
+            if (M::SCAL && ok && qt == 0 && !is_dustbin_row) {
+                float s1 = (red[0 * 128 + row] + red[1 * 128 + row]) + (red[2 * 128 + row] + red[3 * 128 + row]);
+                float s2 = (red[4 * 128 + row] + red[5 * 128 + row]) + (red[6 * 128 + row] + red[7 * 128 + row]);
+                if (d_act && ract) {
+                    if (M::SDP) s1 = fmaf(Pd, dpd, s1);
+                    if (M::SM) s2 = fmaf(Pd, a.m[base + D], s2);
+                }
+                float outv = 0.f;
+                if (ract) {
+                    outv = (a.f ? a.f[base + r] : 1.f) * (s1 + (a.hv ? a.hv[base + r] : 0.f) * s2);
+                    if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+                }
+                a.sout[base + r] = outv;
+            }
+            // The accumulator read is a warp-collective: every lane takes part; only the stores
+            // are predicated (the dustbin row is written by the dense dustbin kernel).
+            if (M::VEC && ok && qt < 2) {
+                const bool have_acc = true;   // an active row tile holds its own diagonal tile
+                bool wacc = ptx::mbar_wait(accfull, jc & 1, abort_flag, a.status);
+                ok = __all_sync(0xffffffffu, wacc);
+                ptx::tc_fence_after();
+                if (ok) {
+                    __nv_bfloat16* vo = static_cast<__nv_bfloat16*>(a.vout) + (base + r) * DH;
+                    const __nv_bfloat16* zD = d_act ? a.Zg + (base + D) * DH : nullptr;
+                    const bool store = !is_dustbin_row;
+#pragma unroll
+                    for (int chh = 0; chh < DH / 64; ++chh) {
+                        const int col = half * (DH / 2) + chh * 32;
+                        float v[32];
+                        if (have_acc) {
+                            ptx::tmem_ld32(tbase + lane_base + C::TM_ACC + uint32_t(col), v);
+                            ptx::tmem_wait_ld(v);
+                            if (chh == DH / 64 - 1) {
+                                // the accumulator is read: the next job's products may start
+                                ptx::tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) ptx::mbar_arrive(accempty);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+                        }
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            float lo = v[2 * j], hi = v[2 * j + 1];
+                            if (ract && d_act && store) {
+                                lo = fmaf(coefd, __bfloat162float(zD[col + 2 * j]), lo);
+                                hi = fmaf(coefd, __bfloat162float(zD[col + 2 * j + 1]), hi);
+                            }
+                            pk[j] = ract ? ptx::pack_bf16(a.vscale * lo, a.vscale * hi) : 0u;
+                        }
+                        if (store) {
+                            uint4* dst = reinterpret_cast<uint4*>(vo + col);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                        }
                     }
                 }
             }
+        ++jc;
         }
     }
     ptx::tc_fence_before();
@@ -1754,8 +1830,14 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.s1part = mode == kModeC1 ? p.s1part : nullptr;
     a.s1stride = p.s1stride;
     a.s1E = p.s1E;
+    if (!p.tile_bits) return cudaErrorInvalidValue;
+    a.BH = g.BH;
+    a.tile_bits = p.tile_bits;
+    a.words = tile_words(g.L);
     const int mt = max_tiles_for(g.L, g.h, 128, 128);
-    dim3 grid(g.L / 128, g.BH);
+    // persistent: one CTA per SM (or per job when there are fewer)
+    const long n_jobs = long(g.BH) * (g.L / 128);
+    dim3 grid(unsigned(std::max(1L, std::min<long>(n_jobs, sm_count()))));
     cudaError_t e = g.d == 128 ? launch_sweep_dh<128>(mode, nmod_k, fold, tmX, tmA, tmY, tmW, ext, a, mt, grid, st)
                                : launch_sweep_dh<64>(mode, nmod_k, fold, tmX, tmA, tmY, tmW, ext, a, mt, grid, st);
     if (e != cudaSuccess || g.D < 0) return e;
