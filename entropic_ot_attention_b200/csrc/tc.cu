@@ -1055,7 +1055,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             ptx::mbar_init(cempty(i), 1);
         }
         ptx::mbar_init(accfull, 1);
-        ptx::mbar_init(xtm, kSweepEpi);
+        ptx::mbar_init(xtm, 1);                     // the commit of the row tiles' copy into TMEM
         ptx::mbar_init(accempty, kSweepEpi / 2);   // the warps of column quarters 0 and 1
         ptx::mbar_fence_init();
     }
@@ -1138,10 +1138,9 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
                 const Job jb = job_of(job);
                 if (!jb.act) continue;
-                // this job's row tiles are in TMEM (and its row modifier tile XE, read from shared
-                // memory by the dP product, has landed)
+                // this job's row tiles are in TMEM (copied once they had landed, with the row
+                // modifier tile XE that the dP product reads from shared memory)
                 ok = ptx::mbar_wait(xtm, jc & 1, abort_flag, a.status);
-                if (FOLD && is_dp) ok = ok && ptx::mbar_wait(xfull, jc & 1, abort_flag, a.status);
                 ++jc;
                 if (!ok) break;
                 ptx::tc_fence_after();
@@ -1182,24 +1181,35 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         }
     } else if (warp == 2 + kSweepEpi) {
         if (lane == 0) {
-            // ---------------- row-tile loads and the product MMA issuer ----------------
-            // The row tiles of a job land in the coefficient buffers (copied from there into
-            // TMEM by the epilogue), so they are loaded here, once the previous job's products
-            // (or, in a pass without products, its copy into TMEM) are done.  The products
-            // acc += coef(j) * Z(j) have a thread of their own, so that score tiles are never
-            // queued behind a product that waits for the epilogue (tcgen05.commit tracks the
-            // issuing thread's MMAs).
+            // ---------------- row tiles into TMEM and the product MMA issuer ----------------
+            // The row tiles X and A of a job land (TMA) in the coefficient buffers and are copied
+            // from there into TMEM as MMA A operands (tcgen05.cp, one row per lane, two bf16 per
+            // 32-bit column; committed to xtm).  The next job's copy starts once this job's
+            // products are done (the coefficient buffers are free and every score product that
+            // read the TMEM row tiles has completed), or, in a pass without products, once its
+            // last score tile has completed, so the next job's scores overlap this job's
+            // read-back.  The products acc += coef(j) * Z(j) have a thread of their own, so that
+            // score tiles are never queued behind a product that waits for the epilogue
+            // (tcgen05.commit tracks the issuing thread's MMAs).
             ptx::prefetch_tmap(&tmX);
             if (M::HASDP) ptx::prefetch_tmap(&tmA);
             if (FOLD) ptx::prefetch_tmap(&tmXE);
             int done = 0, itg = 0, jc = 0;
+            // a pass without products: the previous job's score tiles (global indices) that must
+            // complete before its TMEM row tiles are overwritten, waited for one by one (a wait
+            // on a later tile's phase alone could be satisfied by an earlier phase's parity)
+            int tg = 0, pend_lo = 0, pend_hi = 0;
             bool ok = true, xpending = false;
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
                 const Job jb = job_of(job);
                 if (!jb.act) continue;
                 if (jc > 0) {
-                    ok = M::VEC ? ptx::mbar_wait(accfull, (jc - 1) & 1, abort_flag, a.status)
-                                : ptx::mbar_wait(xtm, (jc - 1) & 1, abort_flag, a.status);
+                    if (M::VEC) {
+                        ok = ptx::mbar_wait(accfull, (jc - 1) & 1, abort_flag, a.status);
+                    } else {
+                        for (int it = pend_lo; it < pend_hi && ok; ++it)
+                            ok = ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
+                    }
                     if (!ok) break;
                 }
                 const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
@@ -1210,6 +1220,20 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 }
                 if (FOLD) ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_XE), &tmXE, 0, int(jb.base) + jb.r0, xfull);
                 xpending = true;
+                if (!ptx::mbar_wait(xfull, jc & 1, abort_flag, a.status)) { ok = false; break; }
+                xpending = false;
+                ptx::tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DH / 16; ++kk) {
+                    const uint32_t koff = uint32_t((kk >> 2) * C::XATOM + (kk & 3) * 32);
+                    ptx::tmem_cp_128x256b(tbase + C::TM_X + uint32_t(kk * 8), ptx::smem_desc(xs + koff, 16, 1024));
+                    if (M::HASDP)
+                        ptx::tmem_cp_128x256b(tbase + C::TM_A + uint32_t(kk * 8), ptx::smem_desc(as + koff, 16, 1024));
+                }
+                ptx::mma_commit(xtm);
+                pend_lo = tg;
+                for (int t = jb.t_lo; t <= jb.t_hi; ++t) tg += tile_bit(jb.bits, t) ? 1 : 0;
+                pend_hi = tg;
                 if (M::VEC) {
                     // the previous job's accumulator has been read back
                     if (jc > 0 && !ptx::mbar_wait(accempty, (jc - 1) & 1, abort_flag, a.status)) { ok = false; break; }
@@ -1219,7 +1243,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                         const int it = itg++;
                         const int cb = it & 1;
                         if (!ptx::mbar_wait(cfull(cb), (it >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                        xpending = false;   // (the epilogue has copied the row tiles)
                         ptx::tc_fence_after();
                         const int sl = it % C::NL;
                         const uint32_t zs = ptx::smem_u32(sm + C::OFF_L + sl * C::YB);   // Z rides the late ring
@@ -1242,7 +1265,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                 volatile int dummy = 0;
                 if (M::VEC && done > 0) ptx::mbar_wait(cempty((done - 1) & 1), ((done - 1) >> 1) & 1, &dummy, a.status);
                 // no row-tile copy may still be writing this CTA's shared memory when it exits
-                if (xpending) ptx::mbar_wait(xfull, (jc - 1) & 1, &dummy, a.status);
+                if (xpending) ptx::mbar_wait(xfull, jc & 1, &dummy, a.status);
             }
         }
     } else {
@@ -1284,37 +1307,12 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         for (int k = 0; k < NMOD; ++k) xr[k] = ract ? -a.xr[k][base + r] : 0.f;
         uint64_t s1a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
         uint64_t s2a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
-        {
-                // Row tiles into TMEM as MMA A operands: warp (q, quarter 0) copies X, (q, quarter 1) A,
-                // rows 32 q .. 32 q + 31 (thread = row), from the 128-byte-swizzled TMA copies.
-                const bool copy = qt == 0 || (qt == 1 && M::HASDP);
-                bool okx = !copy || ptx::mbar_wait(xfull, jc & 1, abort_flag, a.status);
-                okx = __all_sync(0xffffffffu, okx);
-                if (okx && copy) {
-                    const uint32_t src = ptx::smem_u32(sm + C::OFF_C + (half ? C::XB : 0u)) + crow;
-                    const uint32_t dst = tbase + lane_base + (half ? C::TM_A : C::TM_X);
-#pragma unroll
-                    for (int ka = 0; ka < C::KATOMS; ++ka) {
-                        uint32_t w[32];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const uint4 u = ptx::ld_shared_u4(src + ka * C::XATOM + ((uint32_t(j) ^ uint32_t(row & 7)) << 4));
-                            w[4 * j] = u.x;
-                            w[4 * j + 1] = u.y;
-                            w[4 * j + 2] = u.z;
-                            w[4 * j + 3] = u.w;
-                        }
-                        ptx::tmem_st32(dst + uint32_t(ka * 32), w);
-                    }
-                    ptx::tmem_wait_st();
-                }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(xtm);
-            if (!okx) ok = false;
-            // every warp has read its rows of X and A before any coefficient overwrites them
-            ptx::named_bar_sync(2, 32 * kSweepEpi);
-        }
+        // (the row tiles reach TMEM by tcgen05.cp from the coefficient buffers: the first score
+        // tile of the job, which this warp waits for, completes after that copy has read them)
+        // Every epilogue warp has finished the previous job, whose scalar partials the warps of
+        // column quarter 0 read after the shared-memory exchange below, before any warp writes
+        // this job's (a job of one tile would otherwise let a fast warp overwrite them).
+        ptx::named_bar_sync(2, 32 * kSweepEpi);
         for (int tcol = jb.t_lo; tcol <= jb.t_hi; ++tcol) {
             if (!tile_bit(jb.bits, tcol)) continue;
             const int it = itg++;
