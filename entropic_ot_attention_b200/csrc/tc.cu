@@ -148,6 +148,7 @@ constexpr int kFmaPairs = 1;
 struct TcBandArgs {
     int H, L, h, D, n_items, items_per_cta, pairs_per_unit;
     float sl2;                  // scale * log2(e)
+    float isl2;                 // 1 / sl2 (column-bias operand rows)
     const float* logm;
     const uint32_t* tile_bits;  // [B][words]: bit t = positions [128 t, 128 t + 128) hold an active non-dustbin token
     int words;
@@ -196,8 +197,8 @@ struct TcBandArgs {
 // potential, as three bf16 parts (fp32 accuracy); the accumulator then holds S + y and the
 // epilogue forms the exponent with one packed FMA, acc * scale log2 e + st_r.  A column
 // that never enters a band sum (inactive, the dustbin) carries y = -2^100.
-__device__ __forceinline__ void band_ext_row(__nv_bfloat16* dst, float b2, float sl2) {
-    const float y = b2 == kNegInf ? -1.2676506e30f : b2 / sl2;   // -2^100
+__device__ __forceinline__ void band_ext_row(__nv_bfloat16* dst, float b2, float isl2) {
+    const float y = b2 == kNegInf ? -1.2676506e30f : b2 * isl2;   // isl2 = 1 / (scale log2 e); -2^100
     const __nv_bfloat16 hi = __float2bfloat16_rn(y);
     const float r1 = y - __bfloat162float(hi);
     const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
@@ -467,9 +468,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     if (EXT)
                         ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (hs & 1) ? &tmUE : &tmVE, 0,
                                          int(it.base) + c0, full(s));
+                    // (with the column bias in the product the epilogue reads no column vectors)
 #pragma unroll
                     for (int G = 0; G < 2; ++G) {
-                        if (!(G ? use1 : use0)) continue;
+                        if (EXT || !(G ? use1 : use0)) continue;
                         const int vs = gv[G] % C::NV;
                         if (!ptx::mbar_wait(vempty(G, vs), ((gv[G] / C::NV) & 1) ^ 1, abort_flag, a.status)) {
                             ok = false;
@@ -608,7 +610,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     out_hs[pb + r] = 0.f;
                     if (!WSUM) outb_hs[base + r] = kNegInf;
                 }
-                if (!WSUM && hf == 0 && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.sl2);
+                if (!WSUM && hf == 0 && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.isl2);
                 continue;
             }
             const int t_lo = max(0, rg - h) / C::BN, t_hi = min(L - 1, rg + C::BM - 1 + h) / C::BN;
@@ -731,7 +733,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 const int cc0 = c0 + hf * 64, cc1 = cc0 + 32;
                 const int k0 = block_class(cc0), k1 = block_class(cc1);
                 // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-                bool w1 = ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
+                bool w1 = EXT || ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
                 bool w2 = w1 && ptx::mbar_wait(tfull(G, tb), (gg >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
                 ptx::tc_fence_after();
@@ -756,7 +758,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     if (k1 != 0) process(v, cc1, vaddr + 128u, k1 == 2);
                 }
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(vempty(G, vs));
+                if (!EXT && lane == 0) ptx::mbar_arrive(vempty(G, vs));
             }
             // The two column halves of each row meet in shared memory (two parity slots:
             // the partner writes item e + 1 only after this warp has read item e).
@@ -794,9 +796,9 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 }
                 out_hs[pb + r] = outv;
                 if (!WSUM) outb_hs[base + r] = ob;
-                if (!WSUM && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, ob, a.sl2);
+                if (!WSUM && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, ob, a.isl2);
             } else if (!WSUM && hf == 0 && is_dustbin_row && exto_of(hs)) {
-                band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.sl2);   // the dustbin never enters a band sum
+                band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.isl2);   // the dustbin never enters a band sum
             }
         }
         if (MULTI && D >= 0 && __all_sync(0xffffffffu, ok && !*abort_flag)) {
@@ -1633,6 +1635,7 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     a.D = g.D;
     a.dself = g.dself;
     a.sl2 = g.scale * kLog2e;
+    a.isl2 = float(1.0 / double(a.sl2));
     a.words = tile_words(g.L);
     a.pairs_per_unit = (g.L / 128 + 1) / 2;
     a.n_items = g.BH * a.pairs_per_unit;
