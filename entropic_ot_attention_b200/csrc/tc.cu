@@ -232,8 +232,8 @@ struct BandCfg {
     static constexpr uint32_t VB = NVEC * BN * 4;  // column vectors of one tile
     static constexpr uint32_t OFF_Y = NQ * XB;
     static constexpr uint32_t OFF_V = OFF_Y + NS * YB;         // [half][NV][VB]
-    static constexpr uint32_t OFF_RED = OFF_V + 2 * NV * VB;    // [half][parity][m, s][128 rows]
-    static constexpr uint32_t OFF_BITS = OFF_RED + 2 * 2 * 2 * 128 * 4;   // tile bits of the CTA's batch rows
+    static constexpr uint32_t OFF_RED = OFF_V + 2 * NV * VB;    // [half][parity][column half][m, s][128 rows]
+    static constexpr uint32_t OFF_BITS = OFF_RED + 2 * 2 * 2 * 2 * 128 * 4;   // tile bits of the CTA's batch rows
     static constexpr int BITS_WORDS = 512;
     // column-bias operands (EXT): the constant row operand and one column operand per stage,
     // [128 x 16] bf16 each, 32-byte swizzled
@@ -580,7 +580,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         const int q = warp & 3;               // TMEM lane quadrant (fixed by the warp's rank)
         const int row = q * 32 + lane;
         const uint32_t lane_base = uint32_t(q * 32) << 16;
-        float* red = reinterpret_cast<float*>(sm + C::OFF_RED) + G * (2 * 2 * 128);
+        float* red = reinterpret_cast<float*>(sm + C::OFF_RED) + G * (2 * 2 * 2 * 128);
         const uint32_t vsm = ptx::smem_u32(sm + C::OFF_V + G * C::NV * C::VB);
         int gt = 0, ep = 0;
         bool ok = true;
@@ -760,27 +760,30 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 __syncwarp();
                 if (!EXT && lane == 0) ptx::mbar_arrive(vempty(G, vs));
             }
-            // The two column halves of each row meet in shared memory (two parity slots:
-            // the partner writes item e + 1 only after this warp has read item e).
-            float* rd = red + (ep & 1) * (2 * 128);
+            // The two column halves of each row meet in shared memory (two parity slots: the
+            // partner writes item e + 2 only after this warp has read item e).  Both warps form
+            // the same total (half 0's partial first), then half 0 writes the potential and its
+            // log2 copy and half 1 the column-bias operand row.
+            float* rd = red + (ep & 1) * (2 * 2 * 128);
             ++ep;
             const float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-            if (hf == 1) {
-                rd[row] = m_run;
-                rd[128 + row] = part;
-            }
+            rd[hf * 256 + row] = m_run;
+            rd[hf * 256 + 128 + row] = part;
             ptx::named_bar_sync(1 + G * 4 + q, 64);
             const bool is_dustbin_row = (r == D) && lm != kNegInf;
-            if (hf == 0 && ok && !*abort_flag && !is_dustbin_row) {
-                float mm = m_run, sum = part;
-                if (ONLINE) lse2_merge(mm, sum, rd[row], rd[128 + row]);
-                else sum += rd[128 + row];
+            const bool writes_ext = !WSUM && exto_of(hs) != nullptr;
+            if ((hf == 0 || writes_ext) && ok && !*abort_flag && !is_dustbin_row) {
+                const float m1 = rd[(1 - hf) * 256 + row], s1 = rd[(1 - hf) * 256 + 128 + row];
+                float mm = hf == 0 ? m_run : m1, sum = hf == 0 ? part : s1;
+                const float mo = hf == 0 ? m1 : m_run, so = hf == 0 ? s1 : part;
+                if (ONLINE) lse2_merge(mm, sum, mo, so);
+                else sum += so;
                 float outv = 0.f, ob = kNegInf;
                 if (lm != kNegInf) {
                     const bool d_act = D >= 0 && logm[D] != kNegInf;
                     if (ONLINE) {
                         if (d_act) lse2_add(mm, sum, (sdterm_of(hs)[base + r] + colpot_of(hs)[pb + D]) * kLog2e);
-                        outv = lm - (mm + log2f(sum)) * kLn2;
+                        outv = lm - (mm + ptx::lg2(sum)) * kLn2;
                     } else {
                         const float dterm =
                             d_act ? ptx::ex2((sdterm_of(hs)[base + r] + colpot_of(hs)[pb + D]) * kLog2e + st2) : 0.f;
@@ -788,16 +791,19 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                             if (d_act) sum = fmaf(dterm, a.colw[base + D], sum);
                             outv = a.f[base + r] * (a.hv[base + r] * sum + (a.sadd ? a.sadd[base + r] : 0.f));
                         } else {
-                            outv = lm - log2f(sum + dterm) * kLn2 + st;
+                            outv = lm - ptx::lg2(sum + dterm) * kLn2 + st;
                         }
                     }
-                    if (!isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
+                    if (hf == 0 && !isfinite(outv)) atomicOr(a.status, kStatusNonFinite);
                     ob = outv * kLog2e;
                 }
-                out_hs[pb + r] = outv;
-                if (!WSUM) outb_hs[base + r] = ob;
-                if (!WSUM && exto_of(hs)) band_ext_row(exto_of(hs) + (base + r) * 16, ob, a.isl2);
-            } else if (!WSUM && hf == 0 && is_dustbin_row && exto_of(hs)) {
+                if (hf == 0) {
+                    out_hs[pb + r] = outv;
+                    if (!WSUM) outb_hs[base + r] = ob;
+                } else {
+                    band_ext_row(exto_of(hs) + (base + r) * 16, ob, a.isl2);
+                }
+            } else if (writes_ext && hf == 1 && is_dustbin_row) {
                 band_ext_row(exto_of(hs) + (base + r) * 16, kNegInf, a.isl2);   // the dustbin never enters a band sum
             }
         }
