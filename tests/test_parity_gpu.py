@@ -58,6 +58,14 @@ SMALL = {
                                                          name="fp32_dustbin"),
     "bf16_d128_dustbin": lambda: eot_inputs.dustbin_case(1, 2, 250, 128, 90, 5, 2, "bf16", seed=13, mass=0.1,
                                                          name="bf16_d128_dustbin"),
+    # d = 128 with W >= 512: the fused half-steps take the column bias from the score product,
+    # so masked columns and the dustbin run through its -2^100 operand rows
+    "bf16_d128_W512_ragged_L896": lambda: eot_inputs.dense_case(2, 2, 896, 128, 512, 5, 2, "bf16", seed=22,
+                                                                mask=_ragged_mask(2, 896, 22),
+                                                                name="bf16_d128_W512_ragged"),
+    "bf16_d128_W600_dustbin": lambda: eot_inputs.dustbin_case(1, 2, 700, 128, 600, 4, 2, "bf16", seed=23, mass=0.1,
+                                                              mask=_ragged_mask(1, 700, 23),
+                                                              name="bf16_d128_W600_dustbin"),
 }
 
 
