@@ -123,7 +123,9 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 //                per-MMA bookkeeping for both halves was slower than the tensor core.
 //   warp 3       idle (it completes the first warpgroup)
 //   warps 4..11  epilogue of the first half, warps 12..19 of the second: warp (q, hf) reads
-//                TMEM lanes [32 q, 32 q + 32) and columns [64 hf, 64 hf + 64) of each tile
+//                TMEM lanes [32 q, 32 q + 32) of every other tile of its half (tiles whose
+//                running index has parity hf, i.e. the tiles of TMEM buffer hf), all 128 columns,
+//                so that a warp's per-tile waits and hand-backs are paid once per 128 columns
 // Registers: the block is launched at 96 a thread; warpgroup 0 (warps 0-3) gives registers
 // back (setmaxnreg 48) and the four epilogue warpgroups take them (104), so the epilogue's
 // chain of score, exponential and sums keeps more values live (long workload, forward: 5.61 ->
@@ -387,8 +389,10 @@ __global__ void __launch_bounds__(kBandThreads, 1)
         for (int i = 0; i < C::NS; ++i) { ptx::mbar_init(full(i), 1); ptx::mbar_init(empty(i), 2); }
         for (int i = 0; i < C::NQ; ++i) { ptx::mbar_init(qfull(i), 1); ptx::mbar_init(qempty(i), 1); }
         for (int G = 0; G < 2; ++G) {
-            for (int i = 0; i < 2; ++i) { ptx::mbar_init(tfull(G, i), 1); ptx::mbar_init(tempty(G, i), 8); }
-            for (int i = 0; i < C::NV; ++i) { ptx::mbar_init(vfull(G, i), 1); ptx::mbar_init(vempty(G, i), 8); }
+            // a score buffer and a column-vector slot are read by the four quadrant warps of one
+            // column half (tiles alternate between the halves)
+            for (int i = 0; i < 2; ++i) { ptx::mbar_init(tfull(G, i), 1); ptx::mbar_init(tempty(G, i), 4); }
+            for (int i = 0; i < C::NV; ++i) { ptx::mbar_init(vfull(G, i), 1); ptx::mbar_init(vempty(G, i), 4); }
         }
         ptx::mbar_fence_init();
     }
@@ -727,35 +731,40 @@ __global__ void __launch_bounds__(kBandThreads, 1)
             for (int t = t_lo; t <= t_hi; ++t) {
                 if (!bits(t)) continue;
                 const int gg = gt++;
-                if (!ok) continue;
+                // the two column-half warps of a quadrant take alternate tiles (the tile's parity
+                // is also its TMEM buffer), all 128 columns each
+                if ((gg & 1) != hf || !ok) continue;
                 const int c0 = t * C::BN;
                 const int tb = gg & 1, vs = gg % C::NV;
-                const int cc0 = c0 + hf * 64, cc1 = cc0 + 32;
-                const int k0 = block_class(cc0), k1 = block_class(cc1);
                 // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
                 bool w1 = EXT || ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
                 bool w2 = w1 && ptx::mbar_wait(tfull(G, tb), (gg >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
                 ptx::tc_fence_after();
-                const uint32_t vaddr = vsm + uint32_t(vs) * C::VB + uint32_t(hf) * 256u;
-                const uint32_t tcol = tbase + lane_base + uint32_t((G * 2 + tb) * C::BN + hf * 64);
-                if (k0 != 0) {
+                const uint32_t vaddr = vsm + uint32_t(vs) * C::VB;
+                const uint32_t tcol = tbase + lane_base + uint32_t((G * 2 + tb) * C::BN);
+                int last_k = -1;   // the last 32-column chunk with a score read
+                for (int k = 0; k < 4; ++k)
+                    if (block_class(c0 + 32 * k) != 0) last_k = k;
+#pragma unroll 1
+                for (int k = 0; k < 4; ++k) {
+                    const int cc = c0 + 32 * k, kc = block_class(cc);
+                    if (kc == 0) continue;
                     float v[32];
-                    ptx::tmem_ld32(tcol, v);
+                    ptx::tmem_ld32(tcol + uint32_t(32 * k), v);
                     ptx::tmem_wait_ld(v);
-                    process(v, cc0, vaddr, k0 == 2);
-                }
-                {
-                    float v[32];
-                    if (k1 != 0) {
-                        ptx::tmem_ld32(tcol + 32, v);
-                        ptx::tmem_wait_ld(v);
+                    if (k == last_k) {
+                        // this warp's part of the accumulator is read: hand it back
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(tempty(G, tb));
                     }
-                    // this warp's part of the accumulator is read: hand it back
+                    process(v, cc, vaddr + 128u * uint32_t(k), kc == 2);
+                }
+                if (last_k < 0) {
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(tempty(G, tb));
-                    if (k1 != 0) process(v, cc1, vaddr + 128u, k1 == 2);
                 }
                 __syncwarp();
                 if (!EXT && lane == 0) ptx::mbar_arrive(vempty(G, vs));
