@@ -422,6 +422,10 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     va.hv = at<float>(ws, w.hv);
     va.m = at<float>(ws, w.m);
     va.xr = R > 0 ? at<float>(ws, w.xr) : nullptr;
+    // band sums of a wide d = 128 band on the tensor cores take their column bias as operand rows
+    __nv_bfloat16* cext = (impl == EOT_IMPL_TCGEN05 && w.bcext) ? at<__nv_bfloat16>(ws, w.cext) : nullptr;
+    va.cext = cext;
+    va.isl2 = float(1.0 / double(g.scale * kLog2e));
     va.yc = R > 0 ? at<float>(ws, w.yc) : nullptr;
 
     // Row orientation: S = Q K^T, dP = dO V^T.  Column orientation: S^T = K Q^T, dP^T = V dO^T.
@@ -525,6 +529,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
             bp.m = va.m;
             bp.s_dp = 0;
             bp.sadd = at<float>(ws, w.sadd);
+            bp.cext = cext;
             EOT_TRY(run_bwd(impl, bp, st, kProfStair));
         } else {
             BwdPass bp = rowp;
@@ -557,6 +562,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
                 bp.hv = va.hv;
                 bp.m = va.m;
                 bp.s_dp = 0;
+                bp.cext = cext;
                 EOT_TRY(run_bwd(impl, bp, st, kProfStair));
             }
             EOT_TRY(vec(kPassRk, k));
@@ -570,6 +576,7 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
                 bp.hv = va.hv;
                 bp.m = va.m;
                 bp.s_dp = 0;
+                bp.cext = cext;
                 EOT_TRY(run_bwd(impl, bp, st, kProfStair));
             }
         }

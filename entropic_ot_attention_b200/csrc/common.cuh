@@ -98,6 +98,9 @@ struct BwdPass {
     size_t s1stride;
     int s1E;
     const float* sadd;      // staircase-form sweeps: out_r = f_r (hv_r sum_c ... + sadd_r), or nullptr
+    // staircase-form sweeps on the tensor cores (d = 128, W >= 512): the column-bias operand rows
+    // of this pass's column bias pcm2 ([BH L, 16] bf16, see band_ext_row), or nullptr
+    const __nv_bfloat16* cext;
     // dQ / dK (tensor-core kernels, no dustbin): the modifiers as [BH L, 16] bf16 operand rows
     // (xext row side, yext column side; see BwdVecArgs) to fold into the dP product, or nullptr
     const __nv_bfloat16* xext;
@@ -129,6 +132,8 @@ struct WsLayout {
     bool fold;
     size_t ue, ve;          // forward, fused d = 128 half-steps: column-bias operand rows [BH L, 16] bf16 of u and v
     bool bext;
+    size_t cext;            // backward, band sums of wide d = 128 bands: column-bias operand rows [BH L, 16] bf16
+    bool bcext;
     size_t total;
 };
 
@@ -233,6 +238,10 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
             w.s1part = o; o += s1_slots(p.W) * vec;
             w.sadd = o; o += vec;
         }
+        if (p.dtype == EOT_BF16 && p.d == 128 && p.impl != EOT_IMPL_SIMT && p.L % 128 == 0 && p.W / 2 >= 256) {
+            w.bcext = true;
+            w.cext = o; o += align256(BH * L * 32);
+        }
         if (fold_possible(p)) {
             w.fold = true;
             w.xext = o; o += align256(BH * L * 32);
@@ -253,6 +262,35 @@ template <> __device__ __forceinline__ float from_f<float>(float x) { return x; 
 template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+// The column bias enters the score product of the band kernel (d = 128, wide bands: fused
+// half-steps and weighted band sums): one more K = 16 step
+// multiplies a constant row operand (1, 1, 1, 0, ...) with a column operand row
+// (y_hi, y_mid, y_lo, 0, ...) carrying y = b_c / (scale log2 e), b_c the column's masked log2
+// potential, as three bf16 parts (fp32 accuracy); the accumulator then holds S + y and the
+// epilogue forms the exponent with one packed FMA, acc * scale log2 e + st_r.  A column
+// that never enters a band sum (inactive, the dustbin) carries y = -2^100.
+__device__ __forceinline__ void band_ext_row(__nv_bfloat16* dst, float b2, float isl2) {
+    const float y = b2 == neg_inf() ? -1.2676506e30f : b2 * isl2;   // isl2 = 1 / (scale log2 e); -2^100
+    const __nv_bfloat16 hi = __float2bfloat16_rn(y);
+    const float r1 = y - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    __nv_bfloat162 p0, p1;
+    p0.x = hi;
+    p0.y = mid;
+    p1.x = lo;
+    p1.y = __float2bfloat16_rn(0.f);
+    uint4 w0;
+    w0.x = *reinterpret_cast<const uint32_t*>(&p0);
+    w0.y = *reinterpret_cast<const uint32_t*>(&p1);
+    w0.z = 0u;
+    w0.w = 0u;
+    uint4* d = reinterpret_cast<uint4*>(dst);
+    d[0] = w0;
+    d[1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 
 // Merge two (max, sum) log-sum-exp partials in the log2 domain.
 __device__ __forceinline__ void lse2_merge(float& m, float& s, float m2, float s2) {

@@ -31,6 +31,10 @@ struct BwdVecArgs {
     // (bf16 parts), so <xext_r, yext_c> = -sum_k xr_k[r] yc_k[c] up to the lo x lo products.
     __nv_bfloat16* xext;
     __nv_bfloat16* yext;
+    // band-sum passes (kPassR2, kPassCk, kPassRk) of wide d = 128 bands: the column-bias operand
+    // row of pcm2 for every position (band_ext_row with 1 / (scale log2 e) = isl2), or nullptr
+    __nv_bfloat16* cext;
+    float isl2;
 };
 
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,

@@ -626,6 +626,8 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
     if (a.f) a.f[idx] = f;
     if (a.hv) a.hv[idx] = hv;
     if (a.m) a.m[idx] = m;
+    if (a.cext && (a.kind == kPassR2 || a.kind == kPassCk || a.kind == kPassRk))
+        band_ext_row(a.cext + idx * 16, (act && i != a.D) ? pc * kLog2e : neg_inf(), a.isl2);
     if (a.kind == kPassR2 && a.s1part && a.sadd) {
         float t = 0.f;
         if (act)

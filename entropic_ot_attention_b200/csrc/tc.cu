@@ -193,40 +193,15 @@ struct TcBandArgs {
     __nv_bfloat16* ve;
 };
 
-// The column bias enters the fused half-steps' score product (d = 128): one more K = 16 step
-// multiplies a constant row operand (1, 1, 1, 0, ...) with a column operand row
-// (y_hi, y_mid, y_lo, 0, ...) carrying y = b_c / (scale log2 e), b_c the column's masked log2
-// potential, as three bf16 parts (fp32 accuracy); the accumulator then holds S + y and the
-// epilogue forms the exponent with one packed FMA, acc * scale log2 e + st_r.  A column
-// that never enters a band sum (inactive, the dustbin) carries y = -2^100.
-__device__ __forceinline__ void band_ext_row(__nv_bfloat16* dst, float b2, float isl2) {
-    const float y = b2 == kNegInf ? -1.2676506e30f : b2 * isl2;   // isl2 = 1 / (scale log2 e); -2^100
-    const __nv_bfloat16 hi = __float2bfloat16_rn(y);
-    const float r1 = y - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    __nv_bfloat162 p0, p1;
-    p0.x = hi;
-    p0.y = mid;
-    p1.x = lo;
-    p1.y = __float2bfloat16_rn(0.f);
-    uint4 w0;
-    w0.x = *reinterpret_cast<const uint32_t*>(&p0);
-    w0.y = *reinterpret_cast<const uint32_t*>(&p1);
-    w0.z = 0u;
-    w0.w = 0u;
-    uint4* d = reinterpret_cast<uint4*>(dst);
-    d[0] = w0;
-    d[1] = make_uint4(0u, 0u, 0u, 0u);
-}
-
 template <int DH, int KIND, bool EXT = false>
 struct BandCfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int KATOMS = DH / 64;
     static constexpr int NQ = DH == 128 ? 3 : 6;   // row half-tile slots
     static constexpr int NS = DH == 128 ? 3 : 6;   // column-tile stages
-    static constexpr int NV = 4;                   // column-vector slots per half
+    // column-vector slots per half (3 for the weighted sums with the bias in the product, whose
+    // operand tiles take the room of the fourth)
+    static constexpr int NV = (EXT && KIND == kBandWsum) ? 3 : 4;
     static constexpr int NVEC = KIND == kBandWsum ? 2 : 1;
     static constexpr uint32_t XB = BM * DH * 2;    // row half-tile bytes
     static constexpr uint32_t YB = BN * DH * 2;    // column tile bytes
@@ -249,6 +224,7 @@ struct BandCfg {
     static constexpr uint32_t NBARS = HB0 + 2 * HBN;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr size_t SMEM = 1024 + OFF_MISC + 64;
+    static_assert(SMEM <= 227 * 1024, "band kernel shared memory");
     static constexpr uint32_t IDESC = ptx::idesc_bf16(128, 128, false, false);
 };
 
@@ -292,9 +268,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     tc_band_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
                    const __grid_constant__ CUtensorMap tmUE, const __grid_constant__ CUtensorMap tmVE,
                    const TcBandArgs a) {
-    static_assert(!EXT || (MULTI && DH == 128 && KIND == kBandShift), "the folded column bias is a fused d = 128 form");
+    static_assert(!EXT || (DH == 128 && ((MULTI && KIND == kBandShift) || (!MULTI && KIND == kBandWsum))),
+                  "the folded column bias is a d = 128 form of the fused half-steps and of the weighted sums");
     using C = BandCfg<DH, KIND, EXT>;
     constexpr bool ONLINE = KIND == kBandOnline, WSUM = KIND == kBandWsum;
+    // column vectors: none with the bias in the product, except the weights of a weighted sum
+    constexpr bool NOVEC = EXT && !WSUM;
     static_assert(!MULTI || KIND == kBandShift, "fused half-steps are shifted log-sum-exp sweeps");
     // Operands of half-step hs (a single launch uses the fixed pointers of a).
     const int hs_end = a.hs0 + a.nhs;
@@ -460,7 +439,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                             // the stage still expects its column-bias operand: fill it so that
                             // no copy is left pending when the CTA retires
                             if (EXT)
-                                ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (hs & 1) ? &tmUE : &tmVE, 0,
+                                ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (MULTI && !(hs & 1)) ? &tmVE : &tmUE, 0,
                                                  int(it.base) + c0, full(s));
                             ok = false;
                             break;
@@ -470,12 +449,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     }
                     // the column-bias operand rows of half-step hs were written in half-step hs - 1
                     if (EXT)
-                        ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (hs & 1) ? &tmUE : &tmVE, 0,
+                        ptx::tma_load_2d(ptx::smem_u32(sm + C::OFF_YE + s * C::EXTB), (MULTI && !(hs & 1)) ? &tmVE : &tmUE, 0,
                                          int(it.base) + c0, full(s));
                     // (with the column bias in the product the epilogue reads no column vectors)
 #pragma unroll
                     for (int G = 0; G < 2; ++G) {
-                        if (EXT || !(G ? use1 : use0)) continue;
+                        if (NOVEC || !(G ? use1 : use0)) continue;
                         const int vs = gv[G] % C::NV;
                         if (!ptx::mbar_wait(vempty(G, vs), ((gv[G] / C::NV) & 1) ^ 1, abort_flag, a.status)) {
                             ok = false;
@@ -670,10 +649,12 @@ __global__ void __launch_bounds__(kBandThreads, 1)
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4) {
                             const float4 wv = ptx::ld_shared_f4(vaddr + 4u * C::BN + 16u * j4);
-                            acc[0] = fmaf(ptx::ex2(x[4 * j4 + 0] + st2), wv.x, acc[0]);
-                            acc[1] = fmaf(ptx::ex2(x[4 * j4 + 1] + st2), wv.y, acc[1]);
-                            acc[2] = fmaf(ptx::ex2(x[4 * j4 + 2] + st2), wv.z, acc[2]);
-                            acc[3] = fmaf(ptx::ex2(x[4 * j4 + 3] + st2), wv.w, acc[3]);
+                            // (with the bias in the product, x already holds the shift)
+                            const float sh = EXT ? 0.f : st2;
+                            acc[0] = fmaf(ptx::ex2(x[4 * j4 + 0] + sh), wv.x, acc[0]);
+                            acc[1] = fmaf(ptx::ex2(x[4 * j4 + 1] + sh), wv.y, acc[1]);
+                            acc[2] = fmaf(ptx::ex2(x[4 * j4 + 2] + sh), wv.z, acc[2]);
+                            acc[3] = fmaf(ptx::ex2(x[4 * j4 + 3] + sh), wv.w, acc[3]);
                         }
                     } else {
 #pragma unroll
@@ -737,7 +718,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                 const int c0 = t * C::BN;
                 const int tb = gg & 1, vs = gg % C::NV;
                 // Waits are made warp-uniform: the tcgen05.ld below is a warp-collective (.aligned).
-                bool w1 = EXT || ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
+                bool w1 = NOVEC || ptx::mbar_wait(vfull(G, vs), (gg / C::NV) & 1, abort_flag, a.status);
                 bool w2 = w1 && ptx::mbar_wait(tfull(G, tb), (gg >> 1) & 1, abort_flag, a.status);
                 if (!__all_sync(0xffffffffu, w2)) { ok = false; continue; }
                 ptx::tc_fence_after();
@@ -767,7 +748,7 @@ __global__ void __launch_bounds__(kBandThreads, 1)
                     if (lane == 0) ptx::mbar_arrive(tempty(G, tb));
                 }
                 __syncwarp();
-                if (!EXT && lane == 0) ptx::mbar_arrive(vempty(G, vs));
+                if (!NOVEC && lane == 0) ptx::mbar_arrive(vempty(G, vs));
             }
             // The two column halves of each row meet in shared memory (two parity slots: the
             // partner writes item e + 2 only after this warp has read item e).  Both warps form
@@ -1639,8 +1620,12 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     // fused d = 128 half-steps read the column-bias operand rows of both sides
     CUtensorMap tmUE = tmX, tmVE = tmX;
     const bool ext = multi && g.d == 128 && g.h >= 256 && a.ue && a.ve;
+    // a weighted band sum of a wide d = 128 band with its column bias as operand rows (in ue)
+    const bool wext = !multi && kind == kBandWsum && g.d == 128 && g.h >= 256 && a.ue;
     if (ext) {
         if (!make_map_ext(&tmUE, a.ue, rows, 128) || !make_map_ext(&tmVE, a.ve, rows, 128)) return cudaErrorInvalidValue;
+    } else if (wext) {
+        if (!make_map_ext(&tmUE, a.ue, rows, 128)) return cudaErrorInvalidValue;
     } else if (multi) {
         a.ue = a.ve = nullptr;   // (no operand rows written either)
     }
@@ -1672,7 +1657,9 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
         switch (kind) {
             case kBandOnline: return launch_band_variant<128, kBandOnline, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
             case kBandShift: return launch_band_variant<128, kBandShift, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
-            case kBandWsum: return launch_band_variant<128, kBandWsum, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
+            case kBandWsum:
+                return wext ? launch_band_variant<128, kBandWsum, false, true>(tmX, tmY, tmUE, tmVE, a, grid_used, st)
+                            : launch_band_variant<128, kBandWsum, false>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
         }
     } else {
         if (multi) return launch_band_variant<64, kBandShift, true>(tmX, tmY, tmUE, tmVE, a, grid_used, st);
@@ -1791,6 +1778,7 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
         a.sd_term = p.sd_term;
         a.status = p.status;
         a.sadd = p.sadd;
+        a.ue = const_cast<__nv_bfloat16*>(p.cext);   // read only (the column-bias operand rows)
         cudaError_t e = launch_band(g, p.X, p.Y, a, kBandWsum, st);
         if (e != cudaSuccess || g.D < 0) return e;
         return launch_dustbin_bwd(p, st);
