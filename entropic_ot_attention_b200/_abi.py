@@ -66,6 +66,8 @@ lib.eot_sinkhorn_fwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz
 lib.eot_sinkhorn_fwd.restype = ctypes.c_int
 lib.eot_sinkhorn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.eot_sinkhorn_bwd.restype = ctypes.c_int
+lib.eot_band_half_step.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.eot_band_half_step.restype = ctypes.c_int
 lib.eot_last_device_status.argtypes = [_vp, _vp]
 lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -182,6 +184,13 @@ def eot_sinkhorn_bwd(p: eot_problem, Q: int, K: int, V: int, mask: int | None, u
     """Backward; raw device addresses as in eot_sinkhorn_fwd."""
     _check(lib.eot_sinkhorn_bwd(ctypes.byref(p), Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
                                 workspace_bytes, stream), "eot_sinkhorn_bwd")
+
+
+def eot_band_half_step(p: eot_problem, X: int, Y: int, log_marg: int, pot_in: int, pot_out: int,
+                       workspace: int, workspace_bytes: int, stream: int) -> None:
+    """One band half-step; raw device addresses as in eot_sinkhorn_fwd."""
+    _check(lib.eot_band_half_step(ctypes.byref(p), X, Y, log_marg, pot_in, pot_out, workspace, workspace_bytes,
+                                  stream), "eot_band_half_step")
 
 
 def eot_sinkhorn_fwd_static(p: eot_problem, Q: int, K: int, V: int, mask: int | None, O: int, u_tail: int,

@@ -81,6 +81,32 @@ def sinkhorn_fwd(q, k, v, W: int, T: int, R: int, mask=None, scale=None, dustbin
     return O, ut, vt
 
 
+def band_half_step(x, y, log_marg, pot_in, W: int, scale=None, impl: str = "auto", stream=None,
+                   ws: torch.Tensor | None = None):
+    """One band half-step (no dustbin): out[b,h,i] = log_marg[b,i] - LSE_{|i-j| <= W/2, active j}
+    (scale <x_i, y_j> + pot_in[b,h,j]), 0 at inactive positions.  x, y [B,H,L,d] (fp32 or bf16,
+    L a multiple of 128), log_marg [B,L] fp32 (-inf = inactive), pot_in [B,H,L] fp32.  Returns
+    out [B,H,L] fp32.  Row half-step: x = q, y = k, pot_in = v; column half-step: x = k, y = q,
+    pot_in = u."""
+    if x.shape != y.shape or x.dim() != 4 or x.dtype != y.dtype:
+        raise ValueError("x and y must be [B,H,L,d] tensors of one dtype")
+    B, H, L, d = x.shape
+    if log_marg.shape != (B, L) or log_marg.dtype != torch.float32:
+        raise ValueError("log_marg must be a float32 [B, L] tensor")
+    if pot_in.shape != (B, H, L) or pot_in.dtype != torch.float32:
+        raise ValueError("pot_in must be a float32 [B, H, L] tensor")
+    for t in (x, y, log_marg, pot_in):
+        if not t.is_contiguous() or t.device != x.device:
+            raise ValueError("inputs must be contiguous and on one device")
+    p = make_problem(B, H, L, d, W, 0, 0, x.dtype, scale, impl=impl)
+    out = torch.empty((B, H, L), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = workspace(p, False, x.device)
+    _abi.eot_band_half_step(p, x.data_ptr(), y.data_ptr(), log_marg.data_ptr(), pot_in.data_ptr(), out.data_ptr(),
+                            ws.data_ptr(), ws.numel(), _stream(stream))
+    return out
+
+
 def sinkhorn_bwd(q, k, v, u_tail, v_tail, dO, W: int, mask=None, scale=None, dustbin_index=None,
                  dustbin_mass: float = 0.0, dustbin_self: bool = True, impl: str = "auto", stream=None,
                  ws: torch.Tensor | None = None):

@@ -376,6 +376,39 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     return EOT_OK;
 }
 
+// One half-step on its own (§2.1): out = log_marg - LSE over the band of (scale <x_i, y_j> + in_j),
+// with a running maximum (the online form of the first half-step of a solve), so that any finite
+// input potential is accepted.
+eot_status half_step_impl(const eot_problem* p, const void* X, const void* Y, const float* log_marg,
+                          const float* in, float* out, void* ws, cudaStream_t st) {
+    EOT_RANGE("eot band half-step");
+    const Geom g = make_geom(*p);
+    const int impl = resolve_impl(*p);
+    const WsLayout w = ws_layout(*p, false);
+    uint32_t* status = at<uint32_t>(ws, w.status);
+    EOT_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+    float* in_b2 = at<float>(ws, w.vb2);
+    float* out_b2 = at<float>(ws, w.ub2);
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
+    EOT_TRY(aux(st, [&] { return launch_init_bias2(g, log_marg, in_b2, st, in); }));
+    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, log_marg, tbits, st); }));
+    LsePass lp{};
+    lp.g = g;
+    lp.X = X;
+    lp.Y = Y;
+    lp.logm = log_marg;
+    lp.colpot = in;
+    lp.stab = nullptr;
+    lp.out = out;
+    lp.pstride = size_t(p->L);
+    lp.colbias2 = in_b2;
+    lp.out_bias2 = out_b2;
+    lp.tile_bits = tbits;
+    lp.status = status;
+    EOT_TRY(run_lse(impl, lp, st));
+    return EOT_OK;
+}
+
 eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const uint8_t* mask,
                          const float* u_tail, const float* v_tail, const void* dO, void* dQ, void* dK, void* dV,
                          void* ws, cudaStream_t st) {
@@ -667,6 +700,18 @@ eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, 
     if (workspace_bytes < ws_layout(*p, true).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
     return backward_impl(p, Q, K, V, mask, u_tail, v_tail, dO, dQ, dK, dV, workspace,
                          static_cast<cudaStream_t>(stream));
+}
+
+eot_status eot_band_half_step(const eot_problem* p, const void* X, const void* Y, const float* log_marg,
+                              const float* in, float* out, void* workspace, size_t workspace_bytes, void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (p->dustbin) return EOT_ERR_UNSUPPORTED;
+    if (empty(*p)) return EOT_OK;
+    if (!X || !Y || !log_marg || !in || !out || !workspace) return EOT_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
+    return half_step_impl(p, X, Y, log_marg, in, out, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int eot_solve_exp_passes(const eot_problem* p) {

@@ -53,7 +53,9 @@ cudaError_t launch_simt_resident(const LsePass& row, const void* Q, const void* 
                                  int R, cudaStream_t st);
 cudaError_t launch_simt_bwd(const BwdPass& p, cudaStream_t st);
 cudaError_t launch_bwd_vectors(const BwdVecArgs& a, cudaStream_t st);
-cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st);
+// bias2 = log2(e) * pot over the active positions (pot null: a zero potential), -inf elsewhere
+cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st,
+                              const float* pot = nullptr);
 cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, cudaStream_t st);
 cudaError_t launch_sq_norms(const void* a, const void* b, size_t n, int dtype, double* out, int n_sm,
                             cudaStream_t st);

@@ -897,12 +897,14 @@ cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st) {
 }
 
 // Masked log2 bias of the zero potential: 0 for active non-dustbin positions, -inf else.
-__global__ void __launch_bounds__(256) init_bias2_kernel(Geom g, const float* logm, float* bias2) {
+// log2(e) * pot (0 when pot is null), -inf for inactive positions and the dustbin.
+__global__ void __launch_bounds__(256) init_bias2_kernel(Geom g, const float* logm, const float* pot, float* bias2) {
     const int bh = blockIdx.y, b = bh / g.H;
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= g.L) return;
     const bool act = logm[size_t(b) * g.L + i] != neg_inf() && i != g.D;
-    bias2[size_t(bh) * g.L + i] = act ? 0.f : neg_inf();
+    const size_t o = size_t(bh) * g.L + i;
+    bias2[o] = act ? (pot ? pot[o] * kLog2e : 0.f) : neg_inf();
 }
 
 // Bit t of word w of batch row b: positions [128 t, 128 t + 128) hold an active token other
@@ -1117,9 +1119,9 @@ cudaError_t launch_tile_bits(const Geom& g, const float* logm, uint32_t* bits, c
     return cudaGetLastError();
 }
 
-cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st) {
+cudaError_t launch_init_bias2(const Geom& g, const float* logm, float* bias2, cudaStream_t st, const float* pot) {
     dim3 grid((g.L + 255) / 256, g.BH);
-    init_bias2_kernel<<<grid, 256, 0, st>>>(g, logm, bias2);
+    init_bias2_kernel<<<grid, 256, 0, st>>>(g, logm, pot, bias2);
     return cudaGetLastError();
 }
 

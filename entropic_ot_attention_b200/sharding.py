@@ -121,6 +121,44 @@ def allreduce_lse(m: torch.Tensor, s: torch.Tensor, group=None) -> tuple[torch.T
     return M, scaled
 
 
+def device_half_steps(sh: Shard, q_halo: torch.Tensor, k_halo: torch.Tensor, log_marg_halo: torch.Tensor,
+                      W: int, scale: float | None = None, impl: str = "auto"):
+    """``(row_step, col_step)`` for ``sharded_solve`` that run each half-step of this rank's part
+    as one ``eot_band_half_step`` call on the device holding ``q_halo``.
+
+    q_halo, k_halo: [c1 - c0, d] rows of the halo range (float32 or bfloat16, on a CUDA device);
+    log_marg_halo: [c1 - c0] the whole problem's log marginals over the halo range (-inf =
+    inactive).  The range is padded to whole 128-position tiles with inactive positions, which no
+    band sum reads.  The steps take and return potentials in the caller's dtype and device (the
+    device computes in float32); positions of the halo outside [r0, r1) come out truncated and
+    are not returned."""
+    from .api import band_half_step, make_problem, workspace   # needs the built library
+
+    n = sh.c1 - sh.c0
+    if q_halo.shape != k_halo.shape or q_halo.shape[0] != n or log_marg_halo.shape != (n,):
+        raise ValueError("q_halo, k_halo [c1 - c0, d] and log_marg_halo [c1 - c0] expected")
+    Lp = (n + 127) // 128 * 128
+    dev = q_halo.device
+
+    def pad(x):
+        out = torch.zeros((1, 1, Lp, x.shape[1]), dtype=x.dtype, device=dev)
+        out[0, 0, :n] = x
+        return out
+
+    q, k = pad(q_halo), pad(k_halo)
+    lm = torch.full((1, Lp), float("-inf"), dtype=torch.float32, device=dev)
+    lm[0, :n] = log_marg_halo.to(device=dev, dtype=torch.float32)
+    ws = workspace(make_problem(1, 1, Lp, q.shape[-1], W, 0, 0, q.dtype, scale, impl=impl), False, dev)
+
+    def step(x, y, pot_halo):
+        pin = torch.zeros((1, 1, Lp), dtype=torch.float32, device=dev)
+        pin[0, 0, :n] = pot_halo.to(device=dev, dtype=torch.float32)
+        out = band_half_step(x, y, lm, pin, W, scale, impl, ws=ws)
+        return out[0, 0, sh.owned].to(device=pot_halo.device, dtype=pot_halo.dtype)
+
+    return (lambda v_halo: step(q, k, v_halo)), (lambda u_halo: step(k, q, u_halo))
+
+
 def sharded_solve(plan: list[Shard], rank: int, T: int, R: int,
                   row_step: Callable[[torch.Tensor], torch.Tensor],
                   col_step: Callable[[torch.Tensor], torch.Tensor],

@@ -121,6 +121,34 @@ eot_status eot_sinkhorn_bwd(const eot_problem* p, const void* Q, const void* K, 
                             const void* dO, void* dQ, void* dK, void* dV, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/*
+ * One half-step of the band iteration (§2.1) on its own: the step each rank takes when one
+ * unit's sequence is split over several devices (each part updates its own positions from the
+ * potentials over its halo, and the parts exchange their boundary values between half-steps).
+ * For every unit (b, h) and every position i with log_marg[b, i] > -inf:
+ *     out[b, h, i] = log_marg[b, i]
+ *                    - log sum_{j : |i - j| <= W / 2, log_marg[b, j] > -inf}
+ *                          exp( scale * <X[b, h, i], Y[b, h, j]> + in[b, h, j] )
+ * and out[b, h, i] = 0 where log_marg[b, i] = -inf.  A row half-step (u from v) passes X = Q,
+ * Y = K, in = v; a column half-step (v from u) passes X = K, Y = Q, in = u.  The sum keeps a
+ * running maximum, so any finite input potential is accepted.  Device pointers:
+ *   X, Y      [B, H, L, d] p->dtype, read only.
+ *   log_marg  [B, L] float32 log marginals, -inf for positions outside the problem (inactive
+ *             tokens, padding).  A part of a longer sequence passes the whole problem's
+ *             marginals over its positions (they depend on the whole sequence's active count).
+ *   in        [B, H, L] float32, read only (ignored where log_marg is -inf).
+ *   out       [B, H, L] float32, written.
+ *   workspace eot_workspace_bytes(p, 0) bytes, 256-byte aligned, device, contents clobbered.
+ * p->T and p->R are not used.  Errors, all returned before anything is launched except the
+ * last: EOT_ERR_INVALID_ARGUMENT (invalid *p, a NULL pointer, a misaligned workspace),
+ * EOT_ERR_UNSUPPORTED (p->dustbin = 1: the dustbin's dense row and column sum over every
+ * position, which a part cannot form alone), EOT_ERR_WORKSPACE_TOO_SMALL, EOT_ERR_CUDA.
+ * Asynchronous on ``stream``; the device status word is read with eot_last_device_status.
+ */
+eot_status eot_band_half_step(const eot_problem* p, const void* X, const void* Y, const float* log_marg,
+                              const float* in, float* out, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Synchronises ``stream``, reads the device status word that the last fwd/bwd call on this
  * workspace left, clears it, and returns EOT_OK, EOT_ERR_NONFINITE or EOT_ERR_TIMEOUT
  * (EOT_ERR_CUDA if the copy fails). */

@@ -115,6 +115,26 @@ def test_host_errors_launch_nothing(abi):
     assert lib.eot_sinkhorn_fwd(None, None, None, None, None, None, None, None, None, 0, None) == 1
 
 
+def test_half_step_host_errors_launch_nothing(abi):
+    lib, fake = abi.lib, 1 << 20
+    p = _prob(abi)
+    ws_bytes = abi.eot_workspace_bytes(p, False)
+    assert lib.eot_band_half_step(ctypes.byref(p), None, fake, fake, fake, fake, fake, ws_bytes, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT                                  # null X
+    assert lib.eot_band_half_step(ctypes.byref(p), fake, fake, fake, fake, fake, fake, ws_bytes - 1, None) \
+        == abi.EOT_ERR_WORKSPACE_TOO_SMALL
+    assert lib.eot_band_half_step(ctypes.byref(p), fake, fake, fake, fake, fake, fake + 8, ws_bytes, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT                                  # misaligned workspace
+    db = _prob(abi, dustbin=1, dustbin_index=5, dustbin_mass=0.1)
+    assert lib.eot_band_half_step(ctypes.byref(db), fake, fake, fake, fake, fake, fake, 1 << 30, None) \
+        == abi.EOT_ERR_UNSUPPORTED                                       # the dustbin needs every position
+    bad = _prob(abi, L=100)
+    assert lib.eot_band_half_step(ctypes.byref(bad), fake, fake, fake, fake, fake, fake, 1 << 30, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT
+    empty = _prob(abi, H=0)
+    assert lib.eot_band_half_step(ctypes.byref(empty), None, None, None, None, None, None, 0, None) == abi.EOT_OK
+
+
 def test_empty_problem_is_a_noop(abi):
     p = _prob(abi, B=0)
     assert abi.lib.eot_sinkhorn_fwd(ctypes.byref(p), None, None, None, None, None, None, None, None, 0, None) == 0
