@@ -6,8 +6,9 @@ so a step over B x H units can run as a sequence of smaller problems: chunks of 
 rows, or of heads of one batch row.  Three CUDA streams carry the chunks through copy-in, compute
 (eot_sinkhorn_fwd then eot_sinkhorn_bwd through the C ABI) and copy-out; two device staging
 slots alternate, so chunk c + 1's inputs arrive and chunk c - 1's results leave while chunk c
-computes.  Every step of the method still runs in libeot's kernels; this module only moves
-data and orders the streams.
+computes.  Within a chunk the forward starts once Q, K and V are in (dO, which only the backward
+reads, arrives meanwhile) and O leaves while the backward runs.  Every step of the method still
+runs in libeot's kernels; this module only moves data and orders the streams.
 """
 from __future__ import annotations
 
@@ -83,8 +84,10 @@ class HostStep:
             self.slots.append(s)
         self.s_in, self.s_comp, self.s_out = (torch.cuda.Stream(self.dev) for _ in range(3))
         self.ev_comp = [torch.cuda.Event() for _ in range(2)]
+        self.ev_fwd = [torch.cuda.Event() for _ in range(2)]
         self.ev_out = [torch.cuda.Event() for _ in range(2)]
-        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]       # Q, K, V of the slot are in
+        self.ev_in_dO = [torch.cuda.Event() for _ in range(2)]
         self.c = 0   # running chunk counter (slot = counter % 2)
 
     def problem(self, nb: int, nh: int):
@@ -116,9 +119,11 @@ class HostStep:
             with torch.cuda.stream(self.s_in):
                 if not first_use:
                     self.s_in.wait_event(self.ev_comp[i])
-                for name, src in (("q", hq), ("k", hk), ("v", hv), ("dO", hdO)):
+                for name, src in (("q", hq), ("k", hk), ("v", hv)):
                     s[name].copy_(src[b0:b1, h0:h1], non_blocking=True)
                 self.ev_in[i].record(self.s_in)
+                s["dO"].copy_(hdO[b0:b1, h0:h1], non_blocking=True)
+                self.ev_in_dO[i].record(self.s_in)
             # outputs of this slot are free once the copy-out two chunks back has finished
             with torch.cuda.stream(self.s_comp):
                 self.s_comp.wait_event(self.ev_in[i])
@@ -129,14 +134,18 @@ class HostStep:
                 _abi.eot_sinkhorn_fwd(p, s["q"].data_ptr(), s["k"].data_ptr(), s["v"].data_ptr(), m,
                                       s["O"].data_ptr(), s["ut"].data_ptr(), s["vt"].data_ptr(),
                                       ws["wsf"].data_ptr(), ws["wsf"].numel(), sp)
+                self.ev_fwd[i].record(self.s_comp)
+                self.s_comp.wait_event(self.ev_in_dO[i])
                 _abi.eot_sinkhorn_bwd(p, s["q"].data_ptr(), s["k"].data_ptr(), s["v"].data_ptr(), m,
                                       s["ut"].data_ptr(), s["vt"].data_ptr(), s["dO"].data_ptr(),
                                       s["dQ"].data_ptr(), s["dK"].data_ptr(), s["dV"].data_ptr(),
                                       ws["wsb"].data_ptr(), ws["wsb"].numel(), sp)
                 self.ev_comp[i].record(self.s_comp)
             with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_fwd[i])
+                hO[b0:b1, h0:h1].copy_(s["O"], non_blocking=True)
                 self.s_out.wait_event(self.ev_comp[i])
-                for name, dst in (("O", hO), ("dQ", hdQ), ("dK", hdK), ("dV", hdV)):
+                for name, dst in (("dQ", hdQ), ("dK", hdK), ("dV", hdV)):
                     dst[b0:b1, h0:h1].copy_(s[name], non_blocking=True)
                 self.ev_out[i].record(self.s_out)
             self.c += 1
