@@ -68,6 +68,9 @@ lib.eot_sinkhorn_bwd.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp
 lib.eot_sinkhorn_bwd.restype = ctypes.c_int
 lib.eot_band_half_step.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
 lib.eot_band_half_step.restype = ctypes.c_int
+lib.eot_band_half_step_dustbin.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _sz,
+                                           _vp]
+lib.eot_band_half_step_dustbin.restype = ctypes.c_int
 lib.eot_last_device_status.argtypes = [_vp, _vp]
 lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -191,6 +194,14 @@ def eot_band_half_step(p: eot_problem, X: int, Y: int, log_marg: int, pot_in: in
     """One band half-step; raw device addresses as in eot_sinkhorn_fwd."""
     _check(lib.eot_band_half_step(ctypes.byref(p), X, Y, log_marg, pot_in, pot_out, workspace, workspace_bytes,
                                   stream), "eot_band_half_step")
+
+
+def eot_band_half_step_dustbin(p: eot_problem, X: int, Y: int, log_marg: int, pot_in: int, pot_out: int,
+                               own_lo: int, own_hi: int, dust_part: int, workspace: int, workspace_bytes: int,
+                               stream: int) -> None:
+    """One band half-step of a part of a sequence with a dustbin; raw device addresses."""
+    _check(lib.eot_band_half_step_dustbin(ctypes.byref(p), X, Y, log_marg, pot_in, pot_out, int(own_lo), int(own_hi),
+                                          dust_part, workspace, workspace_bytes, stream), "eot_band_half_step_dustbin")
 
 
 def eot_sinkhorn_fwd_static(p: eot_problem, Q: int, K: int, V: int, mask: int | None, O: int, u_tail: int,

@@ -82,12 +82,18 @@ def sinkhorn_fwd(q, k, v, W: int, T: int, R: int, mask=None, scale=None, dustbin
 
 
 def band_half_step(x, y, log_marg, pot_in, W: int, scale=None, impl: str = "auto", stream=None,
-                   ws: torch.Tensor | None = None):
-    """One band half-step (no dustbin): out[b,h,i] = log_marg[b,i] - LSE_{|i-j| <= W/2, active j}
+                   ws: torch.Tensor | None = None, dustbin_index: int | None = None, own=None,
+                   dustbin_self: bool = True):
+    """One band half-step: out[b,h,i] = log_marg[b,i] - LSE_{|i-j| <= W/2, active j}
     (scale <x_i, y_j> + pot_in[b,h,j]), 0 at inactive positions.  x, y [B,H,L,d] (fp32 or bf16,
     L a multiple of 128), log_marg [B,L] fp32 (-inf = inactive), pot_in [B,H,L] fp32.  Returns
     out [B,H,L] fp32.  Row half-step: x = q, y = k, pot_in = v; column half-step: x = k, y = q,
-    pot_in = u."""
+    pot_in = u.
+
+    With ``dustbin_index`` D (a part of a sequence with a dustbin, eot_band_half_step_dustbin):
+    real rows also sum the dustbin term, and the result is (out, part) with part [B,H,2] the
+    (max, sum) partial of the dustbin's dense row over the positions ``own`` = (lo, hi)
+    (default: every real position), (D, D) excluded; out[..., D] is unspecified."""
     if x.shape != y.shape or x.dim() != 4 or x.dtype != y.dtype:
         raise ValueError("x and y must be [B,H,L,d] tensors of one dtype")
     B, H, L, d = x.shape
@@ -98,13 +104,24 @@ def band_half_step(x, y, log_marg, pot_in, W: int, scale=None, impl: str = "auto
     for t in (x, y, log_marg, pot_in):
         if not t.is_contiguous() or t.device != x.device:
             raise ValueError("inputs must be contiguous and on one device")
-    p = make_problem(B, H, L, d, W, 0, 0, x.dtype, scale, impl=impl)
+    if dustbin_index is None:
+        p = make_problem(B, H, L, d, W, 0, 0, x.dtype, scale, impl=impl)
+    else:
+        # (the mass only selects the dustbin's activity in the problem; the step reads log_marg)
+        p = make_problem(B, H, L, d, W, 0, 0, x.dtype, scale, dustbin_index, 0.5, dustbin_self, impl)
     out = torch.empty((B, H, L), dtype=torch.float32, device=x.device)
     if ws is None:
         ws = workspace(p, False, x.device)
-    _abi.eot_band_half_step(p, x.data_ptr(), y.data_ptr(), log_marg.data_ptr(), pot_in.data_ptr(), out.data_ptr(),
-                            ws.data_ptr(), ws.numel(), _stream(stream))
-    return out
+    if dustbin_index is None:
+        _abi.eot_band_half_step(p, x.data_ptr(), y.data_ptr(), log_marg.data_ptr(), pot_in.data_ptr(), out.data_ptr(),
+                                ws.data_ptr(), ws.numel(), _stream(stream))
+        return out
+    part = torch.empty((B, H, 2), dtype=torch.float32, device=x.device)
+    lo, hi = own if own is not None else (0, dustbin_index)
+    _abi.eot_band_half_step_dustbin(p, x.data_ptr(), y.data_ptr(), log_marg.data_ptr(), pot_in.data_ptr(),
+                                    out.data_ptr(), lo, hi, part.data_ptr(), ws.data_ptr(), ws.numel(),
+                                    _stream(stream))
+    return out, part
 
 
 def sinkhorn_bwd(q, k, v, u_tail, v_tail, dO, W: int, mask=None, scale=None, dustbin_index=None,

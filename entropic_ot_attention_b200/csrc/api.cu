@@ -379,14 +379,26 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
 // One half-step on its own (§2.1): out = log_marg - LSE over the band of (scale <x_i, y_j> + in_j),
 // with a running maximum (the online form of the first half-step of a solve), so that any finite
 // input potential is accepted.
+// With a dustbin (own_lo <= own_hi, dust_part not null) every real row also takes the dustbin
+// column term S_iD + in_D, and the dense dustbin row is returned as a (max, sum) partial over the
+// columns [own_lo, own_hi) instead of a finished potential.
 eot_status half_step_impl(const eot_problem* p, const void* X, const void* Y, const float* log_marg,
-                          const float* in, float* out, void* ws, cudaStream_t st) {
+                          const float* in, float* out, void* ws, cudaStream_t st, int own_lo = 0,
+                          int own_hi = 0, float* dust_part = nullptr) {
     EOT_RANGE("eot band half-step");
     const Geom g = make_geom(*p);
     const int impl = resolve_impl(*p);
     const WsLayout w = ws_layout(*p, false);
     uint32_t* status = at<uint32_t>(ws, w.status);
     EOT_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+    float* sd_row = nullptr;
+    float* sd_col = nullptr;
+    if (p->dustbin) {
+        sd_row = at<float>(ws, w.sd_row);
+        sd_col = at<float>(ws, w.sd_col);
+        EOT_TRY(cudaMemsetAsync(at<uint32_t>(ws, w.dcnt), 0, size_t(g.BH) * sizeof(uint32_t), st));
+        EOT_TRY(aux(st, [&] { return launch_dustbin_dots(g, X, Y, g.scale, sd_row, sd_col, st); }));
+    }
     float* in_b2 = at<float>(ws, w.vb2);
     float* out_b2 = at<float>(ws, w.ub2);
     uint32_t* tbits = at<uint32_t>(ws, w.tbits);
@@ -405,7 +417,14 @@ eot_status half_step_impl(const eot_problem* p, const void* X, const void* Y, co
     lp.out_bias2 = out_b2;
     lp.tile_bits = tbits;
     lp.status = status;
+    if (p->dustbin) {
+        lp.sd_term = sd_row;
+        lp.sd_dense = sd_col;
+        lp.dpart = at<float>(ws, w.dpart);
+        lp.dcnt = at<uint32_t>(ws, w.dcnt);
+    }
     EOT_TRY(run_lse(impl, lp, st));
+    if (p->dustbin) EOT_TRY(aux(st, [&] { return launch_dustbin_part(lp, own_lo, own_hi, dust_part, st); }));
     return EOT_OK;
 }
 
@@ -712,6 +731,21 @@ eot_status eot_band_half_step(const eot_problem* p, const void* X, const void* Y
     if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
     if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
     return half_step_impl(p, X, Y, log_marg, in, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+eot_status eot_band_half_step_dustbin(const eot_problem* p, const void* X, const void* Y, const float* log_marg,
+                                      const float* in, float* out, int32_t own_lo, int32_t own_hi, float* dust_part,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (!p->dustbin) return EOT_ERR_INVALID_ARGUMENT;
+    if (own_lo < 0 || own_hi < own_lo || own_hi > p->dustbin_index) return EOT_ERR_INVALID_ARGUMENT;
+    if (empty(*p)) return EOT_OK;
+    if (!X || !Y || !log_marg || !in || !out || !dust_part || !workspace) return EOT_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
+    return half_step_impl(p, X, Y, log_marg, in, out, workspace, static_cast<cudaStream_t>(stream), own_lo, own_hi,
+                          dust_part);
 }
 
 int eot_solve_exp_passes(const eot_problem* p) {

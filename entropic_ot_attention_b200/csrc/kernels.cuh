@@ -75,6 +75,8 @@ struct ContractArgs {
 };
 cudaError_t launch_contraction(const ContractArgs& a, int dtype, int BH, cudaStream_t st);
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st);
+// (max, sum) partial of the dense dustbin row over the columns [lo, hi) (a part of a sequence)
+cudaError_t launch_dustbin_part(const LsePass& p, int lo, int hi, float* part, cudaStream_t st);
 cudaError_t launch_dustbin_bwd(const BwdPass& p, cudaStream_t st);
 
 // Tensor-core (tcgen05 + TMA) kernels; return cudaErrorNotSupported when not built.

@@ -862,6 +862,44 @@ cudaError_t launch_simt_lse_fused(const LsePass& row, const void* Q, const void*
     return row.g.dtype == EOT_BF16 ? launch(simt_lse_fused_kernel<__nv_bfloat16>) : launch(simt_lse_fused_kernel<float>);
 }
 
+// The dense dustbin row of one part of a sequence (a sharded solve): per unit, the (max, sum)
+// partial of x_c = S_Dc + colpot_c over the active real columns c in [lo, hi), natural-log units
+// (sum_c exp(x_c - max)); (-inf, 0) when there is none.  (D, D) is left to the caller.
+__global__ void __launch_bounds__(256) dustbin_part_kernel(LsePass p, int lo, int hi, float* part) {
+    const int bh = blockIdx.x, b = bh / p.g.H, L = p.g.L, D = p.g.D;
+    const size_t base = size_t(bh) * L;
+    const size_t pb = size_t(bh) * p.pstride;
+    const float* logm = p.logm + size_t(b) * L;
+    float m = neg_inf(), s = 0.f;
+    for (int c = lo + int(threadIdx.x); c < hi; c += blockDim.x) {
+        if (c == D || logm[c] == neg_inf()) continue;
+        lse2_add(m, s, (p.sd_dense[base + c] + p.colpot[pb + c]) * kLog2e);
+    }
+    __shared__ float sm_m[256], sm_s[256];
+    sm_m[threadIdx.x] = m;
+    sm_s[threadIdx.x] = s;
+    __syncthreads();
+    for (int st = 128; st > 0; st >>= 1) {
+        if (threadIdx.x < st) {
+            float a = sm_m[threadIdx.x], bb = sm_s[threadIdx.x];
+            lse2_merge(a, bb, sm_m[threadIdx.x + st], sm_s[threadIdx.x + st]);
+            sm_m[threadIdx.x] = a;
+            sm_s[threadIdx.x] = bb;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        part[2 * bh] = sm_m[0] == neg_inf() ? neg_inf() : sm_m[0] * kLn2;
+        part[2 * bh + 1] = sm_s[0];
+    }
+}
+
+cudaError_t launch_dustbin_part(const LsePass& p, int lo, int hi, float* part, cudaStream_t st) {
+    if (!p.sd_dense || !part || p.g.D < 0 || lo < 0 || hi < lo || hi > p.g.L) return cudaErrorInvalidValue;
+    dustbin_part_kernel<<<p.g.BH, 256, 0, st>>>(p, lo, hi, part);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dustbin_lse(const LsePass& p, cudaStream_t st) {
     if (!p.dpart || !p.dcnt) return cudaErrorInvalidValue;
     dustbin_lse_kernel<<<dim3(dustbin_splits(p.g.L), p.g.BH), 256, 0, st>>>(p);

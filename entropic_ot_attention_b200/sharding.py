@@ -181,3 +181,98 @@ def sharded_solve(plan: list[Shard], rank: int, T: int, R: int,
         u_tail[slot] = u
         v_tail[slot] = v
     return u_tail, v_tail
+
+
+def _lse_add(M: torch.Tensor, S: torch.Tensor, x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    """Add one term x to a (max, sum) log-sum-exp pair (elementwise)."""
+    M2 = torch.maximum(M, x)
+    fin = torch.isfinite(M2)
+    base = torch.where(fin, M2, torch.zeros_like(M2))
+    S2 = torch.where(torch.isfinite(M), S * torch.exp(M - base), torch.zeros_like(S)) + \
+        torch.where(torch.isfinite(x), torch.exp(x - base), torch.zeros_like(S))
+    return M2, S2
+
+
+def sharded_solve_dustbin(plan: list[Shard], rank: int, T: int, R: int,
+                          row_step: Callable[[torch.Tensor, torch.Tensor], tuple],
+                          col_step: Callable[[torch.Tensor, torch.Tensor], tuple],
+                          log_mass: float, self_score: float | None,
+                          group=None, dtype=torch.float64, device=None):
+    """``sharded_solve`` for a sequence with a dustbin (§2.3): the dustbin D is linked to every
+    active real position, so its potentials u_D, v_D are held by every rank and its dense row and
+    column are merged from per-rank partials with ``allreduce_lse``.
+
+    ``row_step(v_halo, v_D)`` returns (u of the owned rows, their sums including the dustbin term
+    S_iD + v_D; m, s) with (m, s) the (max, sum) partial of S_Dc + v_c over the owned active
+    columns c; ``col_step(u_halo, u_D)`` the same with rows and columns swapped.  ``log_mass`` is
+    log b_D = log a_D; ``self_score`` is S_DD when (D, D) is in the support, else None.  Returns
+    (u_tail, v_tail, uD_tail, vD_tail): the owned potentials [R + 1, r1 - r0] and the dustbin's
+    [R + 1], slot layout of eot_sinkhorn_fwd."""
+    sh = plan[rank]
+    u_tail = torch.zeros(R + 1, sh.n, dtype=dtype, device=device)
+    v_tail = torch.zeros(R + 1, sh.n, dtype=dtype, device=device)
+    uD_tail = torch.zeros(R + 1, dtype=dtype, device=device)
+    vD_tail = torch.zeros(R + 1, dtype=dtype, device=device)
+    v_halo = torch.zeros(sh.c1 - sh.c0, dtype=dtype, device=device)
+    vD = torch.zeros(1, dtype=dtype, device=device)
+
+    def dense(m, s, other_D):
+        M, S = allreduce_lse(m.reshape(1).to(dtype), s.reshape(1).to(dtype), group)
+        if self_score is not None:
+            M, S = _lse_add(M, S, self_score + other_D)
+        lse = torch.where(S > 0, M + torch.log(torch.where(S > 0, S, torch.ones_like(S))),
+                          torch.full_like(S, float("-inf")))
+        return log_mass - lse
+
+    for k in range(T + R):
+        u, m, s_ = row_step(v_halo, vD)
+        uD = dense(m, s_, vD)
+        v, m, s_ = col_step(halo_exchange(u, plan, rank, group), uD)
+        vD = dense(m, s_, uD)
+        v_halo = halo_exchange(v, plan, rank, group)
+        slot = 0 if k < T else k - T + 1
+        u_tail[slot] = u
+        v_tail[slot] = v
+        uD_tail[slot] = uD[0]
+        vD_tail[slot] = vD[0]
+    return u_tail, v_tail, uD_tail, vD_tail
+
+
+def device_half_steps_dustbin(sh: Shard, q_halo: torch.Tensor, k_halo: torch.Tensor, q_dust: torch.Tensor,
+                              k_dust: torch.Tensor, log_marg_halo: torch.Tensor, log_mass: float, W: int,
+                              scale: float | None = None, impl: str = "auto"):
+    """``(row_step, col_step)`` for ``sharded_solve_dustbin`` on the device holding ``q_halo``:
+    each step is one ``eot_band_half_step_dustbin`` call on the halo range padded to whole tiles,
+    followed by a tile holding the dustbin (its q and k rows ``q_dust``, ``k_dust`` [d]) and
+    inactive fillers; the dustbin's partial covers the owned positions only."""
+    from .api import band_half_step, make_problem, workspace   # needs the built library
+
+    n = sh.c1 - sh.c0
+    if q_halo.shape != k_halo.shape or q_halo.shape[0] != n or log_marg_halo.shape != (n,):
+        raise ValueError("q_halo, k_halo [c1 - c0, d] and log_marg_halo [c1 - c0] expected")
+    D = (n + 127) // 128 * 128
+    Lp = D + 128
+    dev = q_halo.device
+
+    def pad(x, xd):
+        out = torch.zeros((1, 1, Lp, x.shape[1]), dtype=x.dtype, device=dev)
+        out[0, 0, :n] = x
+        out[0, 0, D] = xd.to(device=dev, dtype=x.dtype)
+        return out
+
+    q, k = pad(q_halo, q_dust), pad(k_halo, k_dust)
+    lm = torch.full((1, Lp), float("-inf"), dtype=torch.float32, device=dev)
+    lm[0, :n] = log_marg_halo.to(device=dev, dtype=torch.float32)
+    lm[0, D] = float(log_mass)
+    ws = workspace(make_problem(1, 1, Lp, q.shape[-1], W, 0, 0, q.dtype, scale, D, 0.5, True, impl), False, dev)
+    own = (sh.owned.start, sh.owned.stop)
+
+    def step(x, y, pot_halo, pot_D):
+        pin = torch.zeros((1, 1, Lp), dtype=torch.float32, device=dev)
+        pin[0, 0, :n] = pot_halo.to(device=dev, dtype=torch.float32)
+        pin[0, 0, D] = pot_D.reshape(()).to(device=dev, dtype=torch.float32)
+        out, part = band_half_step(x, y, lm, pin, W, scale, impl, ws=ws, dustbin_index=D, own=own)
+        part = part[0, 0].to(device=pot_halo.device, dtype=pot_halo.dtype)
+        return out[0, 0, sh.owned].to(device=pot_halo.device, dtype=pot_halo.dtype), part[0], part[1]
+
+    return (lambda v_halo, v_D: step(q, k, v_halo, v_D)), (lambda u_halo, u_D: step(k, q, u_halo, u_D))

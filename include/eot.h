@@ -149,6 +149,29 @@ eot_status eot_band_half_step(const eot_problem* p, const void* X, const void* Y
                               const float* in, float* out, void* workspace, size_t workspace_bytes,
                               void* stream);
 
+/*
+ * The same half-step for a part of a sequence that carries a dustbin (§2.3; p->dustbin = 1,
+ * D = p->dustbin_index, positions after D inactive).  The dustbin is linked to every active real
+ * position of the whole sequence, so its row and column are dense over all parts:
+ *   - every active real position i < D gets out[b, h, i] as in eot_band_half_step with the
+ *     dustbin term exp(scale * <X_i, Y_D> + in_D) added to its sum;
+ *   - instead of a finished out[b, h, D], the part's share of the dustbin's sum over the
+ *     positions it owns, [own_lo, own_hi) (0 <= own_lo <= own_hi <= D), excluding (D, D):
+ *       x_c = scale * <X[b, h, D], Y[b, h, c]> + in[b, h, c]  over active c in [own_lo, own_hi),
+ *       dust_part[b, h, 0] = M = max_c x_c,  dust_part[b, h, 1] = sum_c exp(x_c - M)
+ *     ((-inf, 0) when the range holds no active position).  The caller merges the parts'
+ *     partials (a max and a sum over all parts), adds the (D, D) term when it is in the support,
+ *     and forms out_D = log_marg[D] - (M + log(sum)); out[b, h, D] is left unspecified.
+ *   log_marg[b, D] is the dustbin's log marginal (log mass), the real positions' the whole
+ *   problem's (log((1 - mass) / n_real)).  dust_part: [B, H, 2] float32, device, written.
+ * Other arguments, errors and asynchrony as for eot_band_half_step; p->dustbin = 0 or an own range
+ * outside [0, D] is EOT_ERR_INVALID_ARGUMENT.
+ */
+eot_status eot_band_half_step_dustbin(const eot_problem* p, const void* X, const void* Y,
+                                      const float* log_marg, const float* in, float* out, int32_t own_lo,
+                                      int32_t own_hi, float* dust_part, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 /* Synchronises ``stream``, reads the device status word that the last fwd/bwd call on this
  * workspace left, clears it, and returns EOT_OK, EOT_ERR_NONFINITE or EOT_ERR_TIMEOUT
  * (EOT_ERR_CUDA if the copy fails). */

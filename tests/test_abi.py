@@ -133,6 +133,17 @@ def test_half_step_host_errors_launch_nothing(abi):
         == abi.EOT_ERR_INVALID_ARGUMENT
     empty = _prob(abi, H=0)
     assert lib.eot_band_half_step(ctypes.byref(empty), None, None, None, None, None, None, 0, None) == abi.EOT_OK
+    # the dustbin form: a dustbin problem and an own range inside [0, D] are required
+    f = lib.eot_band_half_step_dustbin
+    assert f(ctypes.byref(p), fake, fake, fake, fake, fake, 0, 128, fake, fake, 1 << 30, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT                                  # no dustbin
+    for lo, hi in ((-1, 5), (3, 2), (0, 6)):
+        assert f(ctypes.byref(db), fake, fake, fake, fake, fake, lo, hi, fake, fake, 1 << 30, None) \
+            == abi.EOT_ERR_INVALID_ARGUMENT
+    assert f(ctypes.byref(db), fake, fake, fake, fake, fake, 0, 5, None, fake, 1 << 30, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT                                  # null partial
+    assert f(ctypes.byref(db), fake, fake, fake, fake, fake, 0, 5, fake, fake, 16, None) \
+        == abi.EOT_ERR_WORKSPACE_TOO_SMALL
 
 
 def test_empty_problem_is_a_noop(abi):

@@ -146,3 +146,117 @@ def test_sharded_solve_on_gpu_matches_oracle(world, L, W, d, dtype):
         vt[:, r0:r1] = v
     assert pot_err(ut, ref.u_tail) <= STEP_TOL, pot_err(ut, ref.u_tail)
     assert pot_err(vt, ref.v_tail) <= STEP_TOL, pot_err(vt, ref.v_tail)
+
+
+@pytest.mark.parametrize("dtype,d,W,L_real,impl", [
+    ("bf16", 128, 256, 768, "auto"),
+    ("bf16", 64, 100, 640, "auto"),
+    ("fp32", 32, 60, 384, "auto"),
+])
+def test_half_step_with_dustbin_matches_oracle(dtype, d, W, L_real, impl):
+    import torch
+    from entropic_ot_attention_b200 import band_half_step
+    B, H, mass = 2, 2, 0.1
+    L, D = L_real + 128, L_real
+    rng = np.random.default_rng(L + W + d + 1)
+    real = np.zeros((B, L), np.uint8)
+    real[:, :L_real] = (rng.random((B, L_real)) > 0.2).astype(np.uint8)
+    case = eot_inputs.dense_case(B, H, L, d, W, 0, 0, dtype, seed=4)
+    with np.errstate(divide="ignore"):
+        log_m = np.where(real.astype(bool), np.log((1.0 - mass) / (real.sum(axis=1, keepdims=True) + 37.0)), -np.inf)
+    log_m[:, D] = np.log(mass)
+    pot = (rng.standard_normal((B, H, L)) * 3.0).astype(np.float32)
+    scale = 1.0 / np.sqrt(d)
+    dev = torch.device("cuda:0")
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    q = torch.from_numpy(case.Q).to(dev).to(tdt).contiguous()
+    k = torch.from_numpy(case.K).to(dev).to(tdt).contiguous()
+    lm_t = torch.from_numpy(log_m.astype(np.float32)).to(dev)
+    pin = torch.from_numpy(pot).to(dev)
+    lo, hi = 128, L_real - 128
+    u, part = band_half_step(q, k, lm_t, pin, W, impl=impl, dustbin_index=D, own=(lo, hi))
+    u_all, part_all = band_half_step(q, k, lm_t, pin, W, impl=impl, dustbin_index=D)
+    u, part, part_all = u.cpu().numpy(), part.cpu().numpy(), part_all.cpu().numpy()
+    torch.cuda.synchronize()
+    for b in range(B):
+        act = real[b].astype(bool)
+        st = eo.unit_structure(L, W, mask_row=real[b], dustbin=True, dustbin_index=D, dustbin_mass=mass)
+        for h in range(H):
+            x, y = case.Q[b, h].astype(np.float64), case.K[b, h].astype(np.float64)
+            S = eo.scores(x, y, scale, st.support)
+            want = eo.row_step(S, log_m[b], pot[b, h].astype(np.float64), st.active)
+            assert pot_err(u[b, h, :D], want[:D]) <= STEP_TOL, (b, h, pot_err(u[b, h, :D], want[:D]))
+            # the dustbin's partial over [lo, hi), and over every real position with (D, D) added
+            xs = S[D, :D] + pot[b, h, :D]
+            sel = act[:D] & (np.arange(D) >= lo) & (np.arange(D) < hi)
+            want_part = eo.lse(xs[sel], axis=0)
+            got_part = part[b, h, 0] + np.log(part[b, h, 1])
+            assert abs(got_part - want_part) <= STEP_TOL * max(abs(want_part), 1.0)
+            self_term = S[D, D] + pot[b, h, D]
+            got_D = log_m[b, D] - eo.lse(np.array([part_all[b, h, 0] + np.log(part_all[b, h, 1]), self_term]), axis=0)
+            assert abs(got_D - want[D]) <= STEP_TOL * max(abs(want[D]), 1.0)
+
+
+def _gpu_dustbin_worker(rank, world, port, L_real, d, W, T, R, mass, dtype, out):
+    import torch
+    import torch.distributed as dist
+    from entropic_ot_attention_b200.sharding import device_half_steps_dustbin, shard_plan, sharded_solve_dustbin
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    q, k, mask = _unit_dustbin(L_real, d, dtype, seed=21)
+    D = L_real
+    plan = shard_plan(L_real, W, world)
+    sh = plan[rank]
+    act = mask.astype(bool)
+    n_act = torch.tensor([float(act[sh.r0:sh.r1].sum())], dtype=torch.float64)
+    dist.all_reduce(n_act)
+    lm_halo = torch.from_numpy(np.where(act[sh.c0:sh.c1], np.log((1.0 - mass) / n_act.item()), -np.inf))
+    dev = torch.device("cuda:0")
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(tdt)
+    row_step, col_step = device_half_steps_dustbin(sh, to_dev(q[sh.c0:sh.c1]), to_dev(k[sh.c0:sh.c1]), to_dev(q[D]),
+                                                   to_dev(k[D]), lm_halo, float(np.log(mass)), W)
+    self_score = float(np.float64(q[D]) @ np.float64(k[D]) / np.sqrt(d))
+    ut, vt, uD, vD = sharded_solve_dustbin(plan, rank, T, R, row_step, col_step, float(np.log(mass)), self_score)
+    torch.cuda.synchronize()
+    out[rank] = (sh.r0, sh.r1, ut.numpy(), vt.numpy(), uD.numpy(), vD.numpy())
+    dist.destroy_process_group()
+
+
+def _unit_dustbin(L_real, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    L = L_real + 128
+    mask = np.zeros((1, L), np.uint8)
+    mask[0, :L_real] = (rng.random(L_real) > 0.15).astype(np.uint8)
+    case = eot_inputs.dense_case(1, 1, L, d, 0, 0, 0, dtype, seed=seed)
+    return case.Q[0, 0], case.K[0, 0], mask[0]
+
+
+@pytest.mark.parametrize("world,L_real,W,d,dtype", [(2, 1280, 256, 64, "bf16"), (3, 1536, 300, 128, "bf16")])
+def test_sharded_solve_with_dustbin_on_gpu_matches_oracle(world, L_real, W, d, dtype):
+    import torch.multiprocessing as mp
+    T, R, mass = 5, 2, 0.1
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_gpu_dustbin_worker, args=(r, world, port, L_real, d, W, T, R, mass, dtype, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+        assert p.exitcode == 0
+    q, k, mask = _unit_dustbin(L_real, d, dtype, seed=21)
+    ref = eo.forward_unit(q, k, np.zeros((q.shape[0], 1)), W, T, R, mask_row=mask, dustbin=True,
+                          dustbin_index=L_real, dustbin_mass=mass, dustbin_self=True)
+    ut = np.zeros((R + 1, L_real))
+    vt = np.zeros((R + 1, L_real))
+    for r in range(world):
+        r0, r1, u, v, uD, vD = out[r]
+        ut[:, r0:r1] = u
+        vt[:, r0:r1] = v
+        assert pot_err(uD, ref.u_tail[:, L_real]) <= STEP_TOL
+        assert pot_err(vD, ref.v_tail[:, L_real]) <= STEP_TOL
+    assert pot_err(ut, ref.u_tail[:, :L_real]) <= STEP_TOL, pot_err(ut, ref.u_tail[:, :L_real])
+    assert pot_err(vt, ref.v_tail[:, :L_real]) <= STEP_TOL, pot_err(vt, ref.v_tail[:, :L_real])
