@@ -71,6 +71,8 @@ lib.eot_band_half_step.restype = ctypes.c_int
 lib.eot_band_half_step_dustbin.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _sz,
                                            _vp]
 lib.eot_band_half_step_dustbin.restype = ctypes.c_int
+lib.eot_band_output.argtypes = [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+lib.eot_band_output.restype = ctypes.c_int
 lib.eot_last_device_status.argtypes = [_vp, _vp]
 lib.eot_last_device_status.restype = ctypes.c_int
 lib.eot_device_status_bits.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -202,6 +204,13 @@ def eot_band_half_step_dustbin(p: eot_problem, X: int, Y: int, log_marg: int, po
     """One band half-step of a part of a sequence with a dustbin; raw device addresses."""
     _check(lib.eot_band_half_step_dustbin(ctypes.byref(p), X, Y, log_marg, pot_in, pot_out, int(own_lo), int(own_hi),
                                           dust_part, workspace, workspace_bytes, stream), "eot_band_half_step_dustbin")
+
+
+def eot_band_output(p: eot_problem, Q: int, K: int, V: int, log_marg: int, u: int, v: int, O: int, workspace: int,
+                    workspace_bytes: int, stream: int) -> None:
+    """The output of given potentials; raw device addresses."""
+    _check(lib.eot_band_output(ctypes.byref(p), Q, K, V, log_marg, u, v, O, workspace, workspace_bytes, stream),
+           "eot_band_output")
 
 
 def eot_sinkhorn_fwd_static(p: eot_problem, Q: int, K: int, V: int, mask: int | None, O: int, u_tail: int,

@@ -124,6 +124,31 @@ def band_half_step(x, y, log_marg, pot_in, W: int, scale=None, impl: str = "auto
     return out, part
 
 
+def band_output(q, k, v, log_marg, u, v_pot, W: int, scale=None, impl: str = "auto", stream=None,
+                ws: torch.Tensor | None = None):
+    """O = diag(1/a) P V of given potentials (no dustbin): P_ij = exp(scale <q_i, k_j> + u_i +
+    v_pot_j) on the band, a_i = exp(log_marg_i).  q, k, v [B,H,L,d]; log_marg [B,L] fp32;
+    u, v_pot [B,H,L] fp32.  Returns O [B,H,L,d] in q's dtype."""
+    if not (q.shape == k.shape == v.shape) or q.dim() != 4 or not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must be [B,H,L,d] tensors of one dtype")
+    B, H, L, d = q.shape
+    if log_marg.shape != (B, L) or log_marg.dtype != torch.float32:
+        raise ValueError("log_marg must be a float32 [B, L] tensor")
+    for t in (u, v_pot):
+        if t.shape != (B, H, L) or t.dtype != torch.float32:
+            raise ValueError("u and v_pot must be float32 [B, H, L] tensors")
+    for t in (q, k, v, log_marg, u, v_pot):
+        if not t.is_contiguous() or t.device != q.device:
+            raise ValueError("inputs must be contiguous and on one device")
+    p = make_problem(B, H, L, d, W, 0, 0, q.dtype, scale, impl=impl)
+    O = torch.empty_like(q)
+    if ws is None:
+        ws = workspace(p, False, q.device)
+    _abi.eot_band_output(p, q.data_ptr(), k.data_ptr(), v.data_ptr(), log_marg.data_ptr(), u.data_ptr(),
+                         v_pot.data_ptr(), O.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream))
+    return O
+
+
 def sinkhorn_bwd(q, k, v, u_tail, v_tail, dO, W: int, mask=None, scale=None, dustbin_index=None,
                  dustbin_mass: float = 0.0, dustbin_self: bool = True, impl: str = "auto", stream=None,
                  ws: torch.Tensor | None = None):

@@ -376,6 +376,52 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     return EOT_OK;
 }
 
+// The output of given potentials (§2.1): O = diag(1/a) P V with P_ij = exp(S_ij + u_i + v_j) on the
+// band and a_i = exp(log_marg_i) (no dustbin); the forward's output sweep with a one-slot tail.
+eot_status output_impl(const eot_problem* p, const void* Q, const void* K, const void* V, const float* log_marg,
+                       const float* u, const float* v, void* O, void* ws, cudaStream_t st) {
+    EOT_RANGE("eot band output");
+    const Geom g = make_geom(*p);
+    const int impl = resolve_impl(*p);
+    const WsLayout w = ws_layout(*p, false);
+    uint32_t* status = at<uint32_t>(ws, w.status);
+    EOT_TRY(cudaMemsetAsync(status, 0, sizeof(uint32_t), st));
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
+    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, log_marg, tbits, st); }));
+    BwdVecArgs va{};
+    va.kind = kPassOut;
+    va.R = 0;
+    va.H = g.H;
+    va.BH = g.BH;
+    va.L = g.L;
+    va.logm = log_marg;
+    va.u_tail = u;
+    va.v_tail = v;
+    va.D = g.D;
+    va.pr = at<float>(ws, w.opr);
+    va.pc = at<float>(ws, w.opc);
+    va.pcm2 = at<float>(ws, w.opcm);
+    va.f = va.hv = va.m = nullptr;
+    EOT_TRY(aux(st, [&] { return launch_bwd_vectors(va, st); }));
+    BwdPass op{};
+    op.g = g;
+    op.X = Q;
+    op.Y = K;
+    op.Z = V;
+    op.logm = log_marg;
+    op.pr = va.pr;
+    op.pc = va.pc;
+    op.pcm2 = va.pcm2;
+    op.vout = O;
+    op.vscale = 1.f;
+    op.v_dp = 0;
+    op.nmod = 0;
+    op.status = status;
+    op.tile_bits = tbits;
+    EOT_TRY(run_bwd(impl, op, st, kProfOut));
+    return EOT_OK;
+}
+
 // One half-step on its own (§2.1): out = log_marg - LSE over the band of (scale <x_i, y_j> + in_j),
 // with a running maximum (the online form of the first half-step of a solve), so that any finite
 // input potential is accepted.
@@ -746,6 +792,19 @@ eot_status eot_band_half_step_dustbin(const eot_problem* p, const void* X, const
     if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
     return half_step_impl(p, X, Y, log_marg, in, out, workspace, static_cast<cudaStream_t>(stream), own_lo, own_hi,
                           dust_part);
+}
+
+eot_status eot_band_output(const eot_problem* p, const void* Q, const void* K, const void* V, const float* log_marg,
+                           const float* u, const float* v, void* O, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+    eot_status s = validate(p);
+    if (s != EOT_OK) return s;
+    if (p->dustbin) return EOT_ERR_UNSUPPORTED;
+    if (empty(*p)) return EOT_OK;
+    if (!Q || !K || !V || !log_marg || !u || !v || !O || !workspace) return EOT_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return EOT_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < ws_layout(*p, false).total) return EOT_ERR_WORKSPACE_TOO_SMALL;
+    return output_impl(p, Q, K, V, log_marg, u, v, O, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int eot_solve_exp_passes(const eot_problem* p) {

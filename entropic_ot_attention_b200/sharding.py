@@ -159,6 +159,32 @@ def device_half_steps(sh: Shard, q_halo: torch.Tensor, k_halo: torch.Tensor, log
     return (lambda v_halo: step(q, k, v_halo)), (lambda u_halo: step(k, q, u_halo))
 
 
+def device_output(sh: Shard, q_halo: torch.Tensor, k_halo: torch.Tensor, v_halo: torch.Tensor,
+                  log_marg_halo: torch.Tensor, u_halo: torch.Tensor, vpot_halo: torch.Tensor, W: int,
+                  scale: float | None = None, impl: str = "auto") -> torch.Tensor:
+    """O = diag(1/a) P V of this rank's owned rows (one ``eot_band_output`` call on the halo range,
+    padded to whole tiles with inactive positions), from the potentials over the halo (u and v
+    after the last half-step, exchanged with ``halo_exchange``).  q_halo, k_halo, v_halo:
+    [c1 - c0, d] on a CUDA device; returns [r1 - r0, d] in their dtype on that device."""
+    from .api import band_output   # needs the built library
+
+    n = sh.c1 - sh.c0
+    Lp = (n + 127) // 128 * 128
+    dev = q_halo.device
+
+    def pad(x, dtype=None):
+        shape = (1, 1, Lp) + tuple(x.shape[1:])
+        out = torch.zeros(shape, dtype=dtype or x.dtype, device=dev)
+        out[0, 0, :n] = x.to(device=dev, dtype=dtype or x.dtype)
+        return out
+
+    lm = torch.full((1, Lp), float("-inf"), dtype=torch.float32, device=dev)
+    lm[0, :n] = log_marg_halo.to(device=dev, dtype=torch.float32)
+    O = band_output(pad(q_halo), pad(k_halo), pad(v_halo), lm, pad(u_halo, torch.float32),
+                    pad(vpot_halo, torch.float32), W, scale, impl)
+    return O[0, 0, sh.owned]
+
+
 def sharded_solve(plan: list[Shard], rank: int, T: int, R: int,
                   row_step: Callable[[torch.Tensor], torch.Tensor],
                   col_step: Callable[[torch.Tensor], torch.Tensor],

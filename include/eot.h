@@ -172,6 +172,24 @@ eot_status eot_band_half_step_dustbin(const eot_problem* p, const void* X, const
                                       int32_t own_hi, float* dust_part, void* workspace,
                                       size_t workspace_bytes, void* stream);
 
+/*
+ * The output of given potentials (§2.1) on its own, the last step of a sequence-sharded forward
+ * (each part forms the rows it owns from the potentials over its halo):
+ *     O[b, h, i] = (1 / a_i) sum_{j : |i - j| <= W / 2, active j}
+ *                      exp( scale * <Q[b, h, i], K[b, h, j]> + u[b, h, i] + v[b, h, j] ) V[b, h, j]
+ * with a_i = exp(log_marg[b, i]) for active i; O = 0 at inactive positions.  Device pointers:
+ *   Q, K, V   [B, H, L, d] p->dtype, read only;
+ *   log_marg  [B, L] float32 log marginals (-inf = inactive; a part passes the whole problem's);
+ *   u, v      [B, H, L] float32 potentials, read only;
+ *   O         [B, H, L, d] p->dtype, written;
+ *   workspace eot_workspace_bytes(p, 0) bytes, 256-byte aligned, device, contents clobbered.
+ * p->T and p->R are not used; a dustbin is EOT_ERR_UNSUPPORTED (its dense output row sums over
+ * every position).  Errors and asynchrony as for eot_band_half_step.
+ */
+eot_status eot_band_output(const eot_problem* p, const void* Q, const void* K, const void* V,
+                           const float* log_marg, const float* u, const float* v, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Synchronises ``stream``, reads the device status word that the last fwd/bwd call on this
  * workspace left, clears it, and returns EOT_OK, EOT_ERR_NONFINITE or EOT_ERR_TIMEOUT
  * (EOT_ERR_CUDA if the copy fails). */

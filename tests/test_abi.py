@@ -133,6 +133,13 @@ def test_half_step_host_errors_launch_nothing(abi):
         == abi.EOT_ERR_INVALID_ARGUMENT
     empty = _prob(abi, H=0)
     assert lib.eot_band_half_step(ctypes.byref(empty), None, None, None, None, None, None, 0, None) == abi.EOT_OK
+    # the output of given potentials: no dustbin, no null pointer
+    o = lib.eot_band_output
+    assert o(ctypes.byref(p), fake, fake, None, fake, fake, fake, fake, fake, ws_bytes, None) \
+        == abi.EOT_ERR_INVALID_ARGUMENT
+    assert o(ctypes.byref(db), fake, fake, fake, fake, fake, fake, fake, fake, 1 << 30, None) == abi.EOT_ERR_UNSUPPORTED
+    assert o(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, 16, None) \
+        == abi.EOT_ERR_WORKSPACE_TOO_SMALL
     # the dustbin form: a dustbin problem and an own range inside [0, D] are required
     f = lib.eot_band_half_step_dustbin
     assert f(ctypes.byref(p), fake, fake, fake, fake, fake, 0, 128, fake, fake, 1 << 30, None) \

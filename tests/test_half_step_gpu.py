@@ -80,6 +80,32 @@ def test_half_step_matches_oracle(dtype, d, W, L, impl):
             assert np.all(u[b, h][~act] == 0.0) and np.all(v[b, h][~act] == 0.0)
 
 
+@pytest.mark.parametrize("dtype,d,W,L", [("bf16", 128, 256, 896), ("bf16", 64, 100, 640), ("fp32", 32, 60, 384)])
+def test_output_of_given_potentials_matches_oracle(dtype, d, W, L):
+    import torch
+    from entropic_ot_attention_b200 import band_output
+    from harness import TOL, rel_err
+    B, H = 2, 2
+    rng = np.random.default_rng(L + W + d + 2)
+    mask = (rng.random((B, L)) > 0.2).astype(np.uint8)
+    case = eot_inputs.dense_case(B, H, L, d, W, 0, 0, dtype, seed=6, mask=mask)
+    scale = 1.0 / np.sqrt(d)
+    u = (rng.standard_normal((B, H, L)) * 0.5 - np.log(L)).astype(np.float32)
+    vp = (rng.standard_normal((B, H, L)) * 0.5).astype(np.float32)
+    dev = torch.device("cuda:0")
+    tdt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    t = lambda a: torch.from_numpy(a).to(dev).to(tdt).contiguous()
+    log_m = np.stack([eo.unit_structure(L, W, mask_row=mask[b]).log_a for b in range(B)]).astype(np.float32)
+    O = band_output(t(case.Q), t(case.K), t(case.V), torch.from_numpy(log_m).to(dev), torch.from_numpy(u).to(dev),
+                    torch.from_numpy(vp).to(dev), W).float().cpu().numpy()
+    for b in range(B):
+        st = eo.unit_structure(L, W, mask_row=mask[b])
+        for h in range(H):
+            S = eo.scores(case.Q[b, h], case.K[b, h], scale, st.support)
+            want = eo.output(S, st, u[b, h].astype(np.float64), vp[b, h].astype(np.float64), case.V[b, h])
+            assert rel_err(O[b, h], want) <= TOL[dtype], (b, h, rel_err(O[b, h], want))
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
@@ -95,6 +121,12 @@ def _unit(L, d, dtype, seed):
     return case.Q[0, 0], case.K[0, 0], mask[0]
 
 
+def _unit_v(L, d, dtype, seed):
+    rng = np.random.default_rng(seed)
+    mask = (rng.random((1, L)) > 0.15).astype(np.uint8)
+    return eot_inputs.dense_case(1, 1, L, d, 0, 0, 0, dtype, seed=seed, mask=mask).V[0, 0]
+
+
 def _gpu_solve_worker(rank, world, port, L, d, W, T, R, dtype, out):
     import torch
     import torch.distributed as dist
@@ -102,6 +134,7 @@ def _gpu_solve_worker(rank, world, port, L, d, W, T, R, dtype, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     q, k, mask = _unit(L, d, dtype, seed=9)
+    vv = _unit_v(L, d, dtype, seed=9)
     plan = shard_plan(L, W, world)
     sh = plan[rank]
     act = mask.astype(bool)
@@ -115,8 +148,12 @@ def _gpu_solve_worker(rank, world, port, L, d, W, T, R, dtype, out):
     kh = torch.from_numpy(np.ascontiguousarray(k[sh.c0:sh.c1])).to(dev).to(tdt)
     row_step, col_step = device_half_steps(sh, qh, kh, lm_halo, W)
     ut, vt = sharded_solve(plan, rank, T, R, row_step, col_step)
+    # the owned rows' output from the last potentials over the halo
+    from entropic_ot_attention_b200.sharding import device_output, halo_exchange
+    vh = torch.from_numpy(np.ascontiguousarray(vv[sh.c0:sh.c1])).to(dev).to(tdt)
+    O = device_output(sh, qh, kh, vh, lm_halo, halo_exchange(ut[R], plan, rank), halo_exchange(vt[R], plan, rank), W)
     torch.cuda.synchronize()
-    out[rank] = (sh.r0, sh.r1, ut.numpy(), vt.numpy())
+    out[rank] = (sh.r0, sh.r1, ut.numpy(), vt.numpy(), O.float().cpu().numpy())
     dist.destroy_process_group()
 
 
@@ -136,16 +173,21 @@ def test_sharded_solve_on_gpu_matches_oracle(world, L, W, d, dtype):
     for p in procs:
         p.join(timeout=300)
         assert p.exitcode == 0
+    from harness import TOL, rel_err
     q, k, mask = _unit(L, d, dtype, seed=9)
-    ref = eo.forward_unit(q, k, np.zeros((L, 1)), W, T, R, mask_row=mask)
+    vv = _unit_v(L, d, dtype, seed=9)
+    ref = eo.forward_unit(q, k, vv, W, T, R, mask_row=mask)
     ut = np.zeros((R + 1, L))
     vt = np.zeros((R + 1, L))
+    O = np.zeros((L, d))
     for r in range(world):
-        r0, r1, u, v = out[r]
+        r0, r1, u, v, o = out[r]
         ut[:, r0:r1] = u
         vt[:, r0:r1] = v
+        O[r0:r1] = o
     assert pot_err(ut, ref.u_tail) <= STEP_TOL, pot_err(ut, ref.u_tail)
     assert pot_err(vt, ref.v_tail) <= STEP_TOL, pot_err(vt, ref.v_tail)
+    assert rel_err(O, ref.O) <= TOL[dtype], rel_err(O, ref.O)
 
 
 @pytest.mark.parametrize("dtype,d,W,L_real,impl", [
