@@ -31,10 +31,14 @@ constexpr int kSNT = 256;  // threads per CTA
 // One CTA of 1024 threads per batch row (L is a multiple of 128): count the real tokens (mask
 // bytes read 16 at a time when the mask is 16-byte aligned), then write the row's log marginals
 // 4 at a time.
+// Block (b, j): counts the active real tokens of batch row b (every block of the row reads the
+// whole mask row, from L2 after the first) and writes positions [j kPrepSlice, (j + 1) kPrepSlice).
+constexpr int kPrepSlice = 4096;
 __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint8_t* mask, int dustbin,
                                                               float mass, float* logm, uint32_t* status) {
     const int b = blockIdx.x;
     const int L = g.L;
+    const int w0 = blockIdx.y * kPrepSlice, w1 = min(L, w0 + kPrepSlice);
     const int D = dustbin ? g.D : L;
     const uint8_t* mrow = mask ? mask + size_t(b) * L : nullptr;
     const bool vec = mrow && (reinterpret_cast<uintptr_t>(mask) & 15) == 0;
@@ -62,7 +66,7 @@ __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint
     const double real_mass = use_db ? (1.0 - double(mass)) : 1.0;
     const float lr = n > 0 ? float(log(real_mass / double(n))) : neg_inf();
     const float ld = use_db ? float(log(double(mass))) : neg_inf();
-    for (int i0 = threadIdx.x * 4; i0 < L; i0 += blockDim.x * 4) {
+    for (int i0 = w0 + threadIdx.x * 4; i0 < w1; i0 += blockDim.x * 4) {
         float v[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -73,7 +77,7 @@ __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint
         }
         *reinterpret_cast<float4*>(logm + size_t(b) * L + i0) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    if (b == 0 && threadIdx.x == 0 && status) *status = 0u;
+    if (b == 0 && blockIdx.y == 0 && threadIdx.x == 0 && status) *status = 0u;
 }
 
 // Dustbin link vectors: out_term[r] = s1 * <P_r, Q_D>, out_dense[r] = s1 * <P_D, Q_r> for
@@ -666,7 +670,9 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
 // ---------------------------------------------------------------------------------------
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
                                   uint32_t* status, cudaStream_t st) {
-    prep_marginals_kernel<<<g.B, 1024, 0, st>>>(g, mask, dustbin, mass, logm, status);
+    if (g.B == 0 || g.L == 0) return cudaSuccess;
+    prep_marginals_kernel<<<dim3(g.B, (g.L + kPrepSlice - 1) / kPrepSlice), 1024, 0, st>>>(g, mask, dustbin, mass,
+                                                                                          logm, status);
     return cudaGetLastError();
 }
 
