@@ -776,6 +776,61 @@ __global__ void __launch_bounds__(kResThreads) simt_resident_kernel(LsePass g0, 
     while (G < 32 && G * 2 * L <= int(blockDim.x)) G *= 2;
     const int grp = threadIdx.x / G, gl = threadIdx.x % G, ngrp = blockDim.x / G;
     const float sl2 = g0.g.scale * kLog2e;
+    // Small bands with one row per group: every thread keeps its band entries of row grp (row
+    // half-steps) and of column grp (column half-steps) in registers for the whole solve, so a
+    // half-step is one independent bias load per entry, the exponentials and a group reduction.
+    constexpr int kResRegs = 12;
+    const int ne = (ld + G - 1) / G;
+    if (L <= ngrp && ne <= kResRegs) {
+        const int rc = grp;                    // the row (and the column) of this group
+        float srow[kResRegs], scol[kResRegs];
+#pragma unroll
+        for (int e = 0; e < kResRegs; ++e) {
+            const int j = gl + e * G, c = rc - h + j;   // column of S_rc / row of S_cr
+            const bool ok = e < ne && j < ld && rc < L && c >= 0 && c < L;
+            srow[e] = ok ? sband[size_t(rc) * ld + j] * sl2 : 0.f;
+            scol[e] = ok ? sband[size_t(c) * ld + (2 * h - j)] * sl2 : 0.f;
+        }
+        for (int hs = 0; hs < 2 * (Tb + R); ++hs) {
+            const int it = hs >> 1;
+            const int slot = it < Tb ? 0 : it - Tb + 1;
+            const bool col = hs & 1;
+            const float* bias = col ? ub2 : vb2;   // the other side's log2 potential
+            float* outb = col ? vb2 : ub2;
+            float* out = (col ? v_tail : u_tail) + pb + size_t(slot) * L;
+            float x[kResRegs];
+            float m = neg_inf();
+#pragma unroll
+            for (int e = 0; e < kResRegs; ++e) {
+                const int j = gl + e * G, c = rc - h + j;
+                const bool ok = e < ne && j < ld && rc < L && c >= 0 && c < L;
+                x[e] = ok ? (col ? scol[e] : srow[e]) + bias[ok ? c : 0] : neg_inf();
+                m = fmaxf(m, x[e]);
+            }
+            float s = 0.f;
+            if (m != neg_inf()) {
+#pragma unroll
+                for (int e = 0; e < kResRegs; ++e) s += ptx::ex2(x[e] - m);   // ex2(-inf) = 0
+            }
+            for (int off = G / 2; off > 0; off >>= 1) {
+                const float m2 = __shfl_xor_sync(0xffffffffu, m, off), s2 = __shfl_xor_sync(0xffffffffu, s, off);
+                lse2_merge(m, s, m2, s2);
+            }
+            if (rc < L && gl == 0) {
+                const float lm = lmb[rc];
+                float outv = 0.f, ob = neg_inf();
+                if (lm != neg_inf()) {
+                    outv = lm - (m + log2f(s)) * kLn2;
+                    if (!isfinite(outv)) atomicOr(g0.status, kStatusNonFinite);
+                    ob = outv * kLog2e;
+                }
+                outb[rc] = ob;
+                out[rc] = outv;
+            }
+            __syncthreads();
+        }
+        return;
+    }
     for (int hs = 0; hs < 2 * (Tb + R); ++hs) {
         const int it = hs >> 1;
         const int slot = it < Tb ? 0 : it - Tb + 1;
