@@ -293,7 +293,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         }(), st));
         uint32_t* gbar = at<uint32_t>(ws, w.gbar);
         EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
-        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar, ue, ve};
+        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar, ue, ve, at<int>(ws, w.bounds)};
         const cudaError_t e = tracked(kProfLse, 1, st, [&] { return launch_tc_lse_fused(row, f, st); });
         if (e == cudaSuccess) fused = true;
         else if (e == cudaErrorCooperativeLaunchTooLarge) {

@@ -17,6 +17,7 @@ namespace eot {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxBandCtas = 1024;   // CTAs of a fused half-step launch (one per SM)
 constexpr int kMaxR = 8;
 constexpr int kMaxMods = 2 * kMaxR;
 
@@ -118,6 +119,7 @@ struct WsLayout {
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t gbar;            // forward: grid-barrier counters of the fused half-steps [2 (T + R)]
+    size_t bounds;          // forward: item ranges of the fused half-steps' CTAs [kMaxBandCtas + 1]
     size_t part;            // forward, one exponential per iteration: column partial sums [BH][L/128][window][128]
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
@@ -206,6 +208,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
         w.gbar = o; o += align256(size_t(2) * (size_t(p.T) + size_t(p.R)) * sizeof(uint32_t) + 4);
+        w.bounds = o; o += align256(size_t(kMaxBandCtas + 1) * sizeof(int));
         if (p.dtype == EOT_BF16 && p.d == 128 && p.impl != EOT_IMPL_SIMT && p.L % 128 == 0 && p.W / 2 >= 256) {
             w.bext = true;
             w.ue = o; o += align256(BH * L * 32);

@@ -95,6 +95,8 @@ struct FusedSteps {
     // d = 128: the column-bias operand rows of u and v ([BH L, 16] bf16; the first half-step
     // before this launch writes those of u)
     __nv_bfloat16 *ue, *ve;
+    // scratch for the CTAs' item ranges [kMaxBandCtas + 1], or null for equal ranges
+    int* bounds;
 };
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);

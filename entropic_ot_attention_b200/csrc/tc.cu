@@ -175,6 +175,9 @@ struct TcBandArgs {
     float* ub2;
     float* vb2;
     uint32_t* gbar;
+    // CTA c takes items [bounds[c], bounds[c + 1]) (band_bounds_kernel), or, when null, the
+    // equal ranges of items_per_cta
+    const int* bounds;
     // Fused half-steps with a dustbin: the dustbin links of the rows (sd_row: S between row r
     // and the dustbin column) and of the columns (sd_col: S between the dustbin row and column
     // c); the dense dustbin row of every half-step is summed per item ((max, sum) partials in
@@ -305,8 +308,8 @@ __global__ void __launch_bounds__(kBandThreads, 1)
     uint8_t* sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = a.L, h = a.h, D = a.D;
-    const int item0 = blockIdx.x * a.items_per_cta;
-    const int item1 = min(a.n_items, item0 + a.items_per_cta);
+    const int item0 = a.bounds ? a.bounds[blockIdx.x] : blockIdx.x * a.items_per_cta;
+    const int item1 = a.bounds ? a.bounds[blockIdx.x + 1] : min(a.n_items, item0 + a.items_per_cta);
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
     const uint32_t bar0 = ptx::smem_u32(bars);
@@ -1609,6 +1612,66 @@ cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, 
                                        smem, st);
 }
 
+// Item ranges of the CTAs of a fused launch: contiguous, each holding about the same weight (an
+// item's active 128-row tiles, 0 to 2), so that units with few active tokens (padded sequences)
+// do not leave some CTAs with all-active items and others with none.  bounds[c] = the first item
+// i with (weight before i) * grid >= c * total; the last range runs to the end, so that every
+// item (inactive ones write their rows) belongs to exactly one CTA.  One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) band_bounds_kernel(const uint32_t* bits, int words, int H, int nT, int ppu,
+                                                           int n_items, int grid, int* bounds) {
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    auto weight = [&](int i) {
+        const int bh = i / ppu, b = bh / H, p = i - bh * ppu;
+        const uint32_t* bb = bits + size_t(b) * words;
+        return int(tile_bit(bb, 2 * p)) + ((2 * p + 1 < nT) ? int(tile_bit(bb, 2 * p + 1)) : 0);
+    };
+    // total weight
+    int t = 0;
+    for (int i = tid; i < n_items; i += blockDim.x) t += weight(i);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) wsum[wid] = t;
+    for (int c = tid; c <= grid; c += blockDim.x) bounds[c] = 0;
+    __syncthreads();
+    long long total = 0;
+    for (int k = 0; k < int(blockDim.x >> 5); ++k) total += wsum[k];
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    // inclusive scan of the weights in chunks of blockDim.x; item i owns the boundaries c with
+    // E_i grid < c total <= (E_i + w_i) grid (E_i = weight before i): bounds[c] = i + 1
+    for (int base = 0; base < n_items && total > 0; base += blockDim.x) {
+        const int i = base + tid;
+        const int w = i < n_items ? weight(i) : 0;
+        int x = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        __syncthreads();                       // wsum of the previous chunk is read
+        if (lane == 31) wsum[wid] = x;
+        __syncthreads();
+        int before = carry;
+        for (int k = 0; k < wid; ++k) before += wsum[k];
+        const long long incl = before + x, excl = incl - w;
+        if (w > 0) {
+            const long long c_lo = excl * grid / total + 1;
+            const long long c_hi = incl * grid / total < grid ? incl * grid / total : (long long)grid;
+            for (long long c = c_lo; c <= c_hi; ++c) bounds[c] = i + 1;
+        }
+        __syncthreads();
+        if (tid == blockDim.x - 1) carry = int(incl);
+        __syncthreads();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        bounds[0] = 0;
+        bounds[grid] = n_items;
+    }
+}
+
 // Band row reduction over S = scale X Y^T (geometry, tile bits and the per-kind vectors in a);
 // multi: the fused shifted half-steps a.hs0 .. a.hs0 + a.nhs - 1 in one cooperative launch.
 cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs a, int kind, cudaStream_t st,
@@ -1639,9 +1702,19 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     a.words = tile_words(g.L);
     a.pairs_per_unit = (g.L / 128 + 1) / 2;
     a.n_items = g.BH * a.pairs_per_unit;
-    const int grid = std::max(1, std::min(a.n_items, sm_count()));
+    const int grid = std::max(1, std::min({a.n_items, sm_count(), kMaxBandCtas}));
     a.items_per_cta = (a.n_items + grid - 1) / grid;
-    const int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
+    int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
+    if (multi && a.bounds) {
+        // ranges of equal weight over every CTA of the grid
+        band_bounds_kernel<<<1, 1024, 0, st>>>(a.tile_bits, tile_words(g.L), g.H, g.L / 128, a.pairs_per_unit,
+                                               a.n_items, grid, const_cast<int*>(a.bounds));
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        grid_used = grid;
+    } else {
+        a.bounds = nullptr;
+    }
     if (!multi) {
         a.hs0 = 0;
         a.nhs = 1;
@@ -1711,6 +1784,7 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     a.dcnt = row.dcnt;
     a.ue = f.ue;
     a.ve = f.ve;
+    a.bounds = f.bounds;
     // row half-steps: X = Q (row.X), Y = K (row.Y); the kernel swaps them for column half-steps
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
