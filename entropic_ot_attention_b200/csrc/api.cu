@@ -213,6 +213,12 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     uint32_t* tbits = at<uint32_t>(ws, w.tbits);
     EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
     row.tile_bits = tbits;
+    int* bounds = at<int>(ws, w.bounds);
+    if (impl == EOT_IMPL_TCGEN05) {
+        // every band launch of this call takes item ranges of equal weight
+        EOT_TRY(aux(st, [&] { return launch_band_bounds(g, tbits, bounds, st); }));
+        row.bounds = bounds;
+    }
     row.colbias2 = vb2;
     row.out_bias2 = ub2;
     LsePass col = row;
@@ -293,7 +299,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
         }(), st));
         uint32_t* gbar = at<uint32_t>(ws, w.gbar);
         EOT_TRY(cudaMemsetAsync(gbar, 0, size_t(n_half) * sizeof(uint32_t), st));
-        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar, ue, ve, at<int>(ws, w.bounds)};
+        FusedSteps f{1, n_half - 1, p->T, u_tail, v_tail, ub2, vb2, gbar, ue, ve, row.bounds};
         const cudaError_t e = tracked(kProfLse, 1, st, [&] { return launch_tc_lse_fused(row, f, st); });
         if (e == cudaSuccess) fused = true;
         else if (e == cudaErrorCooperativeLaunchTooLarge) {
@@ -548,6 +554,11 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     uint32_t* tbits = at<uint32_t>(ws, w.tbits);
     EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
     rowp.tile_bits = tbits;
+    if (impl == EOT_IMPL_TCGEN05) {
+        int* bounds = at<int>(ws, w.bounds);
+        EOT_TRY(aux(st, [&] { return launch_band_bounds(g, tbits, bounds, st); }));
+        rowp.bounds = bounds;
+    }
     EOT_TRY(cudaMemsetAsync(at<float>(ws, w.zero), 0, vecn * sizeof(float), st));
     BwdPass colp = rowp;
     colp.X = K;

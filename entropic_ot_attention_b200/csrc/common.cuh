@@ -57,6 +57,8 @@ struct LsePass {
     // tensor-core kernels: also write each output position's column-bias operand row here
     // ([BH L, 16] bf16; read by the fused half-steps that follow), or nullptr
     __nv_bfloat16* ext_out;
+    // tensor-core kernels: the CTAs' item ranges (launch_band_bounds), or nullptr for equal ranges
+    const int* bounds;
 };
 
 // One backward sweep (§2.2).  With Pt_rc = exp(S_rc + pr_r + pc_c) on the support:
@@ -107,6 +109,7 @@ struct BwdPass {
     const __nv_bfloat16* xext;
     const __nv_bfloat16* yext;
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
+    const int* bounds;          // as in LsePass (tensor-core staircase sums)
     float* dpart;           // as in LsePass
     uint32_t* dcnt;
     uint32_t* status;
@@ -119,7 +122,7 @@ struct WsLayout {
     size_t opr, opc, opcm;  // forward output pass: row / column biases
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t gbar;            // forward: grid-barrier counters of the fused half-steps [2 (T + R)]
-    size_t bounds;          // forward: item ranges of the fused half-steps' CTAs [kMaxBandCtas + 1]
+    size_t bounds;          // item ranges of the band kernel's CTAs [kMaxBandCtas + 1]
     size_t part;            // forward, one exponential per iteration: column partial sums [BH][L/128][window][128]
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
@@ -208,7 +211,6 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         w.ub2 = o; o += vec;
         w.vb2 = o; o += vec;
         w.gbar = o; o += align256(size_t(2) * (size_t(p.T) + size_t(p.R)) * sizeof(uint32_t) + 4);
-        w.bounds = o; o += align256(size_t(kMaxBandCtas + 1) * sizeof(int));
         if (p.dtype == EOT_BF16 && p.d == 128 && p.impl != EOT_IMPL_SIMT && p.L % 128 == 0 && p.W / 2 >= 256) {
             w.bext = true;
             w.ue = o; o += align256(BH * L * 32);
@@ -220,6 +222,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
         }
     }
     w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
+    w.bounds = o; o += align256(size_t(kMaxBandCtas + 1) * sizeof(int));
     if (bwd) {
         w.pr = o; o += vec;
         w.pc = o; o += vec;

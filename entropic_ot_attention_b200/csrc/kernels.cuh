@@ -95,10 +95,13 @@ struct FusedSteps {
     // d = 128: the column-bias operand rows of u and v ([BH L, 16] bf16; the first half-step
     // before this launch writes those of u)
     __nv_bfloat16 *ue, *ve;
-    // scratch for the CTAs' item ranges [kMaxBandCtas + 1], or null for equal ranges
-    int* bounds;
+    // the CTAs' item ranges (launch_band_bounds), or null for equal ranges
+    const int* bounds;
 };
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
+// Item ranges of equal weight for the band kernel's CTAs (bounds [kMaxBandCtas + 1], from the
+// tile bits); every band launch of the problem's geometry can then take them.
+cudaError_t launch_band_bounds(const Geom& g, const uint32_t* tile_bits, int* bounds, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
 
 // Staircase sweeps from the cached reference plan (cache.cu): out = f hv sum P m over the band, by

@@ -1672,6 +1672,12 @@ __global__ void __launch_bounds__(1024) band_bounds_kernel(const uint32_t* bits,
     }
 }
 
+// CTAs of a band launch: one per SM, at most one per item.
+int band_grid(const Geom& g) {
+    const int n_items = g.BH * ((g.L / 128 + 1) / 2);
+    return std::max(1, std::min({n_items, sm_count(), kMaxBandCtas}));
+}
+
 // Band row reduction over S = scale X Y^T (geometry, tile bits and the per-kind vectors in a);
 // multi: the fused shifted half-steps a.hs0 .. a.hs0 + a.nhs - 1 in one cooperative launch.
 cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs a, int kind, cudaStream_t st,
@@ -1702,19 +1708,10 @@ cudaError_t launch_band(const Geom& g, const void* X, const void* Y, TcBandArgs 
     a.words = tile_words(g.L);
     a.pairs_per_unit = (g.L / 128 + 1) / 2;
     a.n_items = g.BH * a.pairs_per_unit;
-    const int grid = std::max(1, std::min({a.n_items, sm_count(), kMaxBandCtas}));
+    const int grid = band_grid(g);
     a.items_per_cta = (a.n_items + grid - 1) / grid;
-    int grid_used = (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
-    if (multi && a.bounds) {
-        // ranges of equal weight over every CTA of the grid
-        band_bounds_kernel<<<1, 1024, 0, st>>>(a.tile_bits, tile_words(g.L), g.H, g.L / 128, a.pairs_per_unit,
-                                               a.n_items, grid, const_cast<int*>(a.bounds));
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        grid_used = grid;
-    } else {
-        a.bounds = nullptr;
-    }
+    // (ranges of equal weight cover every CTA of the grid; equal ranges may leave the last empty)
+    const int grid_used = a.bounds ? grid : (a.n_items + a.items_per_cta - 1) / a.items_per_cta;
     if (!multi) {
         a.hs0 = 0;
         a.nhs = 1;
@@ -1758,6 +1755,7 @@ cudaError_t launch_tc_lse(const LsePass& p, cudaStream_t st) {
     a.sd_term = p.sd_term;
     a.status = p.status;
     a.ext_out = p.ext_out;
+    a.bounds = p.bounds;
     cudaError_t e = launch_band(p.g, p.X, p.Y, a, p.stab ? kBandShift : kBandOnline, st);
     if (e != cudaSuccess || p.g.D < 0) return e;
     return launch_dustbin_lse(p, st);
@@ -1787,6 +1785,14 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     a.bounds = f.bounds;
     // row half-steps: X = Q (row.X), Y = K (row.Y); the kernel swaps them for column half-steps
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
+}
+
+cudaError_t launch_band_bounds(const Geom& g, const uint32_t* tile_bits, int* bounds, cudaStream_t st) {
+    if (!tile_bits || !bounds) return cudaErrorInvalidValue;
+    const int ppu = (g.L / 128 + 1) / 2;
+    band_bounds_kernel<<<1, 1024, 0, st>>>(tile_bits, tile_words(g.L), g.H, g.L / 128, ppu, g.BH * ppu, band_grid(g),
+                                           bounds);
+    return cudaGetLastError();
 }
 
 struct ExtMaps {
@@ -1852,6 +1858,7 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
         a.sd_term = p.sd_term;
         a.status = p.status;
         a.sadd = p.sadd;
+        a.bounds = p.bounds;
         a.ue = const_cast<__nv_bfloat16*>(p.cext);   // read only (the column-bias operand rows)
         cudaError_t e = launch_band(g, p.X, p.Y, a, kBandWsum, st);
         if (e != cudaSuccess || g.D < 0) return e;
