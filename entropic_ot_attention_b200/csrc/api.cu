@@ -214,9 +214,12 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
     row.tile_bits = tbits;
     int* bounds = at<int>(ws, w.bounds);
+    int* jobs = nullptr;
     if (impl == EOT_IMPL_TCGEN05) {
-        // every band launch of this call takes item ranges of equal weight
-        EOT_TRY(aux(st, [&] { return launch_band_bounds(g, tbits, bounds, st); }));
+        // every band launch of this call takes item ranges of equal weight, and the output sweep
+        // its row-tile jobs active ones first
+        jobs = at<int>(ws, w.jobs);
+        EOT_TRY(aux(st, [&] { return launch_schedule(g, tbits, bounds, jobs, st); }));
         row.bounds = bounds;
     }
     row.colbias2 = vb2;
@@ -378,6 +381,7 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     op.dcnt = dcnt;
     op.status = status;
     op.tile_bits = tbits;
+    op.jobs = jobs;
     EOT_TRY(run_bwd(impl, op, st, kProfOut));
     return EOT_OK;
 }
@@ -556,8 +560,10 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.tile_bits = tbits;
     if (impl == EOT_IMPL_TCGEN05) {
         int* bounds = at<int>(ws, w.bounds);
-        EOT_TRY(aux(st, [&] { return launch_band_bounds(g, tbits, bounds, st); }));
+        int* jobs = at<int>(ws, w.jobs);
+        EOT_TRY(aux(st, [&] { return launch_schedule(g, tbits, bounds, jobs, st); }));
         rowp.bounds = bounds;
+        rowp.jobs = jobs;
     }
     EOT_TRY(cudaMemsetAsync(at<float>(ws, w.zero), 0, vecn * sizeof(float), st));
     BwdPass colp = rowp;

@@ -57,7 +57,7 @@ struct LsePass {
     // tensor-core kernels: also write each output position's column-bias operand row here
     // ([BH L, 16] bf16; read by the fused half-steps that follow), or nullptr
     __nv_bfloat16* ext_out;
-    // tensor-core kernels: the CTAs' item ranges (launch_band_bounds), or nullptr for equal ranges
+    // tensor-core kernels: the CTAs' item ranges (launch_schedule), or nullptr for equal ranges
     const int* bounds;
 };
 
@@ -110,6 +110,9 @@ struct BwdPass {
     const __nv_bfloat16* yext;
     const uint32_t* tile_bits;  // as in LsePass (tensor-core staircase sums)
     const int* bounds;          // as in LsePass (tensor-core staircase sums)
+    // tensor-core sweeps: the row-tile jobs in the order the persistent CTAs take them by stride
+    // (launch_schedule: the active ones first), or nullptr for the natural order
+    const int* jobs;
     float* dpart;           // as in LsePass
     uint32_t* dcnt;
     uint32_t* status;
@@ -123,6 +126,7 @@ struct WsLayout {
     size_t ub2, vb2;        // forward: masked log2 potentials feeding the next half-step
     size_t gbar;            // forward: grid-barrier counters of the fused half-steps [2 (T + R)]
     size_t bounds;          // item ranges of the band kernel's CTAs [kMaxBandCtas + 1]
+    size_t jobs;            // job order of the sweep kernel [BH L / 128]
     size_t part;            // forward, one exponential per iteration: column partial sums [BH][L/128][window][128]
     size_t tbits;           // active-tile bitmask [B][tile_words(L)]
     size_t pcm;             // backward: masked log2 column bias
@@ -223,6 +227,7 @@ inline WsLayout ws_layout(const eot_problem& p, bool bwd) {
     }
     w.tbits = o; o += align256(size_t(p.B) * size_t((p.L / 128 + 31) / 32) * 4);
     w.bounds = o; o += align256(size_t(kMaxBandCtas + 1) * sizeof(int));
+    w.jobs = o; o += align256(BH * size_t(p.L / 128) * sizeof(int));
     if (bwd) {
         w.pr = o; o += vec;
         w.pc = o; o += vec;

@@ -95,13 +95,15 @@ struct FusedSteps {
     // d = 128: the column-bias operand rows of u and v ([BH L, 16] bf16; the first half-step
     // before this launch writes those of u)
     __nv_bfloat16 *ue, *ve;
-    // the CTAs' item ranges (launch_band_bounds), or null for equal ranges
+    // the CTAs' item ranges (launch_schedule), or null for equal ranges
     const int* bounds;
 };
 cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStream_t st);
-// Item ranges of equal weight for the band kernel's CTAs (bounds [kMaxBandCtas + 1], from the
-// tile bits); every band launch of the problem's geometry can then take them.
-cudaError_t launch_band_bounds(const Geom& g, const uint32_t* tile_bits, int* bounds, cudaStream_t st);
+// From the tile bits, in one launch: item ranges of equal weight for the band kernel's CTAs
+// (bounds [kMaxBandCtas + 1]) and the order of the sweep kernel's row-tile jobs (jobs
+// [BH L / 128]: those whose row tile holds an active token first, then the others, each in their
+// natural order); every band and sweep launch of the problem's geometry can then take them.
+cudaError_t launch_schedule(const Geom& g, const uint32_t* tile_bits, int* bounds, int* jobs, cudaStream_t st);
 cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st);
 
 // Staircase sweeps from the cached reference plan (cache.cu): out = f hv sum P m over the band, by

@@ -175,7 +175,7 @@ struct TcBandArgs {
     float* ub2;
     float* vb2;
     uint32_t* gbar;
-    // CTA c takes items [bounds[c], bounds[c + 1]) (band_bounds_kernel), or, when null, the
+    // CTA c takes items [bounds[c], bounds[c + 1]) (schedule_kernel), or, when null, the
     // equal ranges of items_per_cta
     const int* bounds;
     // Fused half-steps with a dustbin: the dustbin links of the rows (sd_row: S between row r
@@ -897,6 +897,7 @@ struct ModeT {
 
 struct TcVecArgs {
     int H, L, h, D, BH;
+    const int* jobs;            // job order (active row tiles first), or null for the natural order
     const uint32_t* tile_bits;  // [B][words]: 128-position tiles holding an active non-dustbin token
     int words;
     float sc2;              // scale * log2(e)
@@ -1010,6 +1011,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     };
     auto job_of = [&](int job) {
         Job j;
+        if (a.jobs) job = __ldg(a.jobs + job);
         j.bh = job / nT;
         j.b = j.bh / a.H;
         j.r0 = (job - j.bh * nT) * C::BM;
@@ -1617,8 +1619,8 @@ cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, 
 // do not leave some CTAs with all-active items and others with none.  bounds[c] = the first item
 // i with (weight before i) * grid >= c * total; the last range runs to the end, so that every
 // item (inactive ones write their rows) belongs to exactly one CTA.  One CTA of 1024 threads.
-__global__ void __launch_bounds__(1024) band_bounds_kernel(const uint32_t* bits, int words, int H, int nT, int ppu,
-                                                           int n_items, int grid, int* bounds) {
+__device__ void band_bounds_block(const uint32_t* bits, int words, int H, int nT, int ppu, int n_items, int grid,
+                                  int* bounds) {
     __shared__ int wsum[32];
     __shared__ int carry;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -1787,11 +1789,63 @@ cudaError_t launch_tc_lse_fused(const LsePass& row, const FusedSteps& f, cudaStr
     return launch_band(row.g, row.X, row.Y, a, kBandShift, st, true);
 }
 
-cudaError_t launch_band_bounds(const Geom& g, const uint32_t* tile_bits, int* bounds, cudaStream_t st) {
-    if (!tile_bits || !bounds) return cudaErrorInvalidValue;
-    const int ppu = (g.L / 128 + 1) / 2;
-    band_bounds_kernel<<<1, 1024, 0, st>>>(tile_bits, tile_words(g.L), g.H, g.L / 128, ppu, g.BH * ppu, band_grid(g),
-                                           bounds);
+// Job order of the sweep kernel: the CTAs take jobs c, c + grid, ... of this list, so with the
+// active row tiles first every CTA gets as many of them as any other (+-1) and neighbouring
+// CTAs still work on neighbouring active tiles at the same time.  One CTA of 1024 threads:
+// position of job i = (active jobs before i) if active, else (all active) + (inactive before i).
+__device__ void sweep_jobs_block(const uint32_t* bits, int words, int H, int nT, int n_jobs, int* jobs) {
+    __shared__ int wsum[32];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    auto active = [&](int i) {
+        const int bh = i / nT;
+        return int(tile_bit(bits + size_t(bh / H) * words, i - bh * nT));
+    };
+    int t = 0;
+    for (int i = tid; i < n_jobs; i += blockDim.x) t += active(i);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) wsum[wid] = t;
+    __syncthreads();
+    int n_act = 0;
+    for (int k = 0; k < int(blockDim.x >> 5); ++k) n_act += wsum[k];
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < n_jobs; base += blockDim.x) {
+        const int i = base + tid;
+        const int a = i < n_jobs ? active(i) : 0;
+        int x = a;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        __syncthreads();
+        if (lane == 31) wsum[wid] = x;
+        __syncthreads();
+        int before = carry;
+        for (int k = 0; k < wid; ++k) before += wsum[k];
+        const int excl = before + x - a;           // active jobs before i
+        if (i < n_jobs) jobs[a ? excl : n_act + (i - excl)] = i;
+        __syncthreads();
+        if (tid == blockDim.x - 1) carry = before + x;
+        __syncthreads();
+    }
+}
+
+// The band kernel's item ranges and the sweep kernel's job order of one problem, in one launch.
+__global__ void __launch_bounds__(1024) schedule_kernel(const uint32_t* bits, int words, int H, int nT, int ppu,
+                                                        int n_items, int grid, int* bounds, int n_jobs, int* jobs) {
+    band_bounds_block(bits, words, H, nT, ppu, n_items, grid, bounds);
+    __syncthreads();
+    sweep_jobs_block(bits, words, H, nT, n_jobs, jobs);
+}
+
+cudaError_t launch_schedule(const Geom& g, const uint32_t* tile_bits, int* bounds, int* jobs, cudaStream_t st) {
+    if (!tile_bits || !bounds || !jobs) return cudaErrorInvalidValue;
+    const int ppu = (g.L / 128 + 1) / 2, nT = g.L / 128;
+    schedule_kernel<<<1, 1024, 0, st>>>(tile_bits, tile_words(g.L), g.H, nT, ppu, g.BH * ppu, band_grid(g), bounds,
+                                        g.BH * nT, jobs);
     return cudaGetLastError();
 }
 
@@ -1917,6 +1971,7 @@ cudaError_t launch_tc_bwd(const BwdPass& p, cudaStream_t st) {
     a.s1E = p.s1E;
     if (!p.tile_bits) return cudaErrorInvalidValue;
     a.BH = g.BH;
+    a.jobs = p.jobs;
     a.tile_bits = p.tile_bits;
     a.words = tile_words(g.L);
     const int mt = max_tiles_for(g.L, g.h, 128, 128);
