@@ -148,7 +148,7 @@ struct WsLayout {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // The dense dustbin row is split over CTAs of kDCols columns (plus the (D, D) entry).
-constexpr int kDCols = 1024;
+constexpr int kDCols = 256;
 __host__ __device__ inline int dustbin_splits(int L) { return (L + 1 + kDCols - 1) / kDCols; }
 __host__ __device__ inline int tile_words(int L) { return (L / 128 + 31) / 32; }
 

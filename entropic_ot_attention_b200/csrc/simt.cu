@@ -86,26 +86,31 @@ __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint
 template <typename T>
 __global__ void __launch_bounds__(256) prep_dustbin_dots_kernel(Geom g, const T* P, const T* Qm, float s1,
                                                                 float* out_term, float* out_dense) {
-    const int bh = blockIdx.y, lane = threadIdx.x & 31;
-    const int rows_per_block = blockDim.x >> 5;
-    const int r = blockIdx.x * rows_per_block + (threadIdx.x >> 5);
-    if (r >= g.L) return;
+    // 8 lanes per row, each summing its d / 8 consecutive elements (independent loads in flight),
+    // then a 3-step reduction within the 8 lanes; 32 rows per block
+    const int bh = blockIdx.y, sub = threadIdx.x & 7;
+    const int r = blockIdx.x * (blockDim.x >> 3) + (threadIdx.x >> 3);
+    const bool live = r < g.L;
     const size_t base = size_t(bh) * g.L;
-    const T* pr = P + (base + r) * g.d;
-    const T* pD = P + (base + g.D) * g.d;
-    const T* qr = Qm + (base + r) * g.d;
-    const T* qD = Qm + (base + g.D) * g.d;
+    const int per = g.d >> 3, k0 = sub * per;   // d is a multiple of 8
     float a = 0.f, b = 0.f;
-    for (int k = lane; k < g.d; k += 32) {
-        a = fmaf(to_f(pr[k]), to_f(qD[k]), a);
-        b = fmaf(to_f(pD[k]), to_f(qr[k]), b);
+    if (live) {
+        const T* pr = P + (base + r) * g.d + k0;
+        const T* pD = P + (base + g.D) * g.d + k0;
+        const T* qr = Qm + (base + r) * g.d + k0;
+        const T* qD = Qm + (base + g.D) * g.d + k0;
+#pragma unroll 4
+        for (int k = 0; k < per; ++k) {
+            a = fmaf(to_f(pr[k]), to_f(qD[k]), a);
+            b = fmaf(to_f(pD[k]), to_f(qr[k]), b);
+        }
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
+    for (int off = 4; off > 0; off >>= 1) {
         a += __shfl_xor_sync(0xffffffffu, a, off);
         b += __shfl_xor_sync(0xffffffffu, b, off);
     }
-    if (lane == 0) {
+    if (live && sub == 0) {
         out_term[base + r] = s1 * a;
         out_dense[base + r] = s1 * b;
     }
@@ -512,7 +517,7 @@ __global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
     if (p.vout) {
         const T* Z = static_cast<const T*>(p.Z) + base * d;
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+#pragma unroll 8
         for (int j = warp; j < c_end - c_begin; j += 8) {
             const float cf = cs[j];
             if (cf == 0.f) continue;
@@ -678,7 +683,7 @@ cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbi
 
 cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
                                 cudaStream_t st) {
-    dim3 grid((g.L + 7) / 8, g.BH);   // 8 rows (warps) per block
+    dim3 grid((g.L + 31) / 32, g.BH);   // 32 rows (8 lanes each) per block
     if (g.dtype == EOT_BF16)
         prep_dustbin_dots_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
             g, static_cast<const __nv_bfloat16*>(P), static_cast<const __nv_bfloat16*>(Qm), s1, term, dense);
