@@ -478,9 +478,10 @@ def main():
         fwd()
         bwd()
     torch.cuda.synchronize(dev)
-    st = _abi.eot_last_device_status(ws_f.data_ptr(), sp)
-    if st != 0:
-        raise RuntimeError(f"device status after warm-up: {_abi.eot_status_string(st)}")
+    for ws in (ws_f, ws_b):
+        st = _abi.eot_last_device_status(ws.data_ptr(), sp)
+        if st != 0:
+            raise RuntimeError(f"device status after warm-up: {_abi.eot_status_string(st)}")
 
     # ---------------- timed region: K steps, inputs resident (inputs > L2) ----------------
     sampler = ClockSampler(local)
@@ -490,6 +491,10 @@ def main():
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     launches0 = _abi.eot_kernel_launches()
+    # A spin of about 0.2 s ahead of the first event keeps the GPU busy while every step is
+    # enqueued, so that a host-side pause (the clock sampler's queries can hold up launches)
+    # does not leave the GPU idle inside a timed step.  It is outside the timed region.
+    torch.cuda._sleep(int(0.2 * 1.9e9))
     for i in range(args.steps):
         ev[i][0].record(stream)
         fwd()
@@ -500,6 +505,10 @@ def main():
     launches = _abi.eot_kernel_launches() - launches0
     barrier(dev)
     clocks = sampler.stop()
+    for ws in (ws_f, ws_b):
+        st = _abi.eot_last_device_status(ws.data_ptr(), sp)
+        if st != 0:
+            raise RuntimeError(f"device status after the timed steps: {_abi.eot_status_string(st)}")
     t_fwd = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     t_bwd = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     t_step_local = t_fwd + t_bwd

@@ -960,8 +960,8 @@ struct SweepCfg {
     static constexpr uint32_t OFF_YE = OFF_XE + EXTB;
     static constexpr uint32_t OFF_RED = FOLD ? OFF_YE + EXTB : OFF_V + NL * VB;  // [2 sums][4 quarters][128 rows] scalar partials
     static constexpr uint32_t OFF_BAR = OFF_RED + 2 * 4 * 128 * 4;
-    // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm accempty
-    static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1 + 1;
+    // full_l[NL] empty_l[NL] full_e empty_e xfull tfull tempty cfull[2] cempty[2] accfull xtm accempty jobdone
+    static constexpr uint32_t NBARS = 2 * NL + 2 + 1 + 2 + 4 + 1 + 1 + 1 + 1;
     static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr uint32_t OFF_TILES = OFF_MISC + 64;
     static size_t smem_bytes(int max_tiles) { return 1024 + OFF_TILES + 2 * 4 * size_t(max_tiles); }
@@ -1037,6 +1037,14 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
     const uint32_t accfull = bar0 + 8u * (2 * C::NL + 9);
     const uint32_t xtm = bar0 + 8u * (2 * C::NL + 10);       // row tiles copied into TMEM
     const uint32_t accempty = bar0 + 8u * (2 * C::NL + 11);  // accumulator read back
+    // every score product of a job has completed (a pass without products: the next job's row
+    // tiles may then overwrite TMEM).  One phase per job, committed after its last tile, so the
+    // row-tile thread, which copies job k's tiles before phase k can start, is never more than
+    // one phase behind it.  (Waiting instead on the per-tile barrier for each of the previous
+    // job's tiles could block: once two of them had completed, the wait for the first had the
+    // parity of the phase in progress and then waited for a tile of the next job, which needs
+    // this very thread.)
+    const uint32_t jobdone = bar0 + 8u * (2 * C::NL + 12);
     uint32_t* misc = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -1060,6 +1068,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         ptx::mbar_init(accfull, 1);
         ptx::mbar_init(xtm, 1);                     // the commit of the row tiles' copy into TMEM
         ptx::mbar_init(accempty, kSweepEpi / 2);   // the warps of column quarters 0 and 1
+        ptx::mbar_init(jobdone, M::HASDP ? 2 : 1); // the S issuer and the dP issuer
         ptx::mbar_fence_init();
     }
     if (warp == 1) {
@@ -1176,6 +1185,7 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                     else if (!M::VEC) ptx::mma_commit(empty_l(sl));
                     issued = it + 1;
                 }
+                if (!M::VEC && ok) ptx::mma_commit(jobdone);
             }
             if (*abort_flag && issued > 0) {
                 volatile int dummy = 0;
@@ -1198,21 +1208,14 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             if (M::HASDP) ptx::prefetch_tmap(&tmA);
             if (FOLD) ptx::prefetch_tmap(&tmXE);
             int done = 0, itg = 0, jc = 0;
-            // a pass without products: the previous job's score tiles (global indices) that must
-            // complete before its TMEM row tiles are overwritten, waited for one by one (a wait
-            // on a later tile's phase alone could be satisfied by an earlier phase's parity)
-            int tg = 0, pend_lo = 0, pend_hi = 0;
             bool ok = true, xpending = false;
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
                 const Job jb = job_of(job);
                 if (!jb.act) continue;
                 if (jc > 0) {
-                    if (M::VEC) {
-                        ok = ptx::mbar_wait(accfull, (jc - 1) & 1, abort_flag, a.status);
-                    } else {
-                        for (int it = pend_lo; it < pend_hi && ok; ++it)
-                            ok = ptx::mbar_wait(tfull, it & 1, abort_flag, a.status);
-                    }
+                    // the previous job's products (or, in a pass without them, its score
+                    // products) are done with the TMEM row tiles and the coefficient buffers
+                    ok = ptx::mbar_wait(M::VEC ? accfull : jobdone, (jc - 1) & 1, abort_flag, a.status);
                     if (!ok) break;
                 }
                 const uint32_t xs = ptx::smem_u32(sm + C::OFF_C), as = xs + C::XB;
@@ -1234,9 +1237,6 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
                         ptx::tmem_cp_128x256b(tbase + C::TM_A + uint32_t(kk * 8), ptx::smem_desc(as + koff, 16, 1024));
                 }
                 ptx::mma_commit(xtm);
-                pend_lo = tg;
-                for (int t = jb.t_lo; t <= jb.t_hi; ++t) tg += tile_bit(jb.bits, t) ? 1 : 0;
-                pend_hi = tg;
                 if (M::VEC) {
                     // the previous job's accumulator has been read back
                     if (jc > 0 && !ptx::mbar_wait(accempty, (jc - 1) & 1, abort_flag, a.status)) { ok = false; break; }
@@ -1833,18 +1833,18 @@ __device__ void sweep_jobs_block(const uint32_t* bits, int words, int H, int nT,
     }
 }
 
-// The band kernel's item ranges and the sweep kernel's job order of one problem, in one launch.
+// The band kernel's item ranges (CTA 0) and the sweep kernel's job order (CTA 1) of one problem,
+// in one launch.
 __global__ void __launch_bounds__(1024) schedule_kernel(const uint32_t* bits, int words, int H, int nT, int ppu,
                                                         int n_items, int grid, int* bounds, int n_jobs, int* jobs) {
-    band_bounds_block(bits, words, H, nT, ppu, n_items, grid, bounds);
-    __syncthreads();
-    sweep_jobs_block(bits, words, H, nT, n_jobs, jobs);
+    if (blockIdx.x == 0) band_bounds_block(bits, words, H, nT, ppu, n_items, grid, bounds);
+    else sweep_jobs_block(bits, words, H, nT, n_jobs, jobs);
 }
 
 cudaError_t launch_schedule(const Geom& g, const uint32_t* tile_bits, int* bounds, int* jobs, cudaStream_t st) {
     if (!tile_bits || !bounds || !jobs) return cudaErrorInvalidValue;
     const int ppu = (g.L / 128 + 1) / 2, nT = g.L / 128;
-    schedule_kernel<<<1, 1024, 0, st>>>(tile_bits, tile_words(g.L), g.H, nT, ppu, g.BH * ppu, band_grid(g), bounds,
+    schedule_kernel<<<2, 1024, 0, st>>>(tile_bits, tile_words(g.L), g.H, nT, ppu, g.BH * ppu, band_grid(g), bounds,
                                         g.BH * nT, jobs);
     return cudaGetLastError();
 }
