@@ -1614,8 +1614,8 @@ cudaError_t launch_band_variant(const CUtensorMap& tmX, const CUtensorMap& tmY, 
                                        smem, st);
 }
 
-// Item ranges of the CTAs of a fused launch: contiguous, each holding about the same weight (an
-// item's active 128-row tiles, 0 to 2), so that units with few active tokens (padded sequences)
+// Item ranges of the CTAs of a fused launch: contiguous, each holding about the same weight (from
+// an item's active 128-row tiles, see weight below), so that units with few active tokens (padded sequences)
 // do not leave some CTAs with all-active items and others with none.  bounds[c] = the first item
 // i with (weight before i) * grid >= c * total; the last range runs to the end, so that every
 // item (inactive ones write their rows) belongs to exactly one CTA.  One CTA of 1024 threads.
@@ -1627,7 +1627,11 @@ __device__ void band_bounds_block(const uint32_t* bits, int words, int H, int nT
     auto weight = [&](int i) {
         const int bh = i / ppu, b = bh / H, p = i - bh * ppu;
         const uint32_t* bb = bits + size_t(b) * words;
-        return int(tile_bit(bb, 2 * p)) + ((2 * p + 1 < nT) ? int(tile_bit(bb, 2 * p + 1)) : 0);
+        const int halves = int(tile_bit(bb, 2 * p)) + ((2 * p + 1 < nT) ? int(tile_bit(bb, 2 * p + 1)) : 0);
+        // cost model, measured on a padded batch: an item's shared cost (its column tiles, waits
+        // and decode) weighs like one of its active row halves, an inactive item (its rows
+        // written as zeros) like a quarter of one
+        return halves ? 4 + 4 * halves : 1;
     };
     // total weight
     int t = 0;
