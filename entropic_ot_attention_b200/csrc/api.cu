@@ -184,8 +184,14 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     float* logm = at<float>(ws, w.logm);
     float* sd_row = p->dustbin ? at<float>(ws, w.sd_row) : nullptr;
     float* sd_col = p->dustbin ? at<float>(ws, w.sd_col) : nullptr;
+    float* ub2 = at<float>(ws, w.ub2);
+    float* vb2 = at<float>(ws, w.vb2);
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
 
-    EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
+    // marginals, tile bits and the zero potential's masked log2 bias (v = 0) in one launch
+    EOT_TRY(aux(st, [&] {
+        return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st, tbits, vb2);
+    }));
     float* dpart = p->dustbin ? at<float>(ws, w.dpart) : nullptr;
     uint32_t* dcnt = p->dustbin ? at<uint32_t>(ws, w.dcnt) : nullptr;
     if (p->dustbin) {
@@ -207,11 +213,6 @@ eot_status forward_impl(const eot_problem* p, const void* Q, const void* K, cons
     row.dpart = dpart;
     row.dcnt = dcnt;
     row.status = status;
-    float* ub2 = at<float>(ws, w.ub2);
-    float* vb2 = at<float>(ws, w.vb2);
-    EOT_TRY(aux(st, [&] { return launch_init_bias2(g, logm, vb2, st); }));
-    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
-    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
     row.tile_bits = tbits;
     int* bounds = at<int>(ws, w.bounds);
     int* jobs = nullptr;
@@ -496,7 +497,11 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     uint32_t* status = at<uint32_t>(ws, w.status);
     float* logm = at<float>(ws, w.logm);
     float *sd_row = nullptr, *sd_col = nullptr, *e1 = nullptr, *e2 = nullptr;
-    EOT_TRY(aux(st, [&] { return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st); }));
+    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
+    // marginals and tile bits in one launch
+    EOT_TRY(aux(st, [&] {
+        return launch_prep_marginals(g, mask, p->dustbin, p->dustbin_mass, logm, status, st, tbits);
+    }));
     float* dpart = p->dustbin ? at<float>(ws, w.dpart) : nullptr;
     uint32_t* dcnt = p->dustbin ? at<uint32_t>(ws, w.dcnt) : nullptr;
     if (p->dustbin) {
@@ -555,8 +560,6 @@ eot_status backward_impl(const eot_problem* p, const void* Q, const void* K, con
     rowp.dcnt = dcnt;
     rowp.zero_vec = at<float>(ws, w.zero);
     rowp.status = status;
-    uint32_t* tbits = at<uint32_t>(ws, w.tbits);
-    EOT_TRY(aux(st, [&] { return launch_tile_bits(g, logm, tbits, st); }));
     rowp.tile_bits = tbits;
     if (impl == EOT_IMPL_TCGEN05) {
         int* bounds = at<int>(ws, w.bounds);

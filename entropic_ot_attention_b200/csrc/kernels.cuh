@@ -37,8 +37,12 @@ struct BwdVecArgs {
     float isl2;
 };
 
+// Log marginals of every batch row from the mask (and clears the status word); when given, also
+// the tile bits of launch_tile_bits and the zero potential's masked log2 bias of launch_init_bias2
+// ([BH, L]), in the same launch.
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
-                                  uint32_t* status, cudaStream_t st);
+                                  uint32_t* status, cudaStream_t st, uint32_t* bits = nullptr,
+                                  float* bias2 = nullptr);
 cudaError_t launch_dustbin_dots(const Geom& g, const void* P, const void* Qm, float s1, float* term, float* dense,
                                 cudaStream_t st);
 cudaError_t launch_simt_lse(const LsePass& p, cudaStream_t st);

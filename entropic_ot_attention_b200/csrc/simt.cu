@@ -32,10 +32,14 @@ constexpr int kSNT = 256;  // threads per CTA
 // bytes read 16 at a time when the mask is 16-byte aligned), then write the row's log marginals
 // 4 at a time.
 // Block (b, j): counts the active real tokens of batch row b (every block of the row reads the
-// whole mask row, from L2 after the first) and writes positions [j kPrepSlice, (j + 1) kPrepSlice).
+// whole mask row, from L2 after the first) and writes positions [j kPrepSlice, (j + 1) kPrepSlice)
+// of the log marginals and, when asked, of the tile bits (the slice is word j of the row: warp w
+// votes for tile 32 j + w) and of the zero potential's masked log2 bias of every head.
 constexpr int kPrepSlice = 4096;
+static_assert(kPrepSlice == 32 * 128, "one 32-bit word of tile bits per slice");
 __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint8_t* mask, int dustbin,
-                                                              float mass, float* logm, uint32_t* status) {
+                                                              float mass, float* logm, uint32_t* status,
+                                                              uint32_t* bits, float* bias2) {
     const int b = blockIdx.x;
     const int L = g.L;
     const int w0 = blockIdx.y * kPrepSlice, w1 = min(L, w0 + kPrepSlice);
@@ -66,16 +70,34 @@ __global__ void __launch_bounds__(1024) prep_marginals_kernel(Geom g, const uint
     const double real_mass = use_db ? (1.0 - double(mass)) : 1.0;
     const float lr = n > 0 ? float(log(real_mass / double(n))) : neg_inf();
     const float ld = use_db ? float(log(double(mass))) : neg_inf();
-    for (int i0 = w0 + threadIdx.x * 4; i0 < w1; i0 += blockDim.x * 4) {
-        float v[4];
+    __shared__ uint32_t word;
+    if (threadIdx.x == 0) word = 0u;
+    __syncthreads();
+    // one pass of 4 positions a thread covers the slice (kPrepSlice = 4 x 1024)
+    const int i0 = w0 + threadIdx.x * 4;
+    bool any = false;
+    if (i0 < w1) {
+        float v[4], bz[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int i = i0 + j;
             const bool real = (mrow ? (mrow[i] != 0) : true) && (i < D);
+            any |= real;
             v[j] = real ? lr : neg_inf();
+            bz[j] = real ? 0.f : neg_inf();   // the dustbin never enters a band sum
             if (dustbin && i == D) v[j] = ld;
         }
         *reinterpret_cast<float4*>(logm + size_t(b) * L + i0) = make_float4(v[0], v[1], v[2], v[3]);
+        if (bias2)
+            for (int hh = 0; hh < g.H; ++hh)
+                *reinterpret_cast<float4*>(bias2 + (size_t(b) * g.H + hh) * L + i0) = make_float4(bz[0], bz[1], bz[2], bz[3]);
+    }
+    if (bits) {
+        // warp w holds the 128 positions of tile 32 j + w
+        const unsigned vote = __ballot_sync(0xffffffffu, any);
+        if ((threadIdx.x & 31) == 0 && vote) atomicOr(&word, 1u << (threadIdx.x >> 5));
+        __syncthreads();
+        if (threadIdx.x == 0) bits[size_t(b) * tile_words(L) + blockIdx.y] = word;
     }
     if (b == 0 && blockIdx.y == 0 && threadIdx.x == 0 && status) *status = 0u;
 }
@@ -674,10 +696,10 @@ __global__ void __launch_bounds__(256) bwd_vectors_kernel(BwdVecArgs a) {
 // Host launchers
 // ---------------------------------------------------------------------------------------
 cudaError_t launch_prep_marginals(const Geom& g, const uint8_t* mask, int dustbin, float mass, float* logm,
-                                  uint32_t* status, cudaStream_t st) {
+                                  uint32_t* status, cudaStream_t st, uint32_t* bits, float* bias2) {
     if (g.B == 0 || g.L == 0) return cudaSuccess;
     prep_marginals_kernel<<<dim3(g.B, (g.L + kPrepSlice - 1) / kPrepSlice), 1024, 0, st>>>(g, mask, dustbin, mass,
-                                                                                          logm, status);
+                                                                                          logm, status, bits, bias2);
     return cudaGetLastError();
 }
 
