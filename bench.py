@@ -521,6 +521,17 @@ def main():
     total_entries = sum_over_ranks(float(entries), dev)
     value = total_entries / (t_step * 1e-3)
 
+    # ---------------- verification (untimed): the device status after every call ----------------
+    # (each call clears the status word at its start, so the check after the timed steps sees the
+    # last call only; a bounded wait that ran out in an earlier step would go unnoticed)
+    for _ in range(args.steps):
+        fwd()
+        bwd()
+        for ws in (ws_f, ws_b):
+            st = _abi.eot_last_device_status(ws.data_ptr(), sp)
+            if st != 0:
+                raise RuntimeError(f"device status in the verification calls: {_abi.eot_status_string(st)}")
+
     # ---------------- per-kernel timing (CUDA events on the launching stream) ----------------
     _abi.eot_profile_begin()
     fwd()
