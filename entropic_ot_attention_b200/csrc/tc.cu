@@ -1009,9 +1009,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         const uint32_t* bits;
         bool act;
     };
+    // Every role walks list positions blockIdx.x, blockIdx.x + gridDim.x, ...; the job at the next
+    // position is read from the list one job ahead, so that its load is off the critical path.
+    auto list_at = [&](int pos) { return (a.jobs && pos < n_jobs) ? __ldg(a.jobs + pos) : pos; };
     auto job_of = [&](int job) {
         Job j;
-        if (a.jobs) job = __ldg(a.jobs + job);
         j.bh = job / nT;
         j.b = j.bh / a.H;
         j.r0 = (job - j.bh * nT) * C::BM;
@@ -1099,8 +1101,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             constexpr uint32_t late_bytes = C::YB + uint32_t(NV) * C::BN * 4;
             int issued_l = 0, issued_e = 0, itg = 0;
             bool ok = true;
+            int jnext = list_at(blockIdx.x);
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
-                const Job jb = job_of(job);
+                const int jcur = jnext;
+                jnext = list_at(job + gridDim.x);
+                const Job jb = job_of(jcur);
                 if (!jb.act) continue;
                 for (int t = jb.t_lo; t <= jb.t_hi; ++t) {
                     if (!tile_bit(jb.bits, t)) continue;
@@ -1147,8 +1152,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             const uint32_t dtm = tbase + (is_dp ? C::TM_DP : C::TM_S);
             const uint32_t atm = tbase + (is_dp ? C::TM_A : C::TM_X);
             const bool late = is_dp == LATE_W;   // this issuer's column tile (W for dP, Y for S) rides the late ring
+            int jnext = list_at(blockIdx.x);
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
-                const Job jb = job_of(job);
+                const int jcur = jnext;
+                jnext = list_at(job + gridDim.x);
+                const Job jb = job_of(jcur);
                 if (!jb.act) continue;
                 // this job's row tiles are in TMEM (copied once they had landed, with the row
                 // modifier tile XE that the dP product reads from shared memory)
@@ -1209,8 +1217,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
             if (FOLD) ptx::prefetch_tmap(&tmXE);
             int done = 0, itg = 0, jc = 0;
             bool ok = true, xpending = false;
+            int jnext = list_at(blockIdx.x);
             for (int job = blockIdx.x; job < n_jobs && ok; job += gridDim.x) {
-                const Job jb = job_of(job);
+                const int jcur = jnext;
+                jnext = list_at(job + gridDim.x);
+                const Job jb = job_of(jcur);
                 if (!jb.act) continue;
                 if (jc > 0) {
                     // the previous job's products (or, in a pass without them, its score
@@ -1283,8 +1294,11 @@ __global__ void __launch_bounds__(kSweepThreads, 1)
         const uint64_t SC2 = ptx::f2(a.sc2, a.sc2);
         int itg = 0, jc = 0;
         bool ok = true;
+        int jnext = list_at(blockIdx.x);
         for (int job = blockIdx.x; job < n_jobs; job += gridDim.x) {
-        const Job jb = job_of(job);
+        const int jcur = jnext;
+        jnext = list_at(job + gridDim.x);
+        const Job jb = job_of(jcur);
         const int r0 = jb.r0;
         const size_t base = jb.base;
         if (!jb.act) {
