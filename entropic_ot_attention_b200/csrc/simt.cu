@@ -573,20 +573,47 @@ __global__ void __launch_bounds__(256) dustbin_bwd_kernel(BwdPass p) {
     if (!last) return;
     __threadfence();
     const float* parts = p.dpart + size_t(bh) * ns * pw;
-    if (p.sout && threadIdx.x == 0) {
+    // The unit's partials, merged by the whole block in a fixed order (deterministic): the scalars
+    // by a strided sum and a tree, the vector by G = blockDim.x / d groups of d threads, group g
+    // summing partials g, g + G, ..., the groups then added in order.
+    if (p.sout) {
         float s1 = 0.f, s2 = 0.f;
-        for (int i = 0; i < ns; ++i) {
+        for (int i = threadIdx.x; i < ns; i += blockDim.x) {
             s1 += __ldcg(parts + size_t(i) * pw);
             s2 += __ldcg(parts + size_t(i) * pw + 1);
         }
-        float outv = (p.f ? p.f[base + D] : 1.f) * (s1 + (p.hv ? p.hv[base + D] : 0.f) * s2);
-        if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
-        p.sout[base + D] = outv;
+        red1[threadIdx.x] = s1;
+        red2[threadIdx.x] = s2;
     }
-    if (p.vout && threadIdx.x < d) {
+    __syncthreads();
+    if (p.sout) {
+        for (int st = 128; st > 0; st >>= 1) {
+            if (threadIdx.x < st) {
+                red1[threadIdx.x] += red1[threadIdx.x + st];
+                red2[threadIdx.x] += red2[threadIdx.x + st];
+            }
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) {
+            const float outv = (p.f ? p.f[base + D] : 1.f) * (red1[0] + (p.hv ? p.hv[base + D] : 0.f) * red2[0]);
+            if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
+            p.sout[base + D] = outv;
+        }
+    }
+    if (p.vout) {
+        const int G = int(blockDim.x) / d, g = int(threadIdx.x) / d, e = int(threadIdx.x) - g * d;
         float a = 0.f;
-        for (int i = 0; i < ns; ++i) a += __ldcg(parts + size_t(i) * pw + 2 + threadIdx.x);
-        static_cast<T*>(p.vout)[(base + D) * d + threadIdx.x] = from_f<T>(p.vscale * a);
+        if (g < G)
+            for (int i = g; i < ns; i += G) a += __ldcg(parts + size_t(i) * pw + 2 + e);
+        float* vsum = &vred[0][0];                     // (free again: the block's own part is written)
+        __syncthreads();
+        if (g < G) vsum[g * d + e] = a;
+        __syncthreads();
+        if (threadIdx.x < d) {
+            float v = 0.f;
+            for (int k = 0; k < G; ++k) v += vsum[k * d + threadIdx.x];
+            static_cast<T*>(p.vout)[(base + D) * d + threadIdx.x] = from_f<T>(p.vscale * v);
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) p.dcnt[bh] = 0u;   // ready for the next launch of this call
