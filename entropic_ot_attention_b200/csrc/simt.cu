@@ -319,12 +319,26 @@ __global__ void __launch_bounds__(256) dustbin_lse_kernel(LsePass p) {
         last = atomicAdd(p.dcnt + bh, 1u) == unsigned(ns - 1);
     }
     __syncthreads();
-    if (!last || threadIdx.x != 0) return;
+    if (!last) return;
     __threadfence();
+    // the unit's partials, merged by the whole block in a fixed order (strided, then a tree)
     float mm = neg_inf(), ss = 0.f;
-    for (int i = 0; i < ns; ++i) lse2_merge(mm, ss, __ldcg(part + 2 * i), __ldcg(part + 2 * i + 1));
+    for (int i = threadIdx.x; i < ns; i += blockDim.x) lse2_merge(mm, ss, __ldcg(part + 2 * i), __ldcg(part + 2 * i + 1));
+    sm_m[threadIdx.x] = mm;
+    sm_s[threadIdx.x] = ss;
+    __syncthreads();
+    for (int st = 128; st > 0; st >>= 1) {
+        if (threadIdx.x < st) {
+            float a = sm_m[threadIdx.x], bb = sm_s[threadIdx.x];
+            lse2_merge(a, bb, sm_m[threadIdx.x + st], sm_s[threadIdx.x + st]);
+            sm_m[threadIdx.x] = a;
+            sm_s[threadIdx.x] = bb;
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x != 0) return;
     p.dcnt[bh] = 0u;   // ready for the next launch of this call
-    float outv = logm[D] - (mm + log2f(ss)) * kLn2;
+    float outv = logm[D] - (sm_m[0] + log2f(sm_s[0])) * kLn2;
     if (!isfinite(outv)) atomicOr(p.status, kStatusNonFinite);
     p.out[pb + D] = outv;
     p.out_bias2[base + D] = neg_inf();   // the dustbin never enters a band sum
